@@ -1,0 +1,351 @@
+#!/usr/bin/env python
+"""Benchmark of the Llama-3-8B-shaped decoder forward pass on B200.
+
+One step = one full-model prefill (32 layers, embedding, final norm, LM head,
+greedy argmax) of B=1 sequence of 2048 seeded token ids, with N(0, 0.02)
+seeded weights. The line's ``value`` is prefill tokens/s over all GPUs
+(replicas: each rank runs its own model, no data-path collective). The same
+run measures the batch-32 KV-cache decode workload (context 4096 filled with
+N(0,1) K/V entries, 128 greedy steps at positions 4096..4223) under
+``decode``.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = 'tokens/s: 8B-shape prefill & batch-32 decode; % tensor/HBM roofline'
+PREFILL_B, PREFILL_S = 1, 2048
+DECODE_B, DECODE_CTX, DECODE_STEPS = 32, 4096, 128
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, 'MEASURED_PEAKS.json')) as f:
+            p = json.load(f)
+        return p['hbm_gbs'], p['bf16_tflops'], p['bf16_tflops_sustained'], 'measured'
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, 'fallback'
+
+
+# --------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ('index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,'
+              'clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,'
+              'clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap')
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.rows = []
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(['nvidia-smi', '-i', str(self.idx), f'--query-gpu={self.FIELDS}',
+                                      '--format=csv,noheader,nounits'], capture_output=True, text=True, timeout=5)
+                for ln in out.stdout.strip().splitlines():
+                    self.rows.append([c.strip() for c in ln.split(',')])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.rows:
+            return {'sm_mhz': None, 'sm_max_mhz': None, 'reasons': ['nvidia-smi unavailable'], 'samples': 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace('.', '').isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace('.', '').isdigit()]
+        names = ['hw_slowdown', 'hw_thermal_slowdown', 'sw_thermal_slowdown', 'sw_power_cap']
+        reasons = sorted({n for r in self.rows for n, v in zip(names, r[5:9]) if v.strip().lower() == 'active'})
+        return {'sm_mhz': statistics.median(sm) if sm else None, 'sm_max_mhz': max(mx) if mx else None,
+                'reasons': reasons, 'samples': len(self.rows)}
+
+
+# ------------------------------------------------------------ distributed
+def _dist():
+    ws = int(os.environ.get('WORLD_SIZE', '1'))
+    rank = int(os.environ.get('RANK', '0'))
+    local = int(os.environ.get('LOCAL_RANK', '0'))
+    return ws, rank, local
+
+
+def _max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device='cuda')
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(ws: int):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------- CPU oracle sample
+def oracle_prefill_sample(n_layers_model: int = 32, S: int = PREFILL_S):
+    """Time the CPU oracle (float32 numpy, as it stands) on one of the 32 layers
+    of the 8B model at S tokens; returns (tokens/s scaled to the full model,
+    seconds, description)."""
+    import numpy as np
+    from oracle import Oracle, Params
+    import seeded_inputs as si
+    p = Params(4096, n_layers_model, 32, 8, 128256, 14336)
+
+    class W(dict):
+        def __missing__(self, name):
+            if name.endswith('norm.weight'):
+                v = np.ones(4096, np.float32)
+            else:
+                shape = si.weight_shape(name, 4096, 32, 8, 14336, 128256)
+                v = si.bf16_bits_to_f32(si.weight(0, name, shape, n_layers_model, 0.02, 'bf16'))
+            self[name] = v
+            return v
+
+    w = W()
+    for k in si.LAYER_KEYS:                      # inputs are prepared outside the timed region
+        w[f'layers.0.{k}.weight']
+    x = si.bf16_bits_to_f32(si.normal(2, si.STREAM_HIDDEN, S * 4096, 1.0)).reshape(S, 4096)
+    orc = Oracle(p, w, dtype=np.float32)
+    t0 = time.perf_counter()
+    orc.layer(0, x, None, 0)
+    dt = time.perf_counter() - t0
+    tok_s = S / (dt * n_layers_model)
+    return tok_s, dt, f'oracle float32 numpy: 1 of {n_layers_model} layers of the 8B model at S={S}, x{n_layers_model}'
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    cores = os.cpu_count()
+    times = []
+    desc = ''
+    for i in range(args.warmup + args.steps):
+        tok_s, dt, desc = oracle_prefill_sample()
+        if i >= args.warmup:
+            times.append(dt)
+    dt = statistics.mean(times)
+    value = PREFILL_S / (dt * 32)
+    line = {'impl': 'reference', 'metric': METRIC, 'value': value, 'unit': 'tokens/s', 'n_gpus': args.gpus,
+            'steps': args.steps, 'warmup': args.warmup, 'ms_per_step': dt * 32 * 1e3, 'higher_is_better': True,
+            'scaling': 'weak', 'vs_baseline': None, 'dtype': 'f32', 'data': 'synthetic (seeded)',
+            'config': {'workload': 'llama3-8b-shape prefill B=1 S=2048 (CPU oracle on a 1-layer sample)'},
+            'cpu_baseline': {'value': value, 'unit': 'tokens/s', 'cores': cores, 'kind': 'oracle', 'sample': desc},
+            'e2e': {'value': value, 'unit': 'tokens/s', 'h2d_bytes_per_step': 0, 'd2h_bytes_per_step': 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    import numpy as np
+    import torch
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.init_process_group('nccl', timeout=datetime.timedelta(seconds=600), device_id=torch.device('cuda', local))
+    from llama_transformer_decoder_b200 import binding as L
+    from llama_transformer_decoder_b200.configs import LLAMA3_8B, make_config
+    import seeded_inputs as si
+    hbm_peak, tf_burst, tf_sust, peak_src = _peaks()
+
+    max_seq = DECODE_CTX + DECODE_STEPS + max(args.warmup, 1) + 8
+    cfg = make_config(LLAMA3_8B, dtype=L.LLAMA_BF16, max_batch=DECODE_B, max_seq=max_seq,
+                      max_tokens=PREFILL_B * PREFILL_S)
+    st = torch.cuda.Stream()
+    m = L.llama_create(cfg)
+    L.llama_init_weights(m, 0, 0.02, st)
+    toks_h = si.tokens(1, PREFILL_B * PREFILL_S, 128256).reshape(PREFILL_B, PREFILL_S)
+    toks = torch.from_numpy(toks_h).cuda()
+    arg = torch.empty(DECODE_B, dtype=torch.int32, device='cuda')
+    torch.cuda.synchronize()
+
+    def prefill_step():
+        L.llama_reset(m, st)
+        L.llama_prefill(m, toks, PREFILL_B, PREFILL_S, st)
+        L.llama_argmax(m, arg, st)
+
+    for _ in range(args.warmup):
+        prefill_step()
+    torch.cuda.synchronize()
+    assert L.llama_sync_status(m, st) == 0
+    _barrier(ws)
+    # ---- timed prefill region (per-kernel events recorded by the library on `st`)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    L.llama_profile(m, 1)
+    L.llama_profile_read(m)
+    n0 = L.llama_kernel_launches()
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        ev0.record(st)
+        for _ in range(args.steps):
+            prefill_step()
+        ev1.record(st)
+        torch.cuda.synchronize()
+    launches = L.llama_kernel_launches() - n0
+    prof = L.llama_profile_read(m)
+    L.llama_profile(m, 0)
+    _barrier(ws)
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms_max = _max_over_ranks(ms, ws)
+    value = ws * PREFILL_B * PREFILL_S / (ms_max / 1e3)
+
+    # roofline of the dominant kernel: the tcgen05 GEMM (all four projections, M = 2048)
+    D, F, H, Hk, d = 4096, 14336, 32, 8, 128
+    M = PREFILL_B * PREFILL_S
+    flops_layer = 2.0 * M * D * ((H + 2 * Hk) * d + H * d + 2 * F + F)
+    gemm_kinds = ['gemm_qkv_rope', 'gemm_wo_residual', 'gemm_w13_swiglu', 'gemm_w2_residual']
+    gemm_ms = sum(prof[k][0] for k in gemm_kinds)
+    gemm_launches = sum(prof[k][1] for k in gemm_kinds)
+    achieved = flops_layer * 32 * args.steps / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+    kernels = {k: {'ms_per_step': v[0] / args.steps, 'launches_per_step': v[1] / args.steps,
+                   'share': v[0] / max(sum(x[0] for x in prof.values()), 1e-9)} for k, v in prof.items() if v[1]}
+    attn_flops = 4.0 * PREFILL_B * H * d * PREFILL_S * (PREFILL_S + 1) / 2 * 32
+    attn = prof.get('attention_prefill', (0, 0))
+    roofline = {'kernel': 'gemm_wide_kernel (tcgen05, 4 projections)', 'bound': 'tensor',
+                'achieved': achieved, 'peak': tf_sust, 'unit': 'TFLOP/s',
+                'frac': achieved / tf_sust if achieved else None, 'traffic': None,
+                'peak_kind': f'bf16 sustained ({peak_src})', 'launches': gemm_launches // max(args.steps, 1),
+                'attention_tflops': attn_flops * args.steps / (attn[0] / 1e3) / 1e12 if attn[0] else None}
+
+    # ---- end to end through the host API (pinned host buffers)
+    host_toks = torch.from_numpy(toks_h.copy()).pin_memory()
+    host_out = torch.empty(PREFILL_B, dtype=torch.int32).pin_memory()
+    L.llama_reset(m, st)
+    L.llama_generate(m, host_toks, PREFILL_B, PREFILL_S, 0, host_out, st)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(ws)
+    e0.record(st)
+    for _ in range(args.steps):
+        L.llama_reset(m, st)
+        L.llama_generate(m, host_toks, PREFILL_B, PREFILL_S, 0, host_out, st)
+    e1.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, ws)
+    e2e = {'value': ws * PREFILL_B * PREFILL_S / (e2e_ms / 1e3), 'unit': 'tokens/s',
+           'h2d_bytes_per_step': PREFILL_B * PREFILL_S * 4, 'd2h_bytes_per_step': PREFILL_B * 4,
+           'api': 'llama_generate(host tokens, n_new=0)'}
+
+    # ---- batch-32 decode over a 4096-token cache
+    decode = None
+    if not args.no_decode:
+        L.llama_fill_kv_random(m, 3, DECODE_CTX, st)
+        first = torch.from_numpy(si.tokens(1, DECODE_B, 128256, start=PREFILL_B * PREFILL_S)).cuda()
+        lens = np.full(DECODE_B, DECODE_CTX, np.int32)
+
+        def decode_run(n, profile=False):
+            L.llama_set_lengths(m, lens, DECODE_B, st)
+            cur = first
+            for _ in range(n):
+                L.llama_decode_step(m, cur, DECODE_B, st)
+                L.llama_argmax(m, arg, st)
+                cur = arg
+
+        decode_run(max(args.warmup, 2))  # eager first call, then graph capture
+        torch.cuda.synchronize()
+        _barrier(ws)
+        L.llama_set_lengths(m, lens, DECODE_B, st)
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        cur = first
+        n_dec0 = L.llama_kernel_launches()
+        with ClockSampler(local) as dclk:
+            torch.cuda.synchronize()
+            d0.record(st)
+            for _ in range(DECODE_STEPS):
+                L.llama_decode_step(m, cur, DECODE_B, st)
+                L.llama_argmax(m, arg, st)
+                cur = arg
+            d1.record(st)
+            torch.cuda.synchronize()
+        dec_launches = L.llama_kernel_launches() - n_dec0
+        dms = _max_over_ranks(d0.elapsed_time(d1) / DECODE_STEPS, ws)
+        assert L.llama_sync_status(m, st) == 0
+        # profiled pass (eager, per-kernel events) for the breakdown
+        L.llama_profile(m, 1)
+        L.llama_profile_read(m)
+        decode_run(8)
+        dprof = L.llama_profile_read(m)
+        L.llama_profile(m, 0)
+        avg_ctx = DECODE_CTX + (DECODE_STEPS + 1) / 2.0
+        w_bytes = 32 * 2.0 * (D * (H + 2 * Hk) * d + D * H * d + 2 * D * F + D * F) + 2.0 * 128256 * D
+        kv_bytes = 32 * 2.0 * DECODE_B * avg_ctx * Hk * d * 2
+        step_bytes = w_bytes + kv_bytes
+        achieved_gbs = step_bytes / (dms / 1e3) / 1e9
+        decode = {'value': ws * DECODE_B / (dms / 1e3), 'unit': 'tokens/s', 'ms_per_step': dms,
+                  'steps': DECODE_STEPS, 'batch': DECODE_B, 'context': DECODE_CTX, 'graph_replay': True,
+                  'gpu_launches': dec_launches,
+                  'roofline': {'bound': 'hbm', 'achieved': achieved_gbs, 'peak': hbm_peak, 'unit': 'GB/s',
+                               'frac': achieved_gbs / hbm_peak, 'traffic': None,
+                               'algorithmic_bytes_per_step': step_bytes, 'peak_kind': f'hbm copy ({peak_src})'},
+                  'kernels_eager_profile': {k: {'ms_per_step': v[0] / 8, 'launches_per_step': v[1] / 8}
+                                            for k, v in dprof.items() if v[1]},
+                  'clocks': dclk.summary()}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        tok_s, dt, desc = oracle_prefill_sample()
+        cpu = {'value': tok_s, 'unit': 'tokens/s', 'cores': os.cpu_count(), 'kind': 'oracle', 'sample': desc,
+               'seconds': dt}
+
+    L.llama_destroy(m)
+    if rank == 0:
+        line = {'metric': METRIC, 'value': value, 'unit': 'tokens/s', 'n_gpus': ws, 'steps': args.steps,
+                'warmup': args.warmup, 'ms_per_step': ms_max, 'higher_is_better': True, 'scaling': 'weak',
+                'vs_baseline': None, 'dtype': 'bf16',
+                'data': 'synthetic: seeded N(0,0.02) weights of the 8B shapes, uniform token ids',
+                'config': {'workload': 'llama3-8b-shape full-model prefill, B=1, S=2048 (32 layers + LM head '
+                                       '+ argmax); decode: B=32, context 4096, 128 greedy steps',
+                           'batch': PREFILL_B, 'seq_len': PREFILL_S, 'layers': 32,
+                           'l2': 'inputs larger than L2 (16 GB of weights streamed per step)',
+                           'parallelism': f'replicas x{ws}'},
+                'roofline': roofline, 'cpu_baseline': cpu, 'e2e': e2e, 'gpu_launches': launches,
+                'clocks': clk.summary(), 'kernels': kernels, 'decode': decode}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument('--gpus', type=int, default=1)
+    ap.add_argument('--steps', type=int, default=5)
+    ap.add_argument('--warmup', type=int, default=3)
+    ap.add_argument('--impl', choices=['ours', 'reference'], default='ours')
+    ap.add_argument('--no-decode', action='store_true')
+    ap.add_argument('--no-cpu-baseline', action='store_true')
+    args = ap.parse_args()
+    if args.impl == 'reference':
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == '__main__':
+    sys.exit(main())

@@ -1,0 +1,206 @@
+/*
+ * llama_b200.h — C ABI of the Llama-3 decoder forward pass on B200 (sm_100a).
+ *
+ * What is computed follows the Llama-3 walkthrough "250行代码从头搭建Llama 3，
+ * GitHub一天4.6k星！Karpathy大赞" (ai02.cc), cited below as [W] with its section:
+ * token embedding (分词器与编码), RMSNorm (构建Transformer层), per-head Q/K/V
+ * projections (查询向量, 键向量, 值向量), rotary position embedding on adjacent
+ * pairs (位置编码), causal grouped-query attention (查询和键相乘, 掩码,
+ * 多头注意力), the Wo projection plus residual (相加与归一化), the SwiGLU
+ * feed-forward plus residual (前馈神经网络层), the layer stack, the final
+ * norm, last-token logits and greedy argmax (预测下一个输出). The KV cache is
+ * the one described by "Deepdive-llama3-from-scratch" (KV-Cache chapter) and
+ * sized up front by max_seq_len x max_batch_size as the Hacker News thread
+ * "Llama 3 implemented in pure NumPy" explains.
+ *
+ * Conventions for every call:
+ *  - Return value: LLAMA_OK (0) or a negative LLAMA_ERR_* code. No call throws
+ *    or aborts. Errors detected inside a kernel (bad token id, timeout of a
+ *    bounded wait) are latched in a device status word and returned by the
+ *    next llama_sync_status() (model calls) or llama_status() (stateless
+ *    calls).
+ *  - Pointers named "device" are CUDA device pointers; the caller owns them
+ *    and the library never frees them. `stream` is a cudaStream_t passed as
+ *    void* (NULL = legacy default stream); calls are asynchronous on it
+ *    unless stated otherwise.
+ *  - Matrices are row-major and contiguous. Weights use the checkpoint's
+ *    [out, in] convention and y = x W^T ([W] 查询向量).
+ *  - dtype: LLAMA_F32 computes everything in fp32 on the CUDA cores;
+ *    LLAMA_BF16 stores weights, activations and the cache in bf16 and
+ *    accumulates in fp32 on the tensor cores (tcgen05), with an fp32 residual
+ *    stream and fp32 logits.
+ *  - A model and its buffers belong to the device that was current at
+ *    llama_create; make that device current before every later call.
+ */
+#ifndef LLAMA_B200_H
+#define LLAMA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LLAMA_OK 0
+#define LLAMA_ERR_INVALID_ARG (-1)   /* null pointer, bad enum, misaligned buffer */
+#define LLAMA_ERR_SHAPE (-2)         /* sizes violate the model or the call's limits */
+#define LLAMA_ERR_OOM (-3)           /* device allocation failed */
+#define LLAMA_ERR_CUDA (-4)          /* a CUDA runtime/driver call failed */
+#define LLAMA_ERR_DEVICE_TIMEOUT (-5)/* a bounded device-side wait gave up */
+#define LLAMA_ERR_DEVICE_BOUNDS (-6) /* an index checked on the device was out of range */
+#define LLAMA_ERR_UNSUPPORTED (-7)   /* combination not implemented (e.g. bf16 with head_dim != 128) */
+
+typedef enum { LLAMA_F32 = 0, LLAMA_BF16 = 1 } llama_dtype;
+
+/* Model statement: the fields of params.json ([W] 下载并读取模型权重) plus the
+ * cache sizing of the Hacker News thread (max_batch, max_seq). */
+typedef struct llama_config {
+  int32_t dim;                /* 4096 for the 8B model */
+  int32_t n_layers;           /* 32 */
+  int32_t n_heads;            /* 32; head_dim = dim / n_heads */
+  int32_t n_kv_heads;         /* 8; n_heads % n_kv_heads == 0 */
+  int32_t vocab_size;         /* 128256 */
+  int32_t ffn_hidden;         /* SwiGLU width; 0 = derive with llama_ffn_hidden */
+  int32_t multiple_of;        /* 1024 */
+  float ffn_dim_multiplier;   /* 1.3; <= 0 means none */
+  float norm_eps;             /* 1e-5 */
+  float rope_theta;           /* 500000 */
+  int32_t max_batch;          /* sequences held in the KV cache */
+  int32_t max_seq;            /* positions per sequence in the KV cache */
+  int32_t max_tokens;         /* largest B*S of one prefill call; 0 = min(max_batch*max_seq, 16384) */
+  int32_t dtype;              /* llama_dtype */
+} llama_config;
+
+typedef struct llama_model llama_model; /* opaque: weights, KV cache, lengths, workspace */
+
+/* SwiGLU width from params.json: multiple_of * ceil(int(mult * floor(8*dim/3)) / multiple_of),
+ * the multiplier step skipped when mult <= 0. ([W] 下载并读取模型权重 prints multiple_of and
+ * ffn_dim_multiplier only; this reading gives 14336 for dim 4096.) */
+int32_t llama_ffn_hidden(int32_t dim, int32_t multiple_of, float ffn_dim_multiplier);
+
+/* Validates cfg, allocates weights, KV cache ([n_layers][max_batch][n_kv_heads][max_seq][head_dim]
+ * for K and for V), the RoPE table and the workspace on the current device. Weights are zero until
+ * llama_init_weights or llama_set_weight. All sequence lengths start at 0. Synchronous. */
+int llama_create(const llama_config* cfg, llama_model** out);
+void llama_destroy(llama_model* m);
+/* Copy of the resolved configuration (ffn_hidden and max_tokens filled in). */
+int llama_get_config(const llama_model* m, llama_config* out);
+/* Bytes of device memory held by the model. */
+size_t llama_device_bytes(const llama_model* m);
+
+/* Seeded synthetic weights: every matrix N(0, std^2) from the counter-based generator
+ * (SplitMix64 streams + Box-Muller, one stream per checkpoint key in the key order of
+ * [W] 下载并读取模型权重), rounded to the model dtype; every norm weight 1.0. Produces the
+ * same bits as the host generator in the repository's seeded_inputs module. */
+int llama_init_weights(llama_model* m, uint64_t seed, float std, void* stream);
+
+/* Copy one checkpoint tensor in or out, by its checkpoint name ("tok_embeddings.weight",
+ * "layers.{i}.attention.wq.weight", ..., "norm.weight", "output.weight"), in the checkpoint's
+ * [out, in] layout and in the model dtype (norm weights are always fp32). nbytes must equal the
+ * tensor's size. on_device: 1 if src/dst is device memory, 0 for host memory. */
+int llama_set_weight(llama_model* m, const char* name, const void* src, size_t nbytes, int on_device, void* stream);
+int llama_get_weight(llama_model* m, const char* name, void* dst, size_t nbytes, int on_device, void* stream);
+
+/* Prefill: tokens (device int32 [B][S]) are appended to sequences 0..B-1 at positions
+ * len[b] .. len[b]+S-1, their post-RoPE K and V written to the cache, and the last token's
+ * logits of each sequence kept ([W] 预测下一个输出: final norm once, final_embedding[-1] @
+ * output^T). Requires B <= max_batch, B*S <= max_tokens, len[b]+S <= max_seq. len[b] += S. */
+int llama_prefill(llama_model* m, const int32_t* tokens, int32_t B, int32_t S, void* stream);
+
+/* One decode step: token b (device int32 [B]) is processed at position len[b] of sequence b,
+ * attending to keys 0..len[b] through the cache; len[b] += 1. Logits are kept as for prefill.
+ * The step is replayed from a CUDA graph after its first call for a given B. */
+int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t B, void* stream);
+
+/* fp32 logits [B][vocab] (device) of the last prefill or decode step. */
+int llama_logits(llama_model* m, float* dst, void* stream);
+/* Greedy next token of each sequence (device int32 [B]): the largest logit, the lowest index
+ * among equal maxima ([W] 预测下一个输出: torch.argmax). */
+int llama_argmax(llama_model* m, int32_t* dst, void* stream);
+
+/* End to end from host memory: copies tokens (host int32 [B][S]) to the device, prefills, then
+ * runs n_new greedy decode steps feeding each argmax back, and copies the B*(n_new+1) chosen
+ * tokens ([B][n_new+1], host) back. Synchronizes the stream before returning. */
+int llama_generate(llama_model* m, const int32_t* host_tokens, int32_t B, int32_t S, int32_t n_new,
+                   int32_t* host_out, void* stream);
+
+/* One decoder block on given hidden states: x (device fp32 [B][S][dim]) is the residual stream
+ * entering layer `layer` at positions len[b]..len[b]+S-1; y (device fp32, same shape) receives
+ * its output. The layer's cache entries are written; lengths are NOT advanced. */
+int llama_block_forward(llama_model* m, int32_t layer, const float* x, float* y, int32_t B, int32_t S,
+                        void* stream);
+
+/* Cache and length control. llama_fill_kv_random writes N(0,1) K and V entries (taken as
+ * already rotated) for positions 0..c-1 of every layer and every sequence < max_batch from the
+ * seeded generator (layer l: stream 2^21+2l for K, +1 for V, element order [b][g][t][d]) and
+ * sets every length to c. llama_set_kv copies caller K/V (device, model dtype,
+ * [B][n_kv_heads][c][head_dim]) into layer `layer`, positions 0..c-1. Lengths are host-visible
+ * state: set_lengths takes host int32 [B] (B <= max_batch); reset sets all to 0. */
+int llama_fill_kv_random(llama_model* m, uint64_t seed, int32_t c, void* stream);
+int llama_set_kv(llama_model* m, int32_t layer, const void* k, const void* v, int32_t B, int32_t c, void* stream);
+int llama_set_lengths(llama_model* m, const int32_t* host_len, int32_t B, void* stream);
+int llama_get_lengths(const llama_model* m, int32_t* host_len, int32_t B);
+int llama_reset(llama_model* m, void* stream);
+
+/* Per-kernel timing of eager model calls: while enabled (1), an event is recorded on the
+ * launching stream before every kernel launch of prefill/decode/argmax (CUDA-graph replay is
+ * bypassed). llama_profile_read synchronizes, then fills ms[k] (summed time from the launch's
+ * event to the next one) and launches[k] for kinds k < n_kinds, clears the record and returns
+ * the number of kinds (embed, rmsnorm, gemm_qkv_rope, attention_prefill, attention_decode,
+ * gemm_wo_residual, gemm_w13_swiglu, gemm_w2_residual, gemm_lm_head, other). */
+int llama_profile(llama_model* m, int enable);
+int llama_profile_read(llama_model* m, double* ms, int64_t* launches, int n_kinds);
+const char* llama_profile_kind_name(int kind);
+/* Kernels launched by the model entry points in this process so far (graph replays count
+ * their kernels). */
+uint64_t llama_kernel_launches(void);
+
+/* Synchronizes `stream`, then returns and clears the model's latched device status. */
+int llama_sync_status(llama_model* m, void* stream);
+const char* llama_status_string(int status);
+
+/* ---------------------------------------------------------------- stateless kernels
+ * Same kernels as the model, on caller buffers (device pointers, dtype = element type of
+ * q/k/v/o/x/w). They use library-owned scratch on the current device, allocated on first use. */
+
+/* Causal GQA attention for prefill ([W] 查询和键相乘, 掩码, 多头注意力): q [B][H][S][d],
+ * k, v [B][Hk][S][d] (already rotated), o [B][S][H*d]; query s sees keys 0..s; head h reads kv
+ * head h / (H/Hk); scores scaled by 1/sqrt(d). bf16 requires d = 128; fp32 takes d in {32,64,128}. */
+int llama_attention_prefill(const void* q, const void* k, const void* v, void* o, int32_t B, int32_t S, int32_t H,
+                            int32_t Hk, int32_t d, int32_t dtype, void* stream);
+
+/* Single-query attention over a cache (decode): q [B][H][d]; kc, vc [B][Hk][cmax][d]; len
+ * (device int32 [B], 1 <= len[b] <= cmax) = number of valid keys of sequence b; o [B][H*d].
+ * Split over the key range, merged with the log-sum-exp rule. d in {64,128} (bf16) or
+ * {32,64,128} (fp32); H/Hk <= 8. */
+int llama_attention_decode(const void* q, const void* kc, const void* vc, const int32_t* len, void* o, int32_t B,
+                           int32_t cmax, int32_t H, int32_t Hk, int32_t d, int32_t dtype, void* stream);
+
+/* y = x W^T: x [M][K], w [N][K] (dtype), y fp32 [M][N]. variant 0 = automatic, 1 = the wide
+ * persistent tcgen05 kernel, 2 = the skinny split-K tcgen05 kernel (M <= 256); fp32 ignores it.
+ * bf16 requires K % 8 == 0 and 16-byte aligned x and w. */
+int llama_linear(const void* x, const void* w, float* y, int32_t M, int32_t N, int32_t K, int32_t dtype,
+                 int32_t variant, void* stream);
+
+/* y = x * rsqrt(mean(x^2) + eps) * g per row ([W] 构建Transformer层): x fp32 [M][D], g fp32 [D],
+ * y [M][D] in dtype. */
+int llama_rmsnorm(const float* x, const float* g, void* y, int32_t M, int32_t D, float eps, int32_t dtype,
+                  void* stream);
+
+/* Row-wise argmax of fp32 logits [B][V] into int32 [B], lowest index among equal maxima. */
+int llama_argmax_rows(const float* logits, int32_t* out, int32_t B, int32_t V, void* stream);
+
+/* n draws of N(0, std^2) of stream `stream_id` under `seed` (the weight generator) into dst
+ * (device, dtype). */
+int llama_fill_normal(void* dst, int64_t n, uint64_t seed, uint64_t stream_id, float std, int32_t dtype,
+                      void* stream);
+
+/* Synchronizes `stream`, then returns and clears the status word of the stateless calls. */
+int llama_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLAMA_B200_H */

@@ -1,0 +1,553 @@
+// Causal grouped-query attention over the KV cache.
+//
+//  * prefill (bf16): flash-style, one CTA per (64-query tile, q head, batch).
+//    K/V tiles of 64 keys are double-buffered in shared memory with cp.async,
+//    S = Q K^T and O += P V run on the tensor cores (mma.sync m16n8k16, bf16 in,
+//    fp32 accumulate), and the softmax is online in registers with quad
+//    shuffles. P is rounded to bf16 for the PV product, as the walkthrough does
+//    (softmax(...).to(bfloat16)). Query i at absolute position pos0+i sees keys
+//    0 .. pos0+i.
+//  * prefill (fp32): one warp per query row on the CUDA cores.
+//  * decode (both dtypes): split over the cached keys. Each CTA serves the
+//    H/Hk query heads of one kv head, streams its key range through shared
+//    memory with bulk async copies (the step is bound by HBM reads of the
+//    cache), keeps (max, sum, o) per head, and a combine kernel merges the
+//    splits with the log-sum-exp rule.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace llama {
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------ bf16 prefill (mma)
+constexpr int PB_Q = 64, PB_K = 64, PB_D = 128;
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
+  const int n = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Tile rows are 256 B (128 bf16); 16-byte chunk c of row r lives at chunk c ^ (r & 7).
+__device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 256 + ((c ^ (r & 7)) << 4)); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Copy rows [row0, row0+64) of a [rows][128] bf16 matrix into a swizzled tile;
+// rows >= nrows are zero filled.
+__device__ __forceinline__ void load_tile(uint8_t* tile, const bf16* src, int row0, int nrows) {
+  for (int i = threadIdx.x; i < 64 * 16; i += 128) {
+    const int r = i >> 4, c = i & 15;
+    const int gr = row0 + r;
+    const bool ok = gr < nrows;
+    cp_async16(tile + swz(r, c), src + (size_t)(ok ? gr : 0) * PB_D + c * 8, ok);
+  }
+}
+
+__global__ void __launch_bounds__(128) attn_prefill_bf16_kernel(const bf16* __restrict__ q,
+                                                                const bf16* __restrict__ kc,
+                                                                const bf16* __restrict__ vc, bf16* __restrict__ o,
+                                                                const int32_t* __restrict__ pos0, int S, int H,
+                                                                int Hk, int Smax, float scale_log2) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint8_t* sQ = sm;
+  uint8_t* sK = sm + PB_Q * 256;          // 2 buffers of 64 x 256 B
+  uint8_t* sV = sK + 2 * PB_K * 256;
+  const int nqt = gridDim.x;
+  const int qt = nqt - 1 - blockIdx.x;     // longest (last) query tiles first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int g = h / (H / Hk);
+  const int p0 = pos0 ? pos0[b] : 0;
+  const int T = p0 + S;                    // keys visible to the last query
+  const int q_lo = qt * PB_Q;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const bf16* qsrc = q + ((size_t)b * H + h) * S * PB_D;
+  const bf16* ksrc = kc + ((size_t)b * Hk + g) * Smax * PB_D;
+  const bf16* vsrc = vc + ((size_t)b * Hk + g) * Smax * PB_D;
+  const int k_end = min(T, p0 + q_lo + PB_Q);          // keys needed by this tile
+  const int n_kt = (k_end + PB_K - 1) / PB_K;
+
+  load_tile(sQ, qsrc, q_lo, S);
+  load_tile(sK, ksrc, 0, T);
+  load_tile(sV, vsrc, 0, T);
+  cp_async_commit();
+
+  float oacc[16][4];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+  const int r_in = warp * 16 + (lane >> 2);              // this thread's rows: r_in and r_in + 8
+  const int qpos0 = p0 + q_lo + r_in, qpos1 = qpos0 + 8;
+  uint32_t qf[8][4];
+
+  for (int kt = 0; kt < n_kt; ++kt) {
+    const int buf = kt & 1;
+    if (kt + 1 < n_kt) {
+      load_tile(sK + (buf ^ 1) * PB_K * 256, ksrc, (kt + 1) * PB_K, T);
+      load_tile(sV + (buf ^ 1) * PB_K * 256, vsrc, (kt + 1) * PB_K, T);
+    }
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    if (kt == 0) {
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const int r = warp * 16 + (lane & 15), c = ks * 2 + (lane >> 4);
+        ldsm_x4(smem_u32(sQ) + swz(r, c), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+      }
+    }
+    const uint32_t kb = smem_u32(sK + buf * PB_K * 256), vb = smem_u32(sV + buf * PB_K * 256);
+    // S = Q K^T : 16 rows x 64 keys per warp
+    float s[8][4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+      for (int jp = 0; jp < 4; ++jp) {  // two 8-key blocks per ldmatrix.x4
+        const int r = jp * 16 + (lane & 7) + ((lane >> 4) << 3);
+        const int c = ks * 2 + ((lane >> 3) & 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kb + swz(r, c), b0, b1, b2, b3);
+        mma_bf16(s[2 * jp], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b0, b1);
+        mma_bf16(s[2 * jp + 1], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b2, b3);
+      }
+    }
+    // scale, mask, online softmax
+    const int kbase = kt * PB_K;
+    const bool need_mask = kbase + PB_K - 1 > p0 + q_lo;   // some key may be in a query's future
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = kbase + j * 8 + (lane & 3) * 2 + (e & 1);
+        const int qp = (e < 2) ? qpos0 : qpos1;
+        float v = s[j][e] * scale_log2;
+        if (need_mask && key > qp) v = -INFINITY;
+        s[j][e] = v;
+        mx[e >> 1] = fmaxf(mx[e >> 1], v);
+      }
+    }
+    float corr[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
+      mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 2));
+      const float mnew = fmaxf(mrow[i], mx[i]);
+      corr[i] = exp2f(mrow[i] - mnew);
+      mrow[i] = mnew;
+    }
+    float ls[2] = {0.f, 0.f};
+    uint32_t pf[4][4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float p0v = exp2f(s[j][0] - mrow[0]), p1v = exp2f(s[j][1] - mrow[0]);
+      const float p2v = exp2f(s[j][2] - mrow[1]), p3v = exp2f(s[j][3] - mrow[1]);
+      ls[0] += p0v + p1v;
+      ls[1] += p2v + p3v;
+      const int ks = j >> 1;
+      if ((j & 1) == 0) { pf[ks][0] = pack_bf16(p0v, p1v); pf[ks][1] = pack_bf16(p2v, p3v); }
+      else { pf[ks][2] = pack_bf16(p0v, p1v); pf[ks][3] = pack_bf16(p2v, p3v); }
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      ls[i] += __shfl_xor_sync(0xffffffffu, ls[i], 1);
+      ls[i] += __shfl_xor_sync(0xffffffffu, ls[i], 2);
+      lrow[i] = lrow[i] * corr[i] + ls[i];
+    }
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      oacc[n][0] *= corr[0]; oacc[n][1] *= corr[0];
+      oacc[n][2] *= corr[1]; oacc[n][3] *= corr[1];
+    }
+    // O += P V : V tile [64 keys][128 dims], B operand via transposed ldmatrix
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+#pragma unroll
+      for (int np = 0; np < 8; ++np) {  // two 8-dim blocks per ldmatrix.x4
+        const int r = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        const int c = np * 2 + (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vb + swz(r, c), b0, b1, b2, b3);
+        mma_bf16(oacc[2 * np], pf[ks][0], pf[ks][1], pf[ks][2], pf[ks][3], b0, b1);
+        mma_bf16(oacc[2 * np + 1], pf[ks][0], pf[ks][1], pf[ks][2], pf[ks][3], b2, b3);
+      }
+    }
+    __syncthreads();
+  }
+  // normalise and store o[b*S + s][h*128 + :]
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int srow = q_lo + r_in + i * 8;
+    if (srow >= S) continue;
+    const float inv = 1.f / lrow[i];
+    bf16* dst = o + ((size_t)b * S + srow) * H * PB_D + h * PB_D;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      const int col = n * 8 + (lane & 3) * 2;
+      *reinterpret_cast<uint32_t*>(dst + col) = pack_bf16(oacc[n][2 * i] * inv, oacc[n][2 * i + 1] * inv);
+    }
+  }
+}
+
+// ------------------------------------------------------ fp32 prefill (SIMT)
+template <int D>
+__global__ void __launch_bounds__(32) attn_prefill_f32_kernel(const float* __restrict__ q,
+                                                              const float* __restrict__ kc,
+                                                              const float* __restrict__ vc, float* __restrict__ o,
+                                                              const int32_t* __restrict__ pos0, int S, int H,
+                                                              int Hk, int Smax, float scale_log2) {
+  constexpr int DPL = D / 32;
+  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z, lane = threadIdx.x;
+  const int g = h / (H / Hk);
+  const int qp = (pos0 ? pos0[b] : 0) + s;
+  const float* qv = q + (((size_t)b * H + h) * S + s) * D;
+  const float* kb = kc + ((size_t)b * Hk + g) * Smax * D;
+  const float* vb = vc + ((size_t)b * Hk + g) * Smax * D;
+  float acc[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) acc[i] = 0.f;
+  float m = -INFINITY, l = 0.f;
+  for (int j0 = 0; j0 <= qp; j0 += 32) {
+    const int j = j0 + lane;
+    float sc = -INFINITY;
+    if (j <= qp) {
+      float dot = 0.f;
+      for (int t = 0; t < D; ++t) dot = fmaf(qv[t], kb[(size_t)j * D + t], dot);
+      sc = dot * scale_log2;
+    }
+    float cm = sc;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+    const float mn = fmaxf(m, cm);
+    const float corr = exp2f(m - mn);
+    const float p = (j <= qp) ? exp2f(sc - mn) : 0.f;
+    float ps = p;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+    l = l * corr + ps;
+    m = mn;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) acc[i] *= corr;
+    const int nk = min(32, qp + 1 - j0);
+    for (int jj = 0; jj < nk; ++jj) {
+      const float pj = __shfl_sync(0xffffffffu, p, jj);
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) acc[i] = fmaf(pj, vb[(size_t)(j0 + jj) * D + lane + 32 * i], acc[i]);
+    }
+  }
+  float* dst = o + ((size_t)b * S + s) * H * D + h * D;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) dst[lane + 32 * i] = acc[i] / l;
+}
+
+// ------------------------------------------------------------ decode
+constexpr int DEC_STAGES = 3;
+// keys per shared-memory stage: K and V rows of one stage fill at most 64 KB
+template <typename T, int D>
+__host__ __device__ constexpr int dec_sub() { return (32768 / (D * (int)sizeof(T))) < 128 ? (32768 / (D * (int)sizeof(T))) : 128; }
+constexpr int DEC_MAXG = 8;      // query heads per kv head supported
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128) attn_decode_part_kernel(const T* __restrict__ q, const T* __restrict__ kc,
+                                                               const T* __restrict__ vc,
+                                                               const int32_t* __restrict__ nkeys, int add_keys,
+                                                               float* __restrict__ part, int H, int Hk, int Smax,
+                                                               int chunk, float scale_log2, int* status) {
+  constexpr int DPL = D / 32;                       // dims per lane
+  constexpr int DEC_SUB = dec_sub<T, D>();
+  constexpr int ROW = D * (int)sizeof(T);           // bytes per cached key
+  constexpr int STAGE = 2 * DEC_SUB * ROW;          // K and V rows of one stage
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + DEC_STAGES * STAGE);
+  float* red = reinterpret_cast<float*>(bars + DEC_STAGES);   // [4 warps][G][D + 2]
+
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z, splits = gridDim.x;
+  const int G = H / Hk;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = nkeys[b] + add_keys;
+  const int k_lo = split * chunk;
+  const int k_hi = min(n, k_lo + chunk);
+  const int nsub = k_hi > k_lo ? (k_hi - k_lo + DEC_SUB - 1) / DEC_SUB : 0;
+  const T* ksrc = kc + ((size_t)b * Hk + g) * Smax * D;
+  const T* vsrc = vc + ((size_t)b * Hk + g) * Smax * D;
+
+  if (n > Smax && threadIdx.x == 0) set_status(status, LLAMA_ERR_DEVICE_BOUNDS);
+
+  // this lane's slice of the G query vectors, pre-scaled for exp2
+  float qr[DEC_MAXG][DPL];
+#pragma unroll
+  for (int gg = 0; gg < DEC_MAXG; ++gg)
+#pragma unroll
+    for (int i = 0; i < DPL; ++i)
+      qr[gg][i] = gg < G ? to_f<T>(q[((size_t)b * H + g * G + gg) * D + lane * DPL + i]) * scale_log2 : 0.f;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < DEC_STAGES; ++s) mbar_init(&bars[s], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  auto issue = [&](int sub) {
+    const int st = sub % DEC_STAGES;
+    const int k0 = k_lo + sub * DEC_SUB;
+    const int rows = min(DEC_SUB, k_hi - k0);
+    uint8_t* dst = sm + st * STAGE;
+    mbar_arrive_expect_tx(&bars[st], 2 * rows * ROW);
+    bulk_load(dst, ksrc + (size_t)k0 * D, rows * ROW, &bars[st]);
+    bulk_load(dst + DEC_SUB * ROW, vsrc + (size_t)k0 * D, rows * ROW, &bars[st]);
+  };
+  if (threadIdx.x == 0 && n <= Smax)
+    for (int s = 0; s < DEC_STAGES && s < nsub; ++s) issue(s);
+
+  float m[DEC_MAXG], l[DEC_MAXG], acc[DEC_MAXG][DPL];
+#pragma unroll
+  for (int gg = 0; gg < DEC_MAXG; ++gg) {
+    m[gg] = -INFINITY;
+    l[gg] = 0.f;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) acc[gg][i] = 0.f;
+  }
+  bool ok = n <= Smax;
+  int fail_sub = nsub;
+  for (int sub = 0; sub < nsub && ok; ++sub) {
+    const int st = sub % DEC_STAGES;
+    const bool arrived = mbar_wait(&bars[st], (sub / DEC_STAGES) & 1, status);
+    if (!__syncthreads_and(arrived)) { ok = false; fail_sub = sub; break; }
+    const int k0 = k_lo + sub * DEC_SUB;
+    const int rows = min(DEC_SUB, k_hi - k0);
+    const T* sk = reinterpret_cast<const T*>(sm + st * STAGE);
+    const T* sv = reinterpret_cast<const T*>(sm + st * STAGE + DEC_SUB * ROW);
+    // this warp's 32 keys of the stage: lane kk keeps the scores of key kk
+    const int kw = warp * 32;
+    float mine[DEC_MAXG];
+#pragma unroll
+    for (int gg = 0; gg < DEC_MAXG; ++gg) mine[gg] = -INFINITY;
+    const int nk = min(32, rows - kw);
+    for (int kk = 0; kk < nk; ++kk) {
+      float kv[DPL];
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) kv[i] = to_f<T>(sk[(size_t)(kw + kk) * D + lane * DPL + i]);
+#pragma unroll
+      for (int gg = 0; gg < DEC_MAXG; ++gg) {
+        if (gg < G) {
+          float dot = 0.f;
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) dot = fmaf(qr[gg][i], kv[i], dot);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+          if (lane == kk) mine[gg] = dot;
+        }
+      }
+    }
+    float p[DEC_MAXG];
+#pragma unroll
+    for (int gg = 0; gg < DEC_MAXG; ++gg) {
+      if (gg < G && nk > 0) {
+        float cm = mine[gg];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+        const float mn = fmaxf(m[gg], cm);
+        const float corr = exp2f(m[gg] - mn);
+        p[gg] = lane < nk ? exp2f(mine[gg] - mn) : 0.f;
+        float ps = p[gg];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+        l[gg] = l[gg] * corr + ps;
+        m[gg] = mn;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) acc[gg][i] *= corr;
+      } else {
+        p[gg] = 0.f;
+      }
+    }
+    for (int kk = 0; kk < nk; ++kk) {
+      float vv[DPL];
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) vv[i] = to_f<T>(sv[(size_t)(kw + kk) * D + lane * DPL + i]);
+#pragma unroll
+      for (int gg = 0; gg < DEC_MAXG; ++gg) {
+        if (gg < G) {
+          const float pk = __shfl_sync(0xffffffffu, p[gg], kk);
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) acc[gg][i] = fmaf(pk, vv[i], acc[gg][i]);
+        }
+      }
+    }
+    __syncthreads();  // every warp is done with this stage before it is refilled
+    if (threadIdx.x == 0 && sub + DEC_STAGES < nsub) issue(sub + DEC_STAGES);
+  }
+  if (!ok && threadIdx.x == 0) {
+    // do not leave copies in flight: wait (bounded) for every issued stage
+    for (int sub = fail_sub; sub < nsub && sub < fail_sub + DEC_STAGES; ++sub)
+      mbar_wait(&bars[sub % DEC_STAGES], (sub / DEC_STAGES) & 1, status);
+  }
+  // merge the 4 warps' states, then write this split's (o, max, sum) per head
+  for (int gg = 0; gg < G; ++gg) {
+    float* r = red + ((size_t)warp * DEC_MAXG + gg) * (D + 2);
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) r[lane * DPL + i] = acc[gg][i];
+    if (lane == 0) { r[D] = m[gg]; r[D + 1] = l[gg]; }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < G * D; idx += 128) {
+    const int gg = idx / D, dd = idx - gg * D;
+    float M = -INFINITY;
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, red[((size_t)w * DEC_MAXG + gg) * (D + 2) + D]);
+    float L = 0.f, O = 0.f;
+    for (int w = 0; w < 4; ++w) {
+      const float* r = red + ((size_t)w * DEC_MAXG + gg) * (D + 2);
+      const float f = r[D] == -INFINITY ? 0.f : exp2f(r[D] - M);
+      L += r[D + 1] * f;
+      O += r[dd] * f;
+    }
+    float* dst = part + (((size_t)b * H + g * G + gg) * splits + split) * (D + 2);
+    dst[dd] = O;
+    if (dd == 0) { dst[D] = M; dst[D + 1] = L; }
+  }
+}
+
+template <typename T, int D>
+__global__ void attn_decode_combine_kernel(const float* __restrict__ part, T* __restrict__ o, int H, int splits) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const float* base = part + ((size_t)b * H + h) * splits * (D + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, base[(size_t)s * (D + 2) + D]);
+  for (int dd = threadIdx.x; dd < D; dd += blockDim.x) {
+    float L = 0.f, O = 0.f;
+    for (int s = 0; s < splits; ++s) {
+      const float* r = base + (size_t)s * (D + 2);
+      const float f = r[D] == -INFINITY ? 0.f : exp2f(r[D] - M);
+      L += r[D + 1] * f;
+      O += r[dd] * f;
+    }
+    o[((size_t)b * H + h) * D + dd] = from_f<T>(O / L);
+  }
+}
+
+template <typename T, int D>
+int decode_launch(const void* q, const void* kc, const void* vc, const int32_t* nkeys, int add_keys, void* o, int B,
+                  int cmax, int H, int Hk, int Smax, float* part, int splits, int* status, cudaStream_t st) {
+  constexpr int ROW = D * (int)sizeof(T);
+  constexpr int DEC_SUB = dec_sub<T, D>();
+  constexpr int SMEM = DEC_STAGES * 2 * DEC_SUB * ROW + DEC_STAGES * 8 + 4 * DEC_MAXG * (D + 2) * 4;
+  auto kern = attn_decode_part_kernel<T, D>;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
+      return LLAMA_ERR_CUDA;
+    attr = true;
+  }
+  int chunk = (cmax + splits - 1) / splits;
+  chunk = (chunk + 127) / 128 * 128;
+  const float scale_log2 = kLog2e / sqrtf((float)D);
+  kern<<<dim3(splits, Hk, B), 128, SMEM, st>>>(static_cast<const T*>(q), static_cast<const T*>(kc),
+                                               static_cast<const T*>(vc), nkeys, add_keys, part, H, Hk, Smax, chunk,
+                                               scale_log2, status);
+  attn_decode_combine_kernel<T, D><<<dim3(H, B), D < 128 ? D : 128, 0, st>>>(part, static_cast<T*>(o), H, splits);
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+}  // namespace
+
+int attention_prefill(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B, int S,
+                      int H, int Hk, int d, int Smax, int dtype, int* status, cudaStream_t st) {
+  (void)status;
+  if (B <= 0 || S <= 0) return LLAMA_OK;
+  if (H % Hk != 0) return LLAMA_ERR_SHAPE;
+  const float scale_log2 = kLog2e / sqrtf((float)d);
+  if (dtype == LLAMA_BF16) {
+    if (d != PB_D) return LLAMA_ERR_UNSUPPORTED;
+    constexpr int SMEM = PB_Q * 256 + 4 * PB_K * 256;
+    static bool attr = false;
+    if (!attr) {
+      if (cudaFuncSetAttribute(attn_prefill_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
+          cudaSuccess)
+        return LLAMA_ERR_CUDA;
+      attr = true;
+    }
+    dim3 grid((S + PB_Q - 1) / PB_Q, H, B);
+    attn_prefill_bf16_kernel<<<grid, 128, SMEM, st>>>(static_cast<const bf16*>(q), static_cast<const bf16*>(kc),
+                                                      static_cast<const bf16*>(vc), static_cast<bf16*>(o), pos0, S, H,
+                                                      Hk, Smax, scale_log2);
+  } else {
+    dim3 grid(S, H, B);
+#define LLAMA_F32_PREFILL(DD)                                                                                  \
+  attn_prefill_f32_kernel<DD><<<grid, 32, 0, st>>>(static_cast<const float*>(q), static_cast<const float*>(kc), \
+                                                   static_cast<const float*>(vc), static_cast<float*>(o), pos0, S, \
+                                                   H, Hk, Smax, scale_log2)
+    switch (d) {
+      case 32: LLAMA_F32_PREFILL(32); break;
+      case 64: LLAMA_F32_PREFILL(64); break;
+      case 128: LLAMA_F32_PREFILL(128); break;
+      default: return LLAMA_ERR_UNSUPPORTED;
+    }
+#undef LLAMA_F32_PREFILL
+  }
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int decode_splits(int cmax, int B, int Hk) {
+  const int target = 2 * num_sms();
+  int s = (target + B * Hk - 1) / (B * Hk);
+  const int max_s = (cmax + 511) / 512;  // at least ~512 keys per split
+  if (s > max_s) s = max_s;
+  return s < 1 ? 1 : s;
+}
+
+size_t decode_scratch_floats(int B, int H, int d, int splits) { return (size_t)B * H * splits * (d + 2); }
+
+int attention_decode(const void* q, const void* kc, const void* vc, const int32_t* nkeys, int add_keys, void* o,
+                     int B, int cmax, int H, int Hk, int d, int Smax, int dtype, DecodeScratch* scratch, int* status,
+                     cudaStream_t st) {
+  if (B <= 0) return LLAMA_OK;
+  if (H % Hk != 0 || H / Hk > DEC_MAXG) return LLAMA_ERR_SHAPE;
+  const int splits = decode_splits(cmax, B, Hk);
+  if (!scratch || !scratch->part || scratch->floats < decode_scratch_floats(B, H, d, splits))
+    return LLAMA_ERR_INVALID_ARG;
+  if (dtype == LLAMA_BF16) {
+    if (d == 128) return decode_launch<bf16, 128>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch->part,
+                                                  splits, status, st);
+    if (d == 64) return decode_launch<bf16, 64>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch->part,
+                                                splits, status, st);
+  } else {
+    if (d == 128) return decode_launch<float, 128>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax,
+                                                   scratch->part, splits, status, st);
+    if (d == 64) return decode_launch<float, 64>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch->part,
+                                                 splits, status, st);
+    if (d == 32) return decode_launch<float, 32>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch->part,
+                                                 splits, status, st);
+  }
+  return LLAMA_ERR_UNSUPPORTED;
+}
+
+}  // namespace llama

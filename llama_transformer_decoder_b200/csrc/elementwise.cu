@@ -1,0 +1,271 @@
+// Bandwidth-bound kernels around the GEMMs: embedding gather, RMSNorm,
+// greedy argmax, per-sequence length update, and the seeded generator that
+// stands in for checkpoint weights and synthetic inputs.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace llama {
+
+namespace {
+
+// ------------------------------------------------------------- embedding
+// x[m, :] = table[tokens[m], :] widened to fp32 (row gather of tok_embeddings).
+template <typename T>
+__global__ void embed_kernel(const int32_t* __restrict__ tokens, const T* __restrict__ table, int V, int D,
+                             float* __restrict__ x, int* status) {
+  const int m = blockIdx.x;
+  const int tok = tokens[m];
+  float* dst = x + (size_t)m * D;
+  if (tok < 0 || tok >= V) {
+    if (threadIdx.x == 0) set_status(status, LLAMA_ERR_DEVICE_BOUNDS);
+    for (int i = threadIdx.x; i < D; i += blockDim.x) dst[i] = 0.f;
+    return;
+  }
+  const T* src = table + (size_t)tok * D;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) dst[i] = to_f<T>(src[i]);
+}
+
+// ---------------------------------------------------------------- RMSNorm
+// y = x * rsqrt(mean(x^2) + eps) * g over one row of D fp32 values.
+template <typename T>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ g,
+                                                      T* __restrict__ y, int D, float eps, int last_of_S) {
+  const int r = blockIdx.x;
+  const size_t src_row = last_of_S > 0 ? (size_t)(r + 1) * last_of_S - 1 : (size_t)r;
+  const float* xr = x + src_row * D;
+  __shared__ float red[8];
+  float ss = 0.f;
+  const bool vec = (D % 4 == 0);
+  if (vec) {
+    for (int i = threadIdx.x * 4; i < D; i += 1024) {
+      const float4 v = *reinterpret_cast<const float4*>(xr + i);
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+  } else {
+    for (int i = threadIdx.x; i < D; i += 256) ss += xr[i] * xr[i];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) tot += red[w];
+  const float inv = rsqrtf(tot / (float)D + eps);
+  T* yr = y + (size_t)r * D;
+  if (vec) {
+    for (int i = threadIdx.x * 4; i < D; i += 1024) {
+      const float4 v = *reinterpret_cast<const float4*>(xr + i);
+      const float4 w = *reinterpret_cast<const float4*>(g + i);
+      yr[i] = from_f<T>(v.x * inv * w.x);
+      yr[i + 1] = from_f<T>(v.y * inv * w.y);
+      yr[i + 2] = from_f<T>(v.z * inv * w.z);
+      yr[i + 3] = from_f<T>(v.w * inv * w.w);
+    }
+  } else {
+    for (int i = threadIdx.x; i < D; i += 256) yr[i] = from_f<T>(xr[i] * inv * g[i]);
+  }
+}
+
+// ----------------------------------------------------------------- argmax
+// Greedy next token: largest logit, lowest index among equal maxima.
+__device__ __forceinline__ void better(float& bv, int& bi, float v, int i) {
+  if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
+}
+
+__global__ void __launch_bounds__(1024) argmax_kernel(const float* __restrict__ logits, int32_t* out, int V) {
+  const float* row = logits + (size_t)blockIdx.x * V;
+  float bv = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int i = threadIdx.x; i < V; i += 1024) better(bv, bi, row[i], i);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    better(bv, bi, ov, oi);
+  }
+  __shared__ float sv[32];
+  __shared__ int si[32];
+  if ((threadIdx.x & 31) == 0) { sv[threadIdx.x >> 5] = bv; si[threadIdx.x >> 5] = bi; }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    bv = sv[threadIdx.x];
+    bi = si[threadIdx.x];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      better(bv, bi, ov, oi);
+    }
+    if (threadIdx.x == 0) out[blockIdx.x] = bi == 0x7fffffff ? 0 : bi;
+  }
+}
+
+__global__ void add_lengths_kernel(int32_t* len, int B, int add) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) len[b] += add;
+}
+
+// -------------------------------------------------------- seeded generator
+// SplitMix64 counter streams and Box-Muller, with ln and cos(2*pi*t) built
+// from correctly rounded IEEE operations only (explicit _rn intrinsics, so
+// nothing is fused): bit-identical to the host generator.
+#define SG 0x9E3779B97F4A7C15ULL
+#define SM1 0xBF58476D1CE4E5B9ULL
+#define SM2 0x94D049BB133111EBULL
+
+__constant__ double kCos[10] = {0x1.0000000000000p+0, -0x1.0000000000000p-1, 0x1.5555555555555p-5,
+                                -0x1.6c16c16c16c17p-10, 0x1.a01a01a01a01ap-16, -0x1.27e4fb7789f5cp-22,
+                                0x1.1eed8eff8d898p-29, -0x1.93974a8c07c9dp-37, 0x1.ae7f3e733b81fp-45,
+                                -0x1.6827863b97d97p-53};
+__constant__ double kSin[10] = {0x1.0000000000000p+0, -0x1.5555555555555p-3, 0x1.1111111111111p-7,
+                                -0x1.a01a01a01a01ap-13, 0x1.71de3a556c734p-19, -0x1.ae64567f544e4p-26,
+                                0x1.6124613a86d09p-33, -0x1.ae7f3e733b81fp-41, 0x1.952c77030ad4ap-49,
+                                -0x1.2f49b46814157p-57};
+__constant__ double kAtanh[11] = {0x1.0000000000000p+0, 0x1.5555555555555p-2, 0x1.999999999999ap-3,
+                                  0x1.2492492492492p-3, 0x1.c71c71c71c71cp-4, 0x1.745d1745d1746p-4,
+                                  0x1.3b13b13b13b14p-4, 0x1.1111111111111p-4, 0x1.e1e1e1e1e1e1ep-5,
+                                  0x1.af286bca1af28p-5, 0x1.8618618618618p-5};
+
+__host__ __device__ __forceinline__ uint64_t mix64(uint64_t z) {
+  z = (z ^ (z >> 30)) * SM1;
+  z = (z ^ (z >> 27)) * SM2;
+  return z ^ (z >> 31);
+}
+
+__device__ __forceinline__ double det_log(double u) {
+  int e;
+  double m = frexp(u, &e);
+  if (m < 0x1.6a09e667f3bcdp-1) { m = __dmul_rn(m, 2.0); e -= 1; }
+  const double s = __ddiv_rn(__dsub_rn(m, 1.0), __dadd_rn(m, 1.0));
+  const double s2 = __dmul_rn(s, s);
+  double p = kAtanh[10];
+#pragma unroll
+  for (int k = 9; k >= 0; --k) p = __dadd_rn(__dmul_rn(p, s2), kAtanh[k]);
+  return __dadd_rn(__dmul_rn((double)e, 0x1.62e42fefa39efp-1), __dmul_rn(__dmul_rn(2.0, s), p));
+}
+
+__device__ __forceinline__ double det_cos2pi(double t) {
+  if (t > 0.5) t = __dsub_rn(1.0, t);
+  const bool neg = t > 0.25;
+  if (neg) t = __dsub_rn(0.5, t);
+  const bool use_sin = t > 0.125;
+  const double x = __dmul_rn(use_sin ? __dsub_rn(0.25, t) : t, 0x1.921fb54442d18p+2);
+  const double x2 = __dmul_rn(x, x);
+  double r;
+  if (use_sin) {
+    double p = kSin[9];
+#pragma unroll
+    for (int k = 8; k >= 0; --k) p = __dadd_rn(__dmul_rn(p, x2), kSin[k]);
+    r = __dmul_rn(x, p);
+  } else {
+    double p = kCos[9];
+#pragma unroll
+    for (int k = 8; k >= 0; --k) p = __dadd_rn(__dmul_rn(p, x2), kCos[k]);
+    r = p;
+  }
+  return neg ? -r : r;
+}
+
+__device__ __forceinline__ float seeded_normal(uint64_t key, uint64_t i, double sd) {
+  const uint64_t d0 = mix64(key + (2 * i + 1) * SG);
+  const uint64_t d1 = mix64(key + (2 * i + 2) * SG);
+  const double u1 = (double)((d0 >> 11) + 1) * 0x1p-53;
+  const double u2 = (double)(d1 >> 11) * 0x1p-53;
+  const double z = __dmul_rn(__dsqrt_rn(__dmul_rn(-2.0, det_log(u1))), det_cos2pi(u2));
+  return __double2float_rn(__dmul_rn(z, sd));
+}
+
+template <typename T>
+__global__ void fill_normal_kernel(T* __restrict__ dst, FillLayout L, uint64_t key, double sd) {
+  const int64_t n = L.outer * L.rows * L.cols;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c = i % L.cols;
+    const int64_t t = i / L.cols;
+    const int64_t r = t % L.rows;
+    const int64_t o = t / L.rows;
+    const int64_t phys = o * L.outer_stride + (r * L.row_mult + L.row_off) * L.row_stride + c;
+    dst[phys] = from_f<T>(seeded_normal(key, (uint64_t)i, sd));
+  }
+}
+
+__global__ void fill_const_kernel(float* dst, int64_t n, float v) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    dst[i] = v;
+}
+
+__global__ void fill_tokens_kernel(int32_t* dst, int64_t n, uint64_t key, uint32_t vocab) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const uint64_t d = mix64(key + ((uint64_t)i + 1) * SG);
+    dst[i] = (int32_t)(((d >> 32) * (uint64_t)vocab) >> 32);
+  }
+}
+
+int grid_for(int64_t n) {
+  int64_t g = (n + 255) / 256;
+  const int64_t cap = (int64_t)num_sms() * 16;
+  return (int)(g < 1 ? 1 : (g > cap ? cap : g));
+}
+
+}  // namespace
+
+uint64_t stream_key(uint64_t seed, uint64_t stream) { return mix64(seed * SG + stream * SM1 + SG); }
+
+int launch_embed(const int32_t* tokens, int M, const void* table, int V, int D, int dtype, float* x, int* status,
+                 cudaStream_t st) {
+  if (M <= 0) return LLAMA_OK;
+  if (dtype == LLAMA_BF16)
+    embed_kernel<bf16><<<M, 256, 0, st>>>(tokens, static_cast<const bf16*>(table), V, D, x, status);
+  else
+    embed_kernel<float><<<M, 256, 0, st>>>(tokens, static_cast<const float*>(table), V, D, x, status);
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int launch_rmsnorm(const float* x, const float* g, void* y, int rows, int D, float eps, int last_of_S, int dtype,
+                   cudaStream_t st) {
+  if (rows <= 0) return LLAMA_OK;
+  if (dtype == LLAMA_BF16)
+    rmsnorm_kernel<bf16><<<rows, 256, 0, st>>>(x, g, static_cast<bf16*>(y), D, eps, last_of_S);
+  else
+    rmsnorm_kernel<float><<<rows, 256, 0, st>>>(x, g, static_cast<float*>(y), D, eps, last_of_S);
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int launch_argmax(const float* logits, int32_t* out, int B, int V, cudaStream_t st) {
+  if (B <= 0) return LLAMA_OK;
+  argmax_kernel<<<B, 1024, 0, st>>>(logits, out, V);
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int launch_add_lengths(int32_t* len, int B, int add, cudaStream_t st) {
+  if (B <= 0) return LLAMA_OK;
+  add_lengths_kernel<<<(B + 255) / 256, 256, 0, st>>>(len, B, add);
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int launch_fill_normal(void* dst, const FillLayout& L, uint64_t seed, uint64_t stream_id, float std, int dtype,
+                       cudaStream_t st) {
+  const int64_t n = L.outer * L.rows * L.cols;
+  if (n <= 0) return LLAMA_OK;
+  const uint64_t key = stream_key(seed, stream_id);
+  const double sd = (double)std;
+  if (dtype == LLAMA_BF16)
+    fill_normal_kernel<bf16><<<grid_for(n), 256, 0, st>>>(static_cast<bf16*>(dst), L, key, sd);
+  else
+    fill_normal_kernel<float><<<grid_for(n), 256, 0, st>>>(static_cast<float*>(dst), L, key, sd);
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int launch_fill_const(float* dst, int64_t n, float v, cudaStream_t st) {
+  if (n <= 0) return LLAMA_OK;
+  fill_const_kernel<<<grid_for(n), 256, 0, st>>>(dst, n, v);
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int launch_fill_tokens(int32_t* dst, int64_t n, uint64_t seed, uint64_t stream_id, int vocab, cudaStream_t st) {
+  if (n <= 0) return LLAMA_OK;
+  fill_tokens_kernel<<<grid_for(n), 256, 0, st>>>(dst, n, stream_key(seed, stream_id), (uint32_t)vocab);
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+}  // namespace llama

@@ -1,0 +1,160 @@
+// GEMM epilogues shared by the tcgen05 GEMMs and the fp32 SIMT GEMM.
+//
+// A GEMM computes acc[m][n] = sum_k A[m][k] * W[n][k] (y = x W^T, the [out, in]
+// weight convention of the checkpoint). The epilogue turns acc into one of:
+//   STORE_F32  out[m][n] = acc                      (LM-head logits, tests)
+//   RESIDUAL   out[m][n] += acc                     (Wo and w2: h = x + delta)
+//   SWIGLU     g[m][f] = silu(acc[m][2f]) * acc[m][2f+1]
+//              (w1 and w3 rows are interleaved: row 2f = w1[f], 2f+1 = w3[f])
+//   QKV_ROPE   columns [0,H*d) are q, [H*d,(H+Hk)*d) k, then v. Adjacent
+//              pairs of q and k are rotated by angle pos*theta^(-2i/d); q goes
+//              to q_out[b][h][s][:], k and v into the KV cache at pos.
+#pragma once
+#include "common.cuh"
+
+namespace llama {
+
+enum EpiKind { EPI_STORE_F32 = 0, EPI_RESIDUAL = 1, EPI_SWIGLU = 2, EPI_QKV_ROPE = 3 };
+
+struct EpiArgs {
+  int M, N;           // logical output extent (rows = tokens, columns = features)
+  float* out;         // STORE_F32 / RESIDUAL target, row pitch ldo (floats)
+  int ldo;
+  void* g;            // SWIGLU output (T = model dtype), row pitch ldg
+  int ldg;
+  void* q;            // QKV_ROPE: q output [B][H][S][d]
+  void* kc;           // K cache of this layer [Bmax][Hk][Smax][d]
+  void* vc;           // V cache of this layer
+  const float2* rope; // (cos, sin) table [Smax][d/2]
+  const int* pos0;    // per-sequence position of the call's first token
+  int S, H, Hk, d, Smax;
+};
+
+// One rotated (or plain) value of the q/k/v block. n is the column, v its
+// accumulator and partner the accumulator of column n^1.
+template <typename T>
+__device__ __forceinline__ void qkv_store(const EpiArgs& e, int m, int n, float v, float partner) {
+  const int b = m / e.S, s = m - b * e.S;
+  const int pos = e.pos0[b] + s;
+  const int hd = e.H * e.d;
+  float r = v;
+  if (n < hd + e.Hk * e.d) {
+    const int i = (n % e.d) >> 1;
+    const float2 cs = e.rope[(size_t)pos * (e.d >> 1) + i];
+    r = (n & 1) ? (partner * cs.y + v * cs.x) : (v * cs.x - partner * cs.y);
+  }
+  if (n < hd) {
+    const int h = n / e.d, dd = n - h * e.d;
+    static_cast<T*>(e.q)[(((size_t)b * e.H + h) * e.S + s) * e.d + dd] = from_f<T>(r);
+  } else {
+    const bool is_k = n < hd + e.Hk * e.d;
+    const int nn = n - hd - (is_k ? 0 : e.Hk * e.d);
+    const int g = nn / e.d, dd = nn - g * e.d;
+    T* dst = static_cast<T*>(is_k ? e.kc : e.vc);
+    dst[(((size_t)b * e.Hk + g) * e.Smax + pos) * e.d + dd] = from_f<T>(r);
+  }
+}
+
+// Element-wise form (used when consecutive columns live in neighbouring lanes).
+template <int KIND, typename T>
+__device__ __forceinline__ void epi_elem(const EpiArgs& e, int m, int n, float v, float partner) {
+  if (m >= e.M || n >= e.N) return;
+  if (KIND == EPI_STORE_F32) {
+    e.out[(size_t)m * e.ldo + n] = v;
+  } else if (KIND == EPI_RESIDUAL) {
+    float* p = e.out + (size_t)m * e.ldo + n;
+    *p = *p + v;
+  } else if (KIND == EPI_SWIGLU) {
+    if ((n & 1) == 0) static_cast<T*>(e.g)[(size_t)m * e.ldg + (n >> 1)] = from_f<T>(silu_f(v) * partner);
+  } else {
+    qkv_store<T>(e, m, n, v, partner);
+  }
+}
+
+// Row-chunk form: one thread holds 32 consecutive columns [n0, n0+32) of row m
+// (n0 % 32 == 0). Full chunks use 16-byte stores.
+template <int KIND, typename T>
+__device__ __forceinline__ void epi_row32(const EpiArgs& e, int m, int n0, const float (&v)[32]) {
+  if (m >= e.M) return;
+  const bool full = (n0 + 32 <= e.N);
+  if (KIND == EPI_STORE_F32 || KIND == EPI_RESIDUAL) {
+    float* p = e.out + (size_t)m * e.ldo + n0;
+    if (full && ((e.ldo & 3) == 0) && ((reinterpret_cast<uintptr_t>(e.out) & 15) == 0)) {
+      float4* p4 = reinterpret_cast<float4*>(p);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float4 o = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        if (KIND == EPI_RESIDUAL) {
+          const float4 x = p4[j];
+          o.x += x.x; o.y += x.y; o.z += x.z; o.w += x.w;
+        }
+        p4[j] = o;
+      }
+    } else {
+      for (int j = 0; j < 32 && n0 + j < e.N; ++j) {
+        if (KIND == EPI_RESIDUAL) p[j] += v[j];
+        else p[j] = v[j];
+      }
+    }
+  } else if (KIND == EPI_SWIGLU) {
+    T* p = static_cast<T*>(e.g) + (size_t)m * e.ldg + (n0 >> 1);
+    if (sizeof(T) == 2 && full && ((e.ldg & 7) == 0)) {
+      uint32_t w[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(silu_f(v[4 * j]) * v[4 * j + 1], silu_f(v[4 * j + 2]) * v[4 * j + 3]);
+        w[j] = *reinterpret_cast<uint32_t*>(&h2);
+      }
+      uint4* p4 = reinterpret_cast<uint4*>(p);
+      p4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      p4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    } else {
+      for (int j = 0; j < 16 && n0 + 2 * j + 1 < e.N; ++j) p[j] = from_f<T>(silu_f(v[2 * j]) * v[2 * j + 1]);
+    }
+  } else {  // QKV_ROPE: a 32-column chunk never straddles a head when d % 32 == 0
+    if (!full || (e.d & 31) != 0 || sizeof(T) != 2) {
+      for (int j = 0; j < 32 && n0 + j < e.N; ++j) qkv_store<T>(e, m, n0 + j, v[j], v[j ^ 1]);
+      return;
+    }
+    const int b = m / e.S, s = m - b * e.S;
+    const int pos = e.pos0[b] + s;
+    const int hd = e.H * e.d;
+    T* dst;
+    int dd0;
+    float r[32];
+    if (n0 < hd + e.Hk * e.d) {
+      const float2* cs = e.rope + (size_t)pos * (e.d >> 1) + ((n0 % e.d) >> 1);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float2 c = cs[j];
+        r[2 * j] = v[2 * j] * c.x - v[2 * j + 1] * c.y;
+        r[2 * j + 1] = v[2 * j] * c.y + v[2 * j + 1] * c.x;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) r[j] = v[j];
+    }
+    if (n0 < hd) {
+      const int h = n0 / e.d;
+      dd0 = n0 - h * e.d;
+      dst = static_cast<T*>(e.q) + (((size_t)b * e.H + h) * e.S + s) * e.d + dd0;
+    } else {
+      const bool is_k = n0 < hd + e.Hk * e.d;
+      const int nn = n0 - hd - (is_k ? 0 : e.Hk * e.d);
+      const int g = nn / e.d;
+      dd0 = nn - g * e.d;
+      dst = static_cast<T*>(is_k ? e.kc : e.vc) + (((size_t)b * e.Hk + g) * e.Smax + pos) * e.d + dd0;
+    }
+    uint32_t w[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(r[2 * j], r[2 * j + 1]);
+      w[j] = *reinterpret_cast<uint32_t*>(&h2);
+    }
+    uint4* p4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) p4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  }
+}
+
+}  // namespace llama

@@ -1,0 +1,483 @@
+// tcgen05 GEMMs for the bf16 projections: acc = x W^T with x [M,K], W [N,K].
+//
+// Two kernels share the same warp roles (warp 0: TMA producer, warp 1: MMA
+// issuer and TMEM owner, warps 2-5: epilogue reading TMEM):
+//
+//  * gemm_wide  (M large, prefill): persistent, one CTA per SM, 128x256 output
+//    tiles (rows = tokens, cols = weight rows), 4-stage TMA ring of 48 KB,
+//    double-buffered fp32 accumulators in TMEM (2 x 256 columns) so the
+//    epilogue of tile i overlaps the main loop of tile i+1.
+//
+//  * gemm_skinny (M <= 256, decode and short prompts): the weight tile is the
+//    MMA's A operand (128 weight rows) and the tokens are its N side, so a
+//    decode step streams each weight byte exactly once at full MMA width.
+//    The K range is split across CTAs to put every SM on the weight stream;
+//    partial tiles go to a workspace and the last CTA of a tile (atomic
+//    ticket, no spinning) reduces them in split order and runs the epilogue.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "epilogue.cuh"
+#include "kernels.h"
+
+namespace llama {
+
+namespace {
+
+constexpr int BK = 64;                    // K elements per stage (128 B rows, 128B swizzle)
+constexpr int W_BM = 128, W_BN = 256;     // wide tile
+constexpr int W_STAGES = 4;
+constexpr int W_A_BYTES = W_BM * BK * 2;  // 16 KB
+constexpr int W_B_BYTES = W_BN * BK * 2;  // 32 KB
+constexpr int W_STAGE_BYTES = W_A_BYTES + W_B_BYTES;
+constexpr int W_SMEM = W_STAGES * W_STAGE_BYTES + 1024 + 256;
+constexpr int kThreads = 192;
+
+constexpr int S_BM = 128;                 // skinny: weight rows per CTA
+constexpr int S_A_BYTES = S_BM * BK * 2;  // 16 KB
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Wait for the loads this producer issued last (ring positions before
+// (stage, phase)); used only on the error path so no copy is in flight when
+// the CTA exits.
+__device__ void drain_loads(uint64_t* full, int stage, uint32_t phase, int issued, int nstages, int* status) {
+  for (int i = 0; i < issued && i < nstages; ++i) {
+    if (--stage < 0) { stage = nstages - 1; phase ^= 1; }
+    mbar_wait(&full[stage], phase, status);
+  }
+}
+
+// ------------------------------------------------------------------ wide
+template <int KIND, typename T>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
+                     int K, EpiArgs epi, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + W_STAGES * W_STAGE_BYTES);
+  uint64_t* empty = full + W_STAGES;
+  uint64_t* accf = empty + W_STAGES;
+  uint64_t* acce = accf + 2;
+  uint64_t* drain = acce + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tiles = (M + W_BM - 1) / W_BM, n_tiles = (N + W_BN - 1) / W_BN;
+  const int tiles = m_tiles * n_tiles;
+  const int kb = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < W_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&accf[a], 1); mbar_init(&acce[a], 128); }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    const uint64_t pol_a = l2_policy_evict_last(), pol_b = l2_policy_evict_last();
+    int stage = 0, issued = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+      const int m0 = (t % m_tiles) * W_BM, n0 = (t / m_tiles) * W_BN;
+      for (int k = 0; k < kb; ++k) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, status)) { ok = false; break; }
+        uint8_t* sa = smem + stage * W_STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[stage], W_STAGE_BYTES);
+        tma_load_2d(sa, &tmA, &full[stage], k * BK, m0, pol_a);
+        tma_load_2d(sa + W_A_BYTES, &tmB, &full[stage], k * BK, n0, pol_b);
+        ++issued;
+        if (++stage == W_STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+    if (!ok) drain_loads(full, stage, phase, issued, W_STAGES, status);
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = umma_idesc_bf16(W_BM, W_BN);
+    int stage = 0, acc = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    bool ok = true, any = false;
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+      if (!mbar_wait(&acce[acc], acc_phase ^ 1, status)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + acc * W_BN;
+      for (int k = 0; k < kb; ++k) {
+        if (!mbar_wait(&full[stage], phase, status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + stage * W_STAGE_BYTES);
+        const uint32_t b_addr = a_addr + W_A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          umma_bf16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), idesc,
+                    (k | kk) != 0);
+        umma_commit(&empty[stage]);
+        any = true;
+        if (++stage == W_STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      umma_commit(&accf[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+    if (!ok && any) {  // let issued MMAs finish before TMEM is released
+      umma_commit(drain);
+      mbar_wait(drain, 0, status);
+    }
+  } else if (warp >= 2) {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+      const int m0 = (t % m_tiles) * W_BM, n0 = (t / m_tiles) * W_BN;
+      if (!mbar_wait(&accf[acc], acc_phase, status)) break;
+      tc_fence_after();
+      const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + acc * W_BN;
+#pragma unroll 1
+      for (int c = 0; c < W_BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(base + c * 32, v);
+        if (n0 + c * 32 < N) epi_row32<KIND, T>(epi, m0 + row, n0 + c * 32, v);
+      }
+      tc_fence_before();
+      mbar_arrive(&acce[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- skinny
+template <int KIND, typename T, int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, int M,
+                       int N, int K, int splits, int kb_per_split, EpiArgs epi, float* __restrict__ ws,
+                       int* __restrict__ tickets, int* status) {
+  constexpr int B_BYTES = NT * BK * 2;
+  constexpr int STAGE_BYTES = S_A_BYTES + B_BYTES;
+  constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
+  constexpr uint32_t TMEM_COLS = NT <= 32 ? 32 : (NT <= 64 ? 64 : (NT <= 128 ? 128 : 256));
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;
+  uint64_t* drain = accf + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * S_BM;
+  const int split = blockIdx.y;
+  const int kb = (K + BK - 1) / BK;
+  const int k_begin = split * kb_per_split;
+  const int k_end = min(kb, k_begin + kb_per_split);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(accf, 1);
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+    const uint64_t pol_w = l2_policy_evict_first(), pol_x = l2_policy_evict_last();
+    int stage = 0, issued = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int k = k_begin; k < k_end; ++k) {
+      if (!mbar_wait(&empty[stage], phase ^ 1, status)) { ok = false; break; }
+      uint8_t* sa = smem + stage * STAGE_BYTES;
+      mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+      tma_load_2d(sa, &tmW, &full[stage], k * BK, n0, pol_w);
+      tma_load_2d(sa + S_A_BYTES, &tmX, &full[stage], k * BK, 0, pol_x);
+      ++issued;
+      if (++stage == STAGES) { stage = 0; phase ^= 1; }
+    }
+    if (!ok) drain_loads(full, stage, phase, issued, STAGES, status);
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = umma_idesc_bf16(S_BM, NT);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true, any = false;
+    for (int k = k_begin; k < k_end; ++k) {
+      if (!mbar_wait(&full[stage], phase, status)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t a_addr = smem_u32(smem + stage * STAGE_BYTES);
+      const uint32_t b_addr = a_addr + S_A_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk)
+        umma_bf16(tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), idesc,
+                  (k != k_begin) || (kk != 0));
+      umma_commit(&empty[stage]);
+      any = true;
+      if (++stage == STAGES) { stage = 0; phase ^= 1; }
+    }
+    if (ok) {
+      umma_commit(accf);
+    } else if (any) {
+      umma_commit(drain);
+      mbar_wait(drain, 0, status);
+    }
+  } else if (warp >= 2) {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // weight row within the tile
+    const int n = n0 + row;
+    const bool have = k_end > k_begin;
+    bool ok = true;
+    if (have) {
+      ok = mbar_wait(accf, 0, status);
+      tc_fence_after();
+    }
+    const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16);
+    if (splits == 1) {
+#pragma unroll 1
+      for (int c = 0; c < NT / 32; ++c) {
+        float v[32];
+        if (have && ok) tmem_ld32(base + c * 32, v);
+        else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float partner = __shfl_xor_sync(0xffffffffu, v[j], 1);
+          if (ok) epi_elem<KIND, T>(epi, c * 32 + j, n, v[j], partner);
+        }
+      }
+    } else {
+      // 1) publish this split's partial tile [128 rows x NT tokens]
+      float* mine = ws + ((size_t)split * N + n) * NT;
+#pragma unroll 1
+      for (int c = 0; c < NT / 32; ++c) {
+        float v[32];
+        if (have && ok) tmem_ld32(base + c * 32, v);
+        else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        }
+        if (n < N) {
+          float4* p4 = reinterpret_cast<float4*>(mine + c * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) __stcg(p4 + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+        }
+      }
+      __threadfence();
+      named_bar_sync(1, 128);
+      if (threadIdx.x == 64) {
+        const int prev = atomicAdd(&tickets[blockIdx.x], 1);
+        *last_flag = (prev == splits - 1);
+      }
+      named_bar_sync(1, 128);
+      // 2) the last CTA to finish sums the partials in split order
+      if (*last_flag) {
+        __threadfence();
+#pragma unroll 1
+        for (int c = 0; c < NT / 32; ++c) {
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          if (n < N) {
+            for (int s = 0; s < splits; ++s) {
+              const float4* p4 = reinterpret_cast<const float4*>(ws + ((size_t)s * N + n) * NT + c * 32);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float4 x = __ldcg(p4 + j);
+                v[4 * j] += x.x; v[4 * j + 1] += x.y; v[4 * j + 2] += x.z; v[4 * j + 3] += x.w;
+              }
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float partner = __shfl_xor_sync(0xffffffffu, v[j], 1);
+            if (ok) epi_elem<KIND, T>(epi, c * 32 + j, n, v[j], partner);
+          }
+        }
+        if (threadIdx.x == 64) tickets[blockIdx.x] = 0;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// -------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+// bf16 row-major [rows, cols] matrix with row pitch `pitch` elements, boxes of
+// box_rows x 64 elements, 128-byte swizzle, zero fill outside the matrix.
+int make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t pitch, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return LLAMA_ERR_CUDA;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (pitch * 2) % 16 != 0) return LLAMA_ERR_INVALID_ARG;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)(pitch * 2)};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int KIND>
+static int launch_wide(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, const EpiArgs& e,
+                       int* status, cudaStream_t st) {
+  auto kern = gemm_wide_kernel<KIND, bf16>;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, W_SMEM) != cudaSuccess)
+      return LLAMA_ERR_CUDA;
+    attr = true;
+  }
+  const int tiles = ((M + W_BM - 1) / W_BM) * ((N + W_BN - 1) / W_BN);
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  kern<<<grid, kThreads, W_SMEM, st>>>(ta, tb, M, N, K, e, status);
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+template <int KIND, int NT>
+static int launch_skinny_nt(const CUtensorMap& tw, const CUtensorMap& tx, int M, int N, int K, int splits, int kbps,
+                            const EpiArgs& e, float* ws, int* tickets, int* status, cudaStream_t st) {
+  constexpr int B_BYTES = NT * BK * 2;
+  constexpr int STAGE_BYTES = S_A_BYTES + B_BYTES;
+  constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
+  constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+  auto kern = gemm_skinny_kernel<KIND, bf16, NT>;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
+      return LLAMA_ERR_CUDA;
+    attr = true;
+  }
+  dim3 grid((N + S_BM - 1) / S_BM, splits);
+  kern<<<grid, kThreads, SMEM, st>>>(tw, tx, M, N, K, splits, kbps, e, ws, tickets, status);
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+template <int KIND>
+static int launch_skinny(const CUtensorMap& tw, const CUtensorMap& tx, int M, int N, int K, int NT, int splits,
+                         int kbps, const EpiArgs& e, float* ws, int* tickets, int* status, cudaStream_t st) {
+  switch (NT) {
+    case 32: return launch_skinny_nt<KIND, 32>(tw, tx, M, N, K, splits, kbps, e, ws, tickets, status, st);
+    case 64: return launch_skinny_nt<KIND, 64>(tw, tx, M, N, K, splits, kbps, e, ws, tickets, status, st);
+    case 128: return launch_skinny_nt<KIND, 128>(tw, tx, M, N, K, splits, kbps, e, ws, tickets, status, st);
+    case 256: return launch_skinny_nt<KIND, 256>(tw, tx, M, N, K, splits, kbps, e, ws, tickets, status, st);
+  }
+  return LLAMA_ERR_INVALID_ARG;
+}
+
+// Split count that puts about one CTA on every SM without making a split
+// shorter than 4 K-blocks.
+void skinny_plan(int M, int N, int K, int* NT, int* splits, int* kbps) {
+  int nt = 32;
+  while (nt < M) nt *= 2;
+  *NT = nt;
+  const int tiles = (N + S_BM - 1) / S_BM;
+  const int kb = (K + BK - 1) / BK;
+  int s = num_sms() / tiles;
+  if (s < 1) s = 1;
+  if (s > kb / 4) s = kb / 4 > 0 ? kb / 4 : 1;
+  int per = (kb + s - 1) / s;
+  s = (kb + per - 1) / per;  // no empty split
+  *splits = s;
+  *kbps = per;
+}
+
+size_t skinny_workspace_floats(int M, int N, int K) {
+  int nt, s, per;
+  skinny_plan(M, N, K, &nt, &s, &per);
+  return s > 1 ? (size_t)s * N * nt : 0;
+}
+
+int gemm_bf16(const bf16* A, int M, int K, int lda, const bf16* W, int N, int ldw, int kind, const EpiArgs& e,
+              int variant, GemmScratch* scratch, int* status, cudaStream_t st) {
+  if (M <= 0 || N <= 0 || K <= 0) return LLAMA_ERR_SHAPE;
+  if (K % 8 != 0 || lda % 8 != 0 || ldw % 8 != 0) return LLAMA_ERR_SHAPE;
+  const bool skinny = variant == GEMM_SKINNY || (variant == GEMM_AUTO && M <= 128);
+  int rc;
+  if (!skinny) {
+    CUtensorMap ta, tb;
+    if ((rc = make_tmap_bf16(&ta, A, M, K, lda, W_BM)) != LLAMA_OK) return rc;
+    if ((rc = make_tmap_bf16(&tb, W, N, K, ldw, W_BN)) != LLAMA_OK) return rc;
+    switch (kind) {
+      case EPI_STORE_F32: return launch_wide<EPI_STORE_F32>(ta, tb, M, N, K, e, status, st);
+      case EPI_RESIDUAL: return launch_wide<EPI_RESIDUAL>(ta, tb, M, N, K, e, status, st);
+      case EPI_SWIGLU: return launch_wide<EPI_SWIGLU>(ta, tb, M, N, K, e, status, st);
+      case EPI_QKV_ROPE: return launch_wide<EPI_QKV_ROPE>(ta, tb, M, N, K, e, status, st);
+    }
+    return LLAMA_ERR_INVALID_ARG;
+  }
+  if (M > 256) return LLAMA_ERR_SHAPE;
+  int NT, splits, kbps;
+  skinny_plan(M, N, K, &NT, &splits, &kbps);
+  if (splits > 1) {
+    const size_t need = (size_t)splits * N * NT;
+    const int tiles = (N + S_BM - 1) / S_BM;
+    if (!scratch || !scratch->ws || scratch->ws_floats < need || !scratch->tickets || scratch->n_tickets < tiles)
+      return LLAMA_ERR_INVALID_ARG;
+  }
+  CUtensorMap tw, tx;
+  if ((rc = make_tmap_bf16(&tw, W, N, K, ldw, S_BM)) != LLAMA_OK) return rc;
+  if ((rc = make_tmap_bf16(&tx, A, M, K, lda, NT)) != LLAMA_OK) return rc;
+  float* ws = scratch ? scratch->ws : nullptr;
+  int* tk = scratch ? scratch->tickets : nullptr;
+  switch (kind) {
+    case EPI_STORE_F32: return launch_skinny<EPI_STORE_F32>(tw, tx, M, N, K, NT, splits, kbps, e, ws, tk, status, st);
+    case EPI_RESIDUAL: return launch_skinny<EPI_RESIDUAL>(tw, tx, M, N, K, NT, splits, kbps, e, ws, tk, status, st);
+    case EPI_SWIGLU: return launch_skinny<EPI_SWIGLU>(tw, tx, M, N, K, NT, splits, kbps, e, ws, tk, status, st);
+    case EPI_QKV_ROPE: return launch_skinny<EPI_QKV_ROPE>(tw, tx, M, N, K, NT, splits, kbps, e, ws, tk, status, st);
+  }
+  return LLAMA_ERR_INVALID_ARG;
+}
+
+}  // namespace llama

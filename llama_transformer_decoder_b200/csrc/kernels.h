@@ -1,0 +1,72 @@
+// Internal launch interface between the C-ABI host code (model.cu) and the
+// kernels. Not part of the public header.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace llama {
+
+struct EpiArgs;
+
+enum GemmVariant { GEMM_AUTO = 0, GEMM_WIDE = 1, GEMM_SKINNY = 2 };
+
+// Split-K scratch of the skinny GEMM: partial tiles plus one ticket per
+// 128-row weight tile (tickets must start at zero; the kernel leaves them zero).
+struct GemmScratch {
+  float* ws;
+  size_t ws_floats;
+  int* tickets;
+  int n_tickets;
+};
+
+int num_sms();
+int make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t pitch, int box_rows);
+void skinny_plan(int M, int N, int K, int* NT, int* splits, int* kbps);
+size_t skinny_workspace_floats(int M, int N, int K);
+
+int gemm_bf16(const __nv_bfloat16* A, int M, int K, int lda, const __nv_bfloat16* W, int N, int ldw, int kind,
+              const EpiArgs& e, int variant, GemmScratch* scratch, int* status, cudaStream_t st);
+int gemm_f32(const float* A, int M, int K, int lda, const float* W, int N, int ldw, int kind, const EpiArgs& e,
+             int* status, cudaStream_t st);
+
+// Elementwise / reductions. dtype: 0 = fp32, 1 = bf16 (of `y` / tables).
+int launch_embed(const int32_t* tokens, int M, const void* table, int V, int D, int dtype, float* x, int* status,
+                 cudaStream_t st);
+// y[r] = rmsnorm(x[row(r)]) * g; row(r) = r, or (r+1)*S-1 when last_of_S > 0.
+int launch_rmsnorm(const float* x, const float* g, void* y, int rows, int D, float eps, int last_of_S, int dtype,
+                   cudaStream_t st);
+int launch_argmax(const float* logits, int32_t* out, int B, int V, cudaStream_t st);
+int launch_add_lengths(int32_t* len, int B, int add, cudaStream_t st);
+
+// Attention. q [B][H][S][d]; K/V cache [B][Hk][Smax][d] (this layer);
+// o [B*S][H*d]; pos0[b] = position of the call's first query (null = 0).
+int attention_prefill(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B, int S,
+                      int H, int Hk, int d, int Smax, int dtype, int* status, cudaStream_t st);
+// Decode: q [B][H][d]; keys 0 .. nkeys[b]-1 (+ add) of the cache; o [B][H*d].
+struct DecodeScratch {
+  float* part;  // [B][H][splits][d + 2]
+  size_t floats;
+};
+int decode_splits(int cmax, int B, int Hk);
+size_t decode_scratch_floats(int B, int H, int d, int splits);
+int attention_decode(const void* q, const void* kc, const void* vc, const int32_t* nkeys, int add_keys, void* o,
+                     int B, int cmax, int H, int Hk, int d, int Smax, int dtype, DecodeScratch* scratch,
+                     int* status, cudaStream_t st);
+
+// Seeded generator: SplitMix64 counter streams + Box-Muller from IEEE basic ops.
+// Logical element i = ((o * rows + r) * cols + c) of a [outer][rows][cols]
+// tensor lands at  o*outer_stride + (r*row_mult + row_off)*row_stride + c.
+struct FillLayout {
+  int64_t outer, rows, cols;
+  int64_t outer_stride, row_stride;
+  int row_mult, row_off;
+};
+int launch_fill_normal(void* dst, const FillLayout& L, uint64_t seed, uint64_t stream_id, float std, int dtype,
+                       cudaStream_t st);
+int launch_fill_const(float* dst, int64_t n, float v, cudaStream_t st);
+int launch_fill_tokens(int32_t* dst, int64_t n, uint64_t seed, uint64_t stream_id, int vocab, cudaStream_t st);
+
+}  // namespace llama

@@ -1,0 +1,180 @@
+"""Kernel parity on the GPU through the C ABI: generator, GEMMs (wide and
+skinny tcgen05 paths, fp32 SIMT), RMSNorm, argmax, prefill and decode
+attention, each against the CPU oracle on the same seeded inputs."""
+import numpy as np
+import pytest
+
+import seeded_inputs as si
+from oracle import argmax, attention, rms_norm
+from tests.helpers import BF16, F32, normal_values, rel_l2, to_device
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip('torch')
+if not torch.cuda.is_available():  # pragma: no cover
+    pytest.skip('needs a CUDA device', allow_module_level=True)
+
+from llama_transformer_decoder_b200 import binding as L  # noqa: E402
+
+
+def _sync_ok():
+    assert L.llama_status(None) == 0
+
+
+# ----------------------------------------------------------- generator
+@pytest.mark.parametrize('dtype', [BF16, F32])
+def test_device_generator_matches_host(dtype):
+    n = 3_000_017
+    for seed, stream, std in [(0, 1, 0.02), (7, 123456, 1.0), (1, 2 ** 21 + 5, 1.0)]:
+        t = torch.empty(n, dtype=torch.bfloat16 if dtype == BF16 else torch.float32, device='cuda')
+        L.llama_fill_normal(t, n, seed, stream, std, dtype)
+        torch.cuda.synchronize()
+        host = si.normal(seed, stream, n, std, 'bf16' if dtype == BF16 else 'f32')
+        dev = t.view(torch.int16).cpu().numpy().view(np.uint16) if dtype == BF16 else t.cpu().numpy()
+        assert np.array_equal(dev.view(np.uint16 if dtype == BF16 else np.uint32),
+                              host.view(np.uint16 if dtype == BF16 else np.uint32))
+    _sync_ok()
+
+
+# -------------------------------------------------------------- GEMMs
+GEMM_CASES = [
+    # (M, N, K, variant)  variant 1 = wide persistent, 2 = skinny split-K
+    (300, 520, 4104, 1),     # ragged M, N and K tails
+    (128, 256, 64, 1),       # exactly one tile, one k-block
+    (2048, 6144, 4096, 1),   # 8B QKV projection at S = 2048
+    (17, 6144, 4096, 2),     # seq-17 block
+    (32, 4096, 14336, 2),    # decode w2 (long K, split)
+    (1, 1000, 4096, 2),      # one row, ragged N
+    (200, 520, 4104, 2),     # ragged everything, NT = 256
+    (100, 384, 256, 2),      # short K (one split)
+    (64, 1024, 1024, 1),     # wide path with few rows
+]
+
+
+@pytest.mark.parametrize('M,N,K,variant', GEMM_CASES)
+def test_linear_bf16(M, N, K, variant):
+    xv, xr = normal_values(11, 1, (M, K), BF16)
+    wv, wr = normal_values(11, 2, (N, K), BF16, std=0.02)
+    y = torch.full((M, N), float('nan'), device='cuda')
+    L.llama_linear(to_device(xr, BF16), to_device(wr, BF16), y, M, N, K, BF16, variant)
+    torch.cuda.synchronize()
+    _sync_ok()
+    ref = xv.astype(np.float64) @ wv.astype(np.float64).T
+    got = y.cpu().numpy()
+    assert np.all(np.isfinite(got))
+    assert rel_l2(got, ref) < 1e-5
+    # fp32 accumulation of exact bf16 products: per element |err| << 1e-3 * |row scale|
+    scale = np.sqrt((xv.astype(np.float64) ** 2).sum(1, keepdims=True) * (wv.astype(np.float64) ** 2).sum(1)[None, :])
+    assert np.max(np.abs(got - ref) / scale) < 1e-5
+
+
+def test_linear_bf16_repeatable():
+    """Split-K reduction runs in a fixed order: repeated calls agree bit for bit."""
+    M, N, K = 32, 4096, 14336
+    _, xr = normal_values(12, 1, (M, K), BF16)
+    _, wr = normal_values(12, 2, (N, K), BF16, std=0.02)
+    x, w = to_device(xr, BF16), to_device(wr, BF16)
+    outs = []
+    for _ in range(3):
+        y = torch.empty((M, N), device='cuda')
+        L.llama_linear(x, w, y, M, N, K, BF16, 2)
+        outs.append(y.cpu())
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+
+
+@pytest.mark.parametrize('M,N,K', [(17, 768, 256), (70, 130, 33), (1, 1024, 256)])
+def test_linear_f32(M, N, K):
+    xv, xr = normal_values(13, 1, (M, K), F32)
+    wv, wr = normal_values(13, 2, (N, K), F32, std=0.02)
+    y = torch.empty((M, N), device='cuda')
+    L.llama_linear(to_device(xr, F32), to_device(wr, F32), y, M, N, K, F32, 0)
+    ref = xv.astype(np.float64) @ wv.astype(np.float64).T
+    assert rel_l2(y.cpu().numpy(), ref) < 1e-6
+    _sync_ok()
+
+
+# ------------------------------------------------------------ RMSNorm
+@pytest.mark.parametrize('dtype', [BF16, F32])
+@pytest.mark.parametrize('M,D', [(1, 4096), (37, 4096), (5, 256), (3, 100)])
+def test_rmsnorm(dtype, M, D):
+    xv, xr = normal_values(14, 1, (M, D), F32)
+    g = np.linspace(0.5, 1.5, D).astype(np.float32)
+    y = torch.empty((M, D), dtype=torch.bfloat16 if dtype == BF16 else torch.float32, device='cuda')
+    L.llama_rmsnorm(to_device(xr, F32), torch.from_numpy(g).cuda(), y, M, D, 1e-5, dtype)
+    ref = rms_norm(xv.astype(np.float64), g.astype(np.float64), 1e-5)
+    got = y.float().cpu().numpy()
+    assert rel_l2(got, ref) < (4e-3 if dtype == BF16 else 1e-6)
+    _sync_ok()
+
+
+# ------------------------------------------------------------- argmax
+def test_argmax_rows_exact_with_ties():
+    B, V = 5, 128256
+    lv, lr = normal_values(15, 3, (B, V), F32)
+    lv = lv.copy()
+    lv[1, 77] = lv[1, 1000] = lv[1].max() + 1.0        # tie: lowest index wins
+    lv[2, :] = 0.5                                     # all equal -> 0
+    lv[3, V - 1] = 100.0                               # last element
+    out = torch.empty(B, dtype=torch.int32, device='cuda')
+    L.llama_argmax_rows(torch.from_numpy(lv).cuda(), out, B, V)
+    assert list(out.cpu().numpy()) == list(argmax(lv))
+    assert list(out.cpu().numpy())[1:4] == [77, 0, V - 1]
+
+
+# ----------------------------------------------------- prefill attention
+@pytest.mark.parametrize('B,S,H,Hk', [(2, 200, 8, 2), (1, 1, 4, 1), (1, 64, 4, 4), (1, 65, 8, 2),
+                                      (1, 2048, 32, 8)])
+def test_attention_prefill_bf16(B, S, H, Hk):
+    d = 128
+    qv, qr = normal_values(16, 1, (B, H, S, d), BF16)
+    kv, kr = normal_values(16, 2, (B, Hk, S, d), BF16)
+    vv, vr = normal_values(16, 3, (B, Hk, S, d), BF16)
+    o = torch.empty((B, S, H * d), dtype=torch.bfloat16, device='cuda')
+    L.llama_attention_prefill(to_device(qr, BF16), to_device(kr, BF16), to_device(vr, BF16), o, B, S, H, Hk, d, BF16)
+    torch.cuda.synchronize()
+    _sync_ok()
+    got = o.float().cpu().numpy()
+    rows = np.arange(S) if S <= 512 else np.unique(np.r_[np.arange(0, S, 37), S - 1])
+    for b in range(B):
+        ref = attention(qv[b][:, rows].astype(np.float64), kv[b].astype(np.float64), vv[b].astype(np.float64), rows)
+        assert rel_l2(got[b][rows], ref) < 1e-2
+
+
+@pytest.mark.parametrize('d', [32, 128])
+def test_attention_prefill_f32(d):
+    B, S, H, Hk = 2, 17, 8, 2
+    qv, qr = normal_values(17, 1, (B, H, S, d), F32)
+    kv, kr = normal_values(17, 2, (B, Hk, S, d), F32)
+    vv, vr = normal_values(17, 3, (B, Hk, S, d), F32)
+    o = torch.empty((B, S, H * d), device='cuda')
+    L.llama_attention_prefill(to_device(qr, F32), to_device(kr, F32), to_device(vr, F32), o, B, S, H, Hk, d, F32)
+    got = o.cpu().numpy()
+    for b in range(B):
+        ref = attention(qv[b].astype(np.float64), kv[b].astype(np.float64), vv[b].astype(np.float64), np.arange(S))
+        assert rel_l2(got[b], ref) < 1e-5
+    _sync_ok()
+
+
+# ------------------------------------------------------ decode attention
+@pytest.mark.parametrize('dtype,d,B,H,Hk,cmax,lens', [
+    (BF16, 128, 3, 32, 8, 1000, [1, 517, 1000]),
+    (BF16, 128, 2, 8, 8, 4097, [4097, 130]),
+    (F32, 32, 2, 8, 2, 300, [17, 300]),
+    (F32, 128, 1, 4, 1, 64, [64]),
+])
+def test_attention_decode(dtype, d, B, H, Hk, cmax, lens):
+    qv, qr = normal_values(18, 1, (B, H, d), dtype)
+    kv, kr = normal_values(18, 2, (B, Hk, cmax, d), dtype)
+    vv, vr = normal_values(18, 3, (B, Hk, cmax, d), dtype)
+    ln = torch.tensor(lens, dtype=torch.int32, device='cuda')
+    o = torch.empty((B, H * d), dtype=torch.bfloat16 if dtype == BF16 else torch.float32, device='cuda')
+    L.llama_attention_decode(to_device(qr, dtype), to_device(kr, dtype), to_device(vr, dtype), ln, o, B, cmax, H, Hk,
+                             d, dtype)
+    torch.cuda.synchronize()
+    _sync_ok()
+    got = o.float().cpu().numpy()
+    for b in range(B):
+        n = lens[b]
+        ref = attention(qv[b][:, None, :].astype(np.float64), kv[b][:, :n].astype(np.float64),
+                        vv[b][:, :n].astype(np.float64), np.array([n - 1]))[0]
+        assert rel_l2(got[b], ref) < (1e-2 if dtype == BF16 else 1e-5)
