@@ -175,9 +175,11 @@ def run_ours(args):
     import seeded_inputs as si
     hbm_peak, tf_burst, tf_sust, peak_src = _peaks()
 
+    NL = args.layers
     max_seq = DECODE_CTX + DECODE_STEPS + max(args.warmup, 1) + 8
-    cfg = make_config(LLAMA3_8B, dtype=L.LLAMA_BF16, max_batch=DECODE_B, max_seq=max_seq,
-                      max_tokens=PREFILL_B * PREFILL_S)
+    cfg = make_config(LLAMA3_8B, dtype=L.LLAMA_BF16, max_batch=1 if args.no_decode else DECODE_B,
+                      max_seq=PREFILL_S if args.no_decode else max_seq, max_tokens=PREFILL_B * PREFILL_S,
+                      n_layers=NL)
     st = torch.cuda.Stream()
     m = L.llama_create(cfg)
     L.llama_init_weights(m, 0, 0.02, st)
@@ -196,10 +198,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     assert L.llama_sync_status(m, st) == 0
     _barrier(ws)
-    # ---- timed prefill region (per-kernel events recorded by the library on `st`)
+    # ---- timed prefill region (no per-kernel events)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    L.llama_profile(m, 1)
-    L.llama_profile_read(m)
     n0 = L.llama_kernel_launches()
     with ClockSampler(local) as clk:
         torch.cuda.synchronize()
@@ -209,12 +209,22 @@ def run_ours(args):
         ev1.record(st)
         torch.cuda.synchronize()
     launches = L.llama_kernel_launches() - n0
-    prof = L.llama_profile_read(m)
-    L.llama_profile(m, 0)
     _barrier(ws)
     ms = ev0.elapsed_time(ev1) / args.steps
     ms_max = _max_over_ranks(ms, ws)
     value = ws * PREFILL_B * PREFILL_S / (ms_max / 1e3)
+    # ---- the same K steps again with the library's per-launch events on `st`
+    L.llama_profile(m, 1)
+    L.llama_profile_read(m)
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(st)
+    for _ in range(args.steps):
+        prefill_step()
+    p1.record(st)
+    prof = L.llama_profile_read(m)
+    L.llama_profile(m, 0)
+    prof_ms = p0.elapsed_time(p1) / args.steps
+    _barrier(ws)
 
     # roofline of the dominant kernel: the tcgen05 GEMM (all four projections, M = 2048)
     D, F, H, Hk, d = 4096, 14336, 32, 8, 128
@@ -223,16 +233,18 @@ def run_ours(args):
     gemm_kinds = ['gemm_qkv_rope', 'gemm_wo_residual', 'gemm_w13_swiglu', 'gemm_w2_residual']
     gemm_ms = sum(prof[k][0] for k in gemm_kinds)
     gemm_launches = sum(prof[k][1] for k in gemm_kinds)
-    achieved = flops_layer * 32 * args.steps / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+    achieved = flops_layer * NL * args.steps / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
     kernels = {k: {'ms_per_step': v[0] / args.steps, 'launches_per_step': v[1] / args.steps,
                    'share': v[0] / max(sum(x[0] for x in prof.values()), 1e-9)} for k, v in prof.items() if v[1]}
-    attn_flops = 4.0 * PREFILL_B * H * d * PREFILL_S * (PREFILL_S + 1) / 2 * 32
+    attn_flops = 4.0 * PREFILL_B * H * d * PREFILL_S * (PREFILL_S + 1) / 2 * NL
     attn = prof.get('attention_prefill', (0, 0))
     roofline = {'kernel': 'gemm_wide_kernel (tcgen05, 4 projections)', 'bound': 'tensor',
                 'achieved': achieved, 'peak': tf_sust, 'unit': 'TFLOP/s',
                 'frac': achieved / tf_sust if achieved else None, 'traffic': None,
                 'peak_kind': f'bf16 sustained ({peak_src})', 'launches': gemm_launches // max(args.steps, 1),
-                'attention_tflops': attn_flops * args.steps / (attn[0] / 1e3) / 1e12 if attn[0] else None}
+                'attention_tflops': attn_flops * args.steps / (attn[0] / 1e3) / 1e12 if attn[0] else None,
+                'measured': f'per-launch CUDA events on the launching stream over {args.steps} profiled steps '
+                            f'({prof_ms:.2f} ms/step with events vs {ms:.2f} without)'}
 
     # ---- end to end through the host API (pinned host buffers)
     host_toks = torch.from_numpy(toks_h.copy()).pin_memory()
@@ -293,8 +305,8 @@ def run_ours(args):
         dprof = L.llama_profile_read(m)
         L.llama_profile(m, 0)
         avg_ctx = DECODE_CTX + (DECODE_STEPS + 1) / 2.0
-        w_bytes = 32 * 2.0 * (D * (H + 2 * Hk) * d + D * H * d + 2 * D * F + D * F) + 2.0 * 128256 * D
-        kv_bytes = 32 * 2.0 * DECODE_B * avg_ctx * Hk * d * 2
+        w_bytes = NL * 2.0 * (D * (H + 2 * Hk) * d + D * H * d + 2 * D * F + D * F) + 2.0 * 128256 * D
+        kv_bytes = NL * 2.0 * DECODE_B * avg_ctx * Hk * d * 2
         step_bytes = w_bytes + kv_bytes
         achieved_gbs = step_bytes / (dms / 1e3) / 1e9
         decode = {'value': ws * DECODE_B / (dms / 1e3), 'unit': 'tokens/s', 'ms_per_step': dms,
@@ -308,7 +320,7 @@ def run_ours(args):
                   'clocks': dclk.summary()}
 
     cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline and NL == 32:
         tok_s, dt, desc = oracle_prefill_sample()
         cpu = {'value': tok_s, 'unit': 'tokens/s', 'cores': os.cpu_count(), 'kind': 'oracle', 'sample': desc,
                'seconds': dt}
@@ -321,7 +333,7 @@ def run_ours(args):
                 'data': 'synthetic: seeded N(0,0.02) weights of the 8B shapes, uniform token ids',
                 'config': {'workload': 'llama3-8b-shape full-model prefill, B=1, S=2048 (32 layers + LM head '
                                        '+ argmax); decode: B=32, context 4096, 128 greedy steps',
-                           'batch': PREFILL_B, 'seq_len': PREFILL_S, 'layers': 32,
+                           'batch': PREFILL_B, 'seq_len': PREFILL_S, 'layers': NL,
                            'l2': 'inputs larger than L2 (16 GB of weights streamed per step)',
                            'parallelism': f'replicas x{ws}'},
                 'roofline': roofline, 'cpu_baseline': cpu, 'e2e': e2e, 'gpu_launches': launches,
@@ -340,6 +352,7 @@ def main():
     ap.add_argument('--warmup', type=int, default=3)
     ap.add_argument('--impl', choices=['ours', 'reference'], default='ours')
     ap.add_argument('--no-decode', action='store_true')
+    ap.add_argument('--layers', type=int, default=32, help='decoder layers (32 = the 8B model)')
     ap.add_argument('--no-cpu-baseline', action='store_true')
     args = ap.parse_args()
     if args.impl == 'reference':
