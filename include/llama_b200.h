@@ -177,6 +177,28 @@ int llama_attention_prefill(const void* q, const void* k, const void* v, void* o
 int llama_attention_decode(const void* q, const void* kc, const void* vc, const int32_t* len, void* o, int32_t B,
                            int32_t cmax, int32_t H, int32_t Hk, int32_t d, int32_t dtype, void* stream);
 
+/* llama_attention_decode for callers that cannot let this library allocate device memory.
+ * Some programs own all of the GPU's memory through their own allocator or pool (a serving
+ * engine's preallocated cache pool, a framework's caching allocator that has reserved most of
+ * the card): a cudaMalloc made behind their back can fail or fragment that pool, and a
+ * cudaMalloc/cudaFree inside a latency-critical loop synchronizes the whole device. This call
+ * never allocates or frees device memory; everything else is the same as
+ * llama_attention_decode (arguments, layouts, results).
+ * Its split partials live in one static 4 MiB device array that every GPU which loads this
+ * library keeps until the process exits. Calls needing more than 4 MiB of partials
+ * (B * H * splits * (d + 2) * 4 bytes, splits chosen by the library) return
+ * LLAMA_ERR_SHAPE; for H = 32, Hk = 8, d = 128 every B up to 200 fits.
+ * The first call on a device looks up the array's device address for that device
+ * (cudaGetSymbolAddress); make that first call before any stream capture begins.
+ * Every call uses the same array, so calls that may run at the same time on the GPU (e.g. on
+ * two streams) race: order them. Nothing has to be cleared between calls, since every partial
+ * is written before it is read. This call keeps no device status word: a len[b] outside
+ * [1, cmax] gives NaN rows instead of an error code.
+ * The pages have no counterpart of this entry point: it exists for deployment only. */
+int llama_attention_decode_noalloc(const void* q, const void* kc, const void* vc, const int32_t* len, void* o,
+                                   int32_t B, int32_t cmax, int32_t H, int32_t Hk, int32_t d, int32_t dtype,
+                                   void* stream);
+
 /* y = x W^T: x [M][K], w [N][K] (dtype), y fp32 [M][N]. variant 0 = automatic, 1 = the wide
  * persistent tcgen05 kernel, 2 = the skinny split-K tcgen05 kernel (M <= 256); fp32 ignores it.
  * bf16 requires K % 8 == 0 and 16-byte aligned x and w. */

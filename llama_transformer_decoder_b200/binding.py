@@ -75,6 +75,8 @@ _SIGS = {
     'llama_status_string': (ctypes.c_char_p, [ctypes.c_int]),
     'llama_attention_prefill': (ctypes.c_int, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P]),
     'llama_attention_decode': (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P]),
+    'llama_attention_decode_noalloc': (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32,
+                                                      _P]),
     'llama_linear': (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P]),
     'llama_rmsnorm': (ctypes.c_int, [_P, _P, _P, _I32, _I32, _F, _I32, _P]),
     'llama_argmax_rows': (ctypes.c_int, [_P, _P, _I32, _I32, _P]),
@@ -219,6 +221,11 @@ def llama_attention_prefill(q, k, v, o, B, S, H, Hk, d, dtype, stream=None):
 def llama_attention_decode(q, kc, vc, length, o, B, cmax, H, Hk, d, dtype, stream=None):
     _check(_lib.llama_attention_decode(_ptr(q), _ptr(kc), _ptr(vc), _ptr(length), _ptr(o), B, cmax, H, Hk, d, dtype,
                                        _stream(stream)), 'llama_attention_decode')
+
+
+def llama_attention_decode_noalloc(q, kc, vc, length, o, B, cmax, H, Hk, d, dtype, stream=None):
+    _check(_lib.llama_attention_decode_noalloc(_ptr(q), _ptr(kc), _ptr(vc), _ptr(length), _ptr(o), B, cmax, H, Hk,
+                                               d, dtype, _stream(stream)), 'llama_attention_decode_noalloc')
 
 
 def llama_linear(x, w, y, M, N, K, dtype, variant=0, stream=None):
