@@ -42,6 +42,8 @@ def _peaks():
 
 # --------------------------------------------------------------- clocks
 class ClockSampler:
+    """nvidia-smi sampling every 200 ms during a timed region (one background
+    process, started before the region and stopped after it)."""
     FIELDS = ('index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,'
               'clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,'
               'clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap')
@@ -49,37 +51,41 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
         self.rows = []
-        self._stop = threading.Event()
-        self._t = threading.Thread(target=self._run, daemon=True)
-
-    def _run(self):
-        while not self._stop.is_set():
-            try:
-                out = subprocess.run(['nvidia-smi', '-i', str(self.idx), f'--query-gpu={self.FIELDS}',
-                                      '--format=csv,noheader,nounits'], capture_output=True, text=True, timeout=5)
-                for ln in out.stdout.strip().splitlines():
-                    self.rows.append([c.strip() for c in ln.split(',')])
-            except Exception:
-                pass
-            self._stop.wait(0.2)
+        self.proc = None
 
     def __enter__(self):
-        self._t.start()
+        try:
+            self.proc = subprocess.Popen(['nvidia-smi', '-i', str(self.idx), f'--query-gpu={self.FIELDS}',
+                                          '--format=csv,noheader,nounits', '-lms', '200'],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.5)   # first sample before the region starts
+        except Exception:
+            self.proc = None
         return self
 
     def __exit__(self, *a):
-        self._stop.set()
-        self._t.join(timeout=10)
+        if self.proc is None:
+            return
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for ln in (out or '').strip().splitlines():
+            self.rows.append([c.strip() for c in ln.split(',')])
 
     def summary(self):
-        if not self.rows:
+        rows = [r for r in self.rows if len(r) >= 9]
+        if not rows:
             return {'sm_mhz': None, 'sm_max_mhz': None, 'reasons': ['nvidia-smi unavailable'], 'samples': 0}
-        sm = [float(r[1]) for r in self.rows if r[1].replace('.', '').isdigit()]
-        mx = [float(r[2]) for r in self.rows if r[2].replace('.', '').isdigit()]
+        sm = [float(r[1]) for r in rows if r[1].replace('.', '').isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace('.', '').isdigit()]
         names = ['hw_slowdown', 'hw_thermal_slowdown', 'sw_thermal_slowdown', 'sw_power_cap']
-        reasons = sorted({n for r in self.rows for n, v in zip(names, r[5:9]) if v.strip().lower() == 'active'})
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == 'active'})
         return {'sm_mhz': statistics.median(sm) if sm else None, 'sm_max_mhz': max(mx) if mx else None,
-                'reasons': reasons, 'samples': len(self.rows)}
+                'reasons': reasons, 'samples': len(rows)}
 
 
 # ------------------------------------------------------------ distributed

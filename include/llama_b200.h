@@ -185,9 +185,9 @@ int llama_attention_decode(const void* q, const void* kc, const void* vc, const 
  * never allocates or frees device memory; everything else is the same as
  * llama_attention_decode (arguments, layouts, results).
  * Its split partials live in one static 4 MiB device array that every GPU which loads this
- * library keeps until the process exits. Calls needing more than 4 MiB of partials
- * (B * H * splits * (d + 2) * 4 bytes, splits chosen by the library) return
- * LLAMA_ERR_SHAPE; for H = 32, Hk = 8, d = 128 every B up to 200 fits.
+ * library keeps until the process exits. Calls needing more than 4 MiB of partials return
+ * LLAMA_ERR_SHAPE: for bf16 with d = 128 the partials take (B*Hk + 4*SMs) * (H/Hk) * (d+2) * 4
+ * bytes (SMs = 148 on B200), so with H = 32, Hk = 8 every B up to 170 fits.
  * The first call on a device looks up the array's device address for that device
  * (cudaGetSymbolAddress); make that first call before any stream capture begins.
  * Every call uses the same array, so calls that may run at the same time on the GPU (e.g. on

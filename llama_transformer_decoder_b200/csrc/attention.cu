@@ -454,6 +454,270 @@ __global__ void attn_decode_combine_kernel(const float* __restrict__ part, T* __
   }
 }
 
+
+// ---------------------------------------------- decode, bf16 d = 128 (mma)
+// Every warp is an independent flash decoder over a contiguous range of the
+// global tile sequence: (sequence b, kv head g, 32-key tile t) in that order,
+// T tiles in all; warp w of W takes tiles [T*w/W, T*(w+1)/W), so warps differ
+// by at most one tile whatever the lengths. Cutting that sequence at warp and
+// at (b, g) boundaries gives pieces; the piece of (b, g) held by warp w is
+// stored in slot (b*Hk + g) + w, which is unique, so the partials need only
+// (B*Hk + W) slots. A warp streams its tiles through a private 3-stage ring of
+// swizzled shared memory (cp.async, zero fill past the last key) without
+// draining at piece boundaries, computes S = Q K^T and O += P V with mma.sync
+// (the G query heads of the kv head are rows 0..G-1 of a 16-row tile), and
+// writes (o, max, sum) of every piece for the combine kernel.
+constexpr int DM_KEYS = 32;
+constexpr int DM_STAGES = 3;
+constexpr int DM_WARPS = 4;
+constexpr int DM_TILE = DM_KEYS * 256;             // one K (or V) tile: 32 rows x 256 B
+constexpr int DM_STAGE = 2 * DM_TILE;
+constexpr int DM_SMEM = DM_WARPS * DM_STAGES * DM_STAGE;
+
+__device__ __forceinline__ int dm_keys(const int32_t* nkeys, int b, int add, int nmax) {
+  return min(nkeys[b] + add, nmax);
+}
+__device__ __forceinline__ int dm_tiles(int n) { return n > 0 ? (n + DM_KEYS - 1) / DM_KEYS : 0; }
+
+struct TileCursor {
+  int b, g, t;          // sequence, kv head, tile of (b, g)
+  int n, nt;            // keys and tiles of sequence b
+  long long left;       // tiles left in this warp's range, counting the current one
+};
+
+__device__ void tc_seek(TileCursor& c, long long x, long long count, const int32_t* nkeys, int add, int nmax, int B,
+                        int Hk) {
+  c.left = count;
+  long long acc = 0;
+  for (int b = 0; b < B; ++b) {
+    const int n = dm_keys(nkeys, b, add, nmax);
+    const int nt = dm_tiles(n);
+    const long long cnt = (long long)Hk * nt;
+    if (x < acc + cnt) {
+      const int r = (int)(x - acc);
+      c.b = b; c.n = n; c.nt = nt; c.g = r / nt; c.t = r - c.g * nt;
+      return;
+    }
+    acc += cnt;
+  }
+  c.left = 0;
+}
+
+// Advance one tile; true when the piece (this warp's part of one (b, g)) ended.
+__device__ bool tc_next(TileCursor& c, const int32_t* nkeys, int add, int nmax, int B, int Hk) {
+  const bool last_in_range = --c.left <= 0;
+  if (++c.t < c.nt) return last_in_range;
+  c.t = 0;
+  if (++c.g == Hk) {
+    c.g = 0;
+    do {
+      ++c.b;
+      c.n = c.b < B ? dm_keys(nkeys, c.b, add, nmax) : 0;
+      c.nt = dm_tiles(c.n);
+    } while (c.nt == 0 && c.b < B);
+  }
+  return true;
+}
+
+__device__ __forceinline__ void dm_load_tile(uint8_t* stage, const bf16* kc, const bf16* vc, const TileCursor& c,
+                                             int Hk, int Smax, int lane) {
+  const int key0 = c.t * DM_KEYS;
+  const int valid = min(DM_KEYS, c.n - key0);
+  const size_t row0 = ((size_t)c.b * Hk + c.g) * Smax + key0;
+  const bf16* ks = kc + row0 * 128;
+  const bf16* vs = vc + row0 * 128;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int idx = i * 32 + lane;
+    const int r = idx >> 4, ch = idx & 15;
+    const bool ok = r < valid;
+    const size_t off = (size_t)(ok ? r : 0) * 128 + ch * 8;
+    cp_async16(stage + swz(r, ch), ks + off, ok);
+    cp_async16(stage + DM_TILE + swz(r, ch), vs + off, ok);
+  }
+}
+
+__global__ void __launch_bounds__(DM_WARPS * 32, 1)
+    attn_decode_mma_kernel(const bf16* __restrict__ q, const bf16* __restrict__ kc, const bf16* __restrict__ vc,
+                           const int32_t* __restrict__ nkeys, int add_keys, int nmax, float* __restrict__ part, int B,
+                           int H, int Hk, int Smax, float scale_log2, int* status) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = H / Hk;
+  uint8_t* ring = sm + warp * DM_STAGES * DM_STAGE;
+
+  long long total = 0;
+  for (int b = 0; b < B; ++b) {
+    if (nkeys[b] + add_keys > nmax && blockIdx.x == 0 && threadIdx.x == 0) set_status(status, LLAMA_ERR_DEVICE_BOUNDS);
+    total += (long long)Hk * dm_tiles(dm_keys(nkeys, b, add_keys, nmax));
+  }
+  const long long W = (long long)gridDim.x * DM_WARPS;
+  const int w = blockIdx.x * DM_WARPS + warp;
+  const long long x0 = total * w / W, x1 = total * (w + 1) / W;
+  if (x1 <= x0) return;
+
+  TileCursor ld, cp;
+  tc_seek(ld, x0, x1 - x0, nkeys, add_keys, nmax, B, Hk);
+  cp = ld;
+  int issued = 0;
+  bool ld_done = ld.left <= 0;
+  for (int i = 0; i < DM_STAGES - 1; ++i) {
+    if (!ld_done) {
+      dm_load_tile(ring + (issued % DM_STAGES) * DM_STAGE, kc, vc, ld, Hk, Smax, lane);
+      ++issued;
+      tc_next(ld, nkeys, add_keys, nmax, B, Hk);
+      ld_done = ld.left <= 0;
+    }
+    cp_async_commit();
+  }
+
+  const int row = lane >> 2, tq = lane & 3;   // fragment row (query head within the group), column pair
+  const bool real = row < G;
+  uint32_t qa[8][2];
+  float oacc[16][2];
+  float m_r = -INFINITY, l_r = 0.f;
+  int consumed = 0;
+  bool start = true;
+  while (cp.left > 0) {
+    if (start) {   // new piece: reset the state and fetch the G query rows of (b, g)
+      const bf16* qr = q + ((size_t)cp.b * H + cp.g * G + (real ? row : 0)) * 128;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        qa[ks][0] = real ? *reinterpret_cast<const uint32_t*>(qr + ks * 16 + 2 * tq) : 0u;
+        qa[ks][1] = real ? *reinterpret_cast<const uint32_t*>(qr + ks * 16 + 8 + 2 * tq) : 0u;
+      }
+#pragma unroll
+      for (int n = 0; n < 16; ++n) oacc[n][0] = oacc[n][1] = 0.f;
+      m_r = -INFINITY;
+      l_r = 0.f;
+      start = false;
+    }
+    if (!ld_done) {   // keep DM_STAGES-1 tiles in flight
+      dm_load_tile(ring + (issued % DM_STAGES) * DM_STAGE, kc, vc, ld, Hk, Smax, lane);
+      ++issued;
+      tc_next(ld, nkeys, add_keys, nmax, B, Hk);
+      ld_done = ld.left <= 0;
+    }
+    cp_async_commit();
+    cp_async_wait<DM_STAGES - 1>();
+    __syncwarp();
+    const uint8_t* st = ring + (consumed % DM_STAGES) * DM_STAGE;
+    const uint32_t kb = smem_u32(st), vb = smem_u32(st + DM_TILE);
+    const int valid = min(DM_KEYS, cp.n - cp.t * DM_KEYS);
+    // S = Q K^T for 32 keys
+    float sc[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+      for (int jp = 0; jp < 2; ++jp) {
+        const int r = jp * 16 + (lane & 7) + ((lane >> 4) << 3);
+        const int c = ks * 2 + ((lane >> 3) & 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kb + swz(r, c), b0, b1, b2, b3);
+        mma_bf16(sc[2 * jp], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
+        mma_bf16(sc[2 * jp + 1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
+      }
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int kk = j * 8 + 2 * tq + e;
+        const float v = kk < valid ? sc[j][e] * scale_log2 : -INFINITY;
+        sc[j][e] = v;
+        mx = fmaxf(mx, v);
+      }
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float mnew = fmaxf(m_r, mx);
+    const float corr = exp2f(m_r - mnew);
+    m_r = mnew;
+    float ls = 0.f;
+    uint32_t pa[2][2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float p0 = exp2f(sc[j][0] - mnew), p1 = exp2f(sc[j][1] - mnew);
+      ls += p0 + p1;
+      pa[j >> 1][j & 1] = pack_bf16(p0, p1);
+    }
+    ls += __shfl_xor_sync(0xffffffffu, ls, 1);
+    ls += __shfl_xor_sync(0xffffffffu, ls, 2);
+    l_r = l_r * corr + ls;
+    // O += P V  (rows 8..15 of the tiles are zero padding)
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+#pragma unroll
+      for (int np = 0; np < 8; ++np) {
+        const int r = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        const int c = np * 2 + (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vb + swz(r, c), b0, b1, b2, b3);
+        float t0[4] = {ks == 0 ? oacc[2 * np][0] * corr : oacc[2 * np][0],
+                       ks == 0 ? oacc[2 * np][1] * corr : oacc[2 * np][1], 0.f, 0.f};
+        float t1[4] = {ks == 0 ? oacc[2 * np + 1][0] * corr : oacc[2 * np + 1][0],
+                       ks == 0 ? oacc[2 * np + 1][1] * corr : oacc[2 * np + 1][1], 0.f, 0.f};
+        mma_bf16(t0, pa[ks][0], 0u, pa[ks][1], 0u, b0, b1);
+        mma_bf16(t1, pa[ks][0], 0u, pa[ks][1], 0u, b2, b3);
+        oacc[2 * np][0] = t0[0]; oacc[2 * np][1] = t0[1];
+        oacc[2 * np + 1][0] = t1[0]; oacc[2 * np + 1][1] = t1[1];
+      }
+    }
+    __syncwarp();   // the stage may be refilled from the next iteration on
+    ++consumed;
+    const int b_done = cp.b, g_done = cp.g;
+    if (tc_next(cp, nkeys, add_keys, nmax, B, Hk)) {
+      if (real) {
+        const size_t slot = (size_t)b_done * Hk + g_done + w;
+        float* dst = part + (slot * G + row) * 130;
+#pragma unroll
+        for (int n = 0; n < 16; ++n) *reinterpret_cast<float2*>(dst + n * 8 + 2 * tq) = make_float2(oacc[n][0], oacc[n][1]);
+        if (tq == 0) { dst[128] = m_r; dst[129] = l_r; }
+      }
+      start = true;
+    }
+  }
+  cp_async_wait<0>();
+}
+
+// Merge the pieces of every (b, h): the warps holding tiles of (b, g) are
+// owner(T0) .. owner(T1-1), owner(x) = ((x+1)W - 1) / T.
+template <typename T, int D>
+__global__ void attn_decode_combine_pieces_kernel(const float* __restrict__ part, const int32_t* __restrict__ nkeys,
+                                                  int add_keys, int nmax, T* __restrict__ o, int B, int H, int Hk,
+                                                  long long W) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int G = H / Hk, g = h / G, row = h - g * G;
+  long long total = 0, t0 = 0;
+  int nt_b = 0;
+  for (int bb = 0; bb < B; ++bb) {
+    const int nt = dm_tiles(dm_keys(nkeys, bb, add_keys, nmax));
+    if (bb == b) { t0 = total + (long long)g * nt; nt_b = nt; }
+    total += (long long)Hk * nt;
+  }
+  if (nt_b == 0 || total == 0) {
+    for (int dd = threadIdx.x; dd < D; dd += blockDim.x) o[((size_t)b * H + h) * D + dd] = from_f<T>(NAN);
+    return;
+  }
+  const long long w_lo = ((t0 + 1) * W - 1) / total, w_hi = ((t0 + nt_b) * W - 1) / total;
+  const size_t bg = (size_t)b * Hk + g;
+  float M = -INFINITY;
+  for (long long w = w_lo; w <= w_hi; ++w) M = fmaxf(M, part[((bg + w) * G + row) * (D + 2) + D]);
+  for (int dd = threadIdx.x; dd < D; dd += blockDim.x) {
+    float L = 0.f, O = 0.f;
+    for (long long w = w_lo; w <= w_hi; ++w) {
+      const float* r = part + ((bg + w) * G + row) * (D + 2);
+      const float f = exp2f(r[D] - M);
+      L += r[D + 1] * f;
+      O += r[dd] * f;
+    }
+    o[((size_t)b * H + h) * D + dd] = from_f<T>(O / L);
+  }
+}
+
 template <typename T, int D>
 int decode_launch(const void* q, const void* kc, const void* vc, const int32_t* nkeys, int add_keys, void* o, int B,
                   int cmax, int H, int Hk, int Smax, float* part, int splits, int* status, cudaStream_t st) {
@@ -516,6 +780,7 @@ int attention_prefill(const void* q, const void* kc, const void* vc, void* o, co
   return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
+namespace {
 int decode_splits(int cmax, int B, int Hk) {
   const int target = 2 * num_sms();
   int s = (target + B * Hk - 1) / (B * Hk);
@@ -524,19 +789,41 @@ int decode_splits(int cmax, int B, int Hk) {
   return s < 1 ? 1 : s;
 }
 
-size_t decode_scratch_floats(int B, int H, int d, int splits) { return (size_t)B * H * splits * (d + 2); }
+bool use_mma_decode(int d, int dtype) { return dtype == LLAMA_BF16 && d == 128; }
+}  // namespace
+
+size_t decode_scratch_floats(int cmax, int B, int H, int Hk, int d, int dtype) {
+  if (use_mma_decode(d, dtype)) return ((size_t)B * Hk + (size_t)num_sms() * DM_WARPS) * (H / Hk) * (d + 2);
+  return (size_t)B * H * decode_splits(cmax, B, Hk) * (d + 2);
+}
 
 int attention_decode(const void* q, const void* kc, const void* vc, const int32_t* nkeys, int add_keys, void* o,
                      int B, int cmax, int H, int Hk, int d, int Smax, int dtype, DecodeScratch* scratch, int* status,
                      cudaStream_t st) {
   if (B <= 0) return LLAMA_OK;
   if (H % Hk != 0 || H / Hk > DEC_MAXG) return LLAMA_ERR_SHAPE;
-  const int splits = decode_splits(cmax, B, Hk);
-  if (!scratch || !scratch->part || scratch->floats < decode_scratch_floats(B, H, d, splits))
+  if (!scratch || !scratch->part || scratch->floats < decode_scratch_floats(cmax, B, H, Hk, d, dtype))
     return LLAMA_ERR_INVALID_ARG;
+  if (use_mma_decode(d, dtype)) {
+    const int grid = num_sms();
+    static bool attr = false;
+    if (!attr) {
+      if (cudaFuncSetAttribute(attn_decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DM_SMEM) !=
+          cudaSuccess)
+        return LLAMA_ERR_CUDA;
+      attr = true;
+    }
+    const float scale_log2 = kLog2e / sqrtf((float)d);
+    const int nmax = cmax < Smax ? cmax : Smax;
+    attn_decode_mma_kernel<<<grid, DM_WARPS * 32, DM_SMEM, st>>>(
+        static_cast<const bf16*>(q), static_cast<const bf16*>(kc), static_cast<const bf16*>(vc), nkeys, add_keys, nmax,
+        scratch->part, B, H, Hk, Smax, scale_log2, status);
+    attn_decode_combine_pieces_kernel<bf16, 128><<<dim3(H, B), 128, 0, st>>>(
+        scratch->part, nkeys, add_keys, nmax, static_cast<bf16*>(o), B, H, Hk, (long long)grid * DM_WARPS);
+    return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  }
+  const int splits = decode_splits(cmax, B, Hk);
   if (dtype == LLAMA_BF16) {
-    if (d == 128) return decode_launch<bf16, 128>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch->part,
-                                                  splits, status, st);
     if (d == 64) return decode_launch<bf16, 64>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch->part,
                                                 splits, status, st);
   } else {

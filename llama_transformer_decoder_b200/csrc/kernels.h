@@ -50,8 +50,7 @@ struct DecodeScratch {
   float* part;  // [B][H][splits][d + 2]
   size_t floats;
 };
-int decode_splits(int cmax, int B, int Hk);
-size_t decode_scratch_floats(int B, int H, int d, int splits);
+size_t decode_scratch_floats(int cmax, int B, int H, int Hk, int d, int dtype);
 int attention_decode(const void* q, const void* kc, const void* vc, const int32_t* nkeys, int add_keys, void* o,
                      int B, int cmax, int H, int Hk, int d, int Smax, int dtype, DecodeScratch* scratch,
                      int* status, cudaStream_t st);

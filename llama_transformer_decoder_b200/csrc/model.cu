@@ -488,7 +488,7 @@ int llama_create(const llama_config* cfg, llama_model** out) {
   {
     size_t need = 0;
     for (int B = 1; B <= c.max_batch; ++B)
-      need = std::max(need, decode_scratch_floats(B, c.n_heads, m->d, decode_splits(c.max_seq, B, c.n_kv_heads)));
+      need = std::max(need, decode_scratch_floats(c.max_seq, B, c.n_heads, c.n_kv_heads, m->d, c.dtype));
     if (grow_decode_scratch(&m->ds, need) != LLAMA_OK) { delete m; return LLAMA_ERR_OOM; }
     m->allocs.push_back(m->ds.part);
   }
@@ -803,8 +803,7 @@ int llama_attention_decode(const void* q, const void* kc, const void* vc, const 
   if (dtype != LLAMA_F32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
   DevCtx* c = dev_ctx();
   if (!c) return LLAMA_ERR_OOM;
-  const int splits = decode_splits(cmax, B, Hk);
-  RC(grow_decode_scratch(&c->ds, decode_scratch_floats(B, H, d, splits)));
+  RC(grow_decode_scratch(&c->ds, decode_scratch_floats(cmax, B, H, Hk, d, dtype)));
   return attention_decode(q, kc, vc, len, 0, o, B, cmax, H, Hk, d, cmax, dtype, &c->ds, c->status, S_(stream));
 }
 

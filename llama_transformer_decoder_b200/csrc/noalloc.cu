@@ -48,8 +48,7 @@ extern "C" int llama_attention_decode_noalloc(const void* q, const void* kc, con
   if (!q || !kc || !vc || !len || !o) return LLAMA_ERR_INVALID_ARG;
   if (B <= 0 || cmax <= 0 || H <= 0 || Hk <= 0 || H % Hk != 0) return LLAMA_ERR_SHAPE;
   if (dtype != LLAMA_F32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
-  const int splits = llama::decode_splits(cmax, B, Hk);
-  const size_t need = llama::decode_scratch_floats(B, H, d, splits);
+  const size_t need = llama::decode_scratch_floats(cmax, B, H, Hk, d, dtype);
   if (need * sizeof(float) > kScratchBytes) return LLAMA_ERR_SHAPE;
   float* scratch = nullptr;
   const int rc = scratch_address(&scratch);

@@ -45,7 +45,7 @@ def test_noalloc_decode_matches_allocating_entry_point():
 
 
 def test_noalloc_decode_rejects_sizes_beyond_its_array():
-    B, H, Hk, d, cmax = 256, 32, 8, 128, 64        # 256*32*(128+2)*4 B > 4 MiB of partials
+    B, H, Hk, d, cmax = 256, 32, 8, 128, 64        # (256*8 + 4*148)*4*(128+2)*4 B > 4 MiB of partials
     q = torch.zeros((B, H, d), dtype=torch.bfloat16, device='cuda')
     k = torch.zeros((B, Hk, cmax, d), dtype=torch.bfloat16, device='cuda')
     ln = torch.ones(B, dtype=torch.int32, device='cuda')
