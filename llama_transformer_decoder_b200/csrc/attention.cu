@@ -705,10 +705,14 @@ __global__ void attn_decode_combine_pieces_kernel(const float* __restrict__ part
   const long long w_lo = ((t0 + 1) * W - 1) / total, w_hi = ((t0 + nt_b) * W - 1) / total;
   const size_t bg = (size_t)b * Hk + g;
   float M = -INFINITY;
-  for (long long w = w_lo; w <= w_hi; ++w) M = fmaxf(M, part[((bg + w) * G + row) * (D + 2) + D]);
+  // warps whose tile range is empty (fewer tiles than warps) wrote nothing
+  auto owns = [&](long long w) { return total * (w + 1) / W > total * w / W; };
+  for (long long w = w_lo; w <= w_hi; ++w)
+    if (owns(w)) M = fmaxf(M, part[((bg + w) * G + row) * (D + 2) + D]);
   for (int dd = threadIdx.x; dd < D; dd += blockDim.x) {
     float L = 0.f, O = 0.f;
     for (long long w = w_lo; w <= w_hi; ++w) {
+      if (!owns(w)) continue;
       const float* r = part + ((bg + w) * G + row) * (D + 2);
       const float f = exp2f(r[D] - M);
       L += r[D + 1] * f;

@@ -182,3 +182,28 @@ def test_attention_decode(dtype, d, B, H, Hk, cmax, lens):
         ref = attention(qv[b][:, None, :].astype(np.float64), kv[b][:, :n].astype(np.float64),
                         vv[b][:, :n].astype(np.float64), np.array([n - 1]))[0]
         assert rel_l2(got[b], ref) < (1e-2 if dtype == BF16 else 1e-5)
+
+
+def test_attention_decode_few_tiles_after_many():
+    """Fewer 32-key tiles than decoding warps, run right after a large call
+    that filled the library's partial buffers: only the warps that own tiles
+    may contribute to the merge."""
+    big = dict(B=32, H=32, Hk=8, cmax=4224, lens=[4097 + 4 * i for i in range(32)])
+    small = dict(B=2, H=4, Hk=2, cmax=256, lens=[101, 101])
+    outs = []
+    for i, c in enumerate((big, small)):
+        B, H, Hk, cmax, lens = c['B'], c['H'], c['Hk'], c['cmax'], c['lens']
+        qv, qr = normal_values(30 + i, 1, (B, H, 128), BF16)
+        kv, kr = normal_values(30 + i, 2, (B, Hk, cmax, 128), BF16)
+        vv, vr = normal_values(30 + i, 3, (B, Hk, cmax, 128), BF16)
+        o = torch.empty((B, H * 128), dtype=torch.bfloat16, device='cuda')
+        L.llama_attention_decode(to_device(qr, BF16), to_device(kr, BF16), to_device(vr, BF16),
+                                 torch.tensor(lens, dtype=torch.int32, device='cuda'), o, B, cmax, H, Hk, 128, BF16)
+        outs.append((o.float().cpu().numpy(), qv, kv, vv, lens))
+    got, qv, kv, vv, lens = outs[1]
+    for b in range(2):
+        n = lens[b]
+        ref = attention(qv[b][:, None, :].astype(np.float64), kv[b][:, :n].astype(np.float64),
+                        vv[b][:, :n].astype(np.float64), np.array([n - 1]))[0]
+        assert rel_l2(got[b], ref) < 1e-2
+    _sync_ok()
