@@ -168,31 +168,13 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- our arm
-def run_ours(args):
-    import numpy as np
-    import torch
-    ws, rank, local = _dist()
-    torch.cuda.set_device(local)
-    if ws > 1:
-        import torch.distributed as dist
-        dist.init_process_group('nccl', timeout=datetime.timedelta(seconds=600), device_id=torch.device('cuda', local))
-    from llama_transformer_decoder_b200 import binding as L
-    from llama_transformer_decoder_b200.configs import LLAMA3_8B, make_config
-    import seeded_inputs as si
-    hbm_peak, tf_burst, tf_sust, peak_src = _peaks()
+D_, F_, H_, HK_, HD_, V_ = 4096, 14336, 32, 8, 128, 128256
 
-    NL = args.layers
-    max_seq = DECODE_CTX + DECODE_STEPS + max(args.warmup, 1) + 8
-    cfg = make_config(LLAMA3_8B, dtype=L.LLAMA_BF16, max_batch=1 if args.no_decode else DECODE_B,
-                      max_seq=PREFILL_S if args.no_decode else max_seq, max_tokens=PREFILL_B * PREFILL_S,
-                      n_layers=NL)
-    st = torch.cuda.Stream()
-    m = L.llama_create(cfg)
-    L.llama_init_weights(m, 0, 0.02, st)
-    toks_h = si.tokens(1, PREFILL_B * PREFILL_S, 128256).reshape(PREFILL_B, PREFILL_S)
-    toks = torch.from_numpy(toks_h).cuda()
-    arg = torch.empty(DECODE_B, dtype=torch.int32, device='cuda')
-    torch.cuda.synchronize()
+
+def measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust, peak_src):
+    """Timed prefill steps (no per-launch events), then the same steps with
+    the library's per-launch events for the kernel breakdown and roofline."""
+    import torch
 
     def prefill_step():
         L.llama_reset(m, st)
@@ -204,7 +186,6 @@ def run_ours(args):
     torch.cuda.synchronize()
     assert L.llama_sync_status(m, st) == 0
     _barrier(ws)
-    # ---- timed prefill region (no per-kernel events)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n0 = L.llama_kernel_launches()
     with ClockSampler(local) as clk:
@@ -216,10 +197,7 @@ def run_ours(args):
         torch.cuda.synchronize()
     launches = L.llama_kernel_launches() - n0
     _barrier(ws)
-    ms = ev0.elapsed_time(ev1) / args.steps
-    ms_max = _max_over_ranks(ms, ws)
-    value = ws * PREFILL_B * PREFILL_S / (ms_max / 1e3)
-    # ---- the same K steps again with the library's per-launch events on `st`
+    ms = _max_over_ranks(ev0.elapsed_time(ev1) / args.steps, ws)
     L.llama_profile(m, 1)
     L.llama_profile_read(m)
     p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -231,18 +209,16 @@ def run_ours(args):
     L.llama_profile(m, 0)
     prof_ms = p0.elapsed_time(p1) / args.steps
     _barrier(ws)
-
-    # roofline of the dominant kernel: the tcgen05 GEMM (all four projections, M = 2048)
-    D, F, H, Hk, d = 4096, 14336, 32, 8, 128
     M = PREFILL_B * PREFILL_S
-    flops_layer = 2.0 * M * D * ((H + 2 * Hk) * d + H * d + 2 * F + F)
+    flops_layer = 2.0 * M * D_ * ((H_ + 2 * HK_) * HD_ + H_ * HD_ + 2 * F_ + F_)
     gemm_kinds = ['gemm_qkv_rope', 'gemm_wo_residual', 'gemm_w13_swiglu', 'gemm_w2_residual']
     gemm_ms = sum(prof[k][0] for k in gemm_kinds)
     gemm_launches = sum(prof[k][1] for k in gemm_kinds)
     achieved = flops_layer * NL * args.steps / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+    total_prof = max(sum(x[0] for x in prof.values()), 1e-9)
     kernels = {k: {'ms_per_step': v[0] / args.steps, 'launches_per_step': v[1] / args.steps,
-                   'share': v[0] / max(sum(x[0] for x in prof.values()), 1e-9)} for k, v in prof.items() if v[1]}
-    attn_flops = 4.0 * PREFILL_B * H * d * PREFILL_S * (PREFILL_S + 1) / 2 * NL
+                   'share': v[0] / total_prof} for k, v in prof.items() if v[1]}
+    attn_flops = 4.0 * PREFILL_B * H_ * HD_ * PREFILL_S * (PREFILL_S + 1) / 2 * NL
     attn = prof.get('attention_prefill', (0, 0))
     roofline = {'kernel': 'gemm_wide_kernel (tcgen05, 4 projections)', 'bound': 'tensor',
                 'achieved': achieved, 'peak': tf_sust, 'unit': 'TFLOP/s',
@@ -251,8 +227,13 @@ def run_ours(args):
                 'attention_tflops': attn_flops * args.steps / (attn[0] / 1e3) / 1e12 if attn[0] else None,
                 'measured': f'per-launch CUDA events on the launching stream over {args.steps} profiled steps '
                             f'({prof_ms:.2f} ms/step with events vs {ms:.2f} without)'}
+    return ms, launches, clk.summary(), roofline, kernels
 
-    # ---- end to end through the host API (pinned host buffers)
+
+def measure_e2e(L, m, st, toks_h, args, ws):
+    """The same prefill through llama_generate with pinned host buffers:
+    host->device tokens, prefill, argmax, device->host next tokens, per step."""
+    import torch
     host_toks = torch.from_numpy(toks_h.copy()).pin_memory()
     host_out = torch.empty(PREFILL_B, dtype=torch.int32).pin_memory()
     L.llama_reset(m, st)
@@ -266,75 +247,110 @@ def run_ours(args):
     e1.record(st)
     torch.cuda.synchronize()
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, ws)
-    e2e = {'value': ws * PREFILL_B * PREFILL_S / (e2e_ms / 1e3), 'unit': 'tokens/s',
-           'h2d_bytes_per_step': PREFILL_B * PREFILL_S * 4, 'd2h_bytes_per_step': PREFILL_B * 4,
-           'api': 'llama_generate(host tokens, n_new=0)'}
+    return {'value': ws * PREFILL_B * PREFILL_S / (e2e_ms / 1e3), 'unit': 'tokens/s',
+            'h2d_bytes_per_step': PREFILL_B * PREFILL_S * 4, 'd2h_bytes_per_step': PREFILL_B * 4,
+            'api': 'llama_generate(host tokens, n_new=0)'}
 
-    # ---- batch-32 decode over a 4096-token cache
-    decode = None
-    if not args.no_decode:
-        L.llama_fill_kv_random(m, 3, DECODE_CTX, st)
-        first = torch.from_numpy(si.tokens(1, DECODE_B, 128256, start=PREFILL_B * PREFILL_S)).cuda()
-        lens = np.full(DECODE_B, DECODE_CTX, np.int32)
 
-        def decode_run(n, profile=False):
-            L.llama_set_lengths(m, lens, DECODE_B, st)
-            cur = first
-            for _ in range(n):
-                L.llama_decode_step(m, cur, DECODE_B, st)
-                L.llama_argmax(m, arg, st)
-                cur = arg
+def measure_decode(L, m, st, arg, args, ws, local, NL, hbm_peak, peak_src):
+    """Batch-32 greedy decode over a 4096-token cache: 128 graph-replayed steps,
+    then 8 eager steps with per-launch events for the breakdown."""
+    import numpy as np
+    import torch
+    import seeded_inputs as si
+    L.llama_fill_kv_random(m, 3, DECODE_CTX, st)
+    first = torch.from_numpy(si.tokens(1, DECODE_B, V_, start=PREFILL_B * PREFILL_S)).cuda()
+    lens = np.full(DECODE_B, DECODE_CTX, np.int32)
 
-        decode_run(max(args.warmup, 2))  # eager first call, then graph capture
-        torch.cuda.synchronize()
-        _barrier(ws)
+    def decode_run(n):
         L.llama_set_lengths(m, lens, DECODE_B, st)
-        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         cur = first
-        n_dec0 = L.llama_kernel_launches()
-        with ClockSampler(local) as dclk:
-            torch.cuda.synchronize()
-            d0.record(st)
-            for _ in range(DECODE_STEPS):
-                L.llama_decode_step(m, cur, DECODE_B, st)
-                L.llama_argmax(m, arg, st)
-                cur = arg
-            d1.record(st)
-            torch.cuda.synchronize()
-        dec_launches = L.llama_kernel_launches() - n_dec0
-        dms = _max_over_ranks(d0.elapsed_time(d1) / DECODE_STEPS, ws)
-        assert L.llama_sync_status(m, st) == 0
-        # profiled pass (eager, per-kernel events) for the breakdown
-        L.llama_profile(m, 1)
-        L.llama_profile_read(m)
-        decode_run(8)
-        dprof = L.llama_profile_read(m)
-        L.llama_profile(m, 0)
-        avg_ctx = DECODE_CTX + (DECODE_STEPS + 1) / 2.0
-        w_bytes = NL * 2.0 * (D * (H + 2 * Hk) * d + D * H * d + 2 * D * F + D * F) + 2.0 * 128256 * D
-        kv_bytes = NL * 2.0 * DECODE_B * avg_ctx * Hk * d * 2
-        step_bytes = w_bytes + kv_bytes
-        achieved_gbs = step_bytes / (dms / 1e3) / 1e9
-        decode = {'value': ws * DECODE_B / (dms / 1e3), 'unit': 'tokens/s', 'ms_per_step': dms,
-                  'steps': DECODE_STEPS, 'batch': DECODE_B, 'context': DECODE_CTX, 'graph_replay': True,
-                  'gpu_launches': dec_launches,
-                  'roofline': {'bound': 'hbm', 'achieved': achieved_gbs, 'peak': hbm_peak, 'unit': 'GB/s',
-                               'frac': achieved_gbs / hbm_peak, 'traffic': None,
-                               'algorithmic_bytes_per_step': step_bytes, 'peak_kind': f'hbm copy ({peak_src})'},
-                  'kernels_eager_profile': {k: {'ms_per_step': v[0] / 8, 'launches_per_step': v[1] / 8}
-                                            for k, v in dprof.items() if v[1]},
-                  'clocks': dclk.summary()}
+        for _ in range(n):
+            L.llama_decode_step(m, cur, DECODE_B, st)
+            L.llama_argmax(m, arg, st)
+            cur = arg
 
+    decode_run(max(args.warmup, 2))  # eager first call, then graph capture
+    torch.cuda.synchronize()
+    _barrier(ws)
+    L.llama_set_lengths(m, lens, DECODE_B, st)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = first
+    n0 = L.llama_kernel_launches()
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        d0.record(st)
+        for _ in range(DECODE_STEPS):
+            L.llama_decode_step(m, cur, DECODE_B, st)
+            L.llama_argmax(m, arg, st)
+            cur = arg
+        d1.record(st)
+        torch.cuda.synchronize()
+    launches = L.llama_kernel_launches() - n0
+    dms = _max_over_ranks(d0.elapsed_time(d1) / DECODE_STEPS, ws)
+    assert L.llama_sync_status(m, st) == 0
+    L.llama_profile(m, 1)
+    L.llama_profile_read(m)
+    decode_run(8)
+    dprof = L.llama_profile_read(m)
+    L.llama_profile(m, 0)
+    avg_ctx = DECODE_CTX + (DECODE_STEPS + 1) / 2.0
+    w_bytes = NL * 2.0 * (D_ * (H_ + 2 * HK_) * HD_ + D_ * H_ * HD_ + 2 * D_ * F_ + D_ * F_) + 2.0 * V_ * D_
+    kv_bytes = NL * 2.0 * DECODE_B * avg_ctx * HK_ * HD_ * 2
+    step_bytes = w_bytes + kv_bytes
+    achieved = step_bytes / (dms / 1e3) / 1e9
+    return {'value': ws * DECODE_B / (dms / 1e3), 'unit': 'tokens/s', 'ms_per_step': dms,
+            'steps': DECODE_STEPS, 'batch': DECODE_B, 'context': DECODE_CTX, 'graph_replay': True,
+            'gpu_launches': launches,
+            'roofline': {'bound': 'hbm', 'achieved': achieved, 'peak': hbm_peak, 'unit': 'GB/s',
+                         'frac': achieved / hbm_peak, 'traffic': None, 'algorithmic_bytes_per_step': step_bytes,
+                         'peak_kind': f'hbm copy ({peak_src})'},
+            'kernels_eager_profile': {k: {'ms_per_step': v[0] / 8, 'launches_per_step': v[1] / 8}
+                                      for k, v in dprof.items() if v[1]},
+            'clocks': clk.summary()}
+
+
+def run_ours(args):
+    import torch
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.init_process_group('nccl', timeout=datetime.timedelta(seconds=600), device_id=torch.device('cuda', local))
+    from llama_transformer_decoder_b200 import binding as L
+    from llama_transformer_decoder_b200.configs import LLAMA3_8B, make_config
+    import seeded_inputs as si
+    hbm_peak, tf_burst, tf_sust, peak_src = _peaks()
+
+    NL = args.layers
+    max_seq = DECODE_CTX + DECODE_STEPS + max(args.warmup, 2) + 8
+    cfg = make_config(LLAMA3_8B, dtype=L.LLAMA_BF16, max_batch=1 if args.no_decode else DECODE_B,
+                      max_seq=PREFILL_S if args.no_decode else max_seq, max_tokens=PREFILL_B * PREFILL_S,
+                      n_layers=NL)
+    st = torch.cuda.Stream()
+    m = L.llama_create(cfg)
+    L.llama_init_weights(m, 0, 0.02, st)
+    toks_h = si.tokens(1, PREFILL_B * PREFILL_S, V_).reshape(PREFILL_B, PREFILL_S)
+    toks = torch.from_numpy(toks_h).cuda()
+    arg = torch.empty(DECODE_B, dtype=torch.int32, device='cuda')
+    torch.cuda.synchronize()
+
+    ms = launches = clk = roofline = kernels = e2e = None
+    if not args.decode_only:
+        ms, launches, clk, roofline, kernels = measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust,
+                                                               peak_src)
+        e2e = measure_e2e(L, m, st, toks_h, args, ws)
+    decode = None if args.no_decode else measure_decode(L, m, st, arg, args, ws, local, NL, hbm_peak, peak_src)
     cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline and NL == 32:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline and NL == 32 and not args.decode_only:
         tok_s, dt, desc = oracle_prefill_sample()
         cpu = {'value': tok_s, 'unit': 'tokens/s', 'cores': os.cpu_count(), 'kind': 'oracle', 'sample': desc,
                'seconds': dt}
-
     L.llama_destroy(m)
     if rank == 0:
+        value = ws * PREFILL_B * PREFILL_S / (ms / 1e3) if ms else None
         line = {'metric': METRIC, 'value': value, 'unit': 'tokens/s', 'n_gpus': ws, 'steps': args.steps,
-                'warmup': args.warmup, 'ms_per_step': ms_max, 'higher_is_better': True, 'scaling': 'weak',
+                'warmup': args.warmup, 'ms_per_step': ms, 'higher_is_better': True, 'scaling': 'weak',
                 'vs_baseline': None, 'dtype': 'bf16',
                 'data': 'synthetic: seeded N(0,0.02) weights of the 8B shapes, uniform token ids',
                 'config': {'workload': 'llama3-8b-shape full-model prefill, B=1, S=2048 (32 layers + LM head '
@@ -343,7 +359,7 @@ def run_ours(args):
                            'l2': 'inputs larger than L2 (16 GB of weights streamed per step)',
                            'parallelism': f'replicas x{ws}'},
                 'roofline': roofline, 'cpu_baseline': cpu, 'e2e': e2e, 'gpu_launches': launches,
-                'clocks': clk.summary(), 'kernels': kernels, 'decode': decode}
+                'clocks': clk, 'kernels': kernels, 'decode': decode}
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist
@@ -358,6 +374,7 @@ def main():
     ap.add_argument('--warmup', type=int, default=3)
     ap.add_argument('--impl', choices=['ours', 'reference'], default='ours')
     ap.add_argument('--no-decode', action='store_true')
+    ap.add_argument('--decode-only', action='store_true', help='skip the prefill and end-to-end legs (profiling)')
     ap.add_argument('--layers', type=int, default=32, help='decoder layers (32 = the 8B model)')
     ap.add_argument('--no-cpu-baseline', action='store_true')
     args = ap.parse_args()

@@ -77,6 +77,8 @@ __global__ void __launch_bounds__(128) attn_prefill_bf16_kernel(const bf16* __re
                                                                 const bf16* __restrict__ vc, bf16* __restrict__ o,
                                                                 const int32_t* __restrict__ pos0, int S, int H,
                                                                 int Hk, int Smax, float scale_log2) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ __align__(128) uint8_t sm[];
   uint8_t* sQ = sm;
   uint8_t* sK = sm + PB_Q * 256;          // 2 buffers of 64 x 256 B
@@ -227,6 +229,7 @@ __global__ void __launch_bounds__(32) attn_prefill_f32_kernel(const float* __res
                                                               const float* __restrict__ vc, float* __restrict__ o,
                                                               const int32_t* __restrict__ pos0, int S, int H,
                                                               int Hk, int Smax, float scale_log2) {
+  pdl_wait();
   constexpr int DPL = D / 32;
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z, lane = threadIdx.x;
   const int g = h / (H / Hk);
@@ -541,6 +544,8 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
     attn_decode_mma_kernel(const bf16* __restrict__ q, const bf16* __restrict__ kc, const bf16* __restrict__ vc,
                            const int32_t* __restrict__ nkeys, int add_keys, int nmax, float* __restrict__ part, int B,
                            int H, int Hk, int Smax, float scale_log2, int* status) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ __align__(128) uint8_t sm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = H / Hk;
@@ -686,37 +691,60 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
 // Merge the pieces of every (b, h): the warps holding tiles of (b, g) are
 // owner(T0) .. owner(T1-1), owner(x) = ((x+1)W - 1) / T.
 template <typename T, int D>
-__global__ void attn_decode_combine_pieces_kernel(const float* __restrict__ part, const int32_t* __restrict__ nkeys,
-                                                  int add_keys, int nmax, T* __restrict__ o, int B, int H, int Hk,
-                                                  long long W) {
+__global__ void __launch_bounds__(128) attn_decode_combine_pieces_kernel(
+    const float* __restrict__ part, const int32_t* __restrict__ nkeys, int add_keys, int nmax, T* __restrict__ o,
+    int B, int H, int Hk, long long W) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ long long s_tot, s_t0;
+  __shared__ int s_nt, s_cnt;
+  __shared__ int s_w[256];
+  __shared__ float s_f[256];
   const int h = blockIdx.x, b = blockIdx.y;
   const int G = H / Hk, g = h / G, row = h - g * G;
-  long long total = 0, t0 = 0;
-  int nt_b = 0;
-  for (int bb = 0; bb < B; ++bb) {
-    const int nt = dm_tiles(dm_keys(nkeys, bb, add_keys, nmax));
-    if (bb == b) { t0 = total + (long long)g * nt; nt_b = nt; }
-    total += (long long)Hk * nt;
+  if (threadIdx.x == 0) {
+    long long total = 0, t0 = 0;
+    int nt_b = 0;
+    for (int bb = 0; bb < B; ++bb) {
+      const int nt = dm_tiles(dm_keys(nkeys, bb, add_keys, nmax));
+      if (bb == b) { t0 = total + (long long)g * nt; nt_b = nt; }
+      total += (long long)Hk * nt;
+    }
+    s_tot = total; s_t0 = t0; s_nt = nt_b;
   }
+  __syncthreads();
+  const long long total = s_tot, t0 = s_t0;
+  const int nt_b = s_nt;
   if (nt_b == 0 || total == 0) {
     for (int dd = threadIdx.x; dd < D; dd += blockDim.x) o[((size_t)b * H + h) * D + dd] = from_f<T>(NAN);
     return;
   }
+  // warps owning tiles of (b, g): owner(t0) .. owner(t0 + nt_b - 1), skipping warps with empty ranges
   const long long w_lo = ((t0 + 1) * W - 1) / total, w_hi = ((t0 + nt_b) * W - 1) / total;
+  if (threadIdx.x == 0) s_cnt = 0;
+  __syncthreads();
+  for (long long w = w_lo + threadIdx.x; w <= w_hi; w += blockDim.x)
+    if (total * (w + 1) / W > total * w / W) {
+      const int k = atomicAdd(&s_cnt, 1);
+      if (k < 256) s_w[k] = (int)w;
+    }
+  __syncthreads();
+  const int cnt = s_cnt < 256 ? s_cnt : 256;
   const size_t bg = (size_t)b * Hk + g;
-  float M = -INFINITY;
-  // warps whose tile range is empty (fewer tiles than warps) wrote nothing
-  auto owns = [&](long long w) { return total * (w + 1) / W > total * w / W; };
-  for (long long w = w_lo; w <= w_hi; ++w)
-    if (owns(w)) M = fmaxf(M, part[((bg + w) * G + row) * (D + 2) + D]);
+  if (threadIdx.x < 32) {  // merge weights exp2(m_w - M) per piece (order does not matter here)
+    float M = -INFINITY;
+    for (int k = threadIdx.x; k < cnt; k += 32) M = fmaxf(M, part[((bg + s_w[k]) * G + row) * (D + 2) + D]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    for (int k = threadIdx.x; k < cnt; k += 32) s_f[k] = exp2f(part[((bg + s_w[k]) * G + row) * (D + 2) + D] - M);
+  }
+  __syncthreads();
   for (int dd = threadIdx.x; dd < D; dd += blockDim.x) {
     float L = 0.f, O = 0.f;
-    for (long long w = w_lo; w <= w_hi; ++w) {
-      if (!owns(w)) continue;
-      const float* r = part + ((bg + w) * G + row) * (D + 2);
-      const float f = exp2f(r[D] - M);
-      L += r[D + 1] * f;
-      O += r[dd] * f;
+    for (int k = 0; k < cnt; ++k) {
+      const float* r = part + ((bg + s_w[k]) * G + row) * (D + 2);
+      L += r[D + 1] * s_f[k];
+      O += r[dd] * s_f[k];
     }
     o[((size_t)b * H + h) * D + dd] = from_f<T>(O / L);
   }
@@ -764,9 +792,10 @@ int attention_prefill(const void* q, const void* kc, const void* vc, void* o, co
       attr = true;
     }
     dim3 grid((S + PB_Q - 1) / PB_Q, H, B);
-    attn_prefill_bf16_kernel<<<grid, 128, SMEM, st>>>(static_cast<const bf16*>(q), static_cast<const bf16*>(kc),
-                                                      static_cast<const bf16*>(vc), static_cast<bf16*>(o), pos0, S, H,
-                                                      Hk, Smax, scale_log2);
+    if (launch_k(attn_prefill_bf16_kernel, grid, dim3(128), SMEM, st, static_cast<const bf16*>(q),
+                 static_cast<const bf16*>(kc), static_cast<const bf16*>(vc), static_cast<bf16*>(o), pos0, S, H, Hk,
+                 Smax, scale_log2) != cudaSuccess)
+      return LLAMA_ERR_CUDA;
   } else {
     dim3 grid(S, H, B);
 #define LLAMA_F32_PREFILL(DD)                                                                                  \
@@ -819,12 +848,14 @@ int attention_decode(const void* q, const void* kc, const void* vc, const int32_
     }
     const float scale_log2 = kLog2e / sqrtf((float)d);
     const int nmax = cmax < Smax ? cmax : Smax;
-    attn_decode_mma_kernel<<<grid, DM_WARPS * 32, DM_SMEM, st>>>(
-        static_cast<const bf16*>(q), static_cast<const bf16*>(kc), static_cast<const bf16*>(vc), nkeys, add_keys, nmax,
-        scratch->part, B, H, Hk, Smax, scale_log2, status);
-    attn_decode_combine_pieces_kernel<bf16, 128><<<dim3(H, B), 128, 0, st>>>(
-        scratch->part, nkeys, add_keys, nmax, static_cast<bf16*>(o), B, H, Hk, (long long)grid * DM_WARPS);
-    return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+    cudaError_t err = launch_k(attn_decode_mma_kernel, dim3(grid), dim3(DM_WARPS * 32), DM_SMEM, st,
+                               static_cast<const bf16*>(q), static_cast<const bf16*>(kc), static_cast<const bf16*>(vc),
+                               nkeys, add_keys, nmax, scratch->part, B, H, Hk, Smax, scale_log2, status);
+    if (err == cudaSuccess)
+      err = launch_k(attn_decode_combine_pieces_kernel<bf16, 128>, dim3(H, B), dim3(128), 0, st,
+                     (const float*)scratch->part, nkeys, add_keys, nmax, static_cast<bf16*>(o), B, H, Hk,
+                     (long long)grid * DM_WARPS);
+    return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
   }
   const int splits = decode_splits(cmax, B, Hk);
   if (dtype == LLAMA_BF16) {

@@ -188,6 +188,14 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 
 __device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31) == 0; }
 
+// ------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start before
+// its predecessor on the stream has finished: everything before pdl_wait()
+// must not read memory the predecessor writes. Without that launch attribute
+// both calls are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // --------------------------------------------------------------- numerics
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
 

@@ -13,6 +13,8 @@ namespace {
 template <typename T>
 __global__ void embed_kernel(const int32_t* __restrict__ tokens, const T* __restrict__ table, int V, int D,
                              float* __restrict__ x, int* status) {
+  pdl_trigger();
+  pdl_wait();
   const int m = blockIdx.x;
   const int tok = tokens[m];
   float* dst = x + (size_t)m * D;
@@ -30,6 +32,8 @@ __global__ void embed_kernel(const int32_t* __restrict__ tokens, const T* __rest
 template <typename T>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ g,
                                                       T* __restrict__ y, int D, float eps, int last_of_S) {
+  pdl_trigger();
+  pdl_wait();
   const int r = blockIdx.x;
   const size_t src_row = last_of_S > 0 ? (size_t)(r + 1) * last_of_S - 1 : (size_t)r;
   const float* xr = x + src_row * D;
@@ -74,6 +78,8 @@ __device__ __forceinline__ void better(float& bv, int& bi, float v, int i) {
 }
 
 __global__ void __launch_bounds__(1024) argmax_kernel(const float* __restrict__ logits, int32_t* out, int V) {
+  pdl_trigger();
+  pdl_wait();
   const float* row = logits + (size_t)blockIdx.x * V;
   float bv = -INFINITY;
   int bi = 0x7fffffff;
@@ -102,6 +108,8 @@ __global__ void __launch_bounds__(1024) argmax_kernel(const float* __restrict__ 
 }
 
 __global__ void add_lengths_kernel(int32_t* len, int B, int add) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) len[b] += add;
 }
@@ -214,33 +222,39 @@ uint64_t stream_key(uint64_t seed, uint64_t stream) { return mix64(seed * SG + s
 int launch_embed(const int32_t* tokens, int M, const void* table, int V, int D, int dtype, float* x, int* status,
                  cudaStream_t st) {
   if (M <= 0) return LLAMA_OK;
+  cudaError_t err;
   if (dtype == LLAMA_BF16)
-    embed_kernel<bf16><<<M, 256, 0, st>>>(tokens, static_cast<const bf16*>(table), V, D, x, status);
+    err = launch_k(embed_kernel<bf16>, dim3(M), dim3(256), 0, st, tokens, static_cast<const bf16*>(table), V, D, x,
+                   status);
   else
-    embed_kernel<float><<<M, 256, 0, st>>>(tokens, static_cast<const float*>(table), V, D, x, status);
-  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+    err = launch_k(embed_kernel<float>, dim3(M), dim3(256), 0, st, tokens, static_cast<const float*>(table), V, D, x,
+                   status);
+  return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 int launch_rmsnorm(const float* x, const float* g, void* y, int rows, int D, float eps, int last_of_S, int dtype,
                    cudaStream_t st) {
   if (rows <= 0) return LLAMA_OK;
+  cudaError_t err;
   if (dtype == LLAMA_BF16)
-    rmsnorm_kernel<bf16><<<rows, 256, 0, st>>>(x, g, static_cast<bf16*>(y), D, eps, last_of_S);
+    err = launch_k(rmsnorm_kernel<bf16>, dim3(rows), dim3(256), 0, st, x, g, static_cast<bf16*>(y), D, eps, last_of_S);
   else
-    rmsnorm_kernel<float><<<rows, 256, 0, st>>>(x, g, static_cast<float*>(y), D, eps, last_of_S);
-  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+    err = launch_k(rmsnorm_kernel<float>, dim3(rows), dim3(256), 0, st, x, g, static_cast<float*>(y), D, eps,
+                   last_of_S);
+  return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 int launch_argmax(const float* logits, int32_t* out, int B, int V, cudaStream_t st) {
   if (B <= 0) return LLAMA_OK;
-  argmax_kernel<<<B, 1024, 0, st>>>(logits, out, V);
-  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  return launch_k(argmax_kernel, dim3(B), dim3(1024), 0, st, logits, out, V) == cudaSuccess ? LLAMA_OK
+                                                                                           : LLAMA_ERR_CUDA;
 }
 
 int launch_add_lengths(int32_t* len, int B, int add, cudaStream_t st) {
   if (B <= 0) return LLAMA_OK;
-  add_lengths_kernel<<<(B + 255) / 256, 256, 0, st>>>(len, B, add);
-  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  return launch_k(add_lengths_kernel, dim3((B + 255) / 256), dim3(256), 0, st, len, B, add) == cudaSuccess
+             ? LLAMA_OK
+             : LLAMA_ERR_CUDA;
 }
 
 int launch_fill_normal(void* dst, const FillLayout& L, uint64_t seed, uint64_t stream_id, float std, int dtype,

@@ -81,19 +81,24 @@ __device__ __forceinline__ void epi_row32(const EpiArgs& e, int m, int n0, const
     float* p = e.out + (size_t)m * e.ldo + n0;
     if (full && ((e.ldo & 3) == 0) && ((reinterpret_cast<uintptr_t>(e.out) & 15) == 0)) {
       float4* p4 = reinterpret_cast<float4*>(p);
+      float4 x[8];
+      if (KIND == EPI_RESIDUAL) {  // all loads before any store: they do not wait on one another
+#pragma unroll
+        for (int j = 0; j < 8; ++j) x[j] = p4[j];
+      }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         float4 o = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-        if (KIND == EPI_RESIDUAL) {
-          const float4 x = p4[j];
-          o.x += x.x; o.y += x.y; o.z += x.z; o.w += x.w;
-        }
+        if (KIND == EPI_RESIDUAL) { o.x += x[j].x; o.y += x[j].y; o.z += x[j].z; o.w += x[j].w; }
         p4[j] = o;
       }
     } else {
-      for (int j = 0; j < 32 && n0 + j < e.N; ++j) {
-        if (KIND == EPI_RESIDUAL) p[j] += v[j];
-        else p[j] = v[j];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (n0 + j < e.N) {
+          if (KIND == EPI_RESIDUAL) p[j] += v[j];
+          else p[j] = v[j];
+        }
       }
     }
   } else if (KIND == EPI_SWIGLU) {
@@ -109,11 +114,15 @@ __device__ __forceinline__ void epi_row32(const EpiArgs& e, int m, int n0, const
       p4[0] = make_uint4(w[0], w[1], w[2], w[3]);
       p4[1] = make_uint4(w[4], w[5], w[6], w[7]);
     } else {
-      for (int j = 0; j < 16 && n0 + 2 * j + 1 < e.N; ++j) p[j] = from_f<T>(silu_f(v[2 * j]) * v[2 * j + 1]);
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (n0 + 2 * j + 1 < e.N) p[j] = from_f<T>(silu_f(v[2 * j]) * v[2 * j + 1]);
     }
   } else {  // QKV_ROPE: a 32-column chunk never straddles a head when d % 32 == 0
     if (!full || (e.d & 31) != 0 || sizeof(T) != 2) {
-      for (int j = 0; j < 32 && n0 + j < e.N; ++j) qkv_store<T>(e, m, n0 + j, v[j], v[j ^ 1]);
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (n0 + j < e.N) qkv_store<T>(e, m, n0 + j, v[j], v[j ^ 1]);
       return;
     }
     const int b = m / e.S, s = m - b * e.S;
@@ -154,6 +163,71 @@ __device__ __forceinline__ void epi_row32(const EpiArgs& e, int m, int n0, const
     uint4* p4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
     for (int j = 0; j < 4; ++j) p4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  }
+}
+
+// Column form for the swap-AB GEMM: one thread holds feature n for the 32
+// consecutive tokens [m0, m0+32); partner[j] is feature n^1 of token m0+j
+// (from the neighbouring lane). Every global load is issued before the first
+// store, so the loads overlap instead of waiting behind possibly-aliasing stores.
+template <int KIND, typename T>
+__device__ __forceinline__ void epi_col32(const EpiArgs& e, int m0, int n, const float (&v)[32],
+                                          const float (&partner)[32]) {
+  if (n >= e.N) return;
+  const int mcount = e.M - m0 < 32 ? e.M - m0 : 32;
+  if (KIND == EPI_STORE_F32) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < mcount) e.out[(size_t)(m0 + j) * e.ldo + n] = v[j];
+  } else if (KIND == EPI_RESIDUAL) {
+    float x[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) x[j] = j < mcount ? e.out[(size_t)(m0 + j) * e.ldo + n] : 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < mcount) e.out[(size_t)(m0 + j) * e.ldo + n] = x[j] + v[j];
+  } else if (KIND == EPI_SWIGLU) {
+    if ((n & 1) == 0) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < mcount) static_cast<T*>(e.g)[(size_t)(m0 + j) * e.ldg + (n >> 1)] = from_f<T>(silu_f(v[j]) * partner[j]);
+    }
+  } else {
+    const int hd = e.H * e.d;
+    const bool rot = n < hd + e.Hk * e.d;
+    const int i = (n % e.d) >> 1;
+    float2 cs[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      cs[j] = make_float2(1.f, 0.f);
+      if (rot && j < mcount) {
+        const int m = m0 + j, b = m / e.S;
+        cs[j] = e.rope[(size_t)(e.pos0[b] + m - b * e.S) * (e.d >> 1) + i];
+      }
+    }
+    int pos[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int m = m0 + j, b = m / e.S;
+      pos[j] = j < mcount ? e.pos0[b] + m - b * e.S : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (j >= mcount) continue;
+      const int m = m0 + j, b = m / e.S, s = m - b * e.S;
+      const float r = !rot ? v[j] : ((n & 1) ? (partner[j] * cs[j].y + v[j] * cs[j].x)
+                                             : (v[j] * cs[j].x - partner[j] * cs[j].y));
+      if (n < hd) {
+        const int h = n / e.d, dd = n - h * e.d;
+        static_cast<T*>(e.q)[(((size_t)b * e.H + h) * e.S + s) * e.d + dd] = from_f<T>(r);
+      } else {
+        const bool is_k = rot;
+        const int nn = n - hd - (is_k ? 0 : e.Hk * e.d);
+        const int g = nn / e.d, dd = nn - g * e.d;
+        T* dst = static_cast<T*>(is_k ? e.kc : e.vc);
+        dst[(((size_t)b * e.Hk + g) * e.Smax + pos[j]) * e.d + dd] = from_f<T>(r);
+      }
+    }
   }
 }
 

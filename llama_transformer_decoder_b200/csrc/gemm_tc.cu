@@ -11,11 +11,15 @@
 //  * gemm_skinny (M <= 256, decode and short prompts): the weight tile is the
 //    MMA's A operand (128 weight rows) and the tokens are its N side, so a
 //    decode step streams each weight byte exactly once at full MMA width.
-//    The K range is split across CTAs to put every SM on the weight stream;
-//    partial tiles go to a workspace and the last CTA of a tile (atomic
-//    ticket, no spinning) reduces them in split order and runs the epilogue.
+//    Persistent stream-K: every CTA streams an equal share of (tile, k-block)
+//    units; tiles shared by several CTAs are reduced by their last
+//    contributor (atomic ticket, no spinning) in a fixed order.
+//
+// Both are launched with programmatic dependent launch: weight tiles are
+// requested before waiting for the previous kernel, activations after.
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "epilogue.cuh"
@@ -70,6 +74,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tiles = m_tiles * n_tiles;
   const int kb = (K + BK - 1) / BK;
 
+  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < W_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&accf[a], 1); mbar_init(&acce[a], 128); }
@@ -86,12 +91,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     const uint64_t pol_a = l2_policy_evict_last(), pol_b = l2_policy_evict_last();
-    int stage = 0, issued = 0;
-    uint32_t phase = 0;
+    // The weight tiles of the first stages do not depend on the previous
+    // kernel: request them before waiting for it, their activation halves after.
+    const int pre = blockIdx.x < tiles ? (kb < W_STAGES ? kb : W_STAGES) : 0;
+    {
+      const int n0 = (blockIdx.x / m_tiles) * W_BN;
+      for (int k = 0; k < pre; ++k) {
+        mbar_arrive_expect_tx(&full[k], W_STAGE_BYTES);
+        tma_load_2d(smem + k * W_STAGE_BYTES + W_A_BYTES, &tmB, &full[k], k * BK, n0, pol_b);
+      }
+      pdl_wait();
+      const int m0 = (blockIdx.x % m_tiles) * W_BM;
+      for (int k = 0; k < pre; ++k) tma_load_2d(smem + k * W_STAGE_BYTES, &tmA, &full[k], k * BK, m0, pol_a);
+    }
+    int stage = pre % W_STAGES, issued = pre;
+    uint32_t phase = pre == W_STAGES ? 1u : 0u;
     bool ok = true;
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
       const int m0 = (t % m_tiles) * W_BM, n0 = (t / m_tiles) * W_BN;
-      for (int k = 0; k < kb; ++k) {
+      for (int k = (t == (int)blockIdx.x ? pre : 0); k < kb; ++k) {
         if (!mbar_wait(&empty[stage], phase ^ 1, status)) { ok = false; break; }
         uint8_t* sa = smem + stage * W_STAGE_BYTES;
         mbar_arrive_expect_tx(&full[stage], W_STAGE_BYTES);
@@ -133,13 +151,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(drain, 0, status);
     }
   } else if (warp >= 2) {
+    pdl_wait();  // the epilogue reads and writes memory owned by earlier kernels
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int m0 = (t % m_tiles) * W_BM, n0 = (t / m_tiles) * W_BN;
-      if (!mbar_wait(&accf[acc], acc_phase, status)) break;
+      // the whole warp leaves together so the warp-wide TMEM loads stay converged
+      if (!__all_sync(0xffffffffu, mbar_wait(&accf[acc], acc_phase, status))) break;
       tc_fence_after();
       const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + acc * W_BN;
 #pragma unroll 1
@@ -162,38 +182,59 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- skinny
+// Stream-K over (weight tile, k-block) units: of the U = tiles * kb units
+// (tile-major), CTA c of G takes [U*c/G, U*(c+1)/G), so every CTA streams the
+// same number of weight bytes to within one 16 KB block. A CTA's range falls
+// into pieces, one per tile it touches. A piece covering its whole tile runs the
+// epilogue directly; otherwise it leaves its fp32 partial in one of the CTA's
+// two scratch slots (slot 0: the piece holding the CTA's first unit, slot 1:
+// its last), and the tile's last contributor (atomic ticket, no spinning) sums
+// the contributors' partials in CTA order and runs the epilogue. Accumulators
+// are double-buffered in TMEM so the MMA runs on while a piece drains.
+template <int NT>
+struct SkinnyCfg {
+  static constexpr int B_BYTES = NT * BK * 2;
+  static constexpr int STAGE_BYTES = S_A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
+  static constexpr int TRANS_LD = S_BM + 4;                 // padded row of the transpose buffer (floats)
+  static constexpr int TRANS_BYTES = 32 * TRANS_LD * 4;      // 32 tokens x 128 features
+  static constexpr int SMEM = STAGES * STAGE_BYTES + TRANS_BYTES + 1024 + 256;
+  static constexpr uint32_t TMEM_COLS = 2 * NT <= 32 ? 32 : (2 * NT <= 64 ? 64 : (2 * NT <= 128 ? 128 : (2 * NT <= 256 ? 256 : 512)));
+};
+
+__device__ __forceinline__ long long sk_first(long long c, long long U, long long G) { return U * c / G; }
+__device__ __forceinline__ long long sk_owner(long long u, long long U, long long G) { return ((u + 1) * G - 1) / U; }
+
 template <int KIND, typename T, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, int M,
-                       int N, int K, int splits, int kb_per_split, EpiArgs epi, float* __restrict__ ws,
-                       int* __restrict__ tickets, int* status) {
-  constexpr int B_BYTES = NT * BK * 2;
-  constexpr int STAGE_BYTES = S_A_BYTES + B_BYTES;
-  constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
-  constexpr uint32_t TMEM_COLS = NT <= 32 ? 32 : (NT <= 64 ? 64 : (NT <= 128 ? 128 : 256));
+                       int N, int K, EpiArgs epi, float* __restrict__ ws, int* __restrict__ tickets, int* status) {
+  using C = SkinnyCfg<NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint64_t* empty = full + STAGES;
-  uint64_t* accf = empty + STAGES;
-  uint64_t* drain = accf + 1;
+  float* trans = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::TRANS_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* accf = empty + C::STAGES;
+  uint64_t* acce = accf + 2;
+  uint64_t* drain = acce + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * S_BM;
-  const int split = blockIdx.y;
+  const int tiles = (N + S_BM - 1) / S_BM;
   const int kb = (K + BK - 1) / BK;
-  const int k_begin = split * kb_per_split;
-  const int k_end = min(kb, k_begin + kb_per_split);
+  const long long U = (long long)tiles * kb, G = gridDim.x;
+  const long long u0 = sk_first(blockIdx.x, U, G), u1 = sk_first(blockIdx.x + 1, U, G);
 
+  pdl_trigger();
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    mbar_init(accf, 1);
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&accf[a], 1); mbar_init(&acce[a], 128); }
     mbar_init(drain, 1);
     fence_barrier_init();
   }
-  if (warp == 1) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
+  if (warp == 1) { tmem_alloc(tmem_slot, C::TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -203,126 +244,160 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
     const uint64_t pol_w = l2_policy_evict_first(), pol_x = l2_policy_evict_last();
-    int stage = 0, issued = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int k = k_begin; k < k_end; ++k) {
-      if (!mbar_wait(&empty[stage], phase ^ 1, status)) { ok = false; break; }
-      uint8_t* sa = smem + stage * STAGE_BYTES;
-      mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-      tma_load_2d(sa, &tmW, &full[stage], k * BK, n0, pol_w);
-      tma_load_2d(sa + S_A_BYTES, &tmX, &full[stage], k * BK, 0, pol_x);
-      ++issued;
-      if (++stage == STAGES) { stage = 0; phase ^= 1; }
+    // Weight blocks do not depend on the previous kernel: the first stages are
+    // requested before waiting for it, their activation halves after.
+    const int pre = (int)((u1 - u0) < C::STAGES ? (u1 - u0) : C::STAGES);
+    for (int i = 0; i < pre; ++i) {
+      const long long u = u0 + i;
+      mbar_arrive_expect_tx(&full[i], C::STAGE_BYTES);
+      tma_load_2d(smem + i * C::STAGE_BYTES, &tmW, &full[i], (int)(u % kb) * BK, (int)(u / kb) * S_BM, pol_w);
     }
-    if (!ok) drain_loads(full, stage, phase, issued, STAGES, status);
+    pdl_wait();
+    for (int i = 0; i < pre; ++i) {
+      const long long u = u0 + i;
+      tma_load_2d(smem + i * C::STAGE_BYTES + S_A_BYTES, &tmX, &full[i], (int)(u % kb) * BK, 0, pol_x);
+    }
+    int stage = pre % C::STAGES, issued = pre;
+    uint32_t phase = pre == C::STAGES ? 1u : 0u;
+    bool ok = true;
+    for (long long u = u0 + pre; u < u1; ++u) {
+      if (!mbar_wait(&empty[stage], phase ^ 1, status)) { ok = false; break; }
+      uint8_t* sa = smem + stage * C::STAGE_BYTES;
+      mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+      tma_load_2d(sa, &tmW, &full[stage], (int)(u % kb) * BK, (int)(u / kb) * S_BM, pol_w);
+      tma_load_2d(sa + S_A_BYTES, &tmX, &full[stage], (int)(u % kb) * BK, 0, pol_x);
+      ++issued;
+      if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+    }
+    if (!ok) drain_loads(full, stage, phase, issued, C::STAGES, status);
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = umma_idesc_bf16(S_BM, NT);
-    int stage = 0;
-    uint32_t phase = 0;
+    int stage = 0, buf = 0;
+    uint32_t phase = 0, acc_phase = 0;
     bool ok = true, any = false;
-    for (int k = k_begin; k < k_end; ++k) {
-      if (!mbar_wait(&full[stage], phase, status)) { ok = false; break; }
+    for (long long u = u0; u < u1 && ok;) {
+      const int klo = (int)(u % kb);
+      const int n = (int)((u1 - u) < (kb - klo) ? (u1 - u) : (kb - klo));
+      if (!mbar_wait(&acce[buf], acc_phase ^ 1, status)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t a_addr = smem_u32(smem + stage * STAGE_BYTES);
-      const uint32_t b_addr = a_addr + S_A_BYTES;
+      const uint32_t d_tmem = tmem + buf * NT;
+      for (int k = 0; k < n; ++k) {
+        if (!mbar_wait(&full[stage], phase, status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + stage * C::STAGE_BYTES);
+        const uint32_t b_addr = a_addr + S_A_BYTES;
 #pragma unroll
-      for (int kk = 0; kk < BK / 16; ++kk)
-        umma_bf16(tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), idesc,
-                  (k != k_begin) || (kk != 0));
-      umma_commit(&empty[stage]);
-      any = true;
-      if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        for (int kk = 0; kk < BK / 16; ++kk)
+          umma_bf16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), idesc,
+                    (k | kk) != 0);
+        umma_commit(&empty[stage]);
+        any = true;
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      umma_commit(&accf[buf]);
+      if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+      u += n;
     }
-    if (ok) {
-      umma_commit(accf);
-    } else if (any) {
+    if (!ok && any) {
       umma_commit(drain);
       mbar_wait(drain, 0, status);
     }
   } else if (warp >= 2) {
-    const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;  // weight row within the tile
-    const int n = n0 + row;
-    const bool have = k_end > k_begin;
-    bool ok = true;
-    if (have) {
-      ok = mbar_wait(accf, 0, status);
+    pdl_wait();  // the epilogue reads and writes memory owned by earlier kernels
+    // TMEM hands each thread one weight row (feature) across 32 tokens; the
+    // tile is turned around in shared memory so that thread (token = lane,
+    // 32-feature chunk = ew) runs the same row epilogue as the wide GEMM.
+    const int quarter = warp & 3;          // TMEM lanes this warp may read
+    const int ew = warp - 2;               // feature chunk in the row phase
+    int buf = 0;
+    uint32_t acc_phase = 0;
+    for (long long u = u0; u < u1;) {
+      const int tile = (int)(u / kb), klo = (int)(u % kb);
+      const int n = (int)((u1 - u) < (kb - klo) ? (u1 - u) : (kb - klo));
+      const bool whole = klo == 0 && n == kb;
+      const int slot = (u == u0) ? 0 : 1;
+      const int f0 = tile * S_BM + ew * 32;
+      // all lanes of a warp take the same branch so the warp-wide TMEM loads stay converged
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], acc_phase, status));
       tc_fence_after();
-    }
-    const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16);
-    if (splits == 1) {
+      const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + buf * NT;
 #pragma unroll 1
       for (int c = 0; c < NT / 32; ++c) {
         float v[32];
-        if (have && ok) tmem_ld32(base + c * 32, v);
+        if (ok) tmem_ld32(base + c * 32, v);
         else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = 0.f;
         }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float partner = __shfl_xor_sync(0xffffffffu, v[j], 1);
-          if (ok) epi_elem<KIND, T>(epi, c * 32 + j, n, v[j], partner);
+        if (c == NT / 32 - 1) {  // TMEM no longer needed: the MMA may refill this buffer
+          tc_fence_before();
+          mbar_arrive(&acce[buf]);
         }
-      }
-    } else {
-      // 1) publish this split's partial tile [128 rows x NT tokens]
-      float* mine = ws + ((size_t)split * N + n) * NT;
-#pragma unroll 1
-      for (int c = 0; c < NT / 32; ++c) {
-        float v[32];
-        if (have && ok) tmem_ld32(base + c * 32, v);
-        else {
+        named_bar_sync(1, 128);  // earlier readers of the transpose buffer are done
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        for (int j = 0; j < 32; ++j) trans[j * C::TRANS_LD + quarter * 32 + lane] = v[j];
+        named_bar_sync(1, 128);
+        const float4* src = reinterpret_cast<const float4*>(trans + lane * C::TRANS_LD + ew * 32);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 x = src[j];
+          v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
         }
-        if (n < N) {
-          float4* p4 = reinterpret_cast<float4*>(mine + c * 32);
+        const int m = c * 32 + lane;
+        if (whole) {
+          epi_row32<KIND, T>(epi, m, f0, v);
+        } else {  // token-major partial: [slot][token][128 features]
+          float4* p4 = reinterpret_cast<float4*>(ws + (((size_t)blockIdx.x * 2 + slot) * NT + m) * S_BM + ew * 32);
 #pragma unroll
           for (int j = 0; j < 8; ++j) __stcg(p4 + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
         }
       }
-      __threadfence();
-      named_bar_sync(1, 128);
-      if (threadIdx.x == 64) {
-        const int prev = atomicAdd(&tickets[blockIdx.x], 1);
-        *last_flag = (prev == splits - 1);
-      }
-      named_bar_sync(1, 128);
-      // 2) the last CTA to finish sums the partials in split order
-      if (*last_flag) {
+      if (!whole) {
         __threadfence();
+        named_bar_sync(1, 128);
+        const long long t0 = (long long)tile * kb;
+        const long long c_lo = sk_owner(t0, U, G), c_hi = sk_owner(t0 + kb - 1, U, G);
+        if (threadIdx.x == 64) {
+          int contributors = 0;
+          for (long long c = c_lo; c <= c_hi; ++c) contributors += sk_first(c + 1, U, G) > sk_first(c, U, G);
+          const int prev = atomicAdd(&tickets[tile], 1);
+          *last_flag = (prev == contributors - 1);
+        }
+        named_bar_sync(1, 128);
+        if (*last_flag) {  // the tile's last contributor: sum the partials in CTA order
+          __threadfence();
 #pragma unroll 1
-        for (int c = 0; c < NT / 32; ++c) {
-          float v[32];
+          for (int c = 0; c < NT / 32; ++c) {
+            const int m = c * 32 + lane;
+            float v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0.f;
-          if (n < N) {
-            for (int s = 0; s < splits; ++s) {
-              const float4* p4 = reinterpret_cast<const float4*>(ws + ((size_t)s * N + n) * NT + c * 32);
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+            for (long long cc = c_lo; cc <= c_hi; ++cc) {
+              const long long first_unit = sk_first(cc, U, G);
+              if (sk_first(cc + 1, U, G) <= first_unit) continue;   // no units
+              const int sl = first_unit >= t0 ? 0 : 1;              // the tile holds its first unit?
+              const float4* p4 = reinterpret_cast<const float4*>(ws + ((cc * 2 + sl) * NT + m) * S_BM + ew * 32);
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
                 const float4 x = __ldcg(p4 + j);
                 v[4 * j] += x.x; v[4 * j + 1] += x.y; v[4 * j + 2] += x.z; v[4 * j + 3] += x.w;
               }
             }
+            epi_row32<KIND, T>(epi, m, f0, v);
           }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float partner = __shfl_xor_sync(0xffffffffu, v[j], 1);
-            if (ok) epi_elem<KIND, T>(epi, c * 32 + j, n, v[j], partner);
-          }
+          if (threadIdx.x == 64) tickets[tile] = 0;
         }
-        if (threadIdx.x == 64) tickets[blockIdx.x] = 0;
       }
+      if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+      u += n;
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -381,62 +456,49 @@ static int launch_wide(const CUtensorMap& ta, const CUtensorMap& tb, int M, int 
   }
   const int tiles = ((M + W_BM - 1) / W_BM) * ((N + W_BN - 1) / W_BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  kern<<<grid, kThreads, W_SMEM, st>>>(ta, tb, M, N, K, e, status);
-  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  const cudaError_t err = launch_k(kern, dim3(grid), dim3(kThreads), W_SMEM, st, ta, tb, M, N, K, e, status);
+  return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 template <int KIND, int NT>
-static int launch_skinny_nt(const CUtensorMap& tw, const CUtensorMap& tx, int M, int N, int K, int splits, int kbps,
-                            const EpiArgs& e, float* ws, int* tickets, int* status, cudaStream_t st) {
-  constexpr int B_BYTES = NT * BK * 2;
-  constexpr int STAGE_BYTES = S_A_BYTES + B_BYTES;
-  constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
-  constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+static int launch_skinny_nt(const CUtensorMap& tw, const CUtensorMap& tx, int M, int N, int K, const EpiArgs& e,
+                            float* ws, int* tickets, int* status, cudaStream_t st) {
+  using C = SkinnyCfg<NT>;
   auto kern = gemm_skinny_kernel<KIND, bf16, NT>;
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
       return LLAMA_ERR_CUDA;
     attr = true;
   }
-  dim3 grid((N + S_BM - 1) / S_BM, splits);
-  kern<<<grid, kThreads, SMEM, st>>>(tw, tx, M, N, K, splits, kbps, e, ws, tickets, status);
-  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  const cudaError_t err = launch_k(kern, dim3(num_sms()), dim3(kThreads), C::SMEM, st, tw, tx, M, N, K, e, ws,
+                                   tickets, status);
+  return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 template <int KIND>
-static int launch_skinny(const CUtensorMap& tw, const CUtensorMap& tx, int M, int N, int K, int NT, int splits,
-                         int kbps, const EpiArgs& e, float* ws, int* tickets, int* status, cudaStream_t st) {
+static int launch_skinny(const CUtensorMap& tw, const CUtensorMap& tx, int M, int N, int K, int NT, const EpiArgs& e,
+                         float* ws, int* tickets, int* status, cudaStream_t st) {
   switch (NT) {
-    case 32: return launch_skinny_nt<KIND, 32>(tw, tx, M, N, K, splits, kbps, e, ws, tickets, status, st);
-    case 64: return launch_skinny_nt<KIND, 64>(tw, tx, M, N, K, splits, kbps, e, ws, tickets, status, st);
-    case 128: return launch_skinny_nt<KIND, 128>(tw, tx, M, N, K, splits, kbps, e, ws, tickets, status, st);
-    case 256: return launch_skinny_nt<KIND, 256>(tw, tx, M, N, K, splits, kbps, e, ws, tickets, status, st);
+    case 32: return launch_skinny_nt<KIND, 32>(tw, tx, M, N, K, e, ws, tickets, status, st);
+    case 64: return launch_skinny_nt<KIND, 64>(tw, tx, M, N, K, e, ws, tickets, status, st);
+    case 128: return launch_skinny_nt<KIND, 128>(tw, tx, M, N, K, e, ws, tickets, status, st);
+    case 256: return launch_skinny_nt<KIND, 256>(tw, tx, M, N, K, e, ws, tickets, status, st);
   }
   return LLAMA_ERR_INVALID_ARG;
 }
 
-// Split count that puts about one CTA on every SM without making a split
-// shorter than 4 K-blocks.
-void skinny_plan(int M, int N, int K, int* NT, int* splits, int* kbps) {
+static int skinny_nt(int M) {
   int nt = 32;
   while (nt < M) nt *= 2;
-  *NT = nt;
-  const int tiles = (N + S_BM - 1) / S_BM;
-  const int kb = (K + BK - 1) / BK;
-  int s = num_sms() / tiles;
-  if (s < 1) s = 1;
-  if (s > kb / 4) s = kb / 4 > 0 ? kb / 4 : 1;
-  int per = (kb + s - 1) / s;
-  s = (kb + per - 1) / per;  // no empty split
-  *splits = s;
-  *kbps = per;
+  return nt;
 }
 
-size_t skinny_workspace_floats(int M, int N, int K) {
-  int nt, s, per;
-  skinny_plan(M, N, K, &nt, &s, &per);
-  return s > 1 ? (size_t)s * N * nt : 0;
+size_t skinny_workspace_floats(int M) { return (size_t)num_sms() * 2 * S_BM * skinny_nt(M); }
+
+bool pdl_enabled() {
+  static const bool on = getenv("LLAMA_NO_PDL") == nullptr;
+  return on;
 }
 
 int gemm_bf16(const bf16* A, int M, int K, int lda, const bf16* W, int N, int ldw, int kind, const EpiArgs& e,
@@ -458,24 +520,21 @@ int gemm_bf16(const bf16* A, int M, int K, int lda, const bf16* W, int N, int ld
     return LLAMA_ERR_INVALID_ARG;
   }
   if (M > 256) return LLAMA_ERR_SHAPE;
-  int NT, splits, kbps;
-  skinny_plan(M, N, K, &NT, &splits, &kbps);
-  if (splits > 1) {
-    const size_t need = (size_t)splits * N * NT;
-    const int tiles = (N + S_BM - 1) / S_BM;
-    if (!scratch || !scratch->ws || scratch->ws_floats < need || !scratch->tickets || scratch->n_tickets < tiles)
-      return LLAMA_ERR_INVALID_ARG;
-  }
+  const int NT = skinny_nt(M);
+  const int tiles = (N + S_BM - 1) / S_BM;
+  if (!scratch || !scratch->ws || scratch->ws_floats < skinny_workspace_floats(M) || !scratch->tickets ||
+      scratch->n_tickets < tiles)
+    return LLAMA_ERR_INVALID_ARG;
   CUtensorMap tw, tx;
   if ((rc = make_tmap_bf16(&tw, W, N, K, ldw, S_BM)) != LLAMA_OK) return rc;
   if ((rc = make_tmap_bf16(&tx, A, M, K, lda, NT)) != LLAMA_OK) return rc;
-  float* ws = scratch ? scratch->ws : nullptr;
-  int* tk = scratch ? scratch->tickets : nullptr;
+  float* ws = scratch->ws;
+  int* tk = scratch->tickets;
   switch (kind) {
-    case EPI_STORE_F32: return launch_skinny<EPI_STORE_F32>(tw, tx, M, N, K, NT, splits, kbps, e, ws, tk, status, st);
-    case EPI_RESIDUAL: return launch_skinny<EPI_RESIDUAL>(tw, tx, M, N, K, NT, splits, kbps, e, ws, tk, status, st);
-    case EPI_SWIGLU: return launch_skinny<EPI_SWIGLU>(tw, tx, M, N, K, NT, splits, kbps, e, ws, tk, status, st);
-    case EPI_QKV_ROPE: return launch_skinny<EPI_QKV_ROPE>(tw, tx, M, N, K, NT, splits, kbps, e, ws, tk, status, st);
+    case EPI_STORE_F32: return launch_skinny<EPI_STORE_F32>(tw, tx, M, N, K, NT, e, ws, tk, status, st);
+    case EPI_RESIDUAL: return launch_skinny<EPI_RESIDUAL>(tw, tx, M, N, K, NT, e, ws, tk, status, st);
+    case EPI_SWIGLU: return launch_skinny<EPI_SWIGLU>(tw, tx, M, N, K, NT, e, ws, tk, status, st);
+    case EPI_QKV_ROPE: return launch_skinny<EPI_QKV_ROPE>(tw, tx, M, N, K, NT, e, ws, tk, status, st);
   }
   return LLAMA_ERR_INVALID_ARG;
 }

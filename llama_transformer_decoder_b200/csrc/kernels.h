@@ -11,6 +11,25 @@ namespace llama {
 
 struct EpiArgs;
 
+// Launch with programmatic stream serialization (the kernel must call
+// pdl_wait() before reading its predecessor's output). Disabled when the
+// environment variable LLAMA_NO_PDL is set.
+bool pdl_enabled();
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 enum GemmVariant { GEMM_AUTO = 0, GEMM_WIDE = 1, GEMM_SKINNY = 2 };
 
 // Split-K scratch of the skinny GEMM: partial tiles plus one ticket per
@@ -24,8 +43,8 @@ struct GemmScratch {
 
 int num_sms();
 int make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t pitch, int box_rows);
-void skinny_plan(int M, int N, int K, int* NT, int* splits, int* kbps);
-size_t skinny_workspace_floats(int M, int N, int K);
+// Scratch of the stream-K skinny GEMM for M rows: two partial tiles per CTA.
+size_t skinny_workspace_floats(int M);
 
 int gemm_bf16(const __nv_bfloat16* A, int M, int K, int lda, const __nv_bfloat16* W, int N, int ldw, int kind,
               const EpiArgs& e, int variant, GemmScratch* scratch, int* status, cudaStream_t st);

@@ -478,7 +478,7 @@ int llama_create(const llama_config* cfg, llama_model** out) {
     int tickets = 0;
     const int shapes[5][2] = {{m->qkv_n, c.dim}, {c.dim, (int)Hd}, {2 * m->F, c.dim}, {c.dim, m->F}, {c.vocab_size, c.dim}};
     for (auto& sh : shapes) {
-      for (int M = 1; M <= std::min(128, m->Mmax); ++M) ws = std::max(ws, skinny_workspace_floats(M, sh[0], sh[1]));
+      ws = std::max(ws, skinny_workspace_floats(std::min(128, m->Mmax)));
       tickets = std::max(tickets, (sh[0] + 127) / 128);
     }
     if (grow_gemm_scratch(&m->gs, std::max<size_t>(ws, 1), tickets) != LLAMA_OK) { delete m; return LLAMA_ERR_OOM; }
@@ -823,7 +823,7 @@ int llama_linear(const void* x, const void* w, float* y, int32_t M, int32_t N, i
   const bool skinny = variant == GEMM_SKINNY || (variant == GEMM_AUTO && M <= 128);
   if (skinny) {
     if (M > 256) return LLAMA_ERR_SHAPE;
-    RC(grow_gemm_scratch(&c->gs, std::max<size_t>(skinny_workspace_floats(M, N, K), 1), (N + 127) / 128));
+    RC(grow_gemm_scratch(&c->gs, skinny_workspace_floats(M), (N + 127) / 128));
   }
   return gemm_bf16(static_cast<const bf16*>(x), M, K, K, static_cast<const bf16*>(w), N, K, EPI_STORE_F32, e,
                    variant, &c->gs, c->status, S_(stream));
