@@ -152,8 +152,8 @@ int llama_reset(llama_model* m, void* stream);
 int llama_profile(llama_model* m, int enable);
 int llama_profile_read(llama_model* m, double* ms, int64_t* launches, int n_kinds);
 const char* llama_profile_kind_name(int kind);
-/* Kernels launched by the model entry points in this process so far (graph replays count
- * their kernels). */
+/* Kernels launched by this library in this process so far (CUDA-graph replays count the
+ * kernels they contain). */
 uint64_t llama_kernel_launches(void);
 
 /* Synchronizes `stream`, then returns and clears the model's latched device status. */

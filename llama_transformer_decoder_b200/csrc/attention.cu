@@ -766,6 +766,7 @@ int decode_launch(const void* q, const void* kc, const void* vc, const int32_t* 
   int chunk = (cmax + splits - 1) / splits;
   chunk = (chunk + 127) / 128 * 128;
   const float scale_log2 = kLog2e / sqrtf((float)D);
+  count_launches(2);
   kern<<<dim3(splits, Hk, B), 128, SMEM, st>>>(static_cast<const T*>(q), static_cast<const T*>(kc),
                                                static_cast<const T*>(vc), nkeys, add_keys, part, H, Hk, Smax, chunk,
                                                scale_log2, status);
@@ -798,6 +799,7 @@ int attention_prefill(const void* q, const void* kc, const void* vc, void* o, co
       return LLAMA_ERR_CUDA;
   } else {
     dim3 grid(S, H, B);
+    count_launches(1);
 #define LLAMA_F32_PREFILL(DD)                                                                                  \
   attn_prefill_f32_kernel<DD><<<grid, 32, 0, st>>>(static_cast<const float*>(q), static_cast<const float*>(kc), \
                                                    static_cast<const float*>(vc), static_cast<float*>(o), pos0, S, \

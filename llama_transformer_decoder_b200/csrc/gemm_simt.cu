@@ -51,6 +51,7 @@ int gemm_f32(const float* A, int M, int K, int lda, const float* W, int N, int l
   (void)status;
   if (M <= 0 || N <= 0 || K <= 0) return LLAMA_ERR_SHAPE;
   dim3 grid((N + TN - 1) / TN, (M + TM - 1) / TM);
+  count_launches(1);
   switch (kind) {
     case EPI_STORE_F32: gemm_f32_kernel<EPI_STORE_F32><<<grid, 256, 0, st>>>(A, M, K, lda, W, N, ldw, e); break;
     case EPI_RESIDUAL: gemm_f32_kernel<EPI_RESIDUAL><<<grid, 256, 0, st>>>(A, M, K, lda, W, N, ldw, e); break;

@@ -12,8 +12,9 @@
 //    MMA's A operand (128 weight rows) and the tokens are its N side, so a
 //    decode step streams each weight byte exactly once at full MMA width.
 //    Persistent stream-K: every CTA streams an equal share of (tile, k-block)
-//    units; tiles shared by several CTAs are reduced by their last
-//    contributor (atomic ticket, no spinning) in a fixed order.
+//    units. Tiles shared by several CTAs are reduced by their last
+//    contributor (atomic ticket, no spinning) in a fixed order, except for
+//    the residual epilogue, where each contributor adds into x atomically.
 //
 // Both are launched with programmatic dependent launch: weight tiles are
 // requested before waiting for the previous kernel, activations after.
@@ -208,7 +209,8 @@ __device__ __forceinline__ long long sk_owner(long long u, long long U, long lon
 template <int KIND, typename T, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, int M,
-                       int N, int K, EpiArgs epi, float* __restrict__ ws, int* __restrict__ tickets, int* status) {
+                       int N, int K, EpiArgs epi, float* __restrict__ ws, int* __restrict__ tickets,
+                       float* __restrict__ stg, int* status) {
   using C = SkinnyCfg<NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -345,15 +347,45 @@ __global__ void __launch_bounds__(kThreads, 1)
           v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
         }
         const int m = c * 32 + lane;
-        if (whole) {
+        if (KIND == EPI_QKV_ROPE || KIND == EPI_SWIGLU) {
+          // nonlinear epilogues: accumulate into the zeroed fp32 staging
+          // buffer; skinny_finalize_kernel applies the epilogue afterwards
+          if (m < epi.M) {
+            float* dst = stg + (size_t)m * epi.N + f0;
+            if (f0 + 32 <= epi.N && (epi.N & 3) == 0) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                atomicAdd(reinterpret_cast<float4*>(dst) + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (f0 + j < epi.N) atomicAdd(dst + j, v[j]);
+            }
+          }
+        } else if (whole) {
           epi_row32<KIND, T>(epi, m, f0, v);
+        } else if (KIND == EPI_RESIDUAL) {
+          // x += sum of partials is linear: every contributor adds its share
+          // straight into the fp32 residual (summation order is not fixed)
+          if (m < epi.M) {
+            float* dst = epi.out + (size_t)m * epi.ldo + f0;
+            if (f0 + 32 <= epi.N && (epi.ldo & 3) == 0) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                atomicAdd(reinterpret_cast<float4*>(dst) + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (f0 + j < epi.N) atomicAdd(dst + j, v[j]);
+            }
+          }
         } else {  // token-major partial: [slot][token][128 features]
           float4* p4 = reinterpret_cast<float4*>(ws + (((size_t)blockIdx.x * 2 + slot) * NT + m) * S_BM + ew * 32);
 #pragma unroll
           for (int j = 0; j < 8; ++j) __stcg(p4 + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
         }
       }
-      if (!whole) {
+      if (!whole && KIND == EPI_STORE_F32) {
         __threadfence();
         named_bar_sync(1, 128);
         const long long t0 = (long long)tile * kb;
@@ -399,6 +431,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+}
+
+// Apply the QKV/RoPE or SwiGLU epilogue to the summed fp32 staging rows
+// [M][N] left by the skinny GEMM, one (token, 32-feature chunk) per thread,
+// and zero the staging rows for the next GEMM.
+template <int KIND, typename T>
+__global__ void __launch_bounds__(128) skinny_finalize_kernel(EpiArgs epi, float* __restrict__ stg) {
+  pdl_trigger();
+  pdl_wait();
+  const int chunks = (epi.N + 31) / 32;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= epi.M * chunks) return;
+  const int m = idx / chunks, n0 = (idx - m * chunks) * 32;
+  float* src = stg + (size_t)m * epi.N + n0;
+  float v[32];
+  if (n0 + 32 <= epi.N && (epi.N & 3) == 0) {
+    float4* p4 = reinterpret_cast<float4*>(src);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 x = __ldcg(p4 + j);
+      v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) __stcg(p4 + j, make_float4(0.f, 0.f, 0.f, 0.f));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      v[j] = n0 + j < epi.N ? __ldcg(src + j) : 0.f;
+      if (n0 + j < epi.N) src[j] = 0.f;
+    }
+  }
+  epi_row32<KIND, T>(epi, m, n0, v);
 }
 
 // -------------------------------------------------------------- host side
@@ -462,7 +526,7 @@ static int launch_wide(const CUtensorMap& ta, const CUtensorMap& tb, int M, int 
 
 template <int KIND, int NT>
 static int launch_skinny_nt(const CUtensorMap& tw, const CUtensorMap& tx, int M, int N, int K, const EpiArgs& e,
-                            float* ws, int* tickets, int* status, cudaStream_t st) {
+                            float* ws, int* tickets, float* stg, int* status, cudaStream_t st) {
   using C = SkinnyCfg<NT>;
   auto kern = gemm_skinny_kernel<KIND, bf16, NT>;
   static bool attr = false;
@@ -471,19 +535,23 @@ static int launch_skinny_nt(const CUtensorMap& tw, const CUtensorMap& tx, int M,
       return LLAMA_ERR_CUDA;
     attr = true;
   }
-  const cudaError_t err = launch_k(kern, dim3(num_sms()), dim3(kThreads), C::SMEM, st, tw, tx, M, N, K, e, ws,
-                                   tickets, status);
+  cudaError_t err = launch_k(kern, dim3(num_sms()), dim3(kThreads), C::SMEM, st, tw, tx, M, N, K, e, ws, tickets,
+                             stg, status);
+  if (err == cudaSuccess && (KIND == EPI_QKV_ROPE || KIND == EPI_SWIGLU)) {
+    const int items = M * ((N + 31) / 32);
+    err = launch_k(skinny_finalize_kernel<KIND, bf16>, dim3((items + 127) / 128), dim3(128), 0, st, e, stg);
+  }
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 template <int KIND>
 static int launch_skinny(const CUtensorMap& tw, const CUtensorMap& tx, int M, int N, int K, int NT, const EpiArgs& e,
-                         float* ws, int* tickets, int* status, cudaStream_t st) {
+                         float* ws, int* tickets, float* stg, int* status, cudaStream_t st) {
   switch (NT) {
-    case 32: return launch_skinny_nt<KIND, 32>(tw, tx, M, N, K, e, ws, tickets, status, st);
-    case 64: return launch_skinny_nt<KIND, 64>(tw, tx, M, N, K, e, ws, tickets, status, st);
-    case 128: return launch_skinny_nt<KIND, 128>(tw, tx, M, N, K, e, ws, tickets, status, st);
-    case 256: return launch_skinny_nt<KIND, 256>(tw, tx, M, N, K, e, ws, tickets, status, st);
+    case 32: return launch_skinny_nt<KIND, 32>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
+    case 64: return launch_skinny_nt<KIND, 64>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
+    case 128: return launch_skinny_nt<KIND, 128>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
+    case 256: return launch_skinny_nt<KIND, 256>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
   }
   return LLAMA_ERR_INVALID_ARG;
 }
@@ -525,16 +593,18 @@ int gemm_bf16(const bf16* A, int M, int K, int lda, const bf16* W, int N, int ld
   if (!scratch || !scratch->ws || scratch->ws_floats < skinny_workspace_floats(M) || !scratch->tickets ||
       scratch->n_tickets < tiles)
     return LLAMA_ERR_INVALID_ARG;
+  if ((kind == EPI_QKV_ROPE || kind == EPI_SWIGLU) && (!scratch->stg || scratch->stg_floats < (size_t)M * N))
+    return LLAMA_ERR_INVALID_ARG;
   CUtensorMap tw, tx;
   if ((rc = make_tmap_bf16(&tw, W, N, K, ldw, S_BM)) != LLAMA_OK) return rc;
   if ((rc = make_tmap_bf16(&tx, A, M, K, lda, NT)) != LLAMA_OK) return rc;
   float* ws = scratch->ws;
   int* tk = scratch->tickets;
   switch (kind) {
-    case EPI_STORE_F32: return launch_skinny<EPI_STORE_F32>(tw, tx, M, N, K, NT, e, ws, tk, status, st);
-    case EPI_RESIDUAL: return launch_skinny<EPI_RESIDUAL>(tw, tx, M, N, K, NT, e, ws, tk, status, st);
-    case EPI_SWIGLU: return launch_skinny<EPI_SWIGLU>(tw, tx, M, N, K, NT, e, ws, tk, status, st);
-    case EPI_QKV_ROPE: return launch_skinny<EPI_QKV_ROPE>(tw, tx, M, N, K, NT, e, ws, tk, status, st);
+    case EPI_STORE_F32: return launch_skinny<EPI_STORE_F32>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
+    case EPI_RESIDUAL: return launch_skinny<EPI_RESIDUAL>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
+    case EPI_SWIGLU: return launch_skinny<EPI_SWIGLU>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
+    case EPI_QKV_ROPE: return launch_skinny<EPI_QKV_ROPE>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
   }
   return LLAMA_ERR_INVALID_ARG;
 }

@@ -15,6 +15,8 @@ struct EpiArgs;
 // pdl_wait() before reading its predecessor's output). Disabled when the
 // environment variable LLAMA_NO_PDL is set.
 bool pdl_enabled();
+// Process-wide count of kernel launches made by the library.
+void count_launches(unsigned long long n);
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
@@ -27,18 +29,22 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  count_launches(1);
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
 enum GemmVariant { GEMM_AUTO = 0, GEMM_WIDE = 1, GEMM_SKINNY = 2 };
 
-// Split-K scratch of the skinny GEMM: partial tiles plus one ticket per
-// 128-row weight tile (tickets must start at zero; the kernel leaves them zero).
+// Scratch of the skinny GEMM: partial tiles, one ticket per 128-row weight
+// tile and the staging rows (tickets and staging must start at zero; the
+// kernels leave them zero).
 struct GemmScratch {
   float* ws;
   size_t ws_floats;
   int* tickets;
   int n_tickets;
+  float* stg;          // zeroed fp32 [M][N] staging for the QKV/RoPE and SwiGLU epilogues (kept zero)
+  size_t stg_floats;
 };
 
 int num_sms();

@@ -256,8 +256,7 @@ const char* kProfNames[K_COUNT] = {"embed", "rmsnorm", "gemm_qkv_rope", "attenti
                                    "other", "end"};
 std::atomic<unsigned long long> g_launches{0};
 
-void mark(llama_model* m, int kind, cudaStream_t st, int kernels = 1) {
-  g_launches += kernels;
+void mark(llama_model* m, int kind, cudaStream_t st) {
   if (!m->prof_on) return;
   if (m->prof_used == m->prof_pool.size()) {
     cudaEvent_t e;
@@ -314,7 +313,7 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
   mark(m, K_GEMM_QKV, st);
   RC(gemm(m, m->xn, M, D, w.wqkv, m->qkv_n, EPI_QKV_ROPE, e, st));
   if (decode) {
-    mark(m, K_ATTN_DECODE, st, 2);
+    mark(m, K_ATTN_DECODE, st);
     RC(attention_decode(m->q, kc, vc, m->d_len, 1, m->attn, B, cmax, H, Hk, d, c.max_seq, c.dtype, &m->ds,
                         m->d_status, st));
   } else {
@@ -370,6 +369,8 @@ int check_lengths(llama_model* m, int B, int S) {
 }
 
 }  // namespace
+
+void llama::count_launches(unsigned long long n) { g_launches += n; }
 
 // ======================================================================= ABI
 extern "C" {
@@ -484,6 +485,12 @@ int llama_create(const llama_config* cfg, llama_model** out) {
     if (grow_gemm_scratch(&m->gs, std::max<size_t>(ws, 1), tickets) != LLAMA_OK) { delete m; return LLAMA_ERR_OOM; }
     m->allocs.push_back(m->gs.ws);
     m->allocs.push_back(m->gs.tickets);
+    // staging rows for the skinny QKV / SwiGLU epilogues (M <= 128 rows)
+    const size_t stg = (size_t)std::min(128, m->Mmax) * std::max(m->qkv_n, 2 * m->F);
+    m->gs.stg = static_cast<float*>(m->alloc(stg * sizeof(float)));
+    if (!m->gs.stg) { delete m; return LLAMA_ERR_OOM; }
+    cudaMemset(m->gs.stg, 0, stg * sizeof(float));
+    m->gs.stg_floats = stg;
   }
   {
     size_t need = 0;
