@@ -19,7 +19,8 @@ INCLUDE = os.path.join(ROOT, 'include')
 LIB = os.path.join(HERE, 'libllama_b200.so')
 OBJDIR = os.path.join(ROOT, '_build', 'obj')
 
-SOURCES = ['gemm_tc.cu', 'gemm_simt.cu', 'elementwise.cu', 'attention.cu', 'model.cu', 'noalloc.cu']
+SOURCES = ['gemm_tc.cu', 'gemm_simt.cu', 'elementwise.cu', 'attention.cu', 'attention_tc.cu', 'model.cu',
+           'noalloc.cu']
 ARCH = ['-gencode', 'arch=compute_100a,code=sm_100a']
 FLAGS = ['-O3', '-lineinfo', '-std=c++17', '-Xcompiler', '-fPIC', '-I' + INCLUDE]
 

@@ -1,18 +1,14 @@
 // Causal grouped-query attention over the KV cache.
 //
-//  * prefill (bf16): flash-style, one CTA per (64-query tile, q head, batch).
-//    K/V tiles of 64 keys are double-buffered in shared memory with cp.async,
-//    S = Q K^T and O += P V run on the tensor cores (mma.sync m16n8k16, bf16 in,
-//    fp32 accumulate), and the softmax is online in registers with quad
-//    shuffles. P is rounded to bf16 for the PV product, as the walkthrough does
-//    (softmax(...).to(bfloat16)). Query i at absolute position pos0+i sees keys
-//    0 .. pos0+i.
+//  * prefill (bf16): the tcgen05 flash-attention kernel in attention_tc.cu.
 //  * prefill (fp32): one warp per query row on the CUDA cores.
 //  * decode (both dtypes): split over the cached keys. Each CTA serves the
 //    H/Hk query heads of one kv head, streams its key range through shared
 //    memory with bulk async copies (the step is bound by HBM reads of the
 //    cache), keeps (max, sum, o) per head, and a combine kernel merges the
 //    splits with the log-sum-exp rule.
+#include <cstdlib>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -22,8 +18,7 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// ------------------------------------------------------ bf16 prefill (mma)
-constexpr int PB_Q = 64, PB_K = 64, PB_D = 128;
+// ------------------------------------------------------ mma.sync helpers (decode)
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
   const int n = valid ? 16 : 0;
@@ -59,167 +54,6 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
-}
-
-// Copy rows [row0, row0+64) of a [rows][128] bf16 matrix into a swizzled tile;
-// rows >= nrows are zero filled.
-__device__ __forceinline__ void load_tile(uint8_t* tile, const bf16* src, int row0, int nrows) {
-  for (int i = threadIdx.x; i < 64 * 16; i += 128) {
-    const int r = i >> 4, c = i & 15;
-    const int gr = row0 + r;
-    const bool ok = gr < nrows;
-    cp_async16(tile + swz(r, c), src + (size_t)(ok ? gr : 0) * PB_D + c * 8, ok);
-  }
-}
-
-__global__ void __launch_bounds__(128) attn_prefill_bf16_kernel(const bf16* __restrict__ q,
-                                                                const bf16* __restrict__ kc,
-                                                                const bf16* __restrict__ vc, bf16* __restrict__ o,
-                                                                const int32_t* __restrict__ pos0, int S, int H,
-                                                                int Hk, int Smax, float scale_log2) {
-  pdl_trigger();
-  pdl_wait();
-  extern __shared__ __align__(128) uint8_t sm[];
-  uint8_t* sQ = sm;
-  uint8_t* sK = sm + PB_Q * 256;          // 2 buffers of 64 x 256 B
-  uint8_t* sV = sK + 2 * PB_K * 256;
-  const int nqt = gridDim.x;
-  const int qt = nqt - 1 - blockIdx.x;     // longest (last) query tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int g = h / (H / Hk);
-  const int p0 = pos0 ? pos0[b] : 0;
-  const int T = p0 + S;                    // keys visible to the last query
-  const int q_lo = qt * PB_Q;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  const bf16* qsrc = q + ((size_t)b * H + h) * S * PB_D;
-  const bf16* ksrc = kc + ((size_t)b * Hk + g) * Smax * PB_D;
-  const bf16* vsrc = vc + ((size_t)b * Hk + g) * Smax * PB_D;
-  const int k_end = min(T, p0 + q_lo + PB_Q);          // keys needed by this tile
-  const int n_kt = (k_end + PB_K - 1) / PB_K;
-
-  load_tile(sQ, qsrc, q_lo, S);
-  load_tile(sK, ksrc, 0, T);
-  load_tile(sV, vsrc, 0, T);
-  cp_async_commit();
-
-  float oacc[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
-  const int r_in = warp * 16 + (lane >> 2);              // this thread's rows: r_in and r_in + 8
-  const int qpos0 = p0 + q_lo + r_in, qpos1 = qpos0 + 8;
-  uint32_t qf[8][4];
-
-  for (int kt = 0; kt < n_kt; ++kt) {
-    const int buf = kt & 1;
-    if (kt + 1 < n_kt) {
-      load_tile(sK + (buf ^ 1) * PB_K * 256, ksrc, (kt + 1) * PB_K, T);
-      load_tile(sV + (buf ^ 1) * PB_K * 256, vsrc, (kt + 1) * PB_K, T);
-    }
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    if (kt == 0) {
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const int r = warp * 16 + (lane & 15), c = ks * 2 + (lane >> 4);
-        ldsm_x4(smem_u32(sQ) + swz(r, c), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
-      }
-    }
-    const uint32_t kb = smem_u32(sK + buf * PB_K * 256), vb = smem_u32(sV + buf * PB_K * 256);
-    // S = Q K^T : 16 rows x 64 keys per warp
-    float s[8][4];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-#pragma unroll
-      for (int jp = 0; jp < 4; ++jp) {  // two 8-key blocks per ldmatrix.x4
-        const int r = jp * 16 + (lane & 7) + ((lane >> 4) << 3);
-        const int c = ks * 2 + ((lane >> 3) & 1);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(kb + swz(r, c), b0, b1, b2, b3);
-        mma_bf16(s[2 * jp], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b0, b1);
-        mma_bf16(s[2 * jp + 1], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b2, b3);
-      }
-    }
-    // scale, mask, online softmax
-    const int kbase = kt * PB_K;
-    const bool need_mask = kbase + PB_K - 1 > p0 + q_lo;   // some key may be in a query's future
-    float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = kbase + j * 8 + (lane & 3) * 2 + (e & 1);
-        const int qp = (e < 2) ? qpos0 : qpos1;
-        float v = s[j][e] * scale_log2;
-        if (need_mask && key > qp) v = -INFINITY;
-        s[j][e] = v;
-        mx[e >> 1] = fmaxf(mx[e >> 1], v);
-      }
-    }
-    float corr[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
-      mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 2));
-      const float mnew = fmaxf(mrow[i], mx[i]);
-      corr[i] = exp2f(mrow[i] - mnew);
-      mrow[i] = mnew;
-    }
-    float ls[2] = {0.f, 0.f};
-    uint32_t pf[4][4];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float p0v = exp2f(s[j][0] - mrow[0]), p1v = exp2f(s[j][1] - mrow[0]);
-      const float p2v = exp2f(s[j][2] - mrow[1]), p3v = exp2f(s[j][3] - mrow[1]);
-      ls[0] += p0v + p1v;
-      ls[1] += p2v + p3v;
-      const int ks = j >> 1;
-      if ((j & 1) == 0) { pf[ks][0] = pack_bf16(p0v, p1v); pf[ks][1] = pack_bf16(p2v, p3v); }
-      else { pf[ks][2] = pack_bf16(p0v, p1v); pf[ks][3] = pack_bf16(p2v, p3v); }
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      ls[i] += __shfl_xor_sync(0xffffffffu, ls[i], 1);
-      ls[i] += __shfl_xor_sync(0xffffffffu, ls[i], 2);
-      lrow[i] = lrow[i] * corr[i] + ls[i];
-    }
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      oacc[n][0] *= corr[0]; oacc[n][1] *= corr[0];
-      oacc[n][2] *= corr[1]; oacc[n][3] *= corr[1];
-    }
-    // O += P V : V tile [64 keys][128 dims], B operand via transposed ldmatrix
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-#pragma unroll
-      for (int np = 0; np < 8; ++np) {  // two 8-dim blocks per ldmatrix.x4
-        const int r = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-        const int c = np * 2 + (lane >> 4);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vb + swz(r, c), b0, b1, b2, b3);
-        mma_bf16(oacc[2 * np], pf[ks][0], pf[ks][1], pf[ks][2], pf[ks][3], b0, b1);
-        mma_bf16(oacc[2 * np + 1], pf[ks][0], pf[ks][1], pf[ks][2], pf[ks][3], b2, b3);
-      }
-    }
-    __syncthreads();
-  }
-  // normalise and store o[b*S + s][h*128 + :]
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int srow = q_lo + r_in + i * 8;
-    if (srow >= S) continue;
-    const float inv = 1.f / lrow[i];
-    bf16* dst = o + ((size_t)b * S + srow) * H * PB_D + h * PB_D;
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      const int col = n * 8 + (lane & 3) * 2;
-      *reinterpret_cast<uint32_t*>(dst + col) = pack_bf16(oacc[n][2 * i] * inv, oacc[n][2 * i + 1] * inv);
-    }
-  }
 }
 
 // ------------------------------------------------------ fp32 prefill (SIMT)
@@ -783,20 +617,8 @@ int attention_prefill(const void* q, const void* kc, const void* vc, void* o, co
   if (H % Hk != 0) return LLAMA_ERR_SHAPE;
   const float scale_log2 = kLog2e / sqrtf((float)d);
   if (dtype == LLAMA_BF16) {
-    if (d != PB_D) return LLAMA_ERR_UNSUPPORTED;
-    constexpr int SMEM = PB_Q * 256 + 4 * PB_K * 256;
-    static bool attr = false;
-    if (!attr) {
-      if (cudaFuncSetAttribute(attn_prefill_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
-          cudaSuccess)
-        return LLAMA_ERR_CUDA;
-      attr = true;
-    }
-    dim3 grid((S + PB_Q - 1) / PB_Q, H, B);
-    if (launch_k(attn_prefill_bf16_kernel, grid, dim3(128), SMEM, st, static_cast<const bf16*>(q),
-                 static_cast<const bf16*>(kc), static_cast<const bf16*>(vc), static_cast<bf16*>(o), pos0, S, H, Hk,
-                 Smax, scale_log2) != cudaSuccess)
-      return LLAMA_ERR_CUDA;
+    if (d != 128) return LLAMA_ERR_UNSUPPORTED;
+    return attention_prefill_tc(q, kc, vc, o, pos0, B, S, H, Hk, Smax, status, st);
   } else {
     dim3 grid(S, H, B);
     count_launches(1);

@@ -70,6 +70,9 @@ int launch_add_lengths(int32_t* len, int B, int add, cudaStream_t st);
 // o [B*S][H*d]; pos0[b] = position of the call's first query (null = 0).
 int attention_prefill(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B, int S,
                       int H, int Hk, int d, int Smax, int dtype, int* status, cudaStream_t st);
+// tcgen05 flash attention for bf16, d = 128 (same arguments as attention_prefill).
+int attention_prefill_tc(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B, int S,
+                         int H, int Hk, int Smax, int* status, cudaStream_t st);
 // Decode: q [B][H][d]; keys 0 .. nkeys[b]-1 (+ add) of the cache; o [B][H*d].
 struct DecodeScratch {
   float* part;  // [B][H][splits][d + 2]

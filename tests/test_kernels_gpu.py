@@ -123,7 +123,7 @@ def test_argmax_rows_exact_with_ties():
 
 # ----------------------------------------------------- prefill attention
 @pytest.mark.parametrize('B,S,H,Hk', [(2, 200, 8, 2), (1, 1, 4, 1), (1, 64, 4, 4), (1, 65, 8, 2),
-                                      (1, 2048, 32, 8)])
+                                      (1, 2048, 32, 8), (2, 300, 32, 8), (1, 4097, 8, 2), (3, 129, 4, 1)])
 def test_attention_prefill_bf16(B, S, H, Hk):
     d = 128
     qv, qr = normal_values(16, 1, (B, H, S, d), BF16)

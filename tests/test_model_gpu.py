@@ -188,3 +188,25 @@ def test_small_bf16_model_prefill_decode(B, S):
         _check_status(m)
     finally:
         m.close()
+
+
+def test_chunked_prefill_continues_the_cache():
+    """Two prefill calls on the same sequences (the second starts at the cached
+    length) equal one oracle pass over the concatenated prompt: positions,
+    RoPE angles and the causal mask follow the cache length."""
+    m = Model(SMALL_BF16, BF16, max_batch=2, max_seq=512)
+    try:
+        L.llama_init_weights(m.h, 4, 0.02)
+        orc = Oracle(m.p, SeededWeights(m.p, 4, 0.02, BF16))
+        toks = si.tokens(7, 2 * 330, 3000).reshape(2, 330)
+        L.llama_prefill(m.h, torch.from_numpy(np.ascontiguousarray(toks[:, :200])).cuda(), 2, 200)
+        L.llama_prefill(m.h, torch.from_numpy(np.ascontiguousarray(toks[:, 200:])).cuda(), 2, 130)
+        got = m.logits(2).cpu().numpy()
+        ref = np.stack([orc.forward(toks[b]) for b in range(2)])
+        assert rel_l2(got, ref) < 2e-2
+        lens = np.zeros(2, np.int32)
+        L.llama_get_lengths(m.h, lens, 2)
+        assert list(lens) == [330, 330]
+        _check_status(m)
+    finally:
+        m.close()
