@@ -25,10 +25,17 @@
  *    unless stated otherwise.
  *  - Matrices are row-major and contiguous. Weights use the checkpoint's
  *    [out, in] convention and y = x W^T ([W] 查询向量).
- *  - dtype: LLAMA_F32 computes everything in fp32 on the CUDA cores;
- *    LLAMA_BF16 stores weights, activations and the cache in bf16 and
+ *  - dtype: LLAMA_F32 computes everything in fp32 on the CUDA cores.
+ *    LLAMA_F16 stores weights, activations and the cache in fp16 and
  *    accumulates in fp32 on the tensor cores (tcgen05), with an fp32 residual
- *    stream and fp32 logits.
+ *    stream and fp32 logits. LLAMA_BF16 takes bf16 weights (and bf16 K/V in
+ *    llama_set_kv) at the boundary and runs the LLAMA_F16 path on them: each
+ *    bf16 value is stored as the fp16 nearest to it (exact for
+ *    2^-14 <= |w| <= 65504; smaller magnitudes keep an absolute error below
+ *    2^-25, larger ones overflow), and activations are rounded to fp16, whose
+ *    three extra mantissa bits keep the logits of a 32-layer stack within
+ *    2e-2 (relative L2) of the exact result, which bf16 rounding of the
+ *    activations does not. llama_get_weight returns bf16 again.
  *  - A model and its buffers belong to the device that was current at
  *    llama_create; make that device current before every later call.
  */
@@ -49,9 +56,9 @@ extern "C" {
 #define LLAMA_ERR_CUDA (-4)          /* a CUDA runtime/driver call failed */
 #define LLAMA_ERR_DEVICE_TIMEOUT (-5)/* a bounded device-side wait gave up */
 #define LLAMA_ERR_DEVICE_BOUNDS (-6) /* an index checked on the device was out of range */
-#define LLAMA_ERR_UNSUPPORTED (-7)   /* combination not implemented (e.g. bf16 with head_dim != 128) */
+#define LLAMA_ERR_UNSUPPORTED (-7)   /* combination not implemented (e.g. 16-bit model with head_dim != 128) */
 
-typedef enum { LLAMA_F32 = 0, LLAMA_BF16 = 1 } llama_dtype;
+typedef enum { LLAMA_F32 = 0, LLAMA_BF16 = 1, LLAMA_F16 = 2 } llama_dtype;
 
 /* Model statement: the fields of params.json ([W] 下载并读取模型权重) plus the
  * cache sizing of the Hacker News thread (max_batch, max_seq). */
@@ -91,8 +98,9 @@ size_t llama_device_bytes(const llama_model* m);
 
 /* Seeded synthetic weights: every matrix N(0, std^2) from the counter-based generator
  * (SplitMix64 streams + Box-Muller, one stream per checkpoint key in the key order of
- * [W] 下载并读取模型权重), rounded to the model dtype; every norm weight 1.0. Produces the
- * same bits as the host generator in the repository's seeded_inputs module. */
+ * [W] 下载并读取模型权重), rounded to the model dtype (bf16 models: rounded to bf16, then held
+ * as fp16); every norm weight 1.0. Produces the same values as the host generator in the
+ * repository's seeded_inputs module. */
 int llama_init_weights(llama_model* m, uint64_t seed, float std, void* stream);
 
 /* Copy one checkpoint tensor in or out, by its checkpoint name ("tok_embeddings.weight",
@@ -134,7 +142,7 @@ int llama_block_forward(llama_model* m, int32_t layer, const float* x, float* y,
 /* Cache and length control. llama_fill_kv_random writes N(0,1) K and V entries (taken as
  * already rotated) for positions 0..c-1 of every layer and every sequence < max_batch from the
  * seeded generator (layer l: stream 2^21+2l for K, +1 for V, element order [b][g][t][d]) and
- * sets every length to c. llama_set_kv copies caller K/V (device, model dtype,
+ * sets every length to c (rounded as the weights are). llama_set_kv copies caller K/V (device, model dtype,
  * [B][n_kv_heads][c][head_dim]) into layer `layer`, positions 0..c-1. Lengths are host-visible
  * state: set_lengths takes host int32 [B] (B <= max_batch); reset sets all to 0. */
 int llama_fill_kv_random(llama_model* m, uint64_t seed, int32_t c, void* stream);
@@ -166,13 +174,14 @@ const char* llama_status_string(int status);
 
 /* Causal GQA attention for prefill ([W] 查询和键相乘, 掩码, 多头注意力): q [B][H][S][d],
  * k, v [B][Hk][S][d] (already rotated), o [B][S][H*d]; query s sees keys 0..s; head h reads kv
- * head h / (H/Hk); scores scaled by 1/sqrt(d). bf16 requires d = 128; fp32 takes d in {32,64,128}. */
+ * head h / (H/Hk); scores scaled by 1/sqrt(d). bf16 and fp16 require d = 128; fp32 takes d in
+ * {32,64,128}. */
 int llama_attention_prefill(const void* q, const void* k, const void* v, void* o, int32_t B, int32_t S, int32_t H,
                             int32_t Hk, int32_t d, int32_t dtype, void* stream);
 
 /* Single-query attention over a cache (decode): q [B][H][d]; kc, vc [B][Hk][cmax][d]; len
  * (device int32 [B], 1 <= len[b] <= cmax) = number of valid keys of sequence b; o [B][H*d].
- * Split over the key range, merged with the log-sum-exp rule. d in {64,128} (bf16) or
+ * Split over the key range, merged with the log-sum-exp rule. d in {64,128} (bf16, fp16) or
  * {32,64,128} (fp32); H/Hk <= 8. */
 int llama_attention_decode(const void* q, const void* kc, const void* vc, const int32_t* len, void* o, int32_t B,
                            int32_t cmax, int32_t H, int32_t Hk, int32_t d, int32_t dtype, void* stream);
@@ -186,7 +195,7 @@ int llama_attention_decode(const void* q, const void* kc, const void* vc, const 
  * llama_attention_decode (arguments, layouts, results).
  * Its split partials live in one static 4 MiB device array that every GPU which loads this
  * library keeps until the process exits. Calls needing more than 4 MiB of partials return
- * LLAMA_ERR_SHAPE: for bf16 with d = 128 the partials take (B*Hk + 4*SMs) * (H/Hk) * (d+2) * 4
+ * LLAMA_ERR_SHAPE: for bf16 or fp16 with d = 128 the partials take (B*Hk + 4*SMs) * (H/Hk) * (d+2) * 4
  * bytes (SMs = 148 on B200), so with H = 32, Hk = 8 every B up to 170 fits.
  * The first call on a device looks up the array's device address for that device
  * (cudaGetSymbolAddress); make that first call before any stream capture begins.
@@ -201,7 +210,7 @@ int llama_attention_decode_noalloc(const void* q, const void* kc, const void* vc
 
 /* y = x W^T: x [M][K], w [N][K] (dtype), y fp32 [M][N]. variant 0 = automatic, 1 = the wide
  * persistent tcgen05 kernel, 2 = the skinny split-K tcgen05 kernel (M <= 256); fp32 ignores it.
- * bf16 requires K % 8 == 0 and 16-byte aligned x and w. */
+ * bf16 and fp16 require K % 8 == 0 and 16-byte aligned x and w. */
 int llama_linear(const void* x, const void* w, float* y, int32_t M, int32_t N, int32_t K, int32_t dtype,
                  int32_t variant, void* stream);
 
@@ -214,7 +223,7 @@ int llama_rmsnorm(const float* x, const float* g, void* y, int32_t M, int32_t D,
 int llama_argmax_rows(const float* logits, int32_t* out, int32_t B, int32_t V, void* stream);
 
 /* n draws of N(0, std^2) of stream `stream_id` under `seed` (the weight generator) into dst
- * (device, dtype). */
+ * (device, dtype; fp16 rounds the fp32 draw to fp16 directly). */
 int llama_fill_normal(void* dst, int64_t n, uint64_t seed, uint64_t stream_id, float std, int32_t dtype,
                       void* stream);
 

@@ -24,6 +24,7 @@ LLAMA_ERR_DEVICE_BOUNDS = -6
 LLAMA_ERR_UNSUPPORTED = -7
 LLAMA_F32 = 0
 LLAMA_BF16 = 1
+LLAMA_F16 = 2
 
 
 class LlamaError(RuntimeError):

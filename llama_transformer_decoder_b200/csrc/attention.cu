@@ -1,6 +1,6 @@
 // Causal grouped-query attention over the KV cache.
 //
-//  * prefill (bf16): the tcgen05 flash-attention kernel in attention_tc.cu.
+//  * prefill (bf16 / fp16): the tcgen05 flash-attention kernel in attention_tc.cu.
 //  * prefill (fp32): one warp per query row on the CUDA cores.
 //  * decode (both dtypes): split over the cached keys. Each CTA serves the
 //    H/Hk query heads of one kv head, streams its key range through shared
@@ -8,6 +8,7 @@
 //    cache), keeps (max, sum, o) per head, and a combine kernel merges the
 //    splits with the log-sum-exp rule.
 #include <cstdlib>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -30,7 +31,7 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Tile rows are 256 B (128 bf16); 16-byte chunk c of row r lives at chunk c ^ (r & 7).
+// Tile rows are 256 B (128 16-bit values); 16-byte chunk c of row r lives at chunk c ^ (r & 7).
 __device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 256 + ((c ^ (r & 7)) << 4)); }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
@@ -43,17 +44,21 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& a, uint32_t& 
                : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
                : "r"(addr));
 }
-__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
+// m16n8k16 tensor-core product, fp32 accumulate; T = bf16 or fp16 operands.
+template <typename T>
+__device__ __forceinline__ void mma16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                      uint32_t b1) {
+  if constexpr (std::is_same<T, f16>::value) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
 }
 
 // ------------------------------------------------------ fp32 prefill (SIMT)
@@ -292,7 +297,7 @@ __global__ void attn_decode_combine_kernel(const float* __restrict__ part, T* __
 }
 
 
-// ---------------------------------------------- decode, bf16 d = 128 (mma)
+// ---------------------------------------- decode, 16-bit d = 128 (mma)
 // Every warp is an independent flash decoder over a contiguous range of the
 // global tile sequence: (sequence b, kv head g, 32-key tile t) in that order,
 // T tiles in all; warp w of W takes tiles [T*w/W, T*(w+1)/W), so warps differ
@@ -356,13 +361,14 @@ __device__ bool tc_next(TileCursor& c, const int32_t* nkeys, int add, int nmax, 
   return true;
 }
 
-__device__ __forceinline__ void dm_load_tile(uint8_t* stage, const bf16* kc, const bf16* vc, const TileCursor& c,
+template <typename T>
+__device__ __forceinline__ void dm_load_tile(uint8_t* stage, const T* kc, const T* vc, const TileCursor& c,
                                              int Hk, int Smax, int lane) {
   const int key0 = c.t * DM_KEYS;
   const int valid = min(DM_KEYS, c.n - key0);
   const size_t row0 = ((size_t)c.b * Hk + c.g) * Smax + key0;
-  const bf16* ks = kc + row0 * 128;
-  const bf16* vs = vc + row0 * 128;
+  const T* ks = kc + row0 * 128;
+  const T* vs = vc + row0 * 128;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int idx = i * 32 + lane;
@@ -374,8 +380,9 @@ __device__ __forceinline__ void dm_load_tile(uint8_t* stage, const bf16* kc, con
   }
 }
 
+template <typename T>
 __global__ void __launch_bounds__(DM_WARPS * 32, 1)
-    attn_decode_mma_kernel(const bf16* __restrict__ q, const bf16* __restrict__ kc, const bf16* __restrict__ vc,
+    attn_decode_mma_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
                            const int32_t* __restrict__ nkeys, int add_keys, int nmax, float* __restrict__ part, int B,
                            int H, int Hk, int Smax, float scale_log2, int* status) {
   pdl_trigger();
@@ -419,7 +426,7 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
   bool start = true;
   while (cp.left > 0) {
     if (start) {   // new piece: reset the state and fetch the G query rows of (b, g)
-      const bf16* qr = q + ((size_t)cp.b * H + cp.g * G + (real ? row : 0)) * 128;
+      const T* qr = q + ((size_t)cp.b * H + cp.g * G + (real ? row : 0)) * 128;
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         qa[ks][0] = real ? *reinterpret_cast<const uint32_t*>(qr + ks * 16 + 2 * tq) : 0u;
@@ -455,8 +462,8 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
         const int c = ks * 2 + ((lane >> 3) & 1);
         uint32_t b0, b1, b2, b3;
         ldsm_x4(kb + swz(r, c), b0, b1, b2, b3);
-        mma_bf16(sc[2 * jp], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
-        mma_bf16(sc[2 * jp + 1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
+        mma16<T>(sc[2 * jp], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
+        mma16<T>(sc[2 * jp + 1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
       }
     }
     float mx = -INFINITY;
@@ -481,7 +488,7 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
     for (int j = 0; j < 4; ++j) {
       const float p0 = exp2f(sc[j][0] - mnew), p1 = exp2f(sc[j][1] - mnew);
       ls += p0 + p1;
-      pa[j >> 1][j & 1] = pack_bf16(p0, p1);
+      pa[j >> 1][j & 1] = pack2<T>(p0, p1);
     }
     ls += __shfl_xor_sync(0xffffffffu, ls, 1);
     ls += __shfl_xor_sync(0xffffffffu, ls, 2);
@@ -499,8 +506,8 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
                        ks == 0 ? oacc[2 * np][1] * corr : oacc[2 * np][1], 0.f, 0.f};
         float t1[4] = {ks == 0 ? oacc[2 * np + 1][0] * corr : oacc[2 * np + 1][0],
                        ks == 0 ? oacc[2 * np + 1][1] * corr : oacc[2 * np + 1][1], 0.f, 0.f};
-        mma_bf16(t0, pa[ks][0], 0u, pa[ks][1], 0u, b0, b1);
-        mma_bf16(t1, pa[ks][0], 0u, pa[ks][1], 0u, b2, b3);
+        mma16<T>(t0, pa[ks][0], 0u, pa[ks][1], 0u, b0, b1);
+        mma16<T>(t1, pa[ks][0], 0u, pa[ks][1], 0u, b2, b3);
         oacc[2 * np][0] = t0[0]; oacc[2 * np][1] = t0[1];
         oacc[2 * np + 1][0] = t1[0]; oacc[2 * np + 1][1] = t1[1];
       }
@@ -616,9 +623,9 @@ int attention_prefill(const void* q, const void* kc, const void* vc, void* o, co
   if (B <= 0 || S <= 0) return LLAMA_OK;
   if (H % Hk != 0) return LLAMA_ERR_SHAPE;
   const float scale_log2 = kLog2e / sqrtf((float)d);
-  if (dtype == LLAMA_BF16) {
+  if (dtype == LLAMA_BF16 || dtype == LLAMA_F16) {
     if (d != 128) return LLAMA_ERR_UNSUPPORTED;
-    return attention_prefill_tc(q, kc, vc, o, pos0, B, S, H, Hk, Smax, status, st);
+    return attention_prefill_tc(q, kc, vc, o, pos0, B, S, H, Hk, Smax, dtype, status, st);
   } else {
     dim3 grid(S, H, B);
     count_launches(1);
@@ -646,12 +653,36 @@ int decode_splits(int cmax, int B, int Hk) {
   return s < 1 ? 1 : s;
 }
 
-bool use_mma_decode(int d, int dtype) { return dtype == LLAMA_BF16 && d == 128; }
+bool use_mma_decode(int d, int dtype) { return (dtype == LLAMA_BF16 || dtype == LLAMA_F16) && d == 128; }
 }  // namespace
 
 size_t decode_scratch_floats(int cmax, int B, int H, int Hk, int d, int dtype) {
   if (use_mma_decode(d, dtype)) return ((size_t)B * Hk + (size_t)num_sms() * DM_WARPS) * (H / Hk) * (d + 2);
   return (size_t)B * H * decode_splits(cmax, B, Hk) * (d + 2);
+}
+
+template <typename T>
+static int mma_decode_launch(const void* q, const void* kc, const void* vc, const int32_t* nkeys, int add_keys,
+                             void* o, int B, int cmax, int H, int Hk, int Smax, DecodeScratch* scratch, int* status,
+                             cudaStream_t st) {
+  const int grid = num_sms();
+  auto kern = attn_decode_mma_kernel<T>;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DM_SMEM) != cudaSuccess)
+      return LLAMA_ERR_CUDA;
+    attr = true;
+  }
+  const float scale_log2 = kLog2e / sqrtf(128.f);
+  const int nmax = cmax < Smax ? cmax : Smax;
+  cudaError_t err = launch_k(kern, dim3(grid), dim3(DM_WARPS * 32), DM_SMEM, st, static_cast<const T*>(q),
+                             static_cast<const T*>(kc), static_cast<const T*>(vc), nkeys, add_keys, nmax,
+                             scratch->part, B, H, Hk, Smax, scale_log2, status);
+  if (err == cudaSuccess)
+    err = launch_k(attn_decode_combine_pieces_kernel<T, 128>, dim3(H, B), dim3(128), 0, st,
+                   (const float*)scratch->part, nkeys, add_keys, nmax, static_cast<T*>(o), B, H, Hk,
+                   (long long)grid * DM_WARPS);
+  return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 int attention_decode(const void* q, const void* kc, const void* vc, const int32_t* nkeys, int add_keys, void* o,
@@ -662,29 +693,17 @@ int attention_decode(const void* q, const void* kc, const void* vc, const int32_
   if (!scratch || !scratch->part || scratch->floats < decode_scratch_floats(cmax, B, H, Hk, d, dtype))
     return LLAMA_ERR_INVALID_ARG;
   if (use_mma_decode(d, dtype)) {
-    const int grid = num_sms();
-    static bool attr = false;
-    if (!attr) {
-      if (cudaFuncSetAttribute(attn_decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DM_SMEM) !=
-          cudaSuccess)
-        return LLAMA_ERR_CUDA;
-      attr = true;
-    }
-    const float scale_log2 = kLog2e / sqrtf((float)d);
-    const int nmax = cmax < Smax ? cmax : Smax;
-    cudaError_t err = launch_k(attn_decode_mma_kernel, dim3(grid), dim3(DM_WARPS * 32), DM_SMEM, st,
-                               static_cast<const bf16*>(q), static_cast<const bf16*>(kc), static_cast<const bf16*>(vc),
-                               nkeys, add_keys, nmax, scratch->part, B, H, Hk, Smax, scale_log2, status);
-    if (err == cudaSuccess)
-      err = launch_k(attn_decode_combine_pieces_kernel<bf16, 128>, dim3(H, B), dim3(128), 0, st,
-                     (const float*)scratch->part, nkeys, add_keys, nmax, static_cast<bf16*>(o), B, H, Hk,
-                     (long long)grid * DM_WARPS);
-    return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+    if (dtype == LLAMA_F16)
+      return mma_decode_launch<f16>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch, status, st);
+    return mma_decode_launch<bf16>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch, status, st);
   }
   const int splits = decode_splits(cmax, B, Hk);
   if (dtype == LLAMA_BF16) {
     if (d == 64) return decode_launch<bf16, 64>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch->part,
                                                 splits, status, st);
+  } else if (dtype == LLAMA_F16) {
+    if (d == 64) return decode_launch<f16, 64>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch->part,
+                                               splits, status, st);
   } else {
     if (d == 128) return decode_launch<float, 128>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax,
                                                    scratch->part, splits, status, st);

@@ -1,5 +1,5 @@
-// Causal GQA prefill attention on the 5th-generation tensor cores (bf16,
-// head_dim 128).
+// Causal GQA prefill attention on the 5th-generation tensor cores (16-bit
+// q/k/v, bf16 or fp16, head_dim 128).
 //
 // One CTA computes 128 queries of one head. Warp roles: warp 0 issues TMA
 // loads (Q once, then K and V tiles of 128 keys into a 2-stage ring), warp 1
@@ -8,8 +8,8 @@
 //
 //   S_j = Q K_j^T      -> TMEM (two 128-column buffers, so S_{j+1} is computed
 //                         while the softmax works on S_j)
-//   P_j = exp2(S_j*c - m) rounded to bf16 (the walkthrough applies
-//                         softmax(...).to(bfloat16) before the value product)
+//   P_j = exp2(S_j*c - m) rounded to the 16-bit type (the walkthrough rounds
+//                         softmax(...) to 16 bits before the value product)
 //                      -> shared memory, 128-byte swizzled K-major rows
 //   O  += P_j V_j      -> TMEM (128 columns); V is read MN-major straight from
 //                         the cache layout [key][d].
@@ -19,6 +19,8 @@
 // O / l is exact for any m used consistently. Query i of the tile sits at
 // absolute position pos0 + q0 + i and sees keys 0 .. pos0 + q0 + i.
 #include <cudaTypedefs.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -53,9 +55,10 @@ __device__ __forceinline__ uint8_t* fa_align(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+template <typename T>
 __global__ void __launch_bounds__(192, 1)
     attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                           const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ o,
+                           const __grid_constant__ CUtensorMap tmV, T* __restrict__ o,
                            const int32_t* __restrict__ pos0, int S, int H, int Hk, float scale_log2, int* status) {
   extern __shared__ uint8_t fa_smem_raw[];
   uint8_t* smem = fa_align(fa_smem_raw);
@@ -97,8 +100,8 @@ __global__ void __launch_bounds__(192, 1)
   pdl_wait();
 
   const int p0 = pos0 ? pos0[b] : 0;
-  const int T = p0 + S;                                   // keys of this sequence
-  const int k_end = min(T, p0 + q0 + FA_BM);              // keys this tile needs
+  const int n_keys = p0 + S;                              // keys of this sequence
+  const int k_end = min(n_keys, p0 + q0 + FA_BM);         // keys this tile needs
   const int n_kt = (k_end + FA_BN - 1) / FA_BN;
 
   if (warp == 0 && lane == 0) {
@@ -128,8 +131,8 @@ __global__ void __launch_bounds__(192, 1)
       for (int j = issued - 1; j >= 0 && j >= issued - 2; --j) mbar_wait(&kv_full[j & 1], (j >> 1) & 1, status);
     }
   } else if (warp == 1 && lane == 0) {
-    constexpr uint32_t idesc_s = umma_idesc_bf16(FA_BM, FA_BN, false);
-    constexpr uint32_t idesc_o = umma_idesc_bf16(FA_BM, FA_D, true);
+    constexpr uint32_t idesc_s = umma_idesc_16(UmmaFmt<T>::value, FA_BM, FA_BN, false);
+    constexpr uint32_t idesc_o = umma_idesc_16(UmmaFmt<T>::value, FA_BM, FA_D, true);
     const uint32_t q_addr = smem_u32(smem + FA_OFF_Q), p_addr = smem_u32(smem + FA_OFF_P);
     bool ok = mbar_wait(q_full, 0, status), any = false;
     auto issue_s = [&](int j) -> bool {
@@ -219,8 +222,7 @@ __global__ void __launch_bounds__(192, 1)
         const float a = fast_exp2(fmaf(sv[2 * i], scale_log2, -m_used));
         const float c2 = fast_exp2(fmaf(sv[2 * i + 1], scale_log2, -m_used));
         rowsum += a + c2;
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(a, c2);
-        pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+        pk[i] = pack2<T>(a, c2);
       }
       l = l * corr + rowsum;
       // P and O may be touched only once the previous P V product has finished
@@ -256,7 +258,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     const int qi = q0 + r;
     const float inv = 1.f / l;
-    bf16* dst = o + ((size_t)b * S + (qi < S ? qi : 0)) * H * FA_D + (size_t)h * FA_D;
+    T* dst = o + ((size_t)b * S + (qi < S ? qi : 0)) * H * FA_D + (size_t)h * FA_D;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       float t[32];
@@ -268,10 +270,7 @@ __global__ void __launch_bounds__(192, 1)
       if (qi < S) {
         uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(t[2 * i] * inv, t[2 * i + 1] * inv);
-          w[i] = *reinterpret_cast<uint32_t*>(&h2);
-        }
+        for (int i = 0; i < 16; ++i) w[i] = pack2<T>(t[2 * i] * inv, t[2 * i + 1] * inv);
         uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
         for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
@@ -286,8 +285,8 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-// [outer][rows][128] bf16 -> 3-D map with boxes of 64 x 128 x 1, 128-byte swizzle.
-int make_tmap_3d(CUtensorMap* map, const void* base, int64_t outer, int64_t rows) {
+// [outer][rows][128] 16-bit -> 3-D map with boxes of 64 x 128 x 1, 128-byte swizzle.
+int make_tmap_3d(CUtensorMap* map, const void* base, int64_t outer, int64_t rows, bool is_f16) {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
     void* p = nullptr;
@@ -302,7 +301,8 @@ int make_tmap_3d(CUtensorMap* map, const void* base, int64_t outer, int64_t rows
   cuuint64_t gstride[2] = {(cuuint64_t)FA_D * 2, (cuuint64_t)rows * FA_D * 2};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box, estr,
+  const CUresult r = fn(map, is_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                        const_cast<void*>(base), gdim, gstride, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? LLAMA_OK : LLAMA_ERR_CUDA;
@@ -310,24 +310,32 @@ int make_tmap_3d(CUtensorMap* map, const void* base, int64_t outer, int64_t rows
 
 }  // namespace
 
-int attention_prefill_tc(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B, int S,
-                         int H, int Hk, int Smax, int* status, cudaStream_t st) {
+template <typename T>
+static int attention_prefill_tc_t(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B,
+                                  int S, int H, int Hk, int Smax, int* status, cudaStream_t st) {
+  constexpr bool F16 = std::is_same<T, f16>::value;
   CUtensorMap tq, tk, tv;
   int rc;
-  if ((rc = make_tmap_3d(&tq, q, (int64_t)B * H, S)) != LLAMA_OK) return rc;
-  if ((rc = make_tmap_3d(&tk, kc, (int64_t)B * Hk, Smax)) != LLAMA_OK) return rc;
-  if ((rc = make_tmap_3d(&tv, vc, (int64_t)B * Hk, Smax)) != LLAMA_OK) return rc;
+  if ((rc = make_tmap_3d(&tq, q, (int64_t)B * H, S, F16)) != LLAMA_OK) return rc;
+  if ((rc = make_tmap_3d(&tk, kc, (int64_t)B * Hk, Smax, F16)) != LLAMA_OK) return rc;
+  if ((rc = make_tmap_3d(&tv, vc, (int64_t)B * Hk, Smax, F16)) != LLAMA_OK) return rc;
+  auto kern = attn_prefill_tc_kernel<T>;
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(attn_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM) != cudaSuccess)
       return LLAMA_ERR_CUDA;
     attr = true;
   }
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)FA_D);
-  const cudaError_t err = launch_k(attn_prefill_tc_kernel, dim3(((S + FA_BM - 1) / FA_BM) * H * B), dim3(192), FA_SMEM,
-                                   st, tq, tk, tv, static_cast<bf16*>(o), pos0, S, H, Hk, scale_log2, status);
+  const cudaError_t err = launch_k(kern, dim3(((S + FA_BM - 1) / FA_BM) * H * B), dim3(192), FA_SMEM, st, tq, tk, tv,
+                                   static_cast<T*>(o), pos0, S, H, Hk, scale_log2, status);
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int attention_prefill_tc(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B, int S,
+                         int H, int Hk, int Smax, int elt, int* status, cudaStream_t st) {
+  if (elt == LLAMA_F16) return attention_prefill_tc_t<f16>(q, kc, vc, o, pos0, B, S, H, Hk, Smax, status, st);
+  return attention_prefill_tc_t<bf16>(q, kc, vc, o, pos0, B, S, H, Hk, Smax, status, st);
 }
 
 }  // namespace llama

@@ -3,6 +3,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -11,6 +12,7 @@
 namespace llama {
 
 typedef __nv_bfloat16 bf16;
+typedef __half f16;
 
 // ------------------------------------------------------------------ status
 // Device-side errors are latched into a status word (first error wins) and
@@ -123,12 +125,13 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
   return d;
 }
 
-// Instruction descriptor: kind::f16 with bf16 A/B, fp32 accumulator; A K-major,
-// B K-major (b_mn_major = false) or MN-major.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool b_mn_major = false) {
+// Instruction descriptor: kind::f16 with A and B of format `fmt` (0 = f16,
+// 1 = bf16; both operands share it), fp32 accumulator; A K-major, B K-major
+// (b_mn_major = false) or MN-major.
+__host__ __device__ constexpr uint32_t umma_idesc_16(uint32_t fmt, int M, int N, bool b_mn_major = false) {
   return (1u << 4)                    // D format f32
-         | (1u << 7)                  // A format bf16
-         | (1u << 10)                 // B format bf16
+         | (fmt << 7)                 // A format
+         | (fmt << 10)                // B format
          | ((b_mn_major ? 1u : 0u) << 16)
          | ((uint32_t)(N >> 3) << 17) // N / 8
          | ((uint32_t)(M >> 4) << 24);// M / 16
@@ -253,8 +256,17 @@ __device__ __forceinline__ float to_f<bf16>(bf16 v) {
   return __bfloat162float(v);
 }
 
+template <>
+__device__ __forceinline__ float to_f<f16>(f16 v) {
+  return __half2float(v);
+}
+
 template <typename T>
 __device__ __forceinline__ T from_f(float v);
+template <>
+__device__ __forceinline__ f16 from_f<f16>(float v) {
+  return __float2half_rn(v);
+}
 template <>
 __device__ __forceinline__ float from_f<float>(float v) {
   return v;
@@ -263,5 +275,31 @@ template <>
 __device__ __forceinline__ bf16 from_f<bf16>(float v) {
   return __float2bfloat16_rn(v);
 }
+
+// Two floats rounded to a packed pair of 16-bit values (low half = a).
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float a, float b);
+template <>
+__device__ __forceinline__ uint32_t pack2<bf16>(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+template <>
+__device__ __forceinline__ uint32_t pack2<f16>(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// tcgen05 operand format code of a 16-bit element type (kind::f16).
+template <typename T>
+struct UmmaFmt;
+template <>
+struct UmmaFmt<bf16> {
+  static constexpr uint32_t value = 1;
+};
+template <>
+struct UmmaFmt<f16> {
+  static constexpr uint32_t value = 0;
+};
 
 }  // namespace llama

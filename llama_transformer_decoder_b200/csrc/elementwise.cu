@@ -184,7 +184,7 @@ __device__ __forceinline__ float seeded_normal(uint64_t key, uint64_t i, double 
   return __double2float_rn(__dmul_rn(z, sd));
 }
 
-template <typename T>
+template <typename T, bool ROUND_BF16>
 __global__ void fill_normal_kernel(T* __restrict__ dst, FillLayout L, uint64_t key, double sd) {
   const int64_t n = L.outer * L.rows * L.cols;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
@@ -193,7 +193,9 @@ __global__ void fill_normal_kernel(T* __restrict__ dst, FillLayout L, uint64_t k
     const int64_t r = t % L.rows;
     const int64_t o = t / L.rows;
     const int64_t phys = o * L.outer_stride + (r * L.row_mult + L.row_off) * L.row_stride + c;
-    dst[phys] = from_f<T>(seeded_normal(key, (uint64_t)i, sd));
+    float v = seeded_normal(key, (uint64_t)i, sd);
+    if (ROUND_BF16) v = __bfloat162float(__float2bfloat16_rn(v));
+    dst[phys] = from_f<T>(v);
   }
 }
 
@@ -223,7 +225,10 @@ int launch_embed(const int32_t* tokens, int M, const void* table, int V, int D, 
                  cudaStream_t st) {
   if (M <= 0) return LLAMA_OK;
   cudaError_t err;
-  if (dtype == LLAMA_BF16)
+  if (dtype == LLAMA_F16)
+    err = launch_k(embed_kernel<f16>, dim3(M), dim3(256), 0, st, tokens, static_cast<const f16*>(table), V, D, x,
+                   status);
+  else if (dtype == LLAMA_BF16)
     err = launch_k(embed_kernel<bf16>, dim3(M), dim3(256), 0, st, tokens, static_cast<const bf16*>(table), V, D, x,
                    status);
   else
@@ -236,7 +241,9 @@ int launch_rmsnorm(const float* x, const float* g, void* y, int rows, int D, flo
                    cudaStream_t st) {
   if (rows <= 0) return LLAMA_OK;
   cudaError_t err;
-  if (dtype == LLAMA_BF16)
+  if (dtype == LLAMA_F16)
+    err = launch_k(rmsnorm_kernel<f16>, dim3(rows), dim3(256), 0, st, x, g, static_cast<f16*>(y), D, eps, last_of_S);
+  else if (dtype == LLAMA_BF16)
     err = launch_k(rmsnorm_kernel<bf16>, dim3(rows), dim3(256), 0, st, x, g, static_cast<bf16*>(y), D, eps, last_of_S);
   else
     err = launch_k(rmsnorm_kernel<float>, dim3(rows), dim3(256), 0, st, x, g, static_cast<float*>(y), D, eps,
@@ -258,26 +265,62 @@ int launch_add_lengths(int32_t* len, int B, int add, cudaStream_t st) {
 }
 
 int launch_fill_normal(void* dst, const FillLayout& L, uint64_t seed, uint64_t stream_id, float std, int dtype,
-                       cudaStream_t st) {
+                       cudaStream_t st, bool round_bf16) {
   const int64_t n = L.outer * L.rows * L.cols;
   if (n <= 0) return LLAMA_OK;
   const uint64_t key = stream_key(seed, stream_id);
   const double sd = (double)std;
+  count_launches(1);
   if (dtype == LLAMA_BF16)
-    fill_normal_kernel<bf16><<<grid_for(n), 256, 0, st>>>(static_cast<bf16*>(dst), L, key, sd);
+    fill_normal_kernel<bf16, false><<<grid_for(n), 256, 0, st>>>(static_cast<bf16*>(dst), L, key, sd);
+  else if (dtype == LLAMA_F16 && round_bf16)
+    fill_normal_kernel<f16, true><<<grid_for(n), 256, 0, st>>>(static_cast<f16*>(dst), L, key, sd);
+  else if (dtype == LLAMA_F16)
+    fill_normal_kernel<f16, false><<<grid_for(n), 256, 0, st>>>(static_cast<f16*>(dst), L, key, sd);
   else
-    fill_normal_kernel<float><<<grid_for(n), 256, 0, st>>>(static_cast<float*>(dst), L, key, sd);
+    fill_normal_kernel<float, false><<<grid_for(n), 256, 0, st>>>(static_cast<float*>(dst), L, key, sd);
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+namespace {
+// dst[r][c] = src[r][c] converted between 16-bit types (elt codes LLAMA_BF16 / LLAMA_F16).
+template <typename D, typename S>
+__global__ void convert_2d_kernel(D* __restrict__ dst, int64_t dpitch, const S* __restrict__ src, int64_t spitch,
+                                  int64_t rows, int64_t cols) {
+  const int64_t n = rows * cols;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / cols, c = i - r * cols;
+    dst[r * dpitch + c] = from_f<D>(to_f<S>(src[r * spitch + c]));
+  }
+}
+}  // namespace
+
+int launch_convert_2d(void* dst, int64_t dpitch, int dst_elt, const void* src, int64_t spitch, int src_elt,
+                      int64_t rows, int64_t cols, cudaStream_t st) {
+  const int64_t n = rows * cols;
+  if (n <= 0) return LLAMA_OK;
+  count_launches(1);
+  if (dst_elt == LLAMA_F16 && src_elt == LLAMA_BF16)
+    convert_2d_kernel<f16, bf16><<<grid_for(n), 256, 0, st>>>(static_cast<f16*>(dst), dpitch,
+                                                              static_cast<const bf16*>(src), spitch, rows, cols);
+  else if (dst_elt == LLAMA_BF16 && src_elt == LLAMA_F16)
+    convert_2d_kernel<bf16, f16><<<grid_for(n), 256, 0, st>>>(static_cast<bf16*>(dst), dpitch,
+                                                              static_cast<const f16*>(src), spitch, rows, cols);
+  else
+    return LLAMA_ERR_INVALID_ARG;
   return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 int launch_fill_const(float* dst, int64_t n, float v, cudaStream_t st) {
   if (n <= 0) return LLAMA_OK;
+  count_launches(1);
   fill_const_kernel<<<grid_for(n), 256, 0, st>>>(dst, n, v);
   return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 int launch_fill_tokens(int32_t* dst, int64_t n, uint64_t seed, uint64_t stream_id, int vocab, cudaStream_t st) {
   if (n <= 0) return LLAMA_OK;
+  count_launches(1);
   fill_tokens_kernel<<<grid_for(n), 256, 0, st>>>(dst, n, stream_key(seed, stream_id), (uint32_t)vocab);
   return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }

@@ -106,10 +106,7 @@ __device__ __forceinline__ void epi_row32(const EpiArgs& e, int m, int n0, const
     if (sizeof(T) == 2 && full && ((e.ldg & 7) == 0)) {
       uint32_t w[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(silu_f(v[4 * j]) * v[4 * j + 1], silu_f(v[4 * j + 2]) * v[4 * j + 3]);
-        w[j] = *reinterpret_cast<uint32_t*>(&h2);
-      }
+      for (int j = 0; j < 8; ++j) w[j] = pack2<T>(silu_f(v[4 * j]) * v[4 * j + 1], silu_f(v[4 * j + 2]) * v[4 * j + 3]);
       uint4* p4 = reinterpret_cast<uint4*>(p);
       p4[0] = make_uint4(w[0], w[1], w[2], w[3]);
       p4[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -156,10 +153,7 @@ __device__ __forceinline__ void epi_row32(const EpiArgs& e, int m, int n0, const
     }
     uint32_t w[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      __nv_bfloat162 h2 = __floats2bfloat162_rn(r[2 * j], r[2 * j + 1]);
-      w[j] = *reinterpret_cast<uint32_t*>(&h2);
-    }
+    for (int j = 0; j < 16; ++j) w[j] = pack2<T>(r[2 * j], r[2 * j + 1]);
     uint4* p4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
     for (int j = 0; j < 4; ++j) p4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);

@@ -1,4 +1,5 @@
-// tcgen05 GEMMs for the bf16 projections: acc = x W^T with x [M,K], W [N,K].
+// tcgen05 GEMMs for the 16-bit projections: acc = x W^T with x [M,K], W [N,K]
+// (bf16 or fp16 operands, fp32 accumulation).
 //
 // Two kernels share the same warp roles (warp 0: TMA producer, warp 1: MMA
 // issuer and TMEM owner, warps 2-5: epilogue reading TMEM):
@@ -22,6 +23,7 @@
 
 #include <cstdlib>
 #include <mutex>
+#include <type_traits>
 
 #include "epilogue.cuh"
 #include "kernels.h"
@@ -122,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!ok) drain_loads(full, stage, phase, issued, W_STAGES, status);
   } else if (warp == 1 && lane == 0) {
-    constexpr uint32_t idesc = umma_idesc_bf16(W_BM, W_BN);
+    constexpr uint32_t idesc = umma_idesc_16(UmmaFmt<T>::value, W_BM, W_BN);
     int stage = 0, acc = 0;
     uint32_t phase = 0, acc_phase = 0;
     bool ok = true, any = false;
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!ok) drain_loads(full, stage, phase, issued, C::STAGES, status);
   } else if (warp == 1 && lane == 0) {
-    constexpr uint32_t idesc = umma_idesc_bf16(S_BM, NT);
+    constexpr uint32_t idesc = umma_idesc_16(UmmaFmt<T>::value, S_BM, NT);
     int stage = 0, buf = 0;
     uint32_t phase = 0, acc_phase = 0;
     bool ok = true, any = false;
@@ -481,9 +483,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 }  // namespace
 
-// bf16 row-major [rows, cols] matrix with row pitch `pitch` elements, boxes of
-// box_rows x 64 elements, 128-byte swizzle, zero fill outside the matrix.
-int make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t pitch, int box_rows) {
+// 16-bit row-major [rows, cols] matrix with row pitch `pitch` elements, boxes
+// of box_rows x 64 elements, 128-byte swizzle, zero fill outside the matrix.
+int make_tmap_16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t pitch, int box_rows,
+                 bool is_f16) {
   auto fn = encode_fn();
   if (!fn) return LLAMA_ERR_CUDA;
   if ((reinterpret_cast<uintptr_t>(base) & 15) || (pitch * 2) % 16 != 0) return LLAMA_ERR_INVALID_ARG;
@@ -491,7 +494,8 @@ int make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t col
   cuuint64_t gstride[1] = {(cuuint64_t)(pitch * 2)};
   cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estr,
+  CUresult r = fn(map, is_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), gdim, gstride, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? LLAMA_OK : LLAMA_ERR_CUDA;
@@ -508,10 +512,10 @@ int num_sms() {
   return n;
 }
 
-template <int KIND>
+template <int KIND, typename T>
 static int launch_wide(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, const EpiArgs& e,
                        int* status, cudaStream_t st) {
-  auto kern = gemm_wide_kernel<KIND, bf16>;
+  auto kern = gemm_wide_kernel<KIND, T>;
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, W_SMEM) != cudaSuccess)
@@ -524,11 +528,11 @@ static int launch_wide(const CUtensorMap& ta, const CUtensorMap& tb, int M, int 
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
-template <int KIND, int NT>
+template <int KIND, typename T, int NT>
 static int launch_skinny_nt(const CUtensorMap& tw, const CUtensorMap& tx, int M, int N, int K, const EpiArgs& e,
                             float* ws, int* tickets, float* stg, int* status, cudaStream_t st) {
   using C = SkinnyCfg<NT>;
-  auto kern = gemm_skinny_kernel<KIND, bf16, NT>;
+  auto kern = gemm_skinny_kernel<KIND, T, NT>;
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
@@ -539,19 +543,19 @@ static int launch_skinny_nt(const CUtensorMap& tw, const CUtensorMap& tx, int M,
                              stg, status);
   if (err == cudaSuccess && (KIND == EPI_QKV_ROPE || KIND == EPI_SWIGLU)) {
     const int items = M * ((N + 31) / 32);
-    err = launch_k(skinny_finalize_kernel<KIND, bf16>, dim3((items + 127) / 128), dim3(128), 0, st, e, stg);
+    err = launch_k(skinny_finalize_kernel<KIND, T>, dim3((items + 127) / 128), dim3(128), 0, st, e, stg);
   }
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
-template <int KIND>
+template <int KIND, typename T>
 static int launch_skinny(const CUtensorMap& tw, const CUtensorMap& tx, int M, int N, int K, int NT, const EpiArgs& e,
                          float* ws, int* tickets, float* stg, int* status, cudaStream_t st) {
   switch (NT) {
-    case 32: return launch_skinny_nt<KIND, 32>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
-    case 64: return launch_skinny_nt<KIND, 64>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
-    case 128: return launch_skinny_nt<KIND, 128>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
-    case 256: return launch_skinny_nt<KIND, 256>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
+    case 32: return launch_skinny_nt<KIND, T, 32>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
+    case 64: return launch_skinny_nt<KIND, T, 64>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
+    case 128: return launch_skinny_nt<KIND, T, 128>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
+    case 256: return launch_skinny_nt<KIND, T, 256>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
   }
   return LLAMA_ERR_INVALID_ARG;
 }
@@ -569,21 +573,23 @@ bool pdl_enabled() {
   return on;
 }
 
-int gemm_bf16(const bf16* A, int M, int K, int lda, const bf16* W, int N, int ldw, int kind, const EpiArgs& e,
-              int variant, GemmScratch* scratch, int* status, cudaStream_t st) {
+template <typename T>
+static int gemm16_t(const void* A, int M, int K, int lda, const void* W, int N, int ldw, int kind, const EpiArgs& e,
+                    int variant, GemmScratch* scratch, int* status, cudaStream_t st) {
+  constexpr bool F16 = std::is_same<T, f16>::value;
   if (M <= 0 || N <= 0 || K <= 0) return LLAMA_ERR_SHAPE;
   if (K % 8 != 0 || lda % 8 != 0 || ldw % 8 != 0) return LLAMA_ERR_SHAPE;
   const bool skinny = variant == GEMM_SKINNY || (variant == GEMM_AUTO && M <= 128);
   int rc;
   if (!skinny) {
     CUtensorMap ta, tb;
-    if ((rc = make_tmap_bf16(&ta, A, M, K, lda, W_BM)) != LLAMA_OK) return rc;
-    if ((rc = make_tmap_bf16(&tb, W, N, K, ldw, W_BN)) != LLAMA_OK) return rc;
+    if ((rc = make_tmap_16(&ta, A, M, K, lda, W_BM, F16)) != LLAMA_OK) return rc;
+    if ((rc = make_tmap_16(&tb, W, N, K, ldw, W_BN, F16)) != LLAMA_OK) return rc;
     switch (kind) {
-      case EPI_STORE_F32: return launch_wide<EPI_STORE_F32>(ta, tb, M, N, K, e, status, st);
-      case EPI_RESIDUAL: return launch_wide<EPI_RESIDUAL>(ta, tb, M, N, K, e, status, st);
-      case EPI_SWIGLU: return launch_wide<EPI_SWIGLU>(ta, tb, M, N, K, e, status, st);
-      case EPI_QKV_ROPE: return launch_wide<EPI_QKV_ROPE>(ta, tb, M, N, K, e, status, st);
+      case EPI_STORE_F32: return launch_wide<EPI_STORE_F32, T>(ta, tb, M, N, K, e, status, st);
+      case EPI_RESIDUAL: return launch_wide<EPI_RESIDUAL, T>(ta, tb, M, N, K, e, status, st);
+      case EPI_SWIGLU: return launch_wide<EPI_SWIGLU, T>(ta, tb, M, N, K, e, status, st);
+      case EPI_QKV_ROPE: return launch_wide<EPI_QKV_ROPE, T>(ta, tb, M, N, K, e, status, st);
     }
     return LLAMA_ERR_INVALID_ARG;
   }
@@ -596,16 +602,23 @@ int gemm_bf16(const bf16* A, int M, int K, int lda, const bf16* W, int N, int ld
   if ((kind == EPI_QKV_ROPE || kind == EPI_SWIGLU) && (!scratch->stg || scratch->stg_floats < (size_t)M * N))
     return LLAMA_ERR_INVALID_ARG;
   CUtensorMap tw, tx;
-  if ((rc = make_tmap_bf16(&tw, W, N, K, ldw, S_BM)) != LLAMA_OK) return rc;
-  if ((rc = make_tmap_bf16(&tx, A, M, K, lda, NT)) != LLAMA_OK) return rc;
+  if ((rc = make_tmap_16(&tw, W, N, K, ldw, S_BM, F16)) != LLAMA_OK) return rc;
+  if ((rc = make_tmap_16(&tx, A, M, K, lda, NT, F16)) != LLAMA_OK) return rc;
   float* ws = scratch->ws;
   int* tk = scratch->tickets;
   switch (kind) {
-    case EPI_STORE_F32: return launch_skinny<EPI_STORE_F32>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
-    case EPI_RESIDUAL: return launch_skinny<EPI_RESIDUAL>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
-    case EPI_SWIGLU: return launch_skinny<EPI_SWIGLU>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
-    case EPI_QKV_ROPE: return launch_skinny<EPI_QKV_ROPE>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
+    case EPI_STORE_F32: return launch_skinny<EPI_STORE_F32, T>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
+    case EPI_RESIDUAL: return launch_skinny<EPI_RESIDUAL, T>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
+    case EPI_SWIGLU: return launch_skinny<EPI_SWIGLU, T>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
+    case EPI_QKV_ROPE: return launch_skinny<EPI_QKV_ROPE, T>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
   }
+  return LLAMA_ERR_INVALID_ARG;
+}
+
+int gemm16(const void* A, int M, int K, int lda, const void* W, int N, int ldw, int elt, int kind, const EpiArgs& e,
+           int variant, GemmScratch* scratch, int* status, cudaStream_t st) {
+  if (elt == LLAMA_F16) return gemm16_t<f16>(A, M, K, lda, W, N, ldw, kind, e, variant, scratch, status, st);
+  if (elt == LLAMA_BF16) return gemm16_t<bf16>(A, M, K, lda, W, N, ldw, kind, e, variant, scratch, status, st);
   return LLAMA_ERR_INVALID_ARG;
 }
 

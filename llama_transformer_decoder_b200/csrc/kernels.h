@@ -48,16 +48,18 @@ struct GemmScratch {
 };
 
 int num_sms();
-int make_tmap_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t pitch, int box_rows);
+int make_tmap_16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t pitch, int box_rows,
+                 bool is_f16);
 // Scratch of the stream-K skinny GEMM for M rows: two partial tiles per CTA.
 size_t skinny_workspace_floats(int M);
 
-int gemm_bf16(const __nv_bfloat16* A, int M, int K, int lda, const __nv_bfloat16* W, int N, int ldw, int kind,
-              const EpiArgs& e, int variant, GemmScratch* scratch, int* status, cudaStream_t st);
+// 16-bit GEMM; elt = LLAMA_BF16 or LLAMA_F16 (element type of A, W and 16-bit outputs).
+int gemm16(const void* A, int M, int K, int lda, const void* W, int N, int ldw, int elt, int kind, const EpiArgs& e,
+           int variant, GemmScratch* scratch, int* status, cudaStream_t st);
 int gemm_f32(const float* A, int M, int K, int lda, const float* W, int N, int ldw, int kind, const EpiArgs& e,
              int* status, cudaStream_t st);
 
-// Elementwise / reductions. dtype: 0 = fp32, 1 = bf16 (of `y` / tables).
+// Elementwise / reductions. dtype: LLAMA_F32, LLAMA_BF16 or LLAMA_F16 (of `y` / tables).
 int launch_embed(const int32_t* tokens, int M, const void* table, int V, int D, int dtype, float* x, int* status,
                  cudaStream_t st);
 // y[r] = rmsnorm(x[row(r)]) * g; row(r) = r, or (r+1)*S-1 when last_of_S > 0.
@@ -70,9 +72,9 @@ int launch_add_lengths(int32_t* len, int B, int add, cudaStream_t st);
 // o [B*S][H*d]; pos0[b] = position of the call's first query (null = 0).
 int attention_prefill(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B, int S,
                       int H, int Hk, int d, int Smax, int dtype, int* status, cudaStream_t st);
-// tcgen05 flash attention for bf16, d = 128 (same arguments as attention_prefill).
+// tcgen05 flash attention for 16-bit q/k/v (elt = LLAMA_BF16 or LLAMA_F16), d = 128.
 int attention_prefill_tc(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B, int S,
-                         int H, int Hk, int Smax, int* status, cudaStream_t st);
+                         int H, int Hk, int Smax, int elt, int* status, cudaStream_t st);
 // Decode: q [B][H][d]; keys 0 .. nkeys[b]-1 (+ add) of the cache; o [B][H*d].
 struct DecodeScratch {
   float* part;  // [B][H][splits][d + 2]
@@ -91,8 +93,12 @@ struct FillLayout {
   int64_t outer_stride, row_stride;
   int row_mult, row_off;
 };
+// dtype: element type of dst; round_bf16 rounds each value to bf16 first (bf16
+// values kept in an fp16 buffer).
 int launch_fill_normal(void* dst, const FillLayout& L, uint64_t seed, uint64_t stream_id, float std, int dtype,
-                       cudaStream_t st);
+                       cudaStream_t st, bool round_bf16 = false);
+int launch_convert_2d(void* dst, int64_t dpitch, int dst_elt, const void* src, int64_t spitch, int src_elt,
+                      int64_t rows, int64_t cols, cudaStream_t st);
 int launch_fill_const(float* dst, int64_t n, float v, cudaStream_t st);
 int launch_fill_tokens(int32_t* dst, int64_t n, uint64_t seed, uint64_t stream_id, int vocab, cudaStream_t st);
 

@@ -57,6 +57,11 @@ struct llama_model {
   int dev = 0;
   int d = 0, F = 0, qkv_n = 0, Mmax = 0;
   size_t esz = 2;
+  // Element type of weights, activations and cache on the device. A bf16
+  // model keeps its bf16 weight values in fp16 storage and computes with fp16
+  // activations: fp16 has 3 more mantissa bits, which holds the logits of a
+  // 32-layer stack within 2e-2 of the exact result where bf16 activations do not.
+  int adt = LLAMA_F16;
   // weights
   void* wbase = nullptr;
   void* tok_emb = nullptr;
@@ -119,7 +124,7 @@ namespace {
 int resolve(const llama_config* in, llama_config* c) {
   if (!in) return LLAMA_ERR_INVALID_ARG;
   *c = *in;
-  if (c->dtype != LLAMA_F32 && c->dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+  if (c->dtype != LLAMA_F32 && c->dtype != LLAMA_BF16 && c->dtype != LLAMA_F16) return LLAMA_ERR_INVALID_ARG;
   if (c->dim <= 0 || c->n_layers <= 0 || c->n_heads <= 0 || c->n_kv_heads <= 0 || c->vocab_size <= 0 ||
       c->max_batch <= 0 || c->max_seq <= 0)
     return LLAMA_ERR_SHAPE;
@@ -131,7 +136,7 @@ int resolve(const llama_config* in, llama_config* c) {
     if (c->multiple_of <= 0) return LLAMA_ERR_SHAPE;
     c->ffn_hidden = llama_ffn_hidden(c->dim, c->multiple_of, c->ffn_dim_multiplier);
   }
-  if (c->dtype == LLAMA_BF16) {
+  if (c->dtype != LLAMA_F32) {
     if (d != 128) return LLAMA_ERR_UNSUPPORTED;
     if (c->dim % 64 != 0 || c->ffn_hidden % 64 != 0) return LLAMA_ERR_SHAPE;
   }
@@ -272,9 +277,8 @@ void mark(llama_model* m, int kind, cudaStream_t st) {
 // ---------------------------------------------------------------- forward
 int gemm(llama_model* m, const void* A, int M, int K, const void* W, int N, int kind, const EpiArgs& e,
          cudaStream_t st) {
-  if (m->cfg.dtype == LLAMA_BF16)
-    return gemm_bf16(static_cast<const bf16*>(A), M, K, K, static_cast<const bf16*>(W), N, K, kind, e, GEMM_AUTO,
-                     &m->gs, m->d_status, st);
+  if (m->adt != LLAMA_F32)
+    return gemm16(A, M, K, K, W, N, K, m->adt, kind, e, GEMM_AUTO, &m->gs, m->d_status, st);
   return gemm_f32(static_cast<const float*>(A), M, K, K, static_cast<const float*>(W), N, K, kind, e, m->d_status,
                   st);
 }
@@ -298,7 +302,7 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
   char* vc = static_cast<char*>(m->vcache) + (size_t)l * m->layer_cache_elems * m->esz;
 
   mark(m, K_RMSNORM, st);
-  RC(launch_rmsnorm(m->x, w.attn_norm, m->xn, M, D, c.norm_eps, 0, c.dtype, st));
+  RC(launch_rmsnorm(m->x, w.attn_norm, m->xn, M, D, c.norm_eps, 0, m->adt, st));
   EpiArgs e = epi_base(M, m->qkv_n);
   e.q = m->q;
   e.kc = kc;
@@ -314,11 +318,11 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
   RC(gemm(m, m->xn, M, D, w.wqkv, m->qkv_n, EPI_QKV_ROPE, e, st));
   if (decode) {
     mark(m, K_ATTN_DECODE, st);
-    RC(attention_decode(m->q, kc, vc, m->d_len, 1, m->attn, B, cmax, H, Hk, d, c.max_seq, c.dtype, &m->ds,
+    RC(attention_decode(m->q, kc, vc, m->d_len, 1, m->attn, B, cmax, H, Hk, d, c.max_seq, m->adt, &m->ds,
                         m->d_status, st));
   } else {
     mark(m, K_ATTN_PREFILL, st);
-    RC(attention_prefill(m->q, kc, vc, m->attn, m->d_len, B, S, H, Hk, d, c.max_seq, c.dtype, m->d_status, st));
+    RC(attention_prefill(m->q, kc, vc, m->attn, m->d_len, B, S, H, Hk, d, c.max_seq, m->adt, m->d_status, st));
   }
   EpiArgs r = epi_base(M, D);
   r.out = m->x;
@@ -326,7 +330,7 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
   mark(m, K_GEMM_WO, st);
   RC(gemm(m, m->attn, M, H * d, w.wo, D, EPI_RESIDUAL, r, st));
   mark(m, K_RMSNORM, st);
-  RC(launch_rmsnorm(m->x, w.ffn_norm, m->xn, M, D, c.norm_eps, 0, c.dtype, st));
+  RC(launch_rmsnorm(m->x, w.ffn_norm, m->xn, M, D, c.norm_eps, 0, m->adt, st));
   EpiArgs sg = epi_base(M, 2 * m->F);
   sg.g = m->g;
   sg.ldg = m->F;
@@ -341,7 +345,7 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
 int run_head(llama_model* m, int B, int S, cudaStream_t st) {
   const llama_config& c = m->cfg;
   mark(m, K_RMSNORM, st);
-  RC(launch_rmsnorm(m->x, m->norm_w, m->xn, B, c.dim, c.norm_eps, S, c.dtype, st));
+  RC(launch_rmsnorm(m->x, m->norm_w, m->xn, B, c.dim, c.norm_eps, S, m->adt, st));
   EpiArgs e = epi_base(B, c.vocab_size);
   e.out = m->logits;
   e.ldo = c.vocab_size;
@@ -353,7 +357,7 @@ int run_head(llama_model* m, int B, int S, cudaStream_t st) {
 
 int decode_body(llama_model* m, int B, int cmax, cudaStream_t st) {
   mark(m, K_EMBED, st);
-  RC(launch_embed(m->tok_buf, B, m->tok_emb, m->cfg.vocab_size, m->cfg.dim, m->cfg.dtype, m->x, m->d_status, st));
+  RC(launch_embed(m->tok_buf, B, m->tok_emb, m->cfg.vocab_size, m->cfg.dim, m->adt, m->x, m->d_status, st));
   for (int l = 0; l < m->cfg.n_layers; ++l) RC(run_layer(m, l, B, 1, true, cmax, st));
   RC(run_head(m, B, 1, st));
   mark(m, K_OTHER, st);
@@ -405,7 +409,8 @@ int llama_create(const llama_config* cfg, llama_model** out) {
   if (!m) return LLAMA_ERR_OOM;
   m->cfg = c;
   cudaGetDevice(&m->dev);
-  m->esz = c.dtype == LLAMA_BF16 ? 2 : 4;
+  m->esz = c.dtype == LLAMA_F32 ? 4 : 2;
+  m->adt = c.dtype == LLAMA_F32 ? LLAMA_F32 : LLAMA_F16;
   m->d = c.dim / c.n_heads;
   m->F = c.ffn_hidden;
   m->qkv_n = (c.n_heads + 2 * c.n_kv_heads) * m->d;
@@ -474,7 +479,7 @@ int llama_create(const llama_config* cfg, llama_model** out) {
     }
   }
   // ---- split-K scratch for every skinny GEMM shape the model can issue
-  if (c.dtype == LLAMA_BF16) {
+  if (m->adt != LLAMA_F32) {
     size_t ws = 0;
     int tickets = 0;
     const int shapes[5][2] = {{m->qkv_n, c.dim}, {c.dim, (int)Hd}, {2 * m->F, c.dim}, {c.dim, m->F}, {c.vocab_size, c.dim}};
@@ -495,7 +500,7 @@ int llama_create(const llama_config* cfg, llama_model** out) {
   {
     size_t need = 0;
     for (int B = 1; B <= c.max_batch; ++B)
-      need = std::max(need, decode_scratch_floats(c.max_seq, B, c.n_heads, c.n_kv_heads, m->d, c.dtype));
+      need = std::max(need, decode_scratch_floats(c.max_seq, B, c.n_heads, c.n_kv_heads, m->d, m->adt));
     if (grow_decode_scratch(&m->ds, need) != LLAMA_OK) { delete m; return LLAMA_ERR_OOM; }
     m->allocs.push_back(m->ds.part);
   }
@@ -538,7 +543,7 @@ int llama_init_weights(llama_model* m, uint64_t seed, float std, void* stream) {
     }
     // destination row r*row_mult; w3 rows start one row further through p.base
     const FillLayout fl{1, p.rows, p.cols, 0, p.cols, p.row_mult, 0};
-    RC(launch_fill_normal(p.base, fl, seed, p.stream, std, m->cfg.dtype, st));
+    RC(launch_fill_normal(p.base, fl, seed, p.stream, std, m->adt, st, m->cfg.dtype == LLAMA_BF16));
   }
   return LLAMA_OK;
 }
@@ -551,12 +556,37 @@ static int copy_weight(llama_model* m, const char* name, void* host_or_dev, size
   const size_t row_bytes = (size_t)p.cols * p.esz;
   if (nbytes != row_bytes * (size_t)p.rows) return LLAMA_ERR_SHAPE;
   const size_t model_pitch = row_bytes * p.row_mult;
+  cudaStream_t st = S_(stream);
+  if (m->cfg.dtype == LLAMA_BF16 && !p.is_norm) {
+    // bf16 in the caller's buffer, fp16 in the model: convert on the device.
+    void* dev = host_or_dev;
+    if (!on_device) {
+      if (cudaMalloc(&dev, nbytes) != cudaSuccess) { cudaGetLastError(); return LLAMA_ERR_OOM; }
+      if (to_model && cudaMemcpyAsync(dev, host_or_dev, nbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(dev);
+        return LLAMA_ERR_CUDA;
+      }
+    }
+    const int64_t mp = (int64_t)p.cols * p.row_mult;
+    int rc = to_model ? launch_convert_2d(p.base, mp, LLAMA_F16, dev, p.cols, LLAMA_BF16, p.rows, p.cols, st)
+                      : launch_convert_2d(dev, p.cols, LLAMA_BF16, p.base, mp, LLAMA_F16, p.rows, p.cols, st);
+    if (!on_device) {
+      if (rc == LLAMA_OK && !to_model &&
+          cudaMemcpyAsync(host_or_dev, dev, nbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        rc = LLAMA_ERR_CUDA;
+      if (cudaStreamSynchronize(st) != cudaSuccess) rc = LLAMA_ERR_CUDA;
+      cudaGetLastError();
+      cudaFree(dev);
+    }
+    return rc;
+  }
   cudaMemcpyKind kind = on_device ? cudaMemcpyDeviceToDevice : (to_model ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToHost);
   if (to_model)
-    CK(cudaMemcpy2DAsync(p.base, model_pitch, host_or_dev, row_bytes, row_bytes, p.rows, kind, S_(stream)));
+    CK(cudaMemcpy2DAsync(p.base, model_pitch, host_or_dev, row_bytes, row_bytes, p.rows, kind, st));
   else
-    CK(cudaMemcpy2DAsync(host_or_dev, row_bytes, p.base, model_pitch, row_bytes, p.rows, kind, S_(stream)));
-  if (!on_device) CK(cudaStreamSynchronize(S_(stream)));
+    CK(cudaMemcpy2DAsync(host_or_dev, row_bytes, p.base, model_pitch, row_bytes, p.rows, kind, st));
+  if (!on_device) CK(cudaStreamSynchronize(st));
   return LLAMA_OK;
 }
 
@@ -574,7 +604,7 @@ int llama_prefill(llama_model* m, const int32_t* tokens, int32_t B, int32_t S, v
   cudaStream_t st = S_(stream);
   const int M = B * S;
   mark(m, K_EMBED, st);
-  RC(launch_embed(tokens, M, m->tok_emb, m->cfg.vocab_size, m->cfg.dim, m->cfg.dtype, m->x, m->d_status, st));
+  RC(launch_embed(tokens, M, m->tok_emb, m->cfg.vocab_size, m->cfg.dim, m->adt, m->x, m->d_status, st));
   for (int l = 0; l < m->cfg.n_layers; ++l) RC(run_layer(m, l, B, S, false, 0, st));
   RC(run_head(m, B, S, st));
   mark(m, K_OTHER, st);
@@ -692,8 +722,9 @@ int llama_fill_kv_random(llama_model* m, uint64_t seed, int32_t c, void* stream)
   for (int l = 0; l < cf.n_layers; ++l) {
     char* kc = static_cast<char*>(m->kcache) + (size_t)l * m->layer_cache_elems * m->esz;
     char* vc = static_cast<char*>(m->vcache) + (size_t)l * m->layer_cache_elems * m->esz;
-    RC(launch_fill_normal(kc, fl, seed, kStreamKvBase + 2 * (uint64_t)l, 1.0f, cf.dtype, st));
-    RC(launch_fill_normal(vc, fl, seed, kStreamKvBase + 2 * (uint64_t)l + 1, 1.0f, cf.dtype, st));
+    const bool rb = cf.dtype == LLAMA_BF16;
+    RC(launch_fill_normal(kc, fl, seed, kStreamKvBase + 2 * (uint64_t)l, 1.0f, m->adt, st, rb));
+    RC(launch_fill_normal(vc, fl, seed, kStreamKvBase + 2 * (uint64_t)l + 1, 1.0f, m->adt, st, rb));
   }
   std::vector<int32_t> lens(cf.max_batch, c);
   return llama_set_lengths(m, lens.data(), cf.max_batch, stream);
@@ -707,6 +738,11 @@ int llama_set_kv(llama_model* m, int32_t layer, const void* k, const void* v, in
   const size_t rows = (size_t)B * m->cfg.n_kv_heads;
   char* kc = static_cast<char*>(m->kcache) + (size_t)layer * m->layer_cache_elems * m->esz;
   char* vc = static_cast<char*>(m->vcache) + (size_t)layer * m->layer_cache_elems * m->esz;
+  if (m->cfg.dtype == LLAMA_BF16) {  // bf16 from the caller, fp16 in the cache
+    const int64_t cols = (int64_t)c * m->d, dpe = (int64_t)m->cfg.max_seq * m->d;
+    RC(launch_convert_2d(kc, dpe, LLAMA_F16, k, cols, LLAMA_BF16, (int64_t)rows, cols, S_(stream)));
+    return launch_convert_2d(vc, dpe, LLAMA_F16, v, cols, LLAMA_BF16, (int64_t)rows, cols, S_(stream));
+  }
   CK(cudaMemcpy2DAsync(kc, dp, k, w, w, rows, cudaMemcpyDeviceToDevice, S_(stream)));
   CK(cudaMemcpy2DAsync(vc, dp, v, w, w, rows, cudaMemcpyDeviceToDevice, S_(stream)));
   return LLAMA_OK;
@@ -797,7 +833,7 @@ int llama_attention_prefill(const void* q, const void* k, const void* v, void* o
                             int32_t Hk, int32_t d, int32_t dtype, void* stream) {
   if (!q || !k || !v || !o) return LLAMA_ERR_INVALID_ARG;
   if (B <= 0 || S <= 0 || H <= 0 || Hk <= 0 || H % Hk != 0) return LLAMA_ERR_SHAPE;
-  if (dtype != LLAMA_F32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+  if (dtype != LLAMA_F32 && dtype != LLAMA_BF16 && dtype != LLAMA_F16) return LLAMA_ERR_INVALID_ARG;
   DevCtx* c = dev_ctx();
   if (!c) return LLAMA_ERR_OOM;
   return attention_prefill(q, k, v, o, nullptr, B, S, H, Hk, d, S, dtype, c->status, S_(stream));
@@ -807,7 +843,7 @@ int llama_attention_decode(const void* q, const void* kc, const void* vc, const 
                            int32_t cmax, int32_t H, int32_t Hk, int32_t d, int32_t dtype, void* stream) {
   if (!q || !kc || !vc || !len || !o) return LLAMA_ERR_INVALID_ARG;
   if (B <= 0 || cmax <= 0 || H <= 0 || Hk <= 0 || H % Hk != 0) return LLAMA_ERR_SHAPE;
-  if (dtype != LLAMA_F32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+  if (dtype != LLAMA_F32 && dtype != LLAMA_BF16 && dtype != LLAMA_F16) return LLAMA_ERR_INVALID_ARG;
   DevCtx* c = dev_ctx();
   if (!c) return LLAMA_ERR_OOM;
   RC(grow_decode_scratch(&c->ds, decode_scratch_floats(cmax, B, H, Hk, d, dtype)));
@@ -826,21 +862,20 @@ int llama_linear(const void* x, const void* w, float* y, int32_t M, int32_t N, i
   if (dtype == LLAMA_F32)
     return gemm_f32(static_cast<const float*>(x), M, K, K, static_cast<const float*>(w), N, K, EPI_STORE_F32, e,
                     c->status, S_(stream));
-  if (dtype != LLAMA_BF16 || variant < 0 || variant > 2) return LLAMA_ERR_INVALID_ARG;
+  if ((dtype != LLAMA_BF16 && dtype != LLAMA_F16) || variant < 0 || variant > 2) return LLAMA_ERR_INVALID_ARG;
   const bool skinny = variant == GEMM_SKINNY || (variant == GEMM_AUTO && M <= 128);
   if (skinny) {
     if (M > 256) return LLAMA_ERR_SHAPE;
     RC(grow_gemm_scratch(&c->gs, skinny_workspace_floats(M), (N + 127) / 128));
   }
-  return gemm_bf16(static_cast<const bf16*>(x), M, K, K, static_cast<const bf16*>(w), N, K, EPI_STORE_F32, e,
-                   variant, &c->gs, c->status, S_(stream));
+  return gemm16(x, M, K, K, w, N, K, dtype, EPI_STORE_F32, e, variant, &c->gs, c->status, S_(stream));
 }
 
 int llama_rmsnorm(const float* x, const float* g, void* y, int32_t M, int32_t D, float eps, int32_t dtype,
                   void* stream) {
   if (!x || !g || !y) return LLAMA_ERR_INVALID_ARG;
   if (M <= 0 || D <= 0) return LLAMA_ERR_SHAPE;
-  if (dtype != LLAMA_F32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+  if (dtype != LLAMA_F32 && dtype != LLAMA_BF16 && dtype != LLAMA_F16) return LLAMA_ERR_INVALID_ARG;
   return launch_rmsnorm(x, g, y, M, D, eps, 0, dtype, S_(stream));
 }
 
@@ -854,7 +889,7 @@ int llama_fill_normal(void* dst, int64_t n, uint64_t seed, uint64_t stream_id, f
                       void* stream) {
   if (!dst) return LLAMA_ERR_INVALID_ARG;
   if (n < 0) return LLAMA_ERR_SHAPE;
-  if (dtype != LLAMA_F32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+  if (dtype != LLAMA_F32 && dtype != LLAMA_BF16 && dtype != LLAMA_F16) return LLAMA_ERR_INVALID_ARG;
   FillLayout fl{1, 1, n, 0, n, 1, 0};
   return launch_fill_normal(dst, fl, seed, stream_id, std, dtype, S_(stream));
 }

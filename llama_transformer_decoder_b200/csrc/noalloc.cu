@@ -47,7 +47,7 @@ extern "C" int llama_attention_decode_noalloc(const void* q, const void* kc, con
                                               int32_t dtype, void* stream) {
   if (!q || !kc || !vc || !len || !o) return LLAMA_ERR_INVALID_ARG;
   if (B <= 0 || cmax <= 0 || H <= 0 || Hk <= 0 || H % Hk != 0) return LLAMA_ERR_SHAPE;
-  if (dtype != LLAMA_F32 && dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+  if (dtype != LLAMA_F32 && dtype != LLAMA_BF16 && dtype != LLAMA_F16) return LLAMA_ERR_INVALID_ARG;
   const size_t need = llama::decode_scratch_floats(cmax, B, H, Hk, d, dtype);
   if (need * sizeof(float) > kScratchBytes) return LLAMA_ERR_SHAPE;
   float* scratch = nullptr;

@@ -262,12 +262,16 @@ class Oracle:
         """Tokens [S] of one sequence, appended after the cache's current length.
 
         Returns the logits of the last token ([vocab]) and, if asked, the final
-        hidden states before the last norm ([S, dim]).
+        hidden states before the last norm ([S, dim]). Without return_hidden the
+        last layer evaluates only the last row (its keys and values are still
+        computed for every row).
         """
         pos0 = 0 if cache is None else cache.length
         x = self.embed(tokens)
+        S = x.shape[0]
         for i in range(self.p.n_layers):
-            x = self.layer(i, x, cache, pos0)
+            last_only = not return_hidden and i == self.p.n_layers - 1
+            x = self.layer(i, x, cache, pos0, rows=np.array([S - 1]) if last_only else None)
         lg = self.logits(x[-1])
         return (lg, x) if return_hidden else lg
 

@@ -8,7 +8,7 @@ import numpy as np
 import seeded_inputs as si
 from oracle import Params
 
-BF16, F32 = 1, 0
+BF16, F32, F16 = 1, 0, 2
 
 
 def params_from(cfg: dict, ffn_hidden: int) -> Params:
@@ -19,7 +19,7 @@ def params_from(cfg: dict, ffn_hidden: int) -> Params:
 
 class SeededWeights(dict):
     """Checkpoint-named weights of ``llama_init_weights(seed, std)``, generated on
-    the host on first use (float32 values of the exact bf16 or fp32 draws)."""
+    the host on first use (float32 values of the exact bf16, fp16 or fp32 draws)."""
 
     def __init__(self, p: Params, seed: int, std: float, dtype: int, cache: bool = True):
         super().__init__()
@@ -30,6 +30,8 @@ class SeededWeights(dict):
         shape = si.weight_shape(name, p.dim, p.n_heads, p.n_kv_heads, p.ffn_hidden, p.vocab_size)
         if name.endswith('norm.weight'):
             v = np.ones(shape, np.float32)
+        elif self.dtype == F16:
+            v = si.weight(self.seed, name, shape, p.n_layers, self.std, 'f32').astype(np.float16).astype(np.float32)
         else:
             raw = si.weight(self.seed, name, shape, p.n_layers, self.std, 'bf16' if self.dtype == BF16 else 'f32')
             v = si.bf16_bits_to_f32(raw) if self.dtype == BF16 else raw
@@ -39,17 +41,28 @@ class SeededWeights(dict):
 
 
 def normal_values(seed: int, stream: int, shape, dtype: int, std: float = 1.0):
-    """(host float32 values, raw array for upload: uint16 bf16 bits or float32)."""
+    """(host float32 values, raw array for upload: uint16 bf16 bits, float16 or
+    float32). fp16 inputs are the fp32 draws rounded to nearest-even fp16."""
     n = int(np.prod(shape))
+    if dtype == F16:
+        raw = si.normal(seed, stream, n, std, 'f32').reshape(shape).astype(np.float16)
+        return raw.astype(np.float32), raw
     raw = si.normal(seed, stream, n, std, 'bf16' if dtype == BF16 else 'f32').reshape(shape)
     vals = si.bf16_bits_to_f32(raw) if dtype == BF16 else raw
     return vals, raw
+
+
+def torch_dtype(dtype: int):
+    import torch
+    return {BF16: torch.bfloat16, F16: torch.float16, F32: torch.float32}[dtype]
 
 
 def to_device(raw: np.ndarray, dtype: int):
     import torch
     if dtype == BF16:
         t = torch.from_numpy(raw.view(np.int16).copy()).view(torch.bfloat16)
+    elif dtype == F16:
+        t = torch.from_numpy(np.ascontiguousarray(raw, dtype=np.float16))
     else:
         t = torch.from_numpy(np.ascontiguousarray(raw, dtype=np.float32))
     return t.cuda()

@@ -1,0 +1,128 @@
+"""Parity at the full 8B shapes, in the configuration bench.py times.
+
+* Full 32-layer prefill, B = 8 sequences of 2048 seeded token ids: the
+  last-token logits of sequences 0 and 7 against the float32 oracle (the
+  sequences are independent, so checking two of them is exact for those two);
+  B = 1 on the same tokens must agree with sequence 0 of the batch.
+* Batch-32 decode over a 4096-token cache of N(0,1) K/V entries, 128 greedy
+  steps replayed from a CUDA graph on a stream: sequences 0 and 31 are
+  teacher-forced through the oracle (one causal pass over the tokens the GPU
+  chose, after the same cache).
+
+Tolerances: rel-L2 <= 2e-2 on logits; the GPU's greedy token must be the
+oracle's argmax or within the observed logit error of its maximum.
+The oracle runs in float32 here (its float64 twin agrees to ~1e-6, far inside
+the tolerance) to keep the 32-layer passes within about a minute each.
+"""
+import numpy as np
+import pytest
+
+import seeded_inputs as si
+from oracle import Oracle, SequenceCache
+from tests.helpers import BF16, SeededWeights, near_tie_ok, params_from, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip('torch')
+if not torch.cuda.is_available():  # pragma: no cover
+    pytest.skip('needs a CUDA device', allow_module_level=True)
+
+from llama_transformer_decoder_b200 import binding as L  # noqa: E402
+from llama_transformer_decoder_b200.configs import LLAMA3_8B, make_config  # noqa: E402
+
+S_PREFILL, B_PREFILL = 2048, 8
+B_DEC, CTX, STEPS = 32, 4096, 128
+V = 128256
+
+
+@pytest.fixture(scope='module')
+def model8b():
+    cfg = make_config(LLAMA3_8B, dtype=BF16, max_batch=B_DEC, max_seq=CTX + STEPS + 8,
+                      max_tokens=B_PREFILL * S_PREFILL)
+    h = L.llama_create(cfg)
+    L.llama_init_weights(h, 0, 0.02)
+    rc = L.llama_get_config(h)
+    p = params_from(LLAMA3_8B, rc.ffn_hidden)
+    w = SeededWeights(p, 0, 0.02, BF16)
+    for name in si.weight_names(p.n_layers):
+        w[name]                       # host copies, generated once
+    yield h, p, w
+    L.llama_destroy(h)
+
+
+def _logits(h, B):
+    out = torch.empty((B, V), device='cuda')
+    L.llama_logits(h, out)
+    return out.cpu().numpy()
+
+
+def test_8b_prefill_batch8_s2048(model8b):
+    h, p, w = model8b
+    toks = si.tokens(1, B_PREFILL * S_PREFILL, V).reshape(B_PREFILL, S_PREFILL)
+    L.llama_reset(h)
+    L.llama_prefill(h, torch.from_numpy(toks).cuda(), B_PREFILL, S_PREFILL)
+    got8 = _logits(h, B_PREFILL)
+    arg8 = torch.empty(B_PREFILL, dtype=torch.int32, device='cuda')
+    L.llama_argmax(h, arg8)
+    arg8 = arg8.cpu().numpy()
+    L.llama_reset(h)
+    L.llama_prefill(h, torch.from_numpy(np.ascontiguousarray(toks[:1])).cuda(), 1, S_PREFILL)
+    got1 = _logits(h, 1)
+    assert L.llama_sync_status(h) == 0
+    orc = Oracle(p, w, dtype=np.float32)
+    for b in (0, B_PREFILL - 1):
+        ref = orc.forward(toks[b])
+        err = rel_l2(got8[b], ref)
+        print(f'sequence {b}: rel-L2 {err:.3e}, gpu argmax {arg8[b]}, oracle argmax {int(np.argmax(ref))}')
+        assert err < 2e-2
+        assert near_tie_ok(int(arg8[b]), ref, 2 * float(np.max(np.abs(got8[b] - ref))) + 1e-6)
+    assert rel_l2(got1[0], got8[0]) < 5e-3          # batch size does not change a sequence's result
+
+
+def test_8b_decode_batch32_ctx4096_graph(model8b):
+    h, p, w = model8b
+    st = torch.cuda.Stream()
+    watch = (0, B_DEC - 1)
+    toks, rows = [], []
+    with torch.cuda.stream(st):       # torch's reads of lg / arg are ordered after the library's writes
+        L.llama_fill_kv_random(h, 3, CTX, st)
+        cur = torch.from_numpy(si.tokens(1, B_DEC, V, start=B_PREFILL * S_PREFILL)).cuda()
+        arg = torch.empty(B_DEC, dtype=torch.int32, device='cuda')
+        lg = torch.empty((B_DEC, V), device='cuda')
+        for step in range(STEPS):
+            toks.append(cur.cpu().numpy().copy())
+            L.llama_decode_step(h, cur, B_DEC, st)
+            L.llama_logits(h, lg, st)
+            L.llama_argmax(h, arg, st)
+            rows.append(lg[list(watch)].cpu().numpy())
+            cur = arg.clone()
+    torch.cuda.synchronize()
+    assert L.llama_sync_status(h, st) == 0
+    lens = np.zeros(B_DEC, np.int32)
+    L.llama_get_lengths(h, lens, B_DEC)
+    assert np.all(lens == CTX + STEPS)
+    # oracle: the same N(0,1) cache slices for the watched sequences, then teacher forcing
+    orc = Oracle(p, w, dtype=np.float32)
+    d, Hk = p.head_dim, p.n_kv_heads
+    n = Hk * CTX * d
+    worst = 0.0
+    for wi, b in enumerate(watch):
+        cache = SequenceCache()
+        for layer in range(p.n_layers):
+            k = si.normal(3, si.STREAM_KV_BASE + 2 * layer, n, 1.0, 'bf16', start=b * n)
+            v = si.normal(3, si.STREAM_KV_BASE + 2 * layer + 1, n, 1.0, 'bf16', start=b * n)
+            cache.k.append(si.bf16_bits_to_f32(k).reshape(Hk, CTX, d))
+            cache.v.append(si.bf16_bits_to_f32(v).reshape(Hk, CTX, d))
+        # Teacher forcing = one causal pass over the 128 tokens the GPU consumed:
+        # row i of that pass sees the cache plus tokens 0..i, exactly decode step i.
+        seq = np.array([toks[step][b] for step in range(STEPS)])
+        _, hidden = orc.forward(seq, cache, return_hidden=True)
+        refs = orc.logits(hidden)
+        for step in range(STEPS):
+            ref, got = refs[step], rows[step][wi]
+            err = rel_l2(got, ref)
+            worst = max(worst, err)
+            assert err < 2e-2, (b, step, err)
+            if step + 1 < STEPS:
+                assert near_tie_ok(int(toks[step + 1][b]), ref, 2 * float(np.max(np.abs(got - ref))) + 1e-6)
+    print(f'decode: worst logits rel-L2 over {STEPS} steps x {len(watch)} sequences: {worst:.3e}')

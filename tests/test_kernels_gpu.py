@@ -6,7 +6,7 @@ import pytest
 
 import seeded_inputs as si
 from oracle import argmax, attention, rms_norm
-from tests.helpers import BF16, F32, normal_values, rel_l2, to_device
+from tests.helpers import BF16, F16, F32, normal_values, rel_l2, to_device, torch_dtype
 
 pytestmark = pytest.mark.gpu
 
@@ -22,17 +22,21 @@ def _sync_ok():
 
 
 # ----------------------------------------------------------- generator
-@pytest.mark.parametrize('dtype', [BF16, F32])
+@pytest.mark.parametrize('dtype', [BF16, F16, F32])
 def test_device_generator_matches_host(dtype):
     n = 3_000_017
     for seed, stream, std in [(0, 1, 0.02), (7, 123456, 1.0), (1, 2 ** 21 + 5, 1.0)]:
-        t = torch.empty(n, dtype=torch.bfloat16 if dtype == BF16 else torch.float32, device='cuda')
+        t = torch.empty(n, dtype=torch_dtype(dtype), device='cuda')
         L.llama_fill_normal(t, n, seed, stream, std, dtype)
         torch.cuda.synchronize()
-        host = si.normal(seed, stream, n, std, 'bf16' if dtype == BF16 else 'f32')
-        dev = t.view(torch.int16).cpu().numpy().view(np.uint16) if dtype == BF16 else t.cpu().numpy()
-        assert np.array_equal(dev.view(np.uint16 if dtype == BF16 else np.uint32),
-                              host.view(np.uint16 if dtype == BF16 else np.uint32))
+        if dtype == BF16:
+            host = si.normal(seed, stream, n, std, 'bf16')
+        elif dtype == F16:
+            host = si.normal(seed, stream, n, std, 'f32').astype(np.float16).view(np.uint16)
+        else:
+            host = si.normal(seed, stream, n, std, 'f32').view(np.uint32)
+        dev = t.view(torch.int16 if dtype != F32 else torch.int32).cpu().numpy()
+        assert np.array_equal(dev.view(host.dtype), host)
     _sync_ok()
 
 
@@ -51,19 +55,20 @@ GEMM_CASES = [
 ]
 
 
+@pytest.mark.parametrize('dtype', [BF16, F16])
 @pytest.mark.parametrize('M,N,K,variant', GEMM_CASES)
-def test_linear_bf16(M, N, K, variant):
-    xv, xr = normal_values(11, 1, (M, K), BF16)
-    wv, wr = normal_values(11, 2, (N, K), BF16, std=0.02)
+def test_linear_16bit(M, N, K, variant, dtype):
+    xv, xr = normal_values(11, 1, (M, K), dtype)
+    wv, wr = normal_values(11, 2, (N, K), dtype, std=0.02)
     y = torch.full((M, N), float('nan'), device='cuda')
-    L.llama_linear(to_device(xr, BF16), to_device(wr, BF16), y, M, N, K, BF16, variant)
+    L.llama_linear(to_device(xr, dtype), to_device(wr, dtype), y, M, N, K, dtype, variant)
     torch.cuda.synchronize()
     _sync_ok()
     ref = xv.astype(np.float64) @ wv.astype(np.float64).T
     got = y.cpu().numpy()
     assert np.all(np.isfinite(got))
     assert rel_l2(got, ref) < 1e-5
-    # fp32 accumulation of exact bf16 products: per element |err| << 1e-3 * |row scale|
+    # fp32 accumulation of exact 16-bit products: per element |err| << 1e-3 * |row scale|
     scale = np.sqrt((xv.astype(np.float64) ** 2).sum(1, keepdims=True) * (wv.astype(np.float64) ** 2).sum(1)[None, :])
     assert np.max(np.abs(got - ref) / scale) < 1e-5
 
@@ -94,16 +99,16 @@ def test_linear_f32(M, N, K):
 
 
 # ------------------------------------------------------------ RMSNorm
-@pytest.mark.parametrize('dtype', [BF16, F32])
+@pytest.mark.parametrize('dtype', [BF16, F16, F32])
 @pytest.mark.parametrize('M,D', [(1, 4096), (37, 4096), (5, 256), (3, 100)])
 def test_rmsnorm(dtype, M, D):
     xv, xr = normal_values(14, 1, (M, D), F32)
     g = np.linspace(0.5, 1.5, D).astype(np.float32)
-    y = torch.empty((M, D), dtype=torch.bfloat16 if dtype == BF16 else torch.float32, device='cuda')
+    y = torch.empty((M, D), dtype=torch_dtype(dtype), device='cuda')
     L.llama_rmsnorm(to_device(xr, F32), torch.from_numpy(g).cuda(), y, M, D, 1e-5, dtype)
     ref = rms_norm(xv.astype(np.float64), g.astype(np.float64), 1e-5)
     got = y.float().cpu().numpy()
-    assert rel_l2(got, ref) < (4e-3 if dtype == BF16 else 1e-6)
+    assert rel_l2(got, ref) < {BF16: 4e-3, F16: 5e-4, F32: 1e-6}[dtype]
     _sync_ok()
 
 
@@ -122,22 +127,28 @@ def test_argmax_rows_exact_with_ties():
 
 
 # ----------------------------------------------------- prefill attention
-@pytest.mark.parametrize('B,S,H,Hk', [(2, 200, 8, 2), (1, 1, 4, 1), (1, 64, 4, 4), (1, 65, 8, 2),
-                                      (1, 2048, 32, 8), (2, 300, 32, 8), (1, 4097, 8, 2), (3, 129, 4, 1)])
-def test_attention_prefill_bf16(B, S, H, Hk):
+PREFILL_CASES = [(BF16, 2, 200, 8, 2), (BF16, 1, 1, 4, 1), (BF16, 1, 64, 4, 4), (BF16, 1, 65, 8, 2),
+                 (BF16, 1, 2048, 32, 8), (BF16, 2, 300, 32, 8), (BF16, 1, 4097, 8, 2), (BF16, 3, 129, 4, 1),
+                 (F16, 2, 200, 8, 2), (F16, 1, 1, 4, 1), (F16, 1, 2048, 32, 8), (F16, 1, 4097, 8, 2),
+                 (F16, 3, 129, 4, 1)]
+
+
+@pytest.mark.parametrize('dtype,B,S,H,Hk', PREFILL_CASES)
+def test_attention_prefill_16bit(dtype, B, S, H, Hk):
     d = 128
-    qv, qr = normal_values(16, 1, (B, H, S, d), BF16)
-    kv, kr = normal_values(16, 2, (B, Hk, S, d), BF16)
-    vv, vr = normal_values(16, 3, (B, Hk, S, d), BF16)
-    o = torch.empty((B, S, H * d), dtype=torch.bfloat16, device='cuda')
-    L.llama_attention_prefill(to_device(qr, BF16), to_device(kr, BF16), to_device(vr, BF16), o, B, S, H, Hk, d, BF16)
+    qv, qr = normal_values(16, 1, (B, H, S, d), dtype)
+    kv, kr = normal_values(16, 2, (B, Hk, S, d), dtype)
+    vv, vr = normal_values(16, 3, (B, Hk, S, d), dtype)
+    o = torch.empty((B, S, H * d), dtype=torch_dtype(dtype), device='cuda')
+    L.llama_attention_prefill(to_device(qr, dtype), to_device(kr, dtype), to_device(vr, dtype), o, B, S, H, Hk, d,
+                              dtype)
     torch.cuda.synchronize()
     _sync_ok()
     got = o.float().cpu().numpy()
     rows = np.arange(S) if S <= 512 else np.unique(np.r_[np.arange(0, S, 37), S - 1])
     for b in range(B):
         ref = attention(qv[b][:, rows].astype(np.float64), kv[b].astype(np.float64), vv[b].astype(np.float64), rows)
-        assert rel_l2(got[b][rows], ref) < 1e-2
+        assert rel_l2(got[b][rows], ref) < (1e-2 if dtype == BF16 else 2e-3)
 
 
 @pytest.mark.parametrize('d', [32, 128])
@@ -163,6 +174,11 @@ def test_attention_prefill_f32(d):
     (BF16, 128, 32, 32, 8, 4224, [4097 + 4 * i for i in range(32)]),   # batch-32 decode shape
     (BF16, 128, 1, 32, 8, 131072, [131072]),                 # longest cache of the sweep
     (BF16, 128, 64, 32, 8, 1024, [1 + 16 * i for i in range(64)]),
+    (BF16, 64, 2, 8, 2, 300, [17, 300]),
+    (F16, 128, 3, 32, 8, 1000, [1, 517, 1000]),
+    (F16, 128, 32, 32, 8, 4224, [4097 + 4 * i for i in range(32)]),
+    (F16, 128, 2, 16, 2, 300, [300, 45]),
+    (F16, 64, 2, 8, 2, 300, [17, 300]),
     (F32, 32, 2, 8, 2, 300, [17, 300]),
     (F32, 128, 1, 4, 1, 64, [64]),
 ])
@@ -171,7 +187,7 @@ def test_attention_decode(dtype, d, B, H, Hk, cmax, lens):
     kv, kr = normal_values(18, 2, (B, Hk, cmax, d), dtype)
     vv, vr = normal_values(18, 3, (B, Hk, cmax, d), dtype)
     ln = torch.tensor(lens, dtype=torch.int32, device='cuda')
-    o = torch.empty((B, H * d), dtype=torch.bfloat16 if dtype == BF16 else torch.float32, device='cuda')
+    o = torch.empty((B, H * d), dtype=torch_dtype(dtype), device='cuda')
     L.llama_attention_decode(to_device(qr, dtype), to_device(kr, dtype), to_device(vr, dtype), ln, o, B, cmax, H, Hk,
                              d, dtype)
     torch.cuda.synchronize()
@@ -181,7 +197,7 @@ def test_attention_decode(dtype, d, B, H, Hk, cmax, lens):
         n = lens[b]
         ref = attention(qv[b][:, None, :].astype(np.float64), kv[b][:, :n].astype(np.float64),
                         vv[b][:, :n].astype(np.float64), np.array([n - 1]))[0]
-        assert rel_l2(got[b], ref) < (1e-2 if dtype == BF16 else 1e-5)
+        assert rel_l2(got[b], ref) < {BF16: 1e-2, F16: 2e-3, F32: 1e-5}[dtype]
 
 
 def test_attention_decode_few_tiles_after_many():

@@ -5,7 +5,8 @@ import pytest
 
 import seeded_inputs as si
 from oracle import Oracle, argmax
-from tests.helpers import BF16, F32, SeededWeights, near_tie_ok, normal_values, params_from, rel_l2
+from tests.helpers import (BF16, F16, F32, SeededWeights, near_tie_ok, normal_values, params_from, rel_l2,
+                           to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -30,14 +31,14 @@ class Model:
             L.llama_destroy(self.h)
             self.h = None
 
-    def logits(self, B):
+    def logits(self, B, stream=None):
         out = torch.empty((B, self.rc.vocab_size), device='cuda')
-        L.llama_logits(self.h, out)
+        L.llama_logits(self.h, out, stream)
         return out
 
-    def argmax(self, B):
+    def argmax(self, B, stream=None):
         out = torch.empty(B, dtype=torch.int32, device='cuda')
-        L.llama_argmax(self.h, out)
+        L.llama_argmax(self.h, out, stream)
         return out
 
 
@@ -161,30 +162,32 @@ SMALL_BF16 = dict(dim=512, n_layers=3, n_heads=4, n_kv_heads=2, vocab_size=3000,
                   norm_eps=1e-5, rope_theta=500000.0)
 
 
-@pytest.mark.parametrize('B,S', [(3, 40), (2, 100)])
-def test_small_bf16_model_prefill_decode(B, S):
-    """3-layer bf16 model: prefill through the skinny (M <= 128) or wide GEMM
+@pytest.mark.parametrize('dtype,B,S', [(BF16, 3, 40), (BF16, 2, 100), (F16, 2, 100)])
+def test_small_16bit_model_prefill_decode(dtype, B, S):
+    """3-layer 16-bit model: prefill through the skinny (M <= 128) or wide GEMM
     path, then 6 decode steps (graph-replayed from the third); teacher-forced
     oracle, rel-L2 <= 2e-2 on every logits row."""
-    m = Model(SMALL_BF16, BF16, max_batch=4, max_seq=256)
+    m = Model(SMALL_BF16, dtype, max_batch=4, max_seq=256)
     try:
         L.llama_init_weights(m.h, 3, 0.02)
-        orc = Oracle(m.p, SeededWeights(m.p, 3, 0.02, BF16))
+        orc = Oracle(m.p, SeededWeights(m.p, 3, 0.02, dtype))
         toks = si.tokens(1, B * S, 3000).reshape(B, S)
-        L.llama_prefill(m.h, torch.from_numpy(toks).cuda(), B, S)
-        ref, caches = orc.prefill(toks)
-        got = m.logits(B).cpu().numpy()
-        assert rel_l2(got, ref) < 2e-2
-        for step in range(6):
-            nxt = m.argmax(B)
-            tn = nxt.cpu().numpy()
-            slack = 4 * float(np.max(np.abs(got - ref))) + 1e-6
-            for b in range(B):
-                assert near_tie_ok(int(tn[b]), ref[b], slack)
-            L.llama_decode_step(m.h, nxt, B)
-            ref = orc.decode_step(tn, caches)
-            got = m.logits(B).cpu().numpy()
-            assert rel_l2(got, ref) < 2e-2, step
+        st = torch.cuda.Stream()        # graphs are captured on non-default streams only
+        with torch.cuda.stream(st):
+            L.llama_prefill(m.h, torch.from_numpy(toks).cuda(), B, S, st)
+            ref, caches = orc.prefill(toks)
+            got = m.logits(B, st).cpu().numpy()
+            assert rel_l2(got, ref) < 2e-2
+            for step in range(6):
+                nxt = m.argmax(B, st)
+                tn = nxt.cpu().numpy()
+                slack = 4 * float(np.max(np.abs(got - ref))) + 1e-6
+                for b in range(B):
+                    assert near_tie_ok(int(tn[b]), ref[b], slack)
+                L.llama_decode_step(m.h, nxt, B, st)
+                ref = orc.decode_step(tn, caches)
+                got = m.logits(B, st).cpu().numpy()
+                assert rel_l2(got, ref) < 2e-2, step
         _check_status(m)
     finally:
         m.close()
@@ -207,6 +210,66 @@ def test_chunked_prefill_continues_the_cache():
         lens = np.zeros(2, np.int32)
         L.llama_get_lengths(m.h, lens, 2)
         assert list(lens) == [330, 330]
+        _check_status(m)
+    finally:
+        m.close()
+
+
+def test_bf16_weights_and_cache_round_trip():
+    """A bf16 model holds its weights as fp16: set/get return the caller's bf16
+    bits wherever fp16 represents them exactly (|w| >= 2^-14), and within 2^-25
+    below that."""
+    m = Model(SMALL_BF16, BF16, max_batch=2, max_seq=64)
+    try:
+        name = 'layers.1.feed_forward.w3.weight'
+        shape = (m.rc.ffn_hidden, 512)
+        vals, raw = normal_values(21, 5, shape, BF16, std=0.02)
+        raw = raw.copy()
+        raw.flat[:4] = si.f32_to_bf16_bits(np.array([1e-6, -3e-7, 7e-5, 60000.0], np.float32))
+        vals = si.bf16_bits_to_f32(raw)
+        L.llama_set_weight(m.h, name, raw, raw.nbytes, 0)
+        back = np.empty_like(raw)
+        L.llama_get_weight(m.h, name, back, back.nbytes, 0)
+        got = si.bf16_bits_to_f32(back)
+        big = np.abs(vals) >= 2.0 ** -14
+        assert np.array_equal(back[big], raw[big])
+        assert np.max(np.abs(got[~big] - vals[~big])) <= 2.0 ** -25
+        dev = torch.from_numpy(raw.view(np.int16).copy()).cuda()
+        out = torch.empty_like(dev)
+        L.llama_set_weight(m.h, name, dev, raw.nbytes, 1)
+        L.llama_get_weight(m.h, name, out, raw.nbytes, 1)
+        assert np.array_equal(out.cpu().numpy().view(np.uint16)[big], raw[big])
+        _check_status(m)
+    finally:
+        m.close()
+
+
+def test_set_kv_then_decode():
+    """llama_set_kv loads caller K/V (bf16, [B][Hk][c][d]) into every layer;
+    one decode step then attends to exactly those entries (teacher-forced
+    oracle holding the same cache)."""
+    from oracle import SequenceCache
+    B, c = 2, 37
+    m = Model(SMALL_BF16, BF16, max_batch=2, max_seq=64)
+    try:
+        L.llama_init_weights(m.h, 5, 0.02)
+        p = m.p
+        Hk, d = p.n_kv_heads, p.head_dim
+        caches = [SequenceCache() for _ in range(B)]
+        for layer in range(p.n_layers):
+            kv_, kr = normal_values(40 + layer, 1, (B, Hk, c, d), BF16)
+            vv_, vr = normal_values(40 + layer, 2, (B, Hk, c, d), BF16)
+            L.llama_set_kv(m.h, layer, to_device(kr, BF16), to_device(vr, BF16), B, c)
+            for b in range(B):
+                caches[b].k.append(kv_[b].astype(np.float64))
+                caches[b].v.append(vv_[b].astype(np.float64))
+        L.llama_set_lengths(m.h, np.full(B, c, np.int32), B)
+        toks = np.array([11, 2900], np.int32)
+        L.llama_decode_step(m.h, torch.from_numpy(toks).cuda(), B)
+        got = m.logits(B).cpu().numpy()
+        orc = Oracle(p, SeededWeights(p, 5, 0.02, BF16))
+        ref = np.stack([orc.forward(toks[b:b + 1], caches[b]) for b in range(B)])
+        assert rel_l2(got, ref) < 2e-2
         _check_status(m)
     finally:
         m.close()
