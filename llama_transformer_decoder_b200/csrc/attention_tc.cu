@@ -3,8 +3,11 @@
 //
 // One CTA computes 128 queries of one head. Warp roles: warp 0 issues TMA
 // loads (Q once, then K and V tiles of 128 keys into a 2-stage ring), warp 1
-// allocates TMEM and issues tcgen05.mma, warps 2-5 own one query row per
-// thread for the softmax and the final normalisation.
+// allocates TMEM and issues tcgen05.mma, warps 2-9 run the softmax: query row
+// r belongs to two threads, one in warps 2-5 (keys 0-63 of each tile, output
+// columns 0-63) and one in warps 6-9 (keys 64-127, columns 64-127), which
+// exchange their row maxima through shared memory once per tile and their
+// partial row sums once at the end.
 //
 //   S_j = Q K_j^T      -> TMEM (two 128-column buffers, so S_{j+1} is computed
 //                         while the softmax works on S_j)
@@ -38,7 +41,8 @@ constexpr int FA_OFF_Q = 0;
 constexpr int FA_OFF_K = FA_OFF_Q + FA_Q_BYTES;
 constexpr int FA_OFF_V = FA_OFF_K + FA_STAGES * FA_KV_BYTES;
 constexpr int FA_OFF_P = FA_OFF_V + FA_STAGES * FA_KV_BYTES;
-constexpr int FA_OFF_BAR = FA_OFF_P + FA_Q_BYTES;
+constexpr int FA_OFF_RED = FA_OFF_P + FA_Q_BYTES;     // row maxima [2 slots][2 halves][128], sums [2][128]
+constexpr int FA_OFF_BAR = FA_OFF_RED + 6 * 128 * 4;
 constexpr int FA_SMEM = FA_OFF_BAR + 256 + 1024;
 constexpr uint32_t FA_TMEM_O = 0, FA_TMEM_S = 128;   // S buffers at columns 128 and 256
 constexpr float FA_RESCALE = 8.0f;                    // raise the running max only past +8 (log2)
@@ -55,8 +59,10 @@ __device__ __forceinline__ uint8_t* fa_align(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+constexpr int FA_THREADS = 320;
+
 template <typename T>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(FA_THREADS, 1)
     attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, T* __restrict__ o,
                            const int32_t* __restrict__ pos0, int S, int H, int Hk, float scale_log2, int* status) {
@@ -64,13 +70,15 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* smem = fa_align(fa_smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + FA_OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;    // [2]
-  uint64_t* kv_empty = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;     // [2]
-  uint64_t* p_full = bars + 7;
-  uint64_t* o_done = bars + 8;
-  uint64_t* drain = bars + 9;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  uint64_t* k_full = bars + 1;     // [2]
+  uint64_t* k_empty = bars + 3;    // [2] released once S = Q K^T has read the tile
+  uint64_t* v_full = bars + 5;     // [2]
+  uint64_t* v_empty = bars + 7;    // [2] released once O += P V has read the tile
+  uint64_t* s_full = bars + 9;     // [2]
+  uint64_t* p_full = bars + 11;
+  uint64_t* o_done = bars + 12;
+  uint64_t* drain = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Linear block order is longest-first across all heads and sequences
@@ -86,8 +94,12 @@ __global__ void __launch_bounds__(192, 1)
   pdl_trigger();
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); mbar_init(&s_full[i], 1); }
-    mbar_init(p_full, 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+    }
+    mbar_init(p_full, 256);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -111,24 +123,30 @@ __global__ void __launch_bounds__(192, 1)
     mbar_arrive_expect_tx(q_full, FA_Q_BYTES);
     tma_load_3d(smem + FA_OFF_Q, &tmQ, q_full, 0, q0, b * H + h);
     tma_load_3d(smem + FA_OFF_Q + FA_HALF, &tmQ, q_full, 64, q0, b * H + h);
-    int issued = 0;
+    // K and V have rings of their own: K tile j+2 can arrive as soon as
+    // S_j has been computed, while V tile j+2 waits for P_j V_j.
+    int k_issued = 0, v_issued = 0;
     bool ok = true;
-    for (int j = 0; j < n_kt; ++j) {
+    for (int j = 0; j < n_kt && ok; ++j) {
       const int st = j & 1;
       const uint32_t ph = (j >> 1) & 1;
-      if (!mbar_wait(&kv_empty[st], ph ^ 1, status)) { ok = false; break; }
-      mbar_arrive_expect_tx(&kv_full[st], 2 * FA_KV_BYTES);
+      if (!mbar_wait(&k_empty[st], ph ^ 1, status)) { ok = false; break; }
+      mbar_arrive_expect_tx(&k_full[st], FA_KV_BYTES);
       uint8_t* kd = smem + FA_OFF_K + st * FA_KV_BYTES;
+      tma_load_3d(kd, &tmK, &k_full[st], 0, j * FA_BN, b * Hk + g);
+      tma_load_3d(kd + FA_HALF, &tmK, &k_full[st], 64, j * FA_BN, b * Hk + g);
+      ++k_issued;
+      if (!mbar_wait(&v_empty[st], ph ^ 1, status)) { ok = false; break; }
+      mbar_arrive_expect_tx(&v_full[st], FA_KV_BYTES);
       uint8_t* vd = smem + FA_OFF_V + st * FA_KV_BYTES;
-      tma_load_3d(kd, &tmK, &kv_full[st], 0, j * FA_BN, b * Hk + g);
-      tma_load_3d(kd + FA_HALF, &tmK, &kv_full[st], 64, j * FA_BN, b * Hk + g);
-      tma_load_3d(vd, &tmV, &kv_full[st], 0, j * FA_BN, b * Hk + g);
-      tma_load_3d(vd + FA_HALF, &tmV, &kv_full[st], 64, j * FA_BN, b * Hk + g);
-      ++issued;
+      tma_load_3d(vd, &tmV, &v_full[st], 0, j * FA_BN, b * Hk + g);
+      tma_load_3d(vd + FA_HALF, &tmV, &v_full[st], 64, j * FA_BN, b * Hk + g);
+      ++v_issued;
     }
     if (!ok) {  // let issued copies land before the CTA can exit
       mbar_wait(q_full, 0, status);
-      for (int j = issued - 1; j >= 0 && j >= issued - 2; --j) mbar_wait(&kv_full[j & 1], (j >> 1) & 1, status);
+      for (int j = k_issued - 1; j >= 0 && j >= k_issued - 2; --j) mbar_wait(&k_full[j & 1], (j >> 1) & 1, status);
+      for (int j = v_issued - 1; j >= 0 && j >= v_issued - 2; --j) mbar_wait(&v_full[j & 1], (j >> 1) & 1, status);
     }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc_s = umma_idesc_16(UmmaFmt<T>::value, FA_BM, FA_BN, false);
@@ -137,7 +155,7 @@ __global__ void __launch_bounds__(192, 1)
     bool ok = mbar_wait(q_full, 0, status), any = false;
     auto issue_s = [&](int j) -> bool {
       const int st = j & 1;
-      if (!mbar_wait(&kv_full[st], (j >> 1) & 1, status)) return false;
+      if (!mbar_wait(&k_full[st], (j >> 1) & 1, status)) return false;
       tc_fence_after();
       const uint32_t k_addr = smem_u32(smem + FA_OFF_K + st * FA_KV_BYTES);
       const uint32_t d_tmem = tmem + FA_TMEM_S + (uint32_t)st * 128;
@@ -147,6 +165,7 @@ __global__ void __launch_bounds__(192, 1)
         umma_bf16(d_tmem, umma_desc_sw128(q_addr + off), umma_desc_sw128(k_addr + off), idesc_s, ks != 0);
       }
       umma_commit(&s_full[st]);
+      umma_commit(&k_empty[st]);
       any = true;
       return true;
     };
@@ -154,8 +173,9 @@ __global__ void __launch_bounds__(192, 1)
     for (int j = 0; j < n_kt && ok; ++j) {
       if (j + 1 < n_kt && !(ok = issue_s(j + 1))) break;
       if (!(ok = mbar_wait(p_full, j & 1, status))) break;
-      tc_fence_after();
       const int st = j & 1;
+      if (!(ok = mbar_wait(&v_full[st], (j >> 1) & 1, status))) break;
+      tc_fence_after();
       const uint32_t v_addr = smem_u32(smem + FA_OFF_V + st * FA_KV_BYTES);
 #pragma unroll
       for (int ks = 0; ks < FA_BN / 16; ++ks) {
@@ -163,7 +183,7 @@ __global__ void __launch_bounds__(192, 1)
         umma_bf16(tmem + FA_TMEM_O, umma_desc_sw128(p_addr + p_off), umma_desc_sw128_mn(v_addr + ks * 2048, FA_HALF),
                   idesc_o, (j | ks) != 0);
       }
-      umma_commit(&kv_empty[st]);
+      umma_commit(&v_empty[st]);
       umma_commit(o_done);
     }
     if (!ok && any) {
@@ -171,41 +191,51 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(drain, 0, status);
     }
   } else if (warp >= 2) {
-    const int quarter = warp & 3;
+    const int quarter = warp & 3;                       // TMEM lanes this warp may read
+    const int half = (warp - 2) >> 2;                   // 0: keys / columns 0-63, 1: 64-127
     const int r = quarter * 32 + lane;                  // query row in the tile
     const int qpos = p0 + q0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    uint8_t* p_row = smem + FA_OFF_P + r * 128;
+    const uint32_t col0 = (uint32_t)half * 64;
+    uint8_t* p_row = smem + FA_OFF_P + half * FA_HALF + r * 128;
+    float* red_max = reinterpret_cast<float*>(smem + FA_OFF_RED);       // [slot][half][row]
+    float* red_sum = red_max + 4 * 128;                                  // [half][row]
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kt; ++j) {
       const int st = j & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1, status)) && ok;
       tc_fence_after();
-      float sv[128];
+      float sv[64];
       if (ok) {
+        uint32_t t0[32], t1[32];
+        tmem_ld32_nowait(tmem + lane_off + FA_TMEM_S + (uint32_t)st * 128 + col0, t0);
+        tmem_ld32_nowait(tmem + lane_off + FA_TMEM_S + (uint32_t)st * 128 + col0 + 32, t1);
+        tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float t[32];
-          tmem_ld32(tmem + lane_off + FA_TMEM_S + (uint32_t)st * 128 + c * 32, t);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) sv[c * 32 + i] = t[i];
-        }
+        for (int i = 0; i < 32; ++i) { sv[i] = __uint_as_float(t0[i]); sv[32 + i] = __uint_as_float(t1[i]); }
       } else {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) sv[i] = 0.f;
+        for (int i = 0; i < 64; ++i) sv[i] = 0.f;
       }
-      const int kbase = j * FA_BN;
+      const int kbase = j * FA_BN + (int)col0;
       // masked tiles: the last one or two of a causal row block
-      if (kbase + FA_BN - 1 > p0 + q0) {
+      if (j * FA_BN + FA_BN - 1 > p0 + q0) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
+        for (int i = 0; i < 64; ++i)
           if (kbase + i > qpos) sv[i] = -INFINITY;
       }
-      float mx = sv[0];
+      float mx8[8];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, sv[i]);
-      mx *= scale_log2;                       // scale > 0: max of the scaled scores
+      for (int c = 0; c < 8; ++c) mx8[c] = sv[c];
+#pragma unroll
+      for (int i = 8; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+      float mloc = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      red_max[(st * 2 + half) * 128 + r] = mloc;
+      named_bar_sync(1, 256);
+      // both threads of the row see the same maximum and take the same decisions
+      const float mx = fmaxf(mloc, red_max[(st * 2 + (half ^ 1)) * 128 + r]) * scale_log2;
       float corr = 1.f;
       bool rescale = false;
       if (j == 0) {
@@ -215,15 +245,18 @@ __global__ void __launch_bounds__(192, 1)
         m_used = mx;
         rescale = true;
       }
-      float rowsum = 0.f;
-      uint32_t pk[64];
+      float sum8[8];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
+      for (int c = 0; c < 8; ++c) sum8[c] = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
         const float a = fast_exp2(fmaf(sv[2 * i], scale_log2, -m_used));
         const float c2 = fast_exp2(fmaf(sv[2 * i + 1], scale_log2, -m_used));
-        rowsum += a + c2;
+        sum8[i & 7] += a + c2;
         pk[i] = pack2<T>(a, c2);
       }
+      const float rowsum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l = l * corr + rowsum;
       // P and O may be touched only once the previous P V product has finished
       if (j > 0) {
@@ -232,37 +265,41 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (__any_sync(0xffffffffu, rescale) && ok) {
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           float t[32];
-          tmem_ld32(tmem + lane_off + FA_TMEM_O + c * 32, t);
+          tmem_ld32(tmem + lane_off + FA_TMEM_O + col0 + c * 32, t);
 #pragma unroll
           for (int i = 0; i < 32; ++i) t[i] *= corr;
-          tmem_st32(tmem + lane_off + FA_TMEM_O + c * 32, t);
+          tmem_st32(tmem + lane_off + FA_TMEM_O + col0 + c * 32, t);
         }
         tmem_st_wait();
       }
-      // P row: 16-byte chunk cc of 16 goes to block cc/8, swizzled position (cc%8) ^ (r%8)
+      // this thread's 64 keys fill swizzle block `half` of the P row:
+      // 16-byte chunk cc sits at position cc ^ (r % 8)
 #pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        uint4* dst = reinterpret_cast<uint4*>(p_row + (cc >> 3) * FA_HALF + (((cc & 7) ^ (r & 7)) << 4));
+      for (int cc = 0; cc < 8; ++cc) {
+        uint4* dst = reinterpret_cast<uint4*>(p_row + ((cc ^ (r & 7)) << 4));
         *dst = make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    // final: O / l to global memory
+    // final: O / l to global memory, each thread its 64 columns
     if (n_kt > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait(o_done, (n_kt - 1) & 1, status)) && ok;
       tc_fence_after();
     }
+    red_sum[half * 128 + r] = l;
+    named_bar_sync(1, 256);
+    const float ltot = l + red_sum[(half ^ 1) * 128 + r];
     const int qi = q0 + r;
-    const float inv = 1.f / l;
-    T* dst = o + ((size_t)b * S + (qi < S ? qi : 0)) * H * FA_D + (size_t)h * FA_D;
+    const float inv = 1.f / ltot;
+    T* dst = o + ((size_t)b * S + (qi < S ? qi : 0)) * H * FA_D + (size_t)h * FA_D + col0;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
       float t[32];
-      if (ok) tmem_ld32(tmem + lane_off + FA_TMEM_O + c * 32, t);
+      if (ok) tmem_ld32(tmem + lane_off + FA_TMEM_O + col0 + c * 32, t);
       else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) t[i] = 0.f;
@@ -327,7 +364,8 @@ static int attention_prefill_tc_t(const void* q, const void* kc, const void* vc,
     attr = true;
   }
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)FA_D);
-  const cudaError_t err = launch_k(kern, dim3(((S + FA_BM - 1) / FA_BM) * H * B), dim3(192), FA_SMEM, st, tq, tk, tv,
+  const cudaError_t err = launch_k(kern, dim3(((S + FA_BM - 1) / FA_BM) * H * B), dim3(FA_THREADS), FA_SMEM, st, tq,
+                                   tk, tv,
                                    static_cast<T*>(o), pos0, S, H, Hk, scale_log2, status);
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }

@@ -30,6 +30,18 @@ __global__ void embed_kernel(const int32_t* __restrict__ tokens, const T* __rest
 // ---------------------------------------------------------------- RMSNorm
 // y = x * rsqrt(mean(x^2) + eps) * g over one row of D fp32 values.
 template <typename T>
+__device__ __forceinline__ void store4(T* p, float a, float b, float c, float d) {
+  if constexpr (sizeof(T) == 2) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack2<T>(a, b), pack2<T>(c, d));
+  } else {
+    *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+  }
+}
+
+// One row per 256-thread block. Rows with D % 4 == 0 and D <= 8192 stay in
+// registers between the sum of squares and the scaling (x is read once) and
+// are written with 8- or 16-byte stores.
+template <typename T>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ g,
                                                       T* __restrict__ y, int D, float eps, int last_of_S) {
   pdl_trigger();
@@ -37,13 +49,19 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
   const int r = blockIdx.x;
   const size_t src_row = last_of_S > 0 ? (size_t)(r + 1) * last_of_S - 1 : (size_t)r;
   const float* xr = x + src_row * D;
+  T* yr = y + (size_t)r * D;
   __shared__ float red[8];
+  constexpr int NV = 8;  // float4 per thread in the register path
+  const bool vec = (D % 4 == 0) && D <= NV * 4 * 256 && ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(g)) & 15) == 0 &&
+                   (reinterpret_cast<uintptr_t>(y) & 15) == 0;
+  float4 v[NV];
   float ss = 0.f;
-  const bool vec = (D % 4 == 0);
   if (vec) {
-    for (int i = threadIdx.x * 4; i < D; i += 1024) {
-      const float4 v = *reinterpret_cast<const float4*>(xr + i);
-      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+      const int i = (threadIdx.x + k * 256) * 4;
+      v[k] = i < D ? __ldcs(reinterpret_cast<const float4*>(xr + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
     }
   } else {
     for (int i = threadIdx.x; i < D; i += 256) ss += xr[i] * xr[i];
@@ -56,15 +74,14 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
 #pragma unroll
   for (int w = 0; w < 8; ++w) tot += red[w];
   const float inv = rsqrtf(tot / (float)D + eps);
-  T* yr = y + (size_t)r * D;
   if (vec) {
-    for (int i = threadIdx.x * 4; i < D; i += 1024) {
-      const float4 v = *reinterpret_cast<const float4*>(xr + i);
-      const float4 w = *reinterpret_cast<const float4*>(g + i);
-      yr[i] = from_f<T>(v.x * inv * w.x);
-      yr[i + 1] = from_f<T>(v.y * inv * w.y);
-      yr[i + 2] = from_f<T>(v.z * inv * w.z);
-      yr[i + 3] = from_f<T>(v.w * inv * w.w);
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+      const int i = (threadIdx.x + k * 256) * 4;
+      if (i < D) {
+        const float4 w = __ldg(reinterpret_cast<const float4*>(g + i));
+        store4<T>(yr + i, v[k].x * inv * w.x, v[k].y * inv * w.y, v[k].z * inv * w.z, v[k].w * inv * w.w);
+      }
     }
   } else {
     for (int i = threadIdx.x; i < D; i += 256) yr[i] = from_f<T>(xr[i] * inv * g[i]);

@@ -21,6 +21,7 @@
 // requested before waiting for the previous kernel, activations after.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdlib>
 #include <mutex>
 #include <type_traits>
@@ -59,10 +60,64 @@ __device__ void drain_loads(uint64_t* full, int stage, uint32_t phase, int issue
 }
 
 // ------------------------------------------------------------------ wide
+__device__ __forceinline__ long long sk_first(long long c, long long U, long long G) { return U * c / G; }
+__device__ __forceinline__ long long sk_owner(long long u, long long U, long long G) { return ((u + 1) * G - 1) / U; }
+
+// The pieces of work of one wide-GEMM CTA, in order: whole tiles c, c+G, ...
+// below T_dp (data-parallel waves), then its share of the stream-K region.
+// The stream-K region is the tiles [T_dp, T) cut into (tile, k-block) units,
+// tile-major; CTA c < G_sk takes units [U*c/G_sk, U*(c+1)/G_sk). Every role of
+// the CTA walks the same sequence.
+struct WideWork {
+  int c, G, kb, T_dp, i, dp_n;
+  long long u, u1, u_start;
+  __device__ WideWork(int c_, int G_, int kb_, int T, int T_dp_, int G_sk) : c(c_), G(G_), kb(kb_), T_dp(T_dp_), i(0) {
+    dp_n = T_dp > c ? (T_dp - c + G - 1) / G : 0;
+    const long long U = (long long)(T - T_dp) * kb;
+    u = u1 = 0;
+    if (c < G_sk) { u = sk_first(c, U, G_sk); u1 = sk_first(c + 1, U, G_sk); }
+    u_start = u;
+  }
+  // tile index, first k-block and number of k-blocks of the next piece; slot
+  // is 0 for the CTA's first stream-K piece and 1 for any later one
+  __device__ bool next(int& tile, int& klo, int& n, int& slot) {
+    if (i < dp_n) { tile = c + i * G; klo = 0; n = kb; slot = 0; ++i; return true; }
+    if (u < u1) {
+      tile = T_dp + (int)(u / kb);
+      klo = (int)(u % kb);
+      n = (int)((u1 - u) < (kb - klo) ? (u1 - u) : (kb - klo));
+      slot = u == u_start ? 0 : 1;
+      u += n;
+      return true;
+    }
+    return false;
+  }
+  __device__ bool next(int& tile, int& klo, int& n) {
+    int slot;
+    return next(tile, klo, n, slot);
+  }
+};
+
+// A piece that covers its whole tile runs the epilogue from TMEM. A split
+// tile has one owner, the CTA whose piece holds k-block 0: that piece is the
+// last of the owner's range, while every other piece of the tile is the first
+// of its CTA's range (it starts inside the tile), so the other contributors
+// finish their share early. They store it in their CTA's workspace slot and
+// count themselves in the tile's counter; the owner waits (bounded) for the
+// count, adds the shares in CTA order to its own accumulator from TMEM, runs
+// the epilogue and re-arms the counter. The sum order is fixed, so results do
+// not depend on timing. Every CTA of the grid is resident at once (one CTA per
+// SM, grid <= SMs), and an owner only waits for first pieces, which wait for
+// nothing, so the waits always end.
+//
+// Workspace slot layout: float4 (c * 8 + j) * 128 + r holds columns
+// 32c + 4j .. 32c + 4j + 3 of tile row r, so a warp's 32 rows are 512
+// contiguous bytes.
 template <int KIND, typename T>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_wide_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
-                     int K, EpiArgs epi, int* status) {
+                     int K, EpiArgs epi, int T_dp, int G_sk, float* __restrict__ ws, int* __restrict__ counters,
+                     int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + W_STAGES * W_STAGE_BYTES);
@@ -89,6 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  WideWork work(blockIdx.x, gridDim.x, kb, tiles, T_dp, G_sk);
+  int tile, klo, n;
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
@@ -96,28 +153,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t pol_a = l2_policy_evict_last(), pol_b = l2_policy_evict_last();
     // The weight tiles of the first stages do not depend on the previous
     // kernel: request them before waiting for it, their activation halves after.
-    const int pre = blockIdx.x < tiles ? (kb < W_STAGES ? kb : W_STAGES) : 0;
+    bool have = work.next(tile, klo, n);
+    const int pre = have ? (n < W_STAGES ? n : W_STAGES) : 0;
     {
-      const int n0 = (blockIdx.x / m_tiles) * W_BN;
+      const int n0 = have ? (tile / m_tiles) * W_BN : 0;
       for (int k = 0; k < pre; ++k) {
         mbar_arrive_expect_tx(&full[k], W_STAGE_BYTES);
-        tma_load_2d(smem + k * W_STAGE_BYTES + W_A_BYTES, &tmB, &full[k], k * BK, n0, pol_b);
+        tma_load_2d(smem + k * W_STAGE_BYTES + W_A_BYTES, &tmB, &full[k], (klo + k) * BK, n0, pol_b);
       }
       pdl_wait();
-      const int m0 = (blockIdx.x % m_tiles) * W_BM;
-      for (int k = 0; k < pre; ++k) tma_load_2d(smem + k * W_STAGE_BYTES, &tmA, &full[k], k * BK, m0, pol_a);
+      const int m0 = have ? (tile % m_tiles) * W_BM : 0;
+      for (int k = 0; k < pre; ++k) tma_load_2d(smem + k * W_STAGE_BYTES, &tmA, &full[k], (klo + k) * BK, m0, pol_a);
     }
-    int stage = pre % W_STAGES, issued = pre;
+    int stage = pre % W_STAGES, issued = pre, k_start = pre;
     uint32_t phase = pre == W_STAGES ? 1u : 0u;
     bool ok = true;
-    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-      const int m0 = (t % m_tiles) * W_BM, n0 = (t / m_tiles) * W_BN;
-      for (int k = (t == (int)blockIdx.x ? pre : 0); k < kb; ++k) {
+    for (; have && ok; have = work.next(tile, klo, n), k_start = 0) {
+      const int m0 = (tile % m_tiles) * W_BM, n0 = (tile / m_tiles) * W_BN;
+      for (int k = k_start; k < n; ++k) {
         if (!mbar_wait(&empty[stage], phase ^ 1, status)) { ok = false; break; }
         uint8_t* sa = smem + stage * W_STAGE_BYTES;
         mbar_arrive_expect_tx(&full[stage], W_STAGE_BYTES);
-        tma_load_2d(sa, &tmA, &full[stage], k * BK, m0, pol_a);
-        tma_load_2d(sa + W_A_BYTES, &tmB, &full[stage], k * BK, n0, pol_b);
+        tma_load_2d(sa, &tmA, &full[stage], (klo + k) * BK, m0, pol_a);
+        tma_load_2d(sa + W_A_BYTES, &tmB, &full[stage], (klo + k) * BK, n0, pol_b);
         ++issued;
         if (++stage == W_STAGES) { stage = 0; phase ^= 1; }
       }
@@ -128,11 +186,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     int stage = 0, acc = 0;
     uint32_t phase = 0, acc_phase = 0;
     bool ok = true, any = false;
-    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+    while (ok && work.next(tile, klo, n)) {
       if (!mbar_wait(&acce[acc], acc_phase ^ 1, status)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem + acc * W_BN;
-      for (int k = 0; k < kb; ++k) {
+      for (int k = 0; k < n; ++k) {
         if (!mbar_wait(&full[stage], phase, status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_addr = smem_u32(smem + stage * W_STAGE_BYTES);
@@ -157,23 +215,72 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_wait();  // the epilogue reads and writes memory owned by earlier kernels
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
+    const long long U = (long long)(tiles - T_dp) * kb;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
-      const int m0 = (t % m_tiles) * W_BM, n0 = (t / m_tiles) * W_BN;
-      // the whole warp leaves together so the warp-wide TMEM loads stay converged
-      if (!__all_sync(0xffffffffu, mbar_wait(&accf[acc], acc_phase, status))) break;
+    bool failed = false;  // after a timed-out wait the MMA has stopped: no further waits
+    while (work.next(tile, klo, n)) {
+      const int m0 = (tile % m_tiles) * W_BM, n0 = (tile / m_tiles) * W_BN;
+      const bool whole = klo == 0 && n == kb;
+      const int s = tile - T_dp;  // stream-K tile index (split tiles only)
+      // contributors other than the owner: CTAs (c_own, c_hi], each one slot
+      long long c_own = 0, c_hi = 0;
+      if (!whole) {
+        const long long t0 = (long long)s * kb;
+        c_own = sk_owner(t0, U, G_sk);
+        c_hi = sk_owner(t0 + kb - 1, U, G_sk);
+      }
+      if (!whole && klo == 0) {  // owner: wait for the other shares before touching TMEM
+        if (threadIdx.x == 64) {
+          const int need = (int)(c_hi - c_own);
+          counter_wait_geq(&counters[s], need, status);  // a timeout is latched in status
+          counters[s] = 0;  // every other contributor has counted itself: re-arm
+        }
+        named_bar_sync(1, 128);
+        __threadfence();
+      }
+      // the whole warp decides together so the warp-wide TMEM loads stay converged
+      if (!failed) failed = !__all_sync(0xffffffffu, mbar_wait(&accf[acc], acc_phase, status));
       tc_fence_after();
       const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + acc * W_BN;
+      float4* mine = reinterpret_cast<float4*>(ws) + (size_t)blockIdx.x * (W_BM * W_BN / 4) + row;
 #pragma unroll 1
       for (int c = 0; c < W_BN / 32; ++c) {
         float v[32];
-        tmem_ld32(base + c * 32, v);
-        if (n0 + c * 32 < N) epi_row32<KIND, T>(epi, m0 + row, n0 + c * 32, v);
+        if (failed) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        } else {
+          tmem_ld32(base + c * 32, v);
+        }
+        if (whole) {
+          if (!failed && n0 + c * 32 < N) epi_row32<KIND, T>(epi, m0 + row, n0 + c * 32, v);
+        } else if (klo != 0) {  // a share for the owner
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            __stcg(mine + (c * 8 + j) * W_BM, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+        } else {  // owner: add the shares in CTA order, then the epilogue
+          for (long long cc = c_own + 1; cc <= c_hi; ++cc) {
+            const float4* p4 = reinterpret_cast<const float4*>(ws) + (size_t)cc * (W_BM * W_BN / 4) + row;
+            float4 x[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] = __ldcg(p4 + (c * 8 + j) * W_BM);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              v[4 * j] += x[j].x; v[4 * j + 1] += x[j].y; v[4 * j + 2] += x[j].z; v[4 * j + 3] += x[j].w;
+            }
+          }
+          if (!failed && n0 + c * 32 < N) epi_row32<KIND, T>(epi, m0 + row, n0 + c * 32, v);
+        }
       }
       tc_fence_before();
       mbar_arrive(&acce[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      if (!whole && klo != 0) {  // publish the share
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 64) atomicAdd(&counters[s], 1);
+      }
     }
   }
   tc_fence_before();
@@ -204,9 +311,6 @@ struct SkinnyCfg {
   static constexpr int SMEM = STAGES * STAGE_BYTES + TRANS_BYTES + 1024 + 256;
   static constexpr uint32_t TMEM_COLS = 2 * NT <= 32 ? 32 : (2 * NT <= 64 ? 64 : (2 * NT <= 128 ? 128 : (2 * NT <= 256 ? 256 : 512)));
 };
-
-__device__ __forceinline__ long long sk_first(long long c, long long U, long long G) { return U * c / G; }
-__device__ __forceinline__ long long sk_owner(long long u, long long U, long long G) { return ((u + 1) * G - 1) / U; }
 
 template <int KIND, typename T, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -512,9 +616,37 @@ int num_sms() {
   return n;
 }
 
+bool streamk_enabled() {
+  static const bool on = getenv("LLAMA_NO_STREAMK") == nullptr;
+  return on;
+}
+
+// Split of a wide GEMM of T output tiles over G SMs. With fewer tiles than
+// SMs, every tile is cut into (tile, k-block) units spread over up to G CTAs
+// (at least 8 k-blocks each), so all SMs stream the reduction dimension.
+// With at least one full wave the tiles stay data-parallel: measured on the
+// 8B prefill shapes, splitting the tail wave lost more (the fixup, and CTAs
+// no longer walking K in step, which shares A and B slices in L2) than the
+// idle SMs of the last wave cost.
+WideSplit wide_split(int M, int N, int K) {
+  WideSplit w;
+  const int T = ((M + W_BM - 1) / W_BM) * ((N + W_BN - 1) / W_BN), G = num_sms(), kb = (K + BK - 1) / BK;
+  int sk = 0;
+  if (T < G && streamk_enabled()) sk = T;
+  w.tiles = T;
+  w.sk_tiles = sk;
+  w.T_dp = T - sk;
+  const long long U = (long long)sk * kb;
+  w.G_sk = sk ? (int)std::min<long long>(G, std::max<long long>(1, U / 8)) : 0;
+  w.grid = w.T_dp > 0 ? std::min(T, G) : w.G_sk;
+  return w;
+}
+
+size_t wide_workspace_floats() { return (size_t)num_sms() * W_BM * W_BN; }
+
 template <int KIND, typename T>
 static int launch_wide(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, const EpiArgs& e,
-                       int* status, cudaStream_t st) {
+                       GemmScratch* scratch, int* status, cudaStream_t st) {
   auto kern = gemm_wide_kernel<KIND, T>;
   static bool attr = false;
   if (!attr) {
@@ -522,9 +654,23 @@ static int launch_wide(const CUtensorMap& ta, const CUtensorMap& tb, int M, int 
       return LLAMA_ERR_CUDA;
     attr = true;
   }
-  const int tiles = ((M + W_BM - 1) / W_BM) * ((N + W_BN - 1) / W_BN);
-  const int grid = tiles < num_sms() ? tiles : num_sms();
-  const cudaError_t err = launch_k(kern, dim3(grid), dim3(kThreads), W_SMEM, st, ta, tb, M, N, K, e, status);
+  WideSplit w = wide_split(M, N, K);
+  float* ws = nullptr;
+  int* tickets = nullptr;
+  if (w.sk_tiles > 0) {
+    // partial-tile workspace and tickets; without them the tail wave stays data-parallel
+    if (scratch && scratch->ws && scratch->ws_floats >= wide_workspace_floats() && scratch->tickets &&
+        scratch->n_tickets >= w.sk_tiles) {
+      ws = scratch->ws;
+      tickets = scratch->tickets;
+    } else {
+      w.T_dp = w.tiles;
+      w.G_sk = 0;
+      w.grid = std::min(w.tiles, num_sms());
+    }
+  }
+  const cudaError_t err = launch_k(kern, dim3(w.grid), dim3(kThreads), W_SMEM, st, ta, tb, M, N, K, e, w.T_dp,
+                                   w.G_sk, ws, tickets, status);
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
@@ -586,10 +732,10 @@ static int gemm16_t(const void* A, int M, int K, int lda, const void* W, int N, 
     if ((rc = make_tmap_16(&ta, A, M, K, lda, W_BM, F16)) != LLAMA_OK) return rc;
     if ((rc = make_tmap_16(&tb, W, N, K, ldw, W_BN, F16)) != LLAMA_OK) return rc;
     switch (kind) {
-      case EPI_STORE_F32: return launch_wide<EPI_STORE_F32, T>(ta, tb, M, N, K, e, status, st);
-      case EPI_RESIDUAL: return launch_wide<EPI_RESIDUAL, T>(ta, tb, M, N, K, e, status, st);
-      case EPI_SWIGLU: return launch_wide<EPI_SWIGLU, T>(ta, tb, M, N, K, e, status, st);
-      case EPI_QKV_ROPE: return launch_wide<EPI_QKV_ROPE, T>(ta, tb, M, N, K, e, status, st);
+      case EPI_STORE_F32: return launch_wide<EPI_STORE_F32, T>(ta, tb, M, N, K, e, scratch, status, st);
+      case EPI_RESIDUAL: return launch_wide<EPI_RESIDUAL, T>(ta, tb, M, N, K, e, scratch, status, st);
+      case EPI_SWIGLU: return launch_wide<EPI_SWIGLU, T>(ta, tb, M, N, K, e, scratch, status, st);
+      case EPI_QKV_ROPE: return launch_wide<EPI_QKV_ROPE, T>(ta, tb, M, N, K, e, scratch, status, st);
     }
     return LLAMA_ERR_INVALID_ARG;
   }

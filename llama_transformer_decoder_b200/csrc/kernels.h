@@ -43,11 +43,21 @@ struct GemmScratch {
   size_t ws_floats;
   int* tickets;
   int n_tickets;
-  float* stg;          // zeroed fp32 [M][N] staging for the QKV/RoPE and SwiGLU epilogues (kept zero)
+  float* stg;          // zeroed fp32 [M][N] staging for the skinny QKV/RoPE and SwiGLU epilogues (kept zero)
   size_t stg_floats;
 };
 
 int num_sms();
+
+// How a wide (prefill) GEMM is spread over the SMs: tiles [0, T_dp) in
+// data-parallel waves, the rest stream-K over G_sk CTAs (see gemm_tc.cu).
+struct WideSplit {
+  int tiles, sk_tiles, T_dp, G_sk, grid;
+};
+WideSplit wide_split(int M, int N, int K);
+// Partial-tile workspace (floats) a wide GEMM needs for its stream-K tiles
+// (plus sk_tiles tickets).
+size_t wide_workspace_floats();
 int make_tmap_16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t pitch, int box_rows,
                  bool is_f16);
 // Scratch of the stream-K skinny GEMM for M rows: two partial tiles per CTA.

@@ -73,16 +73,17 @@ def test_linear_16bit(M, N, K, variant, dtype):
     assert np.max(np.abs(got - ref) / scale) < 1e-5
 
 
-def test_linear_bf16_repeatable():
-    """Split-K reduction runs in a fixed order: repeated calls agree bit for bit."""
-    M, N, K = 32, 4096, 14336
+@pytest.mark.parametrize('M,N,K,variant', [(32, 4096, 14336, 2), (2048, 4096, 4096, 1), (300, 520, 4104, 1)])
+def test_linear_repeatable(M, N, K, variant):
+    """Split tiles (skinny split-K, wide stream-K tail) are reduced in a fixed
+    order: repeated calls agree bit for bit."""
     _, xr = normal_values(12, 1, (M, K), BF16)
     _, wr = normal_values(12, 2, (N, K), BF16, std=0.02)
     x, w = to_device(xr, BF16), to_device(wr, BF16)
     outs = []
     for _ in range(3):
         y = torch.empty((M, N), device='cuda')
-        L.llama_linear(x, w, y, M, N, K, BF16, 2)
+        L.llama_linear(x, w, y, M, N, K, BF16, variant)
         outs.append(y.cpu())
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
 
@@ -100,7 +101,7 @@ def test_linear_f32(M, N, K):
 
 # ------------------------------------------------------------ RMSNorm
 @pytest.mark.parametrize('dtype', [BF16, F16, F32])
-@pytest.mark.parametrize('M,D', [(1, 4096), (37, 4096), (5, 256), (3, 100)])
+@pytest.mark.parametrize('M,D', [(1, 4096), (37, 4096), (2048, 4096), (5, 256), (3, 100), (2, 12288), (3, 8192)])
 def test_rmsnorm(dtype, M, D):
     xv, xr = normal_values(14, 1, (M, D), F32)
     g = np.linspace(0.5, 1.5, D).astype(np.float32)
