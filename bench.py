@@ -10,6 +10,7 @@ N(0,1) K/V entries, 128 greedy steps at positions 4096..4223) under
 ``decode``.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  python bench.py --kernel attention_prefill|attention_decode|linear [shape flags]
 """
 from __future__ import annotations
 
@@ -97,13 +98,22 @@ def _dist():
 
 
 def _max_over_ranks(x: float, ws: int) -> float:
+    """Largest per-rank value (the replicas' step time is the slowest rank's)."""
     if ws == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device='cuda')
+    dev = 'cpu' if dist.get_backend() == 'gloo' else 'cuda'
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(units_per_rank: float, local_ms: float, ws: int):
+    """Whole-job throughput of ws replicas that each process units_per_rank
+    units in local_ms: (units/s over all ranks, the max-over-ranks ms)."""
+    ms = _max_over_ranks(local_ms, ws)
+    return ws * units_per_rank / (ms / 1e3), ms
 
 
 def _barrier(ws: int):
@@ -247,8 +257,8 @@ def measure_e2e(L, m, st, toks_h, args, ws):
         L.llama_generate(m, host_toks, PREFILL_B, PREFILL_S, 0, host_out, st)
     e1.record(st)
     torch.cuda.synchronize()
-    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, ws)
-    return {'value': ws * PREFILL_B * PREFILL_S / (e2e_ms / 1e3), 'unit': 'tokens/s',
+    e2e_value, _ = replica_throughput(PREFILL_B * PREFILL_S, e0.elapsed_time(e1) / args.steps, ws)
+    return {'value': e2e_value, 'unit': 'tokens/s',
             'h2d_bytes_per_step': PREFILL_B * PREFILL_S * 4, 'd2h_bytes_per_step': PREFILL_B * 4,
             'api': 'llama_generate(host tokens, n_new=0)'}
 
@@ -288,7 +298,7 @@ def measure_decode(L, m, st, arg, args, ws, local, NL, hbm_peak, peak_src):
         d1.record(st)
         torch.cuda.synchronize()
     launches = L.llama_kernel_launches() - n0
-    dms = _max_over_ranks(d0.elapsed_time(d1) / DECODE_STEPS, ws)
+    dvalue, dms = replica_throughput(DECODE_B, d0.elapsed_time(d1) / DECODE_STEPS, ws)
     assert L.llama_sync_status(m, st) == 0
     L.llama_profile(m, 1)
     L.llama_profile_read(m)
@@ -300,7 +310,7 @@ def measure_decode(L, m, st, arg, args, ws, local, NL, hbm_peak, peak_src):
     kv_bytes = NL * 2.0 * DECODE_B * avg_ctx * HK_ * HD_ * 2
     step_bytes = w_bytes + kv_bytes
     achieved = step_bytes / (dms / 1e3) / 1e9
-    return {'value': ws * DECODE_B / (dms / 1e3), 'unit': 'tokens/s', 'ms_per_step': dms,
+    return {'value': dvalue, 'unit': 'tokens/s', 'ms_per_step': dms,
             'steps': DECODE_STEPS, 'batch': DECODE_B, 'context': DECODE_CTX, 'graph_replay': True,
             'gpu_launches': launches,
             'roofline': {'bound': 'hbm', 'achieved': achieved, 'peak': hbm_peak, 'unit': 'GB/s',
@@ -369,6 +379,84 @@ def run_ours(args):
     return 0
 
 
+# ------------------------------------------------------------ one kernel
+def run_kernel(args):
+    """One kernel alone on seeded fp16 inputs from the library's device
+    generator (for ncu captures and shape sweeps): prints one JSON line per
+    shape with its CUDA-event time per call (median over --steps calls, L2
+    flushed by a read before each) and its rate against the burst peaks (it
+    runs alone). --batch, --seq and --ctx take comma-separated lists."""
+    import torch
+    from llama_transformer_decoder_b200 import binding as L
+    torch.cuda.set_device(0)
+    hbm, tf_burst, _, src = _peaks()
+    F16 = L.LLAMA_F16
+    dev = 'cuda'
+
+    def filled(shape, stream_id, std=1.0):
+        t = torch.empty(shape, dtype=torch.float16, device=dev)
+        L.llama_fill_normal(t, t.numel(), 9, stream_id, std, F16)
+        return t
+
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)  # 256 MB > L2
+    H, Hk, d = 32, 8, 128
+    ints = lambda v: [int(x) for x in str(v).split(',')]
+    cases = []
+    if args.kernel == 'attention_prefill':
+        cases = [(B, S) for B in ints(args.batch) for S in ints(args.seq)]
+    elif args.kernel == 'attention_decode':
+        cases = [(B, C) for B in ints(args.batch) for C in ints(args.ctx)]
+    else:
+        cases = [tuple(int(x) for x in args.mnk.split(','))]
+    for case in cases:
+        if args.kernel == 'attention_prefill':
+            B, S = case
+            q, k, v = filled((B, H, S, d), 1), filled((B, Hk, S, d), 2), filled((B, Hk, S, d), 3)
+            o = torch.empty((B, S, H * d), dtype=torch.float16, device=dev)
+            call = lambda: L.llama_attention_prefill(q, k, v, o, B, S, H, Hk, d, F16)
+            work, unit, peak = 4.0 * B * H * d * S * (S + 1) / 2, 'TFLOP/s', tf_burst
+            cfg = {'workload': f'causal GQA prefill attention B={B} S={S} H=32 Hk=8 d=128'}
+        elif args.kernel == 'attention_decode':
+            B, C = case
+            q, kc, vc = filled((B, H, d), 1), filled((B, Hk, C, d), 2), filled((B, Hk, C, d), 3)
+            ln = torch.full((B,), C, dtype=torch.int32, device=dev)
+            o = torch.empty((B, H * d), dtype=torch.float16, device=dev)
+            call = lambda: L.llama_attention_decode(q, kc, vc, ln, o, B, C, H, Hk, d, F16)
+            work, unit, peak = float(B * Hk * C * d * 2 * 2), 'GB/s', hbm
+            cfg = {'workload': f'decode attention B={B} context={C} H=32 Hk=8 d=128'}
+        else:
+            M, N, K = case
+            x, w = filled((M, K), 1), filled((N, K), 2, 0.02)
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            call = lambda: L.llama_linear(x, w, y, M, N, K, F16, 0)
+            if M <= 128:
+                work, unit, peak = float(N * K * 2), 'GB/s', hbm
+            else:
+                work, unit, peak = 2.0 * M * N * K, 'TFLOP/s', tf_burst
+            cfg = {'workload': f'linear y = x W^T, M={M} N={N} K={K}'}
+        for _ in range(args.warmup):
+            call()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(args.steps):
+            float(flush.sum())
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            call()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        assert L.llama_status(None) == 0
+        ms = statistics.median(times)
+        rate = work / (ms / 1e3) / (1e12 if unit == 'TFLOP/s' else 1e9)
+        print(json.dumps({'kernel': args.kernel, 'ms': ms, 'rate': rate, 'unit': unit, 'peak': peak,
+                          'frac': rate / peak, 'peak_kind': f'burst ({src})', 'steps': args.steps,
+                          'warmup': args.warmup, 'config': cfg}), flush=True)
+        del call
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument('--gpus', type=int, default=1)
@@ -379,7 +467,15 @@ def main():
     ap.add_argument('--decode-only', action='store_true', help='skip the prefill and end-to-end legs (profiling)')
     ap.add_argument('--layers', type=int, default=32, help='decoder layers (32 = the 8B model)')
     ap.add_argument('--no-cpu-baseline', action='store_true')
+    ap.add_argument('--kernel', choices=['attention_prefill', 'attention_decode', 'linear'],
+                    help='time one kernel alone on seeded inputs (profiling and sweeps)')
+    ap.add_argument('--batch', default='1', help='--kernel attention_*: sequences (comma list)')
+    ap.add_argument('--seq', default='2048', help='--kernel attention_prefill: tokens per sequence (comma list)')
+    ap.add_argument('--ctx', default='4096', help='--kernel attention_decode: cached keys (comma list)')
+    ap.add_argument('--mnk', default='2048,28672,4096', help='--kernel linear: M,N,K')
     args = ap.parse_args()
+    if args.kernel:
+        return run_kernel(args)
     if args.impl == 'reference':
         return run_reference(args)
     return run_ours(args)

@@ -13,7 +13,8 @@
 //                         while the softmax works on S_j)
 //   P_j = exp2(S_j*c - m) rounded to the 16-bit type (the walkthrough rounds
 //                         softmax(...) to 16 bits before the value product)
-//                      -> shared memory, 128-byte swizzled K-major rows
+//                      -> TMEM (64 columns, two keys per column), the A
+//                         operand of the next product
 //   O  += P_j V_j      -> TMEM (128 columns); V is read MN-major straight from
 //                         the cache layout [key][d].
 //
@@ -40,11 +41,11 @@ constexpr int FA_STAGES = 2;
 constexpr int FA_OFF_Q = 0;
 constexpr int FA_OFF_K = FA_OFF_Q + FA_Q_BYTES;
 constexpr int FA_OFF_V = FA_OFF_K + FA_STAGES * FA_KV_BYTES;
-constexpr int FA_OFF_P = FA_OFF_V + FA_STAGES * FA_KV_BYTES;
-constexpr int FA_OFF_RED = FA_OFF_P + FA_Q_BYTES;     // row maxima [2 slots][2 halves][128], sums [2][128]
+constexpr int FA_OFF_RED = FA_OFF_V + FA_STAGES * FA_KV_BYTES;  // row maxima [2 slots][2 halves][128], sums [2][128]
 constexpr int FA_OFF_BAR = FA_OFF_RED + 6 * 128 * 4;
 constexpr int FA_SMEM = FA_OFF_BAR + 256 + 1024;
 constexpr uint32_t FA_TMEM_O = 0, FA_TMEM_S = 128;   // S buffers at columns 128 and 256
+constexpr uint32_t FA_TMEM_P = 384;                   // P: 64 columns, keys 2c and 2c+1 in column c
 constexpr float FA_RESCALE = 8.0f;                    // raise the running max only past +8 (log2)
 
 // 2^x with the hardware approximation (flushes results below 2^-126 to zero,
@@ -151,7 +152,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc_s = umma_idesc_16(UmmaFmt<T>::value, FA_BM, FA_BN, false);
     constexpr uint32_t idesc_o = umma_idesc_16(UmmaFmt<T>::value, FA_BM, FA_D, true);
-    const uint32_t q_addr = smem_u32(smem + FA_OFF_Q), p_addr = smem_u32(smem + FA_OFF_P);
+    const uint32_t q_addr = smem_u32(smem + FA_OFF_Q);
     bool ok = mbar_wait(q_full, 0, status), any = false;
     auto issue_s = [&](int j) -> bool {
       const int st = j & 1;
@@ -178,11 +179,9 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       tc_fence_after();
       const uint32_t v_addr = smem_u32(smem + FA_OFF_V + st * FA_KV_BYTES);
 #pragma unroll
-      for (int ks = 0; ks < FA_BN / 16; ++ks) {
-        const uint32_t p_off = (uint32_t)(ks >> 2) * FA_HALF + (uint32_t)(ks & 3) * 32;
-        umma_bf16(tmem + FA_TMEM_O, umma_desc_sw128(p_addr + p_off), umma_desc_sw128_mn(v_addr + ks * 2048, FA_HALF),
-                  idesc_o, (j | ks) != 0);
-      }
+      for (int ks = 0; ks < FA_BN / 16; ++ks)   // 16 keys = 8 P columns per step
+        umma_ts(tmem + FA_TMEM_O, tmem + FA_TMEM_P + ks * 8, umma_desc_sw128_mn(v_addr + ks * 2048, FA_HALF), idesc_o,
+                (j | ks) != 0);
       umma_commit(&v_empty[st]);
       umma_commit(o_done);
     }
@@ -197,7 +196,6 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     const int qpos = p0 + q0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t col0 = (uint32_t)half * 64;
-    uint8_t* p_row = smem + FA_OFF_P + half * FA_HALF + r * 128;
     float* red_max = reinterpret_cast<float*>(smem + FA_OFF_RED);       // [slot][half][row]
     float* red_sum = red_max + 4 * 128;                                  // [half][row]
     float m_used = -INFINITY, l = 0.f;
@@ -274,14 +272,9 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         }
         tmem_st_wait();
       }
-      // this thread's 64 keys fill swizzle block `half` of the P row:
-      // 16-byte chunk cc sits at position cc ^ (r % 8)
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        uint4* dst = reinterpret_cast<uint4*>(p_row + ((cc ^ (r & 7)) << 4));
-        *dst = make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-      }
-      fence_proxy_async_smem();
+      // this thread's 64 keys: P columns 32*half .. 32*half+31 of its lane
+      tmem_st32_u(tmem + lane_off + FA_TMEM_P + col0 / 2, pk);
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
     }

@@ -291,6 +291,158 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------- wide, pair
+// The same product on CTA pairs (clusters of 2 SMs): a pair owns a 256x256
+// output tile; each CTA loads its 128 rows of A and its 128 rows of W (half
+// of the tile's columns) per 64-wide k-block, and the leader CTA (rank 0)
+// issues tcgen05.mma.cta_group::2 (M=256, N=256), which reads the operands
+// from both CTAs' shared memory and leaves rows 0-127 of the tile in the
+// leader's TMEM and rows 128-255 in the peer's. Each SM thus moves 32 KB per
+// k-block instead of 48 KB for the same flops. Barriers: the TMA loads of
+// both CTAs count their bytes on the leader's `full` barrier; the leader's
+// commits arrive on `empty` and `accf` in both CTAs; both CTAs' epilogue
+// threads arrive on the leader's `acce`.
+constexpr int P_BM = 128, P_BN = 256;                 // rows per CTA, columns per pair tile
+constexpr int P_A_BYTES = P_BM * BK * 2;              // 16 KB
+constexpr int P_B_BYTES = (P_BN / 2) * BK * 2;        // 16 KB (this CTA's half of the columns)
+constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
+constexpr int P_STAGES = 6;
+constexpr int P_SMEM = P_STAGES * P_STAGE_BYTES + 1024 + 256;
+
+template <int KIND, typename T>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
+                     int K, EpiArgs epi, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES);
+  uint64_t* empty = full + P_STAGES;
+  uint64_t* accf = empty + P_STAGES;
+  uint64_t* acce = accf + 2;
+  uint64_t* drain = acce + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, pairs = gridDim.x >> 1;
+  const int m_tiles = (M + 2 * P_BM - 1) / (2 * P_BM), n_tiles = (N + P_BN - 1) / P_BN;
+  const int tiles = m_tiles * n_tiles;
+  const int kb = (K + BK - 1) / BK;
+
+  pdl_trigger();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&accf[a], 1); mbar_init(&acce[a], 2 * 128); }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) { tmem_alloc2(tmem_slot, 512); tmem_relinquish2(); }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised, TMEM of both allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    const uint64_t pol_a = l2_policy_evict_last(), pol_b = l2_policy_evict_last();
+    const int first = pair < tiles ? pair : -1;
+    const int pre = first >= 0 ? (kb < P_STAGES ? kb : P_STAGES) : 0;
+    {  // weight halves of the first stages before waiting for the previous kernel
+      const int n0 = first >= 0 ? (first / m_tiles) * P_BN + (int)rank * (P_BN / 2) : 0;
+      for (int k = 0; k < pre; ++k) {
+        if (leader) mbar_arrive_expect_tx(&full[k], 2 * P_STAGE_BYTES);
+        tma_load_2d_pair(smem + k * P_STAGE_BYTES + P_A_BYTES, &tmB, mapa_shared(smem_u32(&full[k]), 0), k * BK, n0,
+                         pol_b);
+      }
+      pdl_wait();
+      const int m0 = first >= 0 ? (first % m_tiles) * 2 * P_BM + (int)rank * P_BM : 0;
+      for (int k = 0; k < pre; ++k)
+        tma_load_2d_pair(smem + k * P_STAGE_BYTES, &tmA, mapa_shared(smem_u32(&full[k]), 0), k * BK, m0, pol_a);
+    }
+    int stage = pre % P_STAGES, issued = pre;
+    uint32_t phase = pre == P_STAGES ? 1u : 0u;
+    bool ok = true;
+    for (int t = pair; t < tiles && ok; t += pairs) {
+      const int m0 = (t % m_tiles) * 2 * P_BM + (int)rank * P_BM;
+      const int n0 = (t / m_tiles) * P_BN + (int)rank * (P_BN / 2);
+      for (int k = (t == pair ? pre : 0); k < kb; ++k) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, status)) { ok = false; break; }
+        uint8_t* sa = smem + stage * P_STAGE_BYTES;
+        const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
+        tma_load_2d_pair(sa, &tmA, fb, k * BK, m0, pol_a);
+        tma_load_2d_pair(sa + P_A_BYTES, &tmB, fb, k * BK, n0, pol_b);
+        ++issued;
+        if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+    if (!ok && leader) drain_loads(full, stage, phase, issued, P_STAGES, status);
+  } else if (warp == 1 && lane == 0 && leader) {
+    constexpr uint32_t idesc = umma_idesc_16(UmmaFmt<T>::value, 2 * P_BM, P_BN);
+    int stage = 0, acc = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    bool ok = true, any = false;
+    for (int t = pair; t < tiles && ok; t += pairs) {
+      if (!mbar_wait_cluster(&acce[acc], acc_phase ^ 1, status)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + acc * P_BN;
+      for (int k = 0; k < kb; ++k) {
+        if (!mbar_wait(&full[stage], phase, status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + stage * P_STAGE_BYTES);
+        const uint32_t b_addr = a_addr + P_A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          umma2_f16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), idesc,
+                    (k | kk) != 0);
+        umma2_commit_pair(&empty[stage], 0x3);
+        any = true;
+        if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      umma2_commit_pair(&accf[acc], 0x3);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+    if (!ok && any) {  // let issued MMAs finish before TMEM is released
+      umma2_commit_pair(drain, 0x1);
+      mbar_wait(drain, 0, status);
+    }
+  } else if (warp >= 2) {
+    pdl_wait();  // the epilogue reads and writes memory owned by earlier kernels
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool failed = false;  // after a timed-out wait the MMA has stopped: no further waits
+    for (int t = pair; t < tiles; t += pairs) {
+      const int m0 = (t % m_tiles) * 2 * P_BM + (int)rank * P_BM, n0 = (t / m_tiles) * P_BN;
+      if (!failed) failed = !__all_sync(0xffffffffu, mbar_wait(&accf[acc], acc_phase, status));
+      tc_fence_after();
+      const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + acc * P_BN;
+#pragma unroll 1
+      for (int c = 0; c < P_BN / 32; ++c) {
+        float v[32];
+        if (!failed) {
+          tmem_ld32(base + c * 32, v);
+          if (n0 + c * 32 < N) epi_row32<KIND, T>(epi, m0 + row, n0 + c * 32, v);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(mapa_shared(smem_u32(&acce[acc]), 0));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();  // no MMA of the pair and no epilogue read is left when TMEM goes
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc2(tmem, 512);
+  }
+}
+
 // ---------------------------------------------------------------- skinny
 // Stream-K over (weight tile, k-block) units: of the U = tiles * kb units
 // (tile-major), CTA c of G takes [U*c/G, U*(c+1)/G), so every CTA streams the
@@ -674,6 +826,42 @@ static int launch_wide(const CUtensorMap& ta, const CUtensorMap& tb, int M, int 
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
+bool pair_gemm_enabled() {
+  static const bool on = getenv("LLAMA_NO_PAIR_GEMM") == nullptr;
+  return on;
+}
+
+template <int KIND, typename T>
+static int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, const EpiArgs& e,
+                       int* status, cudaStream_t st) {
+  auto kern = gemm_pair_kernel<KIND, T>;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM) != cudaSuccess)
+      return LLAMA_ERR_CUDA;
+    attr = true;
+  }
+  const int tiles = ((M + 2 * P_BM - 1) / (2 * P_BM)) * ((N + P_BN - 1) / P_BN);
+  const int pairs = std::min(tiles, num_sms() / 2);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = P_SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  count_launches(1);
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, ta, tb, M, N, K, e, status);
+  return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
 template <int KIND, typename T, int NT>
 static int launch_skinny_nt(const CUtensorMap& tw, const CUtensorMap& tx, int M, int N, int K, const EpiArgs& e,
                             float* ws, int* tickets, float* stg, int* status, cudaStream_t st) {
@@ -729,6 +917,18 @@ static int gemm16_t(const void* A, int M, int K, int lda, const void* W, int N, 
   int rc;
   if (!skinny) {
     CUtensorMap ta, tb;
+    if (pair_gemm_enabled() && wide_split(M, N, K).sk_tiles == 0) {
+      // at least one full wave of 128x256 tiles: CTA pairs on 256x256 tiles
+      if ((rc = make_tmap_16(&ta, A, M, K, lda, P_BM, F16)) != LLAMA_OK) return rc;
+      if ((rc = make_tmap_16(&tb, W, N, K, ldw, P_BN / 2, F16)) != LLAMA_OK) return rc;
+      switch (kind) {
+        case EPI_STORE_F32: return launch_pair<EPI_STORE_F32, T>(ta, tb, M, N, K, e, status, st);
+        case EPI_RESIDUAL: return launch_pair<EPI_RESIDUAL, T>(ta, tb, M, N, K, e, status, st);
+        case EPI_SWIGLU: return launch_pair<EPI_SWIGLU, T>(ta, tb, M, N, K, e, status, st);
+        case EPI_QKV_ROPE: return launch_pair<EPI_QKV_ROPE, T>(ta, tb, M, N, K, e, status, st);
+      }
+      return LLAMA_ERR_INVALID_ARG;
+    }
     if ((rc = make_tmap_16(&ta, A, M, K, lda, W_BM, F16)) != LLAMA_OK) return rc;
     if ((rc = make_tmap_16(&tb, W, N, K, ldw, W_BN, F16)) != LLAMA_OK) return rc;
     switch (kind) {

@@ -52,6 +52,8 @@ GEMM_CASES = [
     (200, 520, 4104, 2),     # ragged everything, NT = 256
     (100, 384, 256, 2),      # short K (one split)
     (64, 1024, 1024, 1),     # wide path with few rows
+    (2100, 6000, 4104, 1),   # CTA-pair path with ragged M, N and K
+    (4096, 4096, 1024, 1),   # CTA-pair path, several tiles per pair
 ]
 
 
