@@ -179,6 +179,10 @@ def run_reference(args):
 
 # ---------------------------------------------------------------- our arm
 D_, F_, H_, HK_, HD_, V_ = 4096, 14336, 32, 8, 128, 128256
+# Measured DRAM bytes per launch of the prefill projection GEMM (mean over a
+# layer's QKV, Wo, w1/w3, w2 launches at 2048 tokens; one ncu capture of the
+# current kernel). Set to None when the kernel changes until re-captured.
+PAIR_GEMM_TRAFFIC = 187.6e6
 
 
 def measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust, peak_src):
@@ -230,9 +234,11 @@ def measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust, peak_src)
                    'share': v[0] / total_prof} for k, v in prof.items() if v[1]}
     attn_flops = 4.0 * PREFILL_B * H_ * HD_ * PREFILL_S * (PREFILL_S + 1) / 2 * NL
     attn = prof.get('attention_prefill', (0, 0))
-    roofline = {'kernel': 'gemm_wide_kernel (tcgen05, 4 projections)', 'bound': 'tensor',
+    roofline = {'kernel': 'gemm_pair_kernel (tcgen05 cta_group::2, 4 projections)', 'bound': 'tensor',
                 'achieved': achieved, 'peak': tf_sust, 'unit': 'TFLOP/s',
-                'frac': achieved / tf_sust if achieved else None, 'traffic': None,
+                'frac': achieved / tf_sust if achieved else None, 'traffic': PAIR_GEMM_TRAFFIC,
+                'traffic_note': 'DRAM read+write bytes per launch, mean of one layer\'s four launches, '
+                                'ncu (profiles/gemm_pair_kernel_llama3_8b_prefill_s2048.md)',
                 'peak_kind': f'bf16 sustained ({peak_src}); fp16 has the same nominal tensor rate',
                 'launches': gemm_launches // max(args.steps, 1),
                 'attention_tflops': attn_flops * args.steps / (attn[0] / 1e3) / 1e12 if attn[0] else None,
