@@ -77,6 +77,11 @@ typedef struct llama_config {
   int32_t max_seq;            /* positions per sequence in the KV cache */
   int32_t max_tokens;         /* largest B*S of one prefill call; 0 = min(max_batch*max_seq, 16384) */
   int32_t dtype;              /* llama_dtype */
+  int32_t kv_page_size;       /* 0: contiguous cache [n_layers][max_batch][n_kv_heads][max_seq][head_dim];
+                                 128: paged cache [n_layers][kv_pages][n_kv_heads][128][head_dim] with a block
+                                 table (16-bit models; pages are taken from a pool as sequences grow and
+                                 returned by llama_reset / llama_set_lengths) */
+  int32_t kv_pages;           /* paged: pages in the pool; 0 = max_batch * ceil(max_seq / 128) */
 } llama_config;
 
 typedef struct llama_model llama_model; /* opaque: weights, KV cache, lengths, workspace */
@@ -149,6 +154,10 @@ int llama_fill_kv_random(llama_model* m, uint64_t seed, int32_t c, void* stream)
 int llama_set_kv(llama_model* m, int32_t layer, const void* k, const void* v, int32_t B, int32_t c, void* stream);
 int llama_set_lengths(llama_model* m, const int32_t* host_len, int32_t B, void* stream);
 int llama_get_lengths(const llama_model* m, int32_t* host_len, int32_t B);
+/* Paged models: the block table of sequences 0..B-1 (host int32 [B][ceil(max_seq/128)]): the pool page
+ * holding positions 128j .. 128j+127 of sequence b, -1 past its pages. LLAMA_ERR_UNSUPPORTED when the
+ * cache is contiguous. */
+int llama_get_block_table(const llama_model* m, int32_t* host_table, int32_t B);
 int llama_reset(llama_model* m, void* stream);
 
 /* Per-kernel timing of eager model calls: while enabled (1), an event is recorded on the
@@ -207,6 +216,20 @@ int llama_attention_decode(const void* q, const void* kc, const void* vc, const 
 int llama_attention_decode_noalloc(const void* q, const void* kc, const void* vc, const int32_t* len, void* o,
                                    int32_t B, int32_t cmax, int32_t H, int32_t Hk, int32_t d, int32_t dtype,
                                    void* stream);
+
+/* Paged-cache forms (16-bit, d = 128): k_pages, v_pages [n_pages][Hk][128][d]; table (device int32
+ * [B][max_pages]) gives page j of sequence b (keys 128j .. 128j+127); entries must lie in [-1, n_pages),
+ * -1 marking an unused slot, else LLAMA_ERR_SHAPE (the table is read back to the host to check it).
+ * Prefill: q [B][H][S][d]; sequence b's S queries sit at positions pos0[b] .. pos0[b]+S-1 (pos0 device
+ * int32 [B], NULL = all 0) and see keys 0 .. their own position, which the caller has already written into
+ * the pages; o [B][S][H*d]. Decode: q [B][H][d], len (device int32 [B]) keys per sequence, o [B][H*d].
+ * Same kernels as the model's paged cache ([W] 查询和键相乘, 掩码; [H]: the cache sized by max_seq_len). */
+int llama_attention_prefill_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* table,
+                                  int32_t max_pages, int32_t n_pages, const int32_t* pos0, void* o, int32_t B,
+                                  int32_t S, int32_t H, int32_t Hk, int32_t d, int32_t dtype, void* stream);
+int llama_attention_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* table,
+                                 int32_t max_pages, int32_t n_pages, const int32_t* len, void* o, int32_t B,
+                                 int32_t H, int32_t Hk, int32_t d, int32_t dtype, void* stream);
 
 /* y = x W^T: x [M][K], w [N][K] (dtype), y fp32 [M][N]. variant 0 = automatic, 1 = the wide
  * persistent tcgen05 kernel, 2 = the skinny split-K tcgen05 kernel (M <= 256); fp32 ignores it.

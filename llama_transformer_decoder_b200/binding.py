@@ -38,7 +38,8 @@ class llama_config(ctypes.Structure):
                 ('n_kv_heads', ctypes.c_int32), ('vocab_size', ctypes.c_int32), ('ffn_hidden', ctypes.c_int32),
                 ('multiple_of', ctypes.c_int32), ('ffn_dim_multiplier', ctypes.c_float),
                 ('norm_eps', ctypes.c_float), ('rope_theta', ctypes.c_float), ('max_batch', ctypes.c_int32),
-                ('max_seq', ctypes.c_int32), ('max_tokens', ctypes.c_int32), ('dtype', ctypes.c_int32)]
+                ('max_seq', ctypes.c_int32), ('max_tokens', ctypes.c_int32), ('dtype', ctypes.c_int32),
+                ('kv_page_size', ctypes.c_int32), ('kv_pages', ctypes.c_int32)]
 
 
 if not os.path.exists(LIB_PATH):
@@ -71,6 +72,7 @@ _SIGS = {
     'llama_set_kv': (ctypes.c_int, [_P, _I32, _P, _P, _I32, _I32, _P]),
     'llama_set_lengths': (ctypes.c_int, [_P, _P, _I32, _P]),
     'llama_get_lengths': (ctypes.c_int, [_P, _P, _I32]),
+    'llama_get_block_table': (ctypes.c_int, [_P, _P, _I32]),
     'llama_reset': (ctypes.c_int, [_P, _P]),
     'llama_sync_status': (ctypes.c_int, [_P, _P]),
     'llama_status_string': (ctypes.c_char_p, [ctypes.c_int]),
@@ -78,6 +80,10 @@ _SIGS = {
     'llama_attention_decode': (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P]),
     'llama_attention_decode_noalloc': (ctypes.c_int, [_P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _I32,
                                                       _P]),
+    'llama_attention_prefill_paged': (ctypes.c_int, [_P, _P, _P, _P, _I32, _I32, _P, _P, _I32, _I32, _I32, _I32,
+                                                     _I32, _I32, _P]),
+    'llama_attention_decode_paged': (ctypes.c_int, [_P, _P, _P, _P, _I32, _I32, _P, _P, _I32, _I32, _I32, _I32,
+                                                    _I32, _P]),
     'llama_linear': (ctypes.c_int, [_P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P]),
     'llama_rmsnorm': (ctypes.c_int, [_P, _P, _P, _I32, _I32, _F, _I32, _P]),
     'llama_argmax_rows': (ctypes.c_int, [_P, _P, _I32, _I32, _P]),
@@ -206,6 +212,10 @@ def llama_get_lengths(model, host_len, B):
     _check(_lib.llama_get_lengths(model, _ptr(host_len), B), 'llama_get_lengths')
 
 
+def llama_get_block_table(model, host_table, B):
+    _check(_lib.llama_get_block_table(model, _ptr(host_table), B), 'llama_get_block_table')
+
+
 def llama_reset(model, stream=None):
     _check(_lib.llama_reset(model, _stream(stream)), 'llama_reset')
 
@@ -222,6 +232,20 @@ def llama_attention_prefill(q, k, v, o, B, S, H, Hk, d, dtype, stream=None):
 def llama_attention_decode(q, kc, vc, length, o, B, cmax, H, Hk, d, dtype, stream=None):
     _check(_lib.llama_attention_decode(_ptr(q), _ptr(kc), _ptr(vc), _ptr(length), _ptr(o), B, cmax, H, Hk, d, dtype,
                                        _stream(stream)), 'llama_attention_decode')
+
+
+def llama_attention_prefill_paged(q, k_pages, v_pages, table, max_pages, n_pages, pos0, o, B, S, H, Hk, d, dtype,
+                                  stream=None):
+    _check(_lib.llama_attention_prefill_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(table), max_pages, n_pages,
+                                              _ptr(pos0) if pos0 is not None else None, _ptr(o), B, S, H, Hk, d,
+                                              dtype, _stream(stream)), 'llama_attention_prefill_paged')
+
+
+def llama_attention_decode_paged(q, k_pages, v_pages, table, max_pages, n_pages, length, o, B, H, Hk, d, dtype,
+                                 stream=None):
+    _check(_lib.llama_attention_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(table), max_pages, n_pages,
+                                             _ptr(length), _ptr(o), B, H, Hk, d, dtype, _stream(stream)),
+           'llama_attention_decode_paged')
 
 
 def llama_attention_decode_noalloc(q, kc, vc, length, o, B, cmax, H, Hk, d, dtype, stream=None):

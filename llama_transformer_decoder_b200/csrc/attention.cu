@@ -363,10 +363,10 @@ __device__ bool tc_next(TileCursor& c, const int32_t* nkeys, int add, int nmax, 
 
 template <typename T>
 __device__ __forceinline__ void dm_load_tile(uint8_t* stage, const T* kc, const T* vc, const TileCursor& c,
-                                             int Hk, int Smax, int lane) {
+                                             int Hk, const KvLayout& L, int lane) {
   const int key0 = c.t * DM_KEYS;
   const int valid = min(DM_KEYS, c.n - key0);
-  const size_t row0 = ((size_t)c.b * Hk + c.g) * Smax + key0;
+  const size_t row0 = kv_row(L, Hk, c.b, c.g, key0);   // a 32-key tile never crosses a 128-key page
   const T* ks = kc + row0 * 128;
   const T* vs = vc + row0 * 128;
 #pragma unroll
@@ -384,7 +384,7 @@ template <typename T>
 __global__ void __launch_bounds__(DM_WARPS * 32, 1)
     attn_decode_mma_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
                            const int32_t* __restrict__ nkeys, int add_keys, int nmax, float* __restrict__ part, int B,
-                           int H, int Hk, int Smax, float scale_log2, int* status) {
+                           int H, int Hk, KvLayout L, float scale_log2, int* status) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ __align__(128) uint8_t sm[];
@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
   bool ld_done = ld.left <= 0;
   for (int i = 0; i < DM_STAGES - 1; ++i) {
     if (!ld_done) {
-      dm_load_tile(ring + (issued % DM_STAGES) * DM_STAGE, kc, vc, ld, Hk, Smax, lane);
+      dm_load_tile(ring + (issued % DM_STAGES) * DM_STAGE, kc, vc, ld, Hk, L, lane);
       ++issued;
       tc_next(ld, nkeys, add_keys, nmax, B, Hk);
       ld_done = ld.left <= 0;
@@ -439,7 +439,7 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
       start = false;
     }
     if (!ld_done) {   // keep DM_STAGES-1 tiles in flight
-      dm_load_tile(ring + (issued % DM_STAGES) * DM_STAGE, kc, vc, ld, Hk, Smax, lane);
+      dm_load_tile(ring + (issued % DM_STAGES) * DM_STAGE, kc, vc, ld, Hk, L, lane);
       ++issued;
       tc_next(ld, nkeys, add_keys, nmax, B, Hk);
       ld_done = ld.left <= 0;
@@ -618,15 +618,18 @@ int decode_launch(const void* q, const void* kc, const void* vc, const int32_t* 
 }  // namespace
 
 int attention_prefill(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B, int S,
-                      int H, int Hk, int d, int Smax, int dtype, int* status, cudaStream_t st) {
+                      int H, int Hk, int d, int Smax, int dtype, int* status, cudaStream_t st, const int32_t* kv_table,
+                      int kv_max_pages, int kv_pages) {
   (void)status;
   if (B <= 0 || S <= 0) return LLAMA_OK;
   if (H % Hk != 0) return LLAMA_ERR_SHAPE;
   const float scale_log2 = kLog2e / sqrtf((float)d);
   if (dtype == LLAMA_BF16 || dtype == LLAMA_F16) {
     if (d != 128) return LLAMA_ERR_UNSUPPORTED;
-    return attention_prefill_tc(q, kc, vc, o, pos0, B, S, H, Hk, Smax, dtype, status, st);
+    return attention_prefill_tc(q, kc, vc, o, pos0, B, S, H, Hk, Smax, dtype, status, st, kv_table, kv_max_pages,
+                                kv_pages);
   } else {
+    if (kv_table) return LLAMA_ERR_UNSUPPORTED;   // paged caches: 16-bit, head_dim 128 only
     dim3 grid(S, H, B);
     count_launches(1);
 #define LLAMA_F32_PREFILL(DD)                                                                                  \
@@ -663,8 +666,8 @@ size_t decode_scratch_floats(int cmax, int B, int H, int Hk, int d, int dtype) {
 
 template <typename T>
 static int mma_decode_launch(const void* q, const void* kc, const void* vc, const int32_t* nkeys, int add_keys,
-                             void* o, int B, int cmax, int H, int Hk, int Smax, DecodeScratch* scratch, int* status,
-                             cudaStream_t st) {
+                             void* o, int B, int cmax, int H, int Hk, int Smax, const KvLayout& L,
+                             DecodeScratch* scratch, int* status, cudaStream_t st) {
   const int grid = num_sms();
   auto kern = attn_decode_mma_kernel<T>;
   static bool attr = false;
@@ -677,7 +680,7 @@ static int mma_decode_launch(const void* q, const void* kc, const void* vc, cons
   const int nmax = cmax < Smax ? cmax : Smax;
   cudaError_t err = launch_k(kern, dim3(grid), dim3(DM_WARPS * 32), DM_SMEM, st, static_cast<const T*>(q),
                              static_cast<const T*>(kc), static_cast<const T*>(vc), nkeys, add_keys, nmax,
-                             scratch->part, B, H, Hk, Smax, scale_log2, status);
+                             scratch->part, B, H, Hk, L, scale_log2, status);
   if (err == cudaSuccess)
     err = launch_k(attn_decode_combine_pieces_kernel<T, 128>, dim3(H, B), dim3(128), 0, st,
                    (const float*)scratch->part, nkeys, add_keys, nmax, static_cast<T*>(o), B, H, Hk,
@@ -687,16 +690,18 @@ static int mma_decode_launch(const void* q, const void* kc, const void* vc, cons
 
 int attention_decode(const void* q, const void* kc, const void* vc, const int32_t* nkeys, int add_keys, void* o,
                      int B, int cmax, int H, int Hk, int d, int Smax, int dtype, DecodeScratch* scratch, int* status,
-                     cudaStream_t st) {
+                     cudaStream_t st, const int32_t* kv_table, int kv_max_pages, int kv_pages) {
   if (B <= 0) return LLAMA_OK;
   if (H % Hk != 0 || H / Hk > DEC_MAXG) return LLAMA_ERR_SHAPE;
   if (!scratch || !scratch->part || scratch->floats < decode_scratch_floats(cmax, B, H, Hk, d, dtype))
     return LLAMA_ERR_INVALID_ARG;
+  const KvLayout L{kv_table, kv_max_pages, Smax, kv_pages};
   if (use_mma_decode(d, dtype)) {
     if (dtype == LLAMA_F16)
-      return mma_decode_launch<f16>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch, status, st);
-    return mma_decode_launch<bf16>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch, status, st);
+      return mma_decode_launch<f16>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, L, scratch, status, st);
+    return mma_decode_launch<bf16>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, L, scratch, status, st);
   }
+  if (kv_table) return LLAMA_ERR_UNSUPPORTED;   // paged caches: 16-bit, head_dim 128 only
   const int splits = decode_splits(cmax, B, Hk);
   if (dtype == LLAMA_BF16) {
     if (d == 64) return decode_launch<bf16, 64>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch->part,

@@ -56,6 +56,12 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Page j of sequence b (page 0 for an index outside the pool).
+__device__ __forceinline__ int kv_page(const int32_t* table, int max_pages, int n_pages, int b, int j) {
+  const int p = table[(size_t)b * max_pages + j];
+  return (unsigned)p < (unsigned)n_pages ? p : 0;
+}
+
 __device__ __forceinline__ uint8_t* fa_align(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
@@ -66,7 +72,8 @@ template <typename T>
 __global__ void __launch_bounds__(FA_THREADS, 1)
     attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, T* __restrict__ o,
-                           const int32_t* __restrict__ pos0, int S, int H, int Hk, float scale_log2, int* status) {
+                           const int32_t* __restrict__ pos0, int S, int H, int Hk, float scale_log2,
+                           const int32_t* __restrict__ kv_table, int kv_max_pages, int kv_pages, int* status) {
   extern __shared__ uint8_t fa_smem_raw[];
   uint8_t* smem = fa_align(fa_smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + FA_OFF_BAR);
@@ -132,16 +139,20 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       const int st = j & 1;
       const uint32_t ph = (j >> 1) & 1;
       if (!mbar_wait(&k_empty[st], ph ^ 1, status)) { ok = false; break; }
+      // tile j: 128 keys of (b, g) at row j*128 of the contiguous cache, or
+      // all 128 rows of page kv_table[b][j] of the paged one
+      const int kv_y = kv_table ? 0 : j * FA_BN;
+      const int kv_z = kv_table ? kv_page(kv_table, kv_max_pages, kv_pages, b, j) * Hk + g : b * Hk + g;
       mbar_arrive_expect_tx(&k_full[st], FA_KV_BYTES);
       uint8_t* kd = smem + FA_OFF_K + st * FA_KV_BYTES;
-      tma_load_3d(kd, &tmK, &k_full[st], 0, j * FA_BN, b * Hk + g);
-      tma_load_3d(kd + FA_HALF, &tmK, &k_full[st], 64, j * FA_BN, b * Hk + g);
+      tma_load_3d(kd, &tmK, &k_full[st], 0, kv_y, kv_z);
+      tma_load_3d(kd + FA_HALF, &tmK, &k_full[st], 64, kv_y, kv_z);
       ++k_issued;
       if (!mbar_wait(&v_empty[st], ph ^ 1, status)) { ok = false; break; }
       mbar_arrive_expect_tx(&v_full[st], FA_KV_BYTES);
       uint8_t* vd = smem + FA_OFF_V + st * FA_KV_BYTES;
-      tma_load_3d(vd, &tmV, &v_full[st], 0, j * FA_BN, b * Hk + g);
-      tma_load_3d(vd + FA_HALF, &tmV, &v_full[st], 64, j * FA_BN, b * Hk + g);
+      tma_load_3d(vd, &tmV, &v_full[st], 0, kv_y, kv_z);
+      tma_load_3d(vd + FA_HALF, &tmV, &v_full[st], 64, kv_y, kv_z);
       ++v_issued;
     }
     if (!ok) {  // let issued copies land before the CTA can exit
@@ -342,13 +353,18 @@ int make_tmap_3d(CUtensorMap* map, const void* base, int64_t outer, int64_t rows
 
 template <typename T>
 static int attention_prefill_tc_t(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B,
-                                  int S, int H, int Hk, int Smax, int* status, cudaStream_t st) {
+                                  int S, int H, int Hk, int Smax, int* status, cudaStream_t st,
+                                  const int32_t* kv_table, int kv_max_pages, int kv_pages) {
   constexpr bool F16 = std::is_same<T, f16>::value;
   CUtensorMap tq, tk, tv;
   int rc;
+  // contiguous: [B*Hk][Smax][128]; paged: [kv_pages*Hk][128][128]
+  const int64_t kv_outer = kv_table ? (int64_t)kv_pages * Hk : (int64_t)B * Hk;
+  const int64_t kv_rows = kv_table ? KV_PAGE : Smax;
+  if (kv_table && (kv_pages <= 0 || kv_max_pages <= 0)) return LLAMA_ERR_INVALID_ARG;
   if ((rc = make_tmap_3d(&tq, q, (int64_t)B * H, S, F16)) != LLAMA_OK) return rc;
-  if ((rc = make_tmap_3d(&tk, kc, (int64_t)B * Hk, Smax, F16)) != LLAMA_OK) return rc;
-  if ((rc = make_tmap_3d(&tv, vc, (int64_t)B * Hk, Smax, F16)) != LLAMA_OK) return rc;
+  if ((rc = make_tmap_3d(&tk, kc, kv_outer, kv_rows, F16)) != LLAMA_OK) return rc;
+  if ((rc = make_tmap_3d(&tv, vc, kv_outer, kv_rows, F16)) != LLAMA_OK) return rc;
   auto kern = attn_prefill_tc_kernel<T>;
   static bool attr = false;
   if (!attr) {
@@ -359,14 +375,19 @@ static int attention_prefill_tc_t(const void* q, const void* kc, const void* vc,
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)FA_D);
   const cudaError_t err = launch_k(kern, dim3(((S + FA_BM - 1) / FA_BM) * H * B), dim3(FA_THREADS), FA_SMEM, st, tq,
                                    tk, tv,
-                                   static_cast<T*>(o), pos0, S, H, Hk, scale_log2, status);
+                                   static_cast<T*>(o), pos0, S, H, Hk, scale_log2, kv_table, kv_max_pages, kv_pages,
+                                   status);
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 int attention_prefill_tc(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B, int S,
-                         int H, int Hk, int Smax, int elt, int* status, cudaStream_t st) {
-  if (elt == LLAMA_F16) return attention_prefill_tc_t<f16>(q, kc, vc, o, pos0, B, S, H, Hk, Smax, status, st);
-  return attention_prefill_tc_t<bf16>(q, kc, vc, o, pos0, B, S, H, Hk, Smax, status, st);
+                         int H, int Hk, int Smax, int elt, int* status, cudaStream_t st, const int32_t* kv_table,
+                         int kv_max_pages, int kv_pages) {
+  if (elt == LLAMA_F16)
+    return attention_prefill_tc_t<f16>(q, kc, vc, o, pos0, B, S, H, Hk, Smax, status, st, kv_table, kv_max_pages,
+                                       kv_pages);
+  return attention_prefill_tc_t<bf16>(q, kc, vc, o, pos0, B, S, H, Hk, Smax, status, st, kv_table, kv_max_pages,
+                                      kv_pages);
 }
 
 }  // namespace llama

@@ -63,6 +63,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// ------------------------------------------------------------ KV cache rows
+// K and V caches are arrays of 128-element rows (one head_dim-128 key or value
+// per row; head_dim 32 and 64 rows are used contiguously only). Contiguous:
+// [sequence][kv head][Smax] rows. Paged: pages of KV_PAGE positions,
+// [page][kv head][KV_PAGE] rows, page j of sequence b = table[b*max_pages + j].
+constexpr int KV_PAGE = 128;
+struct KvLayout {
+  const int32_t* table;  // nullptr: contiguous
+  int max_pages;         // row pitch of the table
+  int Smax;              // contiguous: positions per (sequence, kv head)
+  int n_pages;           // paged: pages in the pool (a page index outside [0, n_pages) reads page 0)
+};
+__host__ __device__ __forceinline__ size_t kv_row(const KvLayout& L, int Hk, int b, int g, int pos) {
+  if (!L.table) return ((size_t)b * Hk + g) * L.Smax + pos;
+  int page = L.table[(size_t)b * L.max_pages + pos / KV_PAGE];
+  if ((unsigned)page >= (unsigned)L.n_pages) page = 0;   // memory safety; hosts validate tables
+  return ((size_t)page * Hk + g) * KV_PAGE + (pos % KV_PAGE);
+}
+
 // ------------------------------------------------------- CTA pairs (clusters of 2)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

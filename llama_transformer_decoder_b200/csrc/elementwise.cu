@@ -328,6 +328,72 @@ int launch_convert_2d(void* dst, int64_t dpitch, int dst_elt, const void* src, i
   return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
+namespace {
+// Element i of the logical cache [B][Hk][c][d] (the generator's order) is
+// written through the cache layout L.
+template <typename T, bool ROUND_BF16>
+__global__ void fill_kv_kernel(T* __restrict__ dst, KvLayout L, int Hk, int c, int d, int64_t n, uint64_t key,
+                               double sd) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int dd = (int)(i % d);
+    const int64_t r = i / d;
+    const int t = (int)(r % c);
+    const int64_t bg = r / c;
+    const int g = (int)(bg % Hk), b = (int)(bg / Hk);
+    float v = seeded_normal(key, (uint64_t)i, sd);
+    if (ROUND_BF16) v = __bfloat162float(__float2bfloat16_rn(v));
+    dst[kv_row(L, Hk, b, g, t) * d + dd] = from_f<T>(v);
+  }
+}
+
+// dst (through L) <- src [B][Hk][c][d], converting S -> D.
+template <typename D, typename S>
+__global__ void kv_scatter_kernel(D* __restrict__ dst, KvLayout L, int Hk, int c, int d, const S* __restrict__ src,
+                                  int64_t n) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int dd = (int)(i % d);
+    const int64_t r = i / d;
+    const int t = (int)(r % c);
+    const int64_t bg = r / c;
+    const int g = (int)(bg % Hk), b = (int)(bg / Hk);
+    dst[kv_row(L, Hk, b, g, t) * d + dd] = from_f<D>(to_f<S>(src[i]));
+  }
+}
+}  // namespace
+
+int launch_fill_kv(void* dst, const KvLayout& L, int B, int Hk, int c, int d, uint64_t seed, uint64_t stream_id,
+                   float std, int dtype, bool round_bf16, cudaStream_t st) {
+  const int64_t n = (int64_t)B * Hk * c * d;
+  if (n <= 0) return LLAMA_OK;
+  const uint64_t key = stream_key(seed, stream_id);
+  count_launches(1);
+  if (dtype == LLAMA_F16 && round_bf16)
+    fill_kv_kernel<f16, true><<<grid_for(n), 256, 0, st>>>(static_cast<f16*>(dst), L, Hk, c, d, n, key, std);
+  else if (dtype == LLAMA_F16)
+    fill_kv_kernel<f16, false><<<grid_for(n), 256, 0, st>>>(static_cast<f16*>(dst), L, Hk, c, d, n, key, std);
+  else if (dtype == LLAMA_BF16)
+    fill_kv_kernel<bf16, false><<<grid_for(n), 256, 0, st>>>(static_cast<bf16*>(dst), L, Hk, c, d, n, key, std);
+  else
+    fill_kv_kernel<float, false><<<grid_for(n), 256, 0, st>>>(static_cast<float*>(dst), L, Hk, c, d, n, key, std);
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int launch_kv_scatter(void* dst, int dst_elt, const KvLayout& L, int B, int Hk, int c, int d, const void* src,
+                      int src_elt, cudaStream_t st) {
+  const int64_t n = (int64_t)B * Hk * c * d;
+  if (n <= 0) return LLAMA_OK;
+  count_launches(1);
+#define LLAMA_SCATTER(DT, ST) \
+  kv_scatter_kernel<DT, ST><<<grid_for(n), 256, 0, st>>>(static_cast<DT*>(dst), L, Hk, c, d, static_cast<const ST*>(src), n)
+  if (dst_elt == LLAMA_F16 && src_elt == LLAMA_BF16) LLAMA_SCATTER(f16, bf16);
+  else if (dst_elt == LLAMA_F16 && src_elt == LLAMA_F16) LLAMA_SCATTER(f16, f16);
+  else if (dst_elt == LLAMA_BF16 && src_elt == LLAMA_BF16) LLAMA_SCATTER(bf16, bf16);
+  else if (dst_elt == LLAMA_F32 && src_elt == LLAMA_F32) LLAMA_SCATTER(float, float);
+  else return LLAMA_ERR_INVALID_ARG;
+#undef LLAMA_SCATTER
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
 int launch_fill_const(float* dst, int64_t n, float v, cudaStream_t st) {
   if (n <= 0) return LLAMA_OK;
   count_launches(1);

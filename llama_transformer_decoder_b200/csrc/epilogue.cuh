@@ -23,12 +23,20 @@ struct EpiArgs {
   void* g;            // SWIGLU output (T = model dtype), row pitch ldg
   int ldg;
   void* q;            // QKV_ROPE: q output [B][H][S][d]
-  void* kc;           // K cache of this layer [Bmax][Hk][Smax][d]
+  void* kc;           // K cache of this layer: [Bmax][Hk][Smax][d], or paged [pages][Hk][128][d]
   void* vc;           // V cache of this layer
   const float2* rope; // (cos, sin) table [Smax][d/2]
   const int* pos0;    // per-sequence position of the call's first token
   int S, H, Hk, d, Smax;
+  const int32_t* kv_table;  // paged cache block table (nullptr: contiguous)
+  int kv_max_pages, kv_pages;
 };
+
+// Element offset of (sequence b, kv head g, position pos, dim 0) in a K/V cache.
+__device__ __forceinline__ size_t kv_elem(const EpiArgs& e, int b, int g, int pos) {
+  const KvLayout L{e.kv_table, e.kv_max_pages, e.Smax, e.kv_pages};
+  return kv_row(L, e.Hk, b, g, pos) * (size_t)e.d;
+}
 
 // One rotated (or plain) value of the q/k/v block. n is the column, v its
 // accumulator and partner the accumulator of column n^1.
@@ -51,7 +59,7 @@ __device__ __forceinline__ void qkv_store(const EpiArgs& e, int m, int n, float 
     const int nn = n - hd - (is_k ? 0 : e.Hk * e.d);
     const int g = nn / e.d, dd = nn - g * e.d;
     T* dst = static_cast<T*>(is_k ? e.kc : e.vc);
-    dst[(((size_t)b * e.Hk + g) * e.Smax + pos) * e.d + dd] = from_f<T>(r);
+    dst[kv_elem(e, b, g, pos) + dd] = from_f<T>(r);
   }
 }
 
@@ -149,7 +157,7 @@ __device__ __forceinline__ void epi_row32(const EpiArgs& e, int m, int n0, const
       const int nn = n0 - hd - (is_k ? 0 : e.Hk * e.d);
       const int g = nn / e.d;
       dd0 = nn - g * e.d;
-      dst = static_cast<T*>(is_k ? e.kc : e.vc) + (((size_t)b * e.Hk + g) * e.Smax + pos) * e.d + dd0;
+      dst = static_cast<T*>(is_k ? e.kc : e.vc) + kv_elem(e, b, g, pos) + dd0;
     }
     uint32_t w[16];
 #pragma unroll
@@ -219,7 +227,7 @@ __device__ __forceinline__ void epi_col32(const EpiArgs& e, int m0, int n, const
         const int nn = n - hd - (is_k ? 0 : e.Hk * e.d);
         const int g = nn / e.d, dd = nn - g * e.d;
         T* dst = static_cast<T*>(is_k ? e.kc : e.vc);
-        dst[(((size_t)b * e.Hk + g) * e.Smax + pos[j]) * e.d + dd] = from_f<T>(r);
+        dst[kv_elem(e, b, g, pos[j]) + dd] = from_f<T>(r);
       }
     }
   }

@@ -10,6 +10,7 @@
 namespace llama {
 
 struct EpiArgs;
+struct KvLayout;
 
 // Launch with programmatic stream serialization (the kernel must call
 // pdl_wait() before reading its predecessor's output). Disabled when the
@@ -80,11 +81,16 @@ int launch_add_lengths(int32_t* len, int B, int add, cudaStream_t st);
 
 // Attention. q [B][H][S][d]; K/V cache [B][Hk][Smax][d] (this layer);
 // o [B*S][H*d]; pos0[b] = position of the call's first query (null = 0).
+// Caches: contiguous [B][Hk][Smax][d] (kv_table == nullptr), or paged: pages
+// [kv_pages][Hk][128][d] with page j of sequence b at kv_table[b*kv_max_pages + j]
+// (16-bit, d = 128 only; Smax is then the per-sequence capacity).
 int attention_prefill(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B, int S,
-                      int H, int Hk, int d, int Smax, int dtype, int* status, cudaStream_t st);
+                      int H, int Hk, int d, int Smax, int dtype, int* status, cudaStream_t st,
+                      const int32_t* kv_table = nullptr, int kv_max_pages = 0, int kv_pages = 0);
 // tcgen05 flash attention for 16-bit q/k/v (elt = LLAMA_BF16 or LLAMA_F16), d = 128.
 int attention_prefill_tc(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B, int S,
-                         int H, int Hk, int Smax, int elt, int* status, cudaStream_t st);
+                         int H, int Hk, int Smax, int elt, int* status, cudaStream_t st,
+                         const int32_t* kv_table = nullptr, int kv_max_pages = 0, int kv_pages = 0);
 // Decode: q [B][H][d]; keys 0 .. nkeys[b]-1 (+ add) of the cache; o [B][H*d].
 struct DecodeScratch {
   float* part;  // [B][H][splits][d + 2]
@@ -93,7 +99,8 @@ struct DecodeScratch {
 size_t decode_scratch_floats(int cmax, int B, int H, int Hk, int d, int dtype);
 int attention_decode(const void* q, const void* kc, const void* vc, const int32_t* nkeys, int add_keys, void* o,
                      int B, int cmax, int H, int Hk, int d, int Smax, int dtype, DecodeScratch* scratch,
-                     int* status, cudaStream_t st);
+                     int* status, cudaStream_t st, const int32_t* kv_table = nullptr, int kv_max_pages = 0,
+                     int kv_pages = 0);
 
 // Seeded generator: SplitMix64 counter streams + Box-Muller from IEEE basic ops.
 // Logical element i = ((o * rows + r) * cols + c) of a [outer][rows][cols]
@@ -110,6 +117,13 @@ int launch_fill_normal(void* dst, const FillLayout& L, uint64_t seed, uint64_t s
 int launch_convert_2d(void* dst, int64_t dpitch, int dst_elt, const void* src, int64_t spitch, int src_elt,
                       int64_t rows, int64_t cols, cudaStream_t st);
 int launch_fill_const(float* dst, int64_t n, float v, cudaStream_t st);
+// N(0, std^2) draws of stream `stream_id` in the logical order [B][Hk][c][d]
+// (the cache generator's order), written through a cache layout.
+int launch_fill_kv(void* dst, const KvLayout& L, int B, int Hk, int c, int d, uint64_t seed, uint64_t stream_id,
+                   float std, int dtype, bool round_bf16, cudaStream_t st);
+// Cache (through L) <- src [B][Hk][c][d], converting src_elt -> dst_elt.
+int launch_kv_scatter(void* dst, int dst_elt, const KvLayout& L, int B, int Hk, int c, int d, const void* src,
+                      int src_elt, cudaStream_t st);
 int launch_fill_tokens(int32_t* dst, int64_t n, uint64_t seed, uint64_t stream_id, int vocab, cudaStream_t st);
 
 }  // namespace llama

@@ -72,6 +72,15 @@ struct llama_model {
   void* kcache = nullptr;
   void* vcache = nullptr;
   size_t layer_cache_elems = 0;
+  // paged cache: pool of n_pages pages of KV_PAGE positions, block table
+  // [max_batch][max_pages] on the device and its host copy, free pages, and
+  // the pages each sequence holds (table row prefix)
+  bool paged = false;
+  int max_pages = 0, n_pages = 0;
+  int32_t* d_table = nullptr;
+  std::vector<int32_t> h_table;
+  std::vector<int32_t> free_pages;
+  std::vector<int> seq_pages;
   int32_t* d_len = nullptr;
   std::vector<int32_t> h_len;
   float2* rope = nullptr;
@@ -139,6 +148,16 @@ int resolve(const llama_config* in, llama_config* c) {
   if (c->dtype != LLAMA_F32) {
     if (d != 128) return LLAMA_ERR_UNSUPPORTED;
     if (c->dim % 64 != 0 || c->ffn_hidden % 64 != 0) return LLAMA_ERR_SHAPE;
+  }
+  if (c->kv_page_size != 0) {
+    if (c->kv_page_size != KV_PAGE) return LLAMA_ERR_UNSUPPORTED;
+    if (c->dtype == LLAMA_F32) return LLAMA_ERR_UNSUPPORTED;   // paged attention kernels are 16-bit
+    if (c->kv_pages < 0) return LLAMA_ERR_SHAPE;
+    if (c->kv_pages == 0)
+      c->kv_pages = (int32_t)std::min<int64_t>((int64_t)c->max_batch * ((c->max_seq + KV_PAGE - 1) / KV_PAGE),
+                                               INT32_MAX);
+  } else {
+    c->kv_pages = 0;
   }
   if (c->max_tokens <= 0) {
     const int64_t mt = (int64_t)c->max_batch * c->max_seq;
@@ -314,15 +333,19 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
   e.Hk = Hk;
   e.d = d;
   e.Smax = c.max_seq;
+  e.kv_table = m->paged ? m->d_table : nullptr;
+  e.kv_max_pages = m->max_pages;
+  e.kv_pages = m->n_pages;
   mark(m, K_GEMM_QKV, st);
   RC(gemm(m, m->xn, M, D, w.wqkv, m->qkv_n, EPI_QKV_ROPE, e, st));
   if (decode) {
     mark(m, K_ATTN_DECODE, st);
     RC(attention_decode(m->q, kc, vc, m->d_len, 1, m->attn, B, cmax, H, Hk, d, c.max_seq, m->adt, &m->ds,
-                        m->d_status, st));
+                        m->d_status, st, e.kv_table, m->max_pages, m->n_pages));
   } else {
     mark(m, K_ATTN_PREFILL, st);
-    RC(attention_prefill(m->q, kc, vc, m->attn, m->d_len, B, S, H, Hk, d, c.max_seq, m->adt, m->d_status, st));
+    RC(attention_prefill(m->q, kc, vc, m->attn, m->d_len, B, S, H, Hk, d, c.max_seq, m->adt, m->d_status, st,
+                         e.kv_table, m->max_pages, m->n_pages));
   }
   EpiArgs r = epi_base(M, D);
   r.out = m->x;
@@ -362,6 +385,43 @@ int decode_body(llama_model* m, int B, int cmax, cudaStream_t st) {
   RC(run_head(m, B, 1, st));
   mark(m, K_OTHER, st);
   RC(launch_add_lengths(m->d_len, B, 1, st));
+  return LLAMA_OK;
+}
+
+KvLayout kv_layout(const llama_model* m) {
+  return KvLayout{m->paged ? m->d_table : nullptr, m->max_pages, m->cfg.max_seq, m->n_pages};
+}
+
+// Give sequence b exactly the pages that positions [0, len) need, taking
+// pages from (or returning them to) the pool, and upload the changed part of
+// its block-table row on `st`. Contiguous caches need nothing.
+int fit_pages(llama_model* m, int b, int len, cudaStream_t st) {
+  if (!m->paged) return LLAMA_OK;
+  const int need = (len + KV_PAGE - 1) / KV_PAGE;
+  int& have = m->seq_pages[b];
+  if (need > m->max_pages) return LLAMA_ERR_SHAPE;
+  if (need - have > (int)m->free_pages.size()) return LLAMA_ERR_SHAPE;   // pool exhausted
+  const int first = have;
+  while (have < need) {
+    m->h_table[(size_t)b * m->max_pages + have] = m->free_pages.back();
+    m->free_pages.pop_back();
+    ++have;
+  }
+  while (have > need) {
+    --have;
+    m->free_pages.push_back(m->h_table[(size_t)b * m->max_pages + have]);
+    m->h_table[(size_t)b * m->max_pages + have] = 0;
+  }
+  if (need > first) {
+    const size_t off = (size_t)b * m->max_pages + first;
+    CK(cudaMemcpyAsync(m->d_table + off, m->h_table.data() + off, (size_t)(need - first) * sizeof(int32_t),
+                       cudaMemcpyHostToDevice, st));
+  }
+  return LLAMA_OK;
+}
+
+int fit_pages_all(llama_model* m, int B, int add, cudaStream_t st) {
+  for (int b = 0; b < B; ++b) RC(fit_pages(m, b, m->h_len[b] + add, st));
   return LLAMA_OK;
 }
 
@@ -437,7 +497,28 @@ int llama_create(const llama_config* cfg, llama_model** out) {
     w.ffn_norm = reinterpret_cast<float*>(wb); wb += align256(D * 4);
   }
   // ---- KV cache
-  m->layer_cache_elems = (size_t)c.max_batch * c.n_kv_heads * c.max_seq * m->d;
+  m->paged = c.kv_page_size != 0;
+  if (m->paged) {
+    m->max_pages = (c.max_seq + KV_PAGE - 1) / KV_PAGE;
+    m->n_pages = c.kv_pages;
+    m->layer_cache_elems = (size_t)m->n_pages * c.n_kv_heads * KV_PAGE * m->d;
+    m->d_table = static_cast<int32_t*>(m->alloc((size_t)c.max_batch * m->max_pages * sizeof(int32_t)));
+    if (!m->d_table) { delete m; return LLAMA_ERR_OOM; }
+    cudaMemset(m->d_table, 0, (size_t)c.max_batch * m->max_pages * sizeof(int32_t));
+    m->h_table.assign((size_t)c.max_batch * m->max_pages, 0);
+    m->seq_pages.assign(c.max_batch, 0);
+    // The pool hands pages out in a scattered order (stride coprime with the
+    // pool size), so consecutive pages of a sequence are not neighbours.
+    int stride = 7919 % m->n_pages;
+    auto gcd = [](int a, int b) { while (b) { const int t = a % b; a = b; b = t; } return a; };
+    while (stride <= 0 || gcd(stride, m->n_pages) != 1) stride = (stride + 1) % std::max(m->n_pages, 2);
+    if (m->n_pages == 1) stride = 1;
+    m->free_pages.resize(m->n_pages);
+    for (int i = 0; i < m->n_pages; ++i)   // back of the vector is handed out first
+      m->free_pages[m->n_pages - 1 - i] = (int32_t)(((int64_t)i * stride) % m->n_pages);
+  } else {
+    m->layer_cache_elems = (size_t)c.max_batch * c.n_kv_heads * c.max_seq * m->d;
+  }
   m->kcache = m->alloc(m->layer_cache_elems * c.n_layers * es);
   m->vcache = m->alloc(m->layer_cache_elems * c.n_layers * es);
   m->d_len = static_cast<int32_t*>(m->alloc(c.max_batch * sizeof(int32_t)));
@@ -606,6 +687,7 @@ int llama_prefill(llama_model* m, const int32_t* tokens, int32_t B, int32_t S, v
   RC(check_lengths(m, B, S));
   if ((int64_t)B * S > m->Mmax) return LLAMA_ERR_SHAPE;
   cudaStream_t st = S_(stream);
+  RC(fit_pages_all(m, B, S, st));
   const int M = B * S;
   mark(m, K_EMBED, st);
   RC(launch_embed(tokens, M, m->tok_emb, m->cfg.vocab_size, m->cfg.dim, m->adt, m->x, m->d_status, st));
@@ -621,6 +703,7 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t B, void* st
   if (!m || !tokens) return LLAMA_ERR_INVALID_ARG;
   RC(check_lengths(m, B, 1));
   cudaStream_t st = S_(stream);
+  RC(fit_pages_all(m, B, 1, st));   // before the (possibly graph-replayed) step reads the table
   int maxlen = 0;
   for (int b = 0; b < B; ++b) maxlen = std::max(maxlen, m->h_len[b] + 1);
   const int cmax = std::min(m->cfg.max_seq, (maxlen + 511) / 512 * 512);
@@ -710,6 +793,7 @@ int llama_block_forward(llama_model* m, int32_t layer, const float* x, float* y,
   RC(check_lengths(m, B, S));
   if ((int64_t)B * S > m->Mmax) return LLAMA_ERR_SHAPE;
   cudaStream_t st = S_(stream);
+  RC(fit_pages_all(m, B, S, st));
   const size_t bytes = (size_t)B * S * m->cfg.dim * sizeof(float);
   CK(cudaMemcpyAsync(m->x, x, bytes, cudaMemcpyDeviceToDevice, st));
   RC(run_layer(m, layer, B, S, false, 0, st));
@@ -722,13 +806,16 @@ int llama_fill_kv_random(llama_model* m, uint64_t seed, int32_t c, void* stream)
   if (c < 0 || c > m->cfg.max_seq) return LLAMA_ERR_SHAPE;
   cudaStream_t st = S_(stream);
   const llama_config& cf = m->cfg;
-  FillLayout fl{(int64_t)cf.max_batch * cf.n_kv_heads, c, m->d, (int64_t)cf.max_seq * m->d, m->d, 1, 0};
+  for (int b = 0; b < cf.max_batch; ++b) RC(fit_pages(m, b, c, st));   // pages first: the fill writes through them
+  const KvLayout L = kv_layout(m);
   for (int l = 0; l < cf.n_layers; ++l) {
     char* kc = static_cast<char*>(m->kcache) + (size_t)l * m->layer_cache_elems * m->esz;
     char* vc = static_cast<char*>(m->vcache) + (size_t)l * m->layer_cache_elems * m->esz;
     const bool rb = cf.dtype == LLAMA_BF16;
-    RC(launch_fill_normal(kc, fl, seed, kStreamKvBase + 2 * (uint64_t)l, 1.0f, m->adt, st, rb));
-    RC(launch_fill_normal(vc, fl, seed, kStreamKvBase + 2 * (uint64_t)l + 1, 1.0f, m->adt, st, rb));
+    RC(launch_fill_kv(kc, L, cf.max_batch, cf.n_kv_heads, c, m->d, seed, kStreamKvBase + 2 * (uint64_t)l, 1.0f,
+                      m->adt, rb, st));
+    RC(launch_fill_kv(vc, L, cf.max_batch, cf.n_kv_heads, c, m->d, seed, kStreamKvBase + 2 * (uint64_t)l + 1, 1.0f,
+                      m->adt, rb, st));
   }
   std::vector<int32_t> lens(cf.max_batch, c);
   return llama_set_lengths(m, lens.data(), cf.max_batch, stream);
@@ -738,18 +825,14 @@ int llama_set_kv(llama_model* m, int32_t layer, const void* k, const void* v, in
   if (!m || !k || !v) return LLAMA_ERR_INVALID_ARG;
   if (layer < 0 || layer >= m->cfg.n_layers) return LLAMA_ERR_INVALID_ARG;
   if (B <= 0 || B > m->cfg.max_batch || c <= 0 || c > m->cfg.max_seq) return LLAMA_ERR_SHAPE;
-  const size_t w = (size_t)c * m->d * m->esz, dp = (size_t)m->cfg.max_seq * m->d * m->esz;
-  const size_t rows = (size_t)B * m->cfg.n_kv_heads;
+  cudaStream_t st = S_(stream);
+  for (int b = 0; b < B; ++b) RC(fit_pages(m, b, std::max(m->h_len[b], (int)c), st));
   char* kc = static_cast<char*>(m->kcache) + (size_t)layer * m->layer_cache_elems * m->esz;
   char* vc = static_cast<char*>(m->vcache) + (size_t)layer * m->layer_cache_elems * m->esz;
-  if (m->cfg.dtype == LLAMA_BF16) {  // bf16 from the caller, fp16 in the cache
-    const int64_t cols = (int64_t)c * m->d, dpe = (int64_t)m->cfg.max_seq * m->d;
-    RC(launch_convert_2d(kc, dpe, LLAMA_F16, k, cols, LLAMA_BF16, (int64_t)rows, cols, S_(stream)));
-    return launch_convert_2d(vc, dpe, LLAMA_F16, v, cols, LLAMA_BF16, (int64_t)rows, cols, S_(stream));
-  }
-  CK(cudaMemcpy2DAsync(kc, dp, k, w, w, rows, cudaMemcpyDeviceToDevice, S_(stream)));
-  CK(cudaMemcpy2DAsync(vc, dp, v, w, w, rows, cudaMemcpyDeviceToDevice, S_(stream)));
-  return LLAMA_OK;
+  // caller's dtype in, the model's storage type (fp16 for bf16 models) in the cache
+  const KvLayout L = kv_layout(m);
+  RC(launch_kv_scatter(kc, m->adt, L, B, m->cfg.n_kv_heads, c, m->d, k, m->cfg.dtype, st));
+  return launch_kv_scatter(vc, m->adt, L, B, m->cfg.n_kv_heads, c, m->d, v, m->cfg.dtype, st);
 }
 
 int llama_set_lengths(llama_model* m, const int32_t* host_len, int32_t B, void* stream) {
@@ -758,8 +841,19 @@ int llama_set_lengths(llama_model* m, const int32_t* host_len, int32_t B, void* 
   for (int b = 0; b < B; ++b)
     if (host_len[b] < 0 || host_len[b] > m->cfg.max_seq) return LLAMA_ERR_SHAPE;
   for (int b = 0; b < B; ++b) m->h_len[b] = host_len[b];
+  for (int b = 0; b < B; ++b) RC(fit_pages(m, b, m->h_len[b], S_(stream)));
   CK(cudaMemcpyAsync(m->d_len, m->h_len.data(), B * sizeof(int32_t), cudaMemcpyHostToDevice, S_(stream)));
   CK(cudaStreamSynchronize(S_(stream)));
+  return LLAMA_OK;
+}
+
+int llama_get_block_table(const llama_model* m, int32_t* host_table, int32_t B) {
+  if (!m || !host_table) return LLAMA_ERR_INVALID_ARG;
+  if (!m->paged) return LLAMA_ERR_UNSUPPORTED;
+  if (B <= 0 || B > m->cfg.max_batch) return LLAMA_ERR_SHAPE;
+  for (int b = 0; b < B; ++b)
+    for (int j = 0; j < m->max_pages; ++j)
+      host_table[(size_t)b * m->max_pages + j] = j < m->seq_pages[b] ? m->h_table[(size_t)b * m->max_pages + j] : -1;
   return LLAMA_OK;
 }
 
@@ -773,6 +867,7 @@ int llama_get_lengths(const llama_model* m, int32_t* host_len, int32_t B) {
 int llama_reset(llama_model* m, void* stream) {
   if (!m) return LLAMA_ERR_INVALID_ARG;
   std::fill(m->h_len.begin(), m->h_len.end(), 0);
+  for (int b = 0; b < m->cfg.max_batch; ++b) RC(fit_pages(m, b, 0, S_(stream)));   // every page back to the pool
   m->last_B = 0;
   CK(cudaMemsetAsync(m->d_len, 0, m->cfg.max_batch * sizeof(int32_t), S_(stream)));
   return LLAMA_OK;
@@ -852,6 +947,47 @@ int llama_attention_decode(const void* q, const void* kc, const void* vc, const 
   if (!c) return LLAMA_ERR_OOM;
   RC(grow_decode_scratch(&c->ds, decode_scratch_floats(cmax, B, H, Hk, d, dtype)));
   return attention_decode(q, kc, vc, len, 0, o, B, cmax, H, Hk, d, cmax, dtype, &c->ds, c->status, S_(stream));
+}
+
+// Validates a caller's block table (device [B][max_pages]): every entry in
+// [-1, n_pages) (-1 marks an unused slot).
+static int check_block_table(const int32_t* table, int B, int max_pages, int n_pages, cudaStream_t st) {
+  std::vector<int32_t> h((size_t)B * max_pages);
+  CK(cudaMemcpyAsync(h.data(), table, h.size() * sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+  CK(cudaStreamSynchronize(st));
+  for (int32_t p : h)
+    if (p < -1 || p >= n_pages) return LLAMA_ERR_SHAPE;
+  return LLAMA_OK;
+}
+
+int llama_attention_prefill_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* table,
+                                  int32_t max_pages, int32_t n_pages, const int32_t* pos0, void* o, int32_t B,
+                                  int32_t S, int32_t H, int32_t Hk, int32_t d, int32_t dtype, void* stream) {
+  if (!q || !k_pages || !v_pages || !table || !o) return LLAMA_ERR_INVALID_ARG;
+  if (B <= 0 || S <= 0 || H <= 0 || Hk <= 0 || H % Hk != 0 || max_pages <= 0 || n_pages <= 0) return LLAMA_ERR_SHAPE;
+  if (dtype != LLAMA_BF16 && dtype != LLAMA_F16) return LLAMA_ERR_UNSUPPORTED;
+  if (d != 128) return LLAMA_ERR_UNSUPPORTED;
+  DevCtx* c = dev_ctx();
+  if (!c) return LLAMA_ERR_OOM;
+  RC(check_block_table(table, B, max_pages, n_pages, S_(stream)));
+  return attention_prefill(q, k_pages, v_pages, o, pos0, B, S, H, Hk, d, max_pages * KV_PAGE, dtype, c->status,
+                           S_(stream), table, max_pages, n_pages);
+}
+
+int llama_attention_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* table,
+                                 int32_t max_pages, int32_t n_pages, const int32_t* len, void* o, int32_t B,
+                                 int32_t H, int32_t Hk, int32_t d, int32_t dtype, void* stream) {
+  if (!q || !k_pages || !v_pages || !table || !len || !o) return LLAMA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || Hk <= 0 || H % Hk != 0 || max_pages <= 0 || n_pages <= 0) return LLAMA_ERR_SHAPE;
+  if (dtype != LLAMA_BF16 && dtype != LLAMA_F16) return LLAMA_ERR_UNSUPPORTED;
+  if (d != 128) return LLAMA_ERR_UNSUPPORTED;
+  DevCtx* c = dev_ctx();
+  if (!c) return LLAMA_ERR_OOM;
+  RC(check_block_table(table, B, max_pages, n_pages, S_(stream)));
+  const int cmax = max_pages * KV_PAGE;
+  RC(grow_decode_scratch(&c->ds, decode_scratch_floats(cmax, B, H, Hk, d, dtype)));
+  return attention_decode(q, k_pages, v_pages, len, 0, o, B, cmax, H, Hk, d, cmax, dtype, &c->ds, c->status,
+                          S_(stream), table, max_pages, n_pages);
 }
 
 int llama_linear(const void* x, const void* w, float* y, int32_t M, int32_t N, int32_t K, int32_t dtype,

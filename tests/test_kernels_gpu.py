@@ -226,3 +226,81 @@ def test_attention_decode_few_tiles_after_many():
                         vv[b][:, :n].astype(np.float64), np.array([n - 1]))[0]
         assert rel_l2(got[b], ref) < 1e-2
     _sync_ok()
+
+
+# ------------------------------------------------------- paged KV cache
+def _paginate(raw, n_pages, seed):
+    """Scatter a logical cache [B][Hk][C][d] into pages [n_pages][Hk][128][d]
+    under a random block table (distinct pages, unused slots -1)."""
+    B, Hk, C, d = raw.shape
+    max_pages = (C + 127) // 128
+    rng = np.random.RandomState(seed)
+    perm = rng.permutation(n_pages)[:B * max_pages].reshape(B, max_pages).astype(np.int32)
+    pages = np.zeros((n_pages, Hk, 128, d), raw.dtype)
+    for b in range(B):
+        for j in range(max_pages):
+            rows = raw[b, :, j * 128:(j + 1) * 128]
+            pages[perm[b, j], :, :rows.shape[1]] = rows
+    return pages, perm, max_pages
+
+
+@pytest.mark.parametrize('dtype', [F16, BF16])
+def test_attention_decode_paged(dtype):
+    B, H, Hk, d, C = 3, 32, 8, 128, 1000
+    lens = [1, 300, 1000]
+    qv, qr = normal_values(50, 1, (B, H, d), dtype)
+    kv, kr = normal_values(50, 2, (B, Hk, C, d), dtype)
+    vv, vr = normal_values(50, 3, (B, Hk, C, d), dtype)
+    n_pages = 3 * 8 + 5
+    kp, table, max_pages = _paginate(kr, n_pages, 1)
+    vp, _, _ = _paginate(vr, n_pages, 1)
+    o = torch.empty((B, H * d), dtype=torch_dtype(dtype), device='cuda')
+    L.llama_attention_decode_paged(to_device(qr, dtype), to_device(kp, dtype), to_device(vp, dtype),
+                                   torch.from_numpy(table).cuda(), max_pages, n_pages,
+                                   torch.tensor(lens, dtype=torch.int32, device='cuda'), o, B, H, Hk, d, dtype)
+    torch.cuda.synchronize()
+    _sync_ok()
+    got = o.float().cpu().numpy()
+    for b in range(B):
+        n = lens[b]
+        ref = attention(qv[b][:, None, :].astype(np.float64), kv[b][:, :n].astype(np.float64),
+                        vv[b][:, :n].astype(np.float64), np.array([n - 1]))[0]
+        assert rel_l2(got[b], ref) < (1e-2 if dtype == BF16 else 2e-3)
+
+
+def test_attention_prefill_paged_continues_a_cache():
+    """Queries at positions pos0[b] .. pos0[b]+S-1 over a paged cache that
+    already holds their keys (a prompt continued across page boundaries)."""
+    dtype, B, S, H, Hk, d = F16, 2, 300, 32, 8, 128
+    pos0 = [0, 200]
+    C = max(pos0) + S
+    qv, qr = normal_values(51, 1, (B, H, S, d), dtype)
+    kv, kr = normal_values(51, 2, (B, Hk, C, d), dtype)
+    vv, vr = normal_values(51, 3, (B, Hk, C, d), dtype)
+    n_pages = 11
+    kp, table, max_pages = _paginate(kr, n_pages, 2)
+    vp, _, _ = _paginate(vr, n_pages, 2)
+    o = torch.empty((B, S, H * d), dtype=torch.float16, device='cuda')
+    L.llama_attention_prefill_paged(to_device(qr, dtype), to_device(kp, dtype), to_device(vp, dtype),
+                                    torch.from_numpy(table).cuda(), max_pages, n_pages,
+                                    torch.tensor(pos0, dtype=torch.int32, device='cuda'), o, B, S, H, Hk, d, dtype)
+    torch.cuda.synchronize()
+    _sync_ok()
+    got = o.float().cpu().numpy()
+    for b in range(B):
+        n = pos0[b] + S
+        ref = attention(qv[b].astype(np.float64), kv[b][:, :n].astype(np.float64), vv[b][:, :n].astype(np.float64),
+                        pos0[b] + np.arange(S))
+        assert rel_l2(got[b], ref) < 2e-3
+
+
+def test_attention_paged_rejects_bad_tables():
+    B, H, Hk, d = 1, 8, 2, 128
+    q = torch.zeros((B, H, d), dtype=torch.float16, device='cuda')
+    pages = torch.zeros((2, Hk, 128, d), dtype=torch.float16, device='cuda')
+    o = torch.empty((B, H * d), dtype=torch.float16, device='cuda')
+    bad = torch.tensor([[0, 5]], dtype=torch.int32, device='cuda')      # page 5 of a 2-page pool
+    with pytest.raises(L.LlamaError) as e:
+        L.llama_attention_decode_paged(q, pages, pages, bad, 2, 2, torch.tensor([200], dtype=torch.int32,
+                                                                                 device='cuda'), o, B, H, Hk, d, F16)
+    assert e.value.status == L.LLAMA_ERR_SHAPE

@@ -273,3 +273,65 @@ def test_set_kv_then_decode():
         _check_status(m)
     finally:
         m.close()
+
+
+# ------------------------------------------------------------ paged cache
+def test_paged_cache_matches_contiguous_across_pages():
+    """A model with a paged cache (128-position pages from a scattered pool)
+    gives the contiguous model's logits through a chunked prefill that crosses
+    a page boundary and decode steps that cross the next one; both agree with
+    the oracle."""
+    B = 2
+    cont = Model(SMALL_BF16, BF16, max_batch=B, max_seq=512)
+    paged = Model(dict(SMALL_BF16, kv_page_size=128), BF16, max_batch=B, max_seq=512)
+    try:
+        for m in (cont, paged):
+            L.llama_init_weights(m.h, 6, 0.02)
+        toks = si.tokens(8, B * 270, 3000).reshape(B, 270)
+        st = torch.cuda.Stream()
+        outs = {}
+        with torch.cuda.stream(st):
+            for name, m in (('cont', cont), ('paged', paged)):
+                L.llama_prefill(m.h, torch.from_numpy(np.ascontiguousarray(toks[:, :100])).cuda(), B, 100, st)
+                L.llama_prefill(m.h, torch.from_numpy(np.ascontiguousarray(toks[:, 100:250])).cuda(), B, 150, st)
+                rows = [m.logits(B, st).cpu().numpy()]
+                for i in range(250, 270):           # positions 250..269 cross the page boundary at 256
+                    L.llama_decode_step(m.h, torch.from_numpy(np.ascontiguousarray(toks[:, i])).cuda(), B, st)
+                    rows.append(m.logits(B, st).cpu().numpy())
+                outs[name] = np.stack(rows)
+        _check_status(cont)
+        _check_status(paged)
+        assert rel_l2(outs['paged'], outs['cont']) < 1e-3
+        orc = Oracle(paged.p, SeededWeights(paged.p, 6, 0.02, BF16))
+        for b in range(B):
+            ref = orc.forward(toks[b, :250])
+            assert rel_l2(outs['paged'][0, b], ref) < 2e-2
+            ref = orc.forward(toks[b, :270])
+            assert rel_l2(outs['paged'][-1, b], ref) < 2e-2
+        max_pages = (512 + 127) // 128
+        tab = np.zeros((B, max_pages), np.int32)
+        L.llama_get_block_table(paged.h, tab, B)
+        used = tab[:, :3]                           # 270 positions -> 3 pages each
+        assert np.all(used >= 0) and len(set(used.ravel())) == used.size and np.all(tab[:, 3:] == -1)
+        assert not all(used[b, j + 1] == used[b, j] + 1 for b in range(B) for j in range(2))
+        L.llama_reset(paged.h)
+        L.llama_get_block_table(paged.h, tab, B)
+        assert np.all(tab == -1)
+    finally:
+        cont.close()
+        paged.close()
+
+
+def test_paged_pool_exhaustion_is_an_error():
+    m = Model(dict(SMALL_BF16, kv_page_size=128, kv_pages=3), BF16, max_batch=2, max_seq=512)
+    try:
+        L.llama_init_weights(m.h, 6, 0.02)
+        toks = torch.from_numpy(si.tokens(9, 2 * 200, 3000)).cuda()
+        with pytest.raises(L.LlamaError) as e:          # 2 x 2 pages needed, 3 in the pool
+            L.llama_prefill(m.h, toks, 2, 200)
+        assert e.value.status == L.LLAMA_ERR_SHAPE
+        L.llama_reset(m.h)
+        L.llama_prefill(m.h, toks[:200], 1, 200)        # fits after the reset
+        _check_status(m)
+    finally:
+        m.close()
