@@ -447,12 +447,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Stream-K over (weight tile, k-block) units: of the U = tiles * kb units
 // (tile-major), CTA c of G takes [U*c/G, U*(c+1)/G), so every CTA streams the
 // same number of weight bytes to within one 16 KB block. A CTA's range falls
-// into pieces, one per tile it touches. A piece covering its whole tile runs the
-// epilogue directly; otherwise it leaves its fp32 partial in one of the CTA's
-// two scratch slots (slot 0: the piece holding the CTA's first unit, slot 1:
-// its last), and the tile's last contributor (atomic ticket, no spinning) sums
-// the contributors' partials in CTA order and runs the epilogue. Accumulators
-// are double-buffered in TMEM so the MMA runs on while a piece drains.
+// into pieces, one per tile it touches. A piece covering its whole tile runs
+// the epilogue directly. A split tile is finished by its owner, the CTA whose
+// piece holds k-block 0 (always the last piece of the owner's range); every
+// other piece of the tile is the first piece of its CTA's range, stored in
+// that CTA's workspace slot and counted in the tile's counter. The owner waits
+// (bounded) for the count, adds the shares in CTA order, runs the epilogue and
+// re-arms the counter: results do not depend on timing. Residual tiles are the
+// exception: x += sum is linear, so every piece adds its share into x with
+// vector atomics and nothing waits (measured faster on decode than the owner
+// fixup, whose x read-modify-write lands at the end of the kernel); their
+// summation order varies from run to run at fp32 rounding level. All CTAs of the grid
+// (one per SM) are resident together and owners wait only for first pieces,
+// which wait for nothing, so the waits end. Accumulators are double-buffered
+// in TMEM so the MMA runs on while a piece drains.
 template <int NT>
 struct SkinnyCfg {
   static constexpr int B_BYTES = NT * BK * 2;
@@ -467,8 +475,8 @@ struct SkinnyCfg {
 template <int KIND, typename T, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, int M,
-                       int N, int K, EpiArgs epi, float* __restrict__ ws, int* __restrict__ tickets,
-                       float* __restrict__ stg, int* status) {
+                       int N, int K, EpiArgs epi, float* __restrict__ ws, int* __restrict__ counters,
+                       int* status) {
   using C = SkinnyCfg<NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -479,7 +487,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acce = accf + 2;
   uint64_t* drain = acce + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles = (N + S_BM - 1) / S_BM;
@@ -570,14 +577,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     // 32-feature chunk = ew) runs the same row epilogue as the wide GEMM.
     const int quarter = warp & 3;          // TMEM lanes this warp may read
     const int ew = warp - 2;               // feature chunk in the row phase
+    const int tid = ew * 32 + lane;        // 0..127
     int buf = 0;
     uint32_t acc_phase = 0;
     for (long long u = u0; u < u1;) {
       const int tile = (int)(u / kb), klo = (int)(u % kb);
       const int n = (int)((u1 - u) < (kb - klo) ? (u1 - u) : (kb - klo));
       const bool whole = klo == 0 && n == kb;
-      const int slot = (u == u0) ? 0 : 1;
+      // residual tiles: every piece adds its share into x atomically (linear,
+      // no waiting at the end of the kernel; the summation order varies);
+      // other split tiles: owner fixup
+      const bool atomic_piece = KIND == EPI_RESIDUAL && !whole;
+      const bool owner = !whole && !atomic_piece && klo == 0;   // k-block 0: the last piece of this CTA's range
+      const bool share = !whole && !atomic_piece && klo != 0;   // the first piece of this CTA's range
       const int f0 = tile * S_BM + ew * 32;
+      const long long t0 = (long long)tile * kb;
+      long long c_own = 0, c_hi = 0;
+      if (!whole) { c_own = sk_owner(t0, U, G); c_hi = sk_owner(t0 + kb - 1, U, G); }
+      if (owner) {  // the other shares of this tile (their CTAs' first pieces) before the epilogue
+        if (threadIdx.x == 64) {
+          int need = 0;
+          for (long long cc = c_own + 1; cc <= c_hi; ++cc) need += sk_first(cc + 1, U, G) > sk_first(cc, U, G);
+          counter_wait_geq(&counters[tile], need, status);   // a timeout is latched in status
+          counters[tile] = 0;
+        }
+        named_bar_sync(1, 128);
+        __threadfence();
+      }
       // all lanes of a warp take the same branch so the warp-wide TMEM loads stay converged
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], acc_phase, status));
       tc_fence_after();
@@ -605,26 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
         }
         const int m = c * 32 + lane;
-        if (KIND == EPI_QKV_ROPE || KIND == EPI_SWIGLU) {
-          // nonlinear epilogues: accumulate into the zeroed fp32 staging
-          // buffer; skinny_finalize_kernel applies the epilogue afterwards
-          if (m < epi.M) {
-            float* dst = stg + (size_t)m * epi.N + f0;
-            if (f0 + 32 <= epi.N && (epi.N & 3) == 0) {
-#pragma unroll
-              for (int j = 0; j < 8; ++j)
-                atomicAdd(reinterpret_cast<float4*>(dst) + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (f0 + j < epi.N) atomicAdd(dst + j, v[j]);
-            }
-          }
-        } else if (whole) {
-          epi_row32<KIND, T>(epi, m, f0, v);
-        } else if (KIND == EPI_RESIDUAL) {
-          // x += sum of partials is linear: every contributor adds its share
-          // straight into the fp32 residual (summation order is not fixed)
+        if (atomic_piece) {
           if (m < epi.M) {
             float* dst = epi.out + (size_t)m * epi.ldo + f0;
             if (f0 + 32 <= epi.N && (epi.ldo & 3) == 0) {
@@ -637,47 +644,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (f0 + j < epi.N) atomicAdd(dst + j, v[j]);
             }
           }
-        } else {  // token-major partial: [slot][token][128 features]
-          float4* p4 = reinterpret_cast<float4*>(ws + (((size_t)blockIdx.x * 2 + slot) * NT + m) * S_BM + ew * 32);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) __stcg(p4 + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+          continue;
         }
+        // a share: float4 (c*8 + j)*128 + tid of the CTA's slot, so a warp's
+        // accesses are 512 contiguous bytes
+        if (share) {
+          float4* p4 = reinterpret_cast<float4*>(ws) + (size_t)blockIdx.x * (NT * S_BM / 4) + tid;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            __stcg(p4 + (c * 8 + j) * 128, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+          continue;
+        }
+        if (owner) {  // add the other shares in CTA order
+          for (long long cc = c_own + 1; cc <= c_hi; ++cc) {
+            if (sk_first(cc + 1, U, G) <= sk_first(cc, U, G)) continue;   // no units
+            const float4* p4 = reinterpret_cast<const float4*>(ws) + (size_t)cc * (NT * S_BM / 4) + tid;
+            float4 x[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] = __ldcg(p4 + (c * 8 + j) * 128);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              v[4 * j] += x[j].x; v[4 * j + 1] += x[j].y; v[4 * j + 2] += x[j].z; v[4 * j + 3] += x[j].w;
+            }
+          }
+        }
+        epi_row32<KIND, T>(epi, m, f0, v);
       }
-      if (!whole && KIND == EPI_STORE_F32) {
+      if (share) {  // publish the share
         __threadfence();
         named_bar_sync(1, 128);
-        const long long t0 = (long long)tile * kb;
-        const long long c_lo = sk_owner(t0, U, G), c_hi = sk_owner(t0 + kb - 1, U, G);
-        if (threadIdx.x == 64) {
-          int contributors = 0;
-          for (long long c = c_lo; c <= c_hi; ++c) contributors += sk_first(c + 1, U, G) > sk_first(c, U, G);
-          const int prev = atomicAdd(&tickets[tile], 1);
-          *last_flag = (prev == contributors - 1);
-        }
-        named_bar_sync(1, 128);
-        if (*last_flag) {  // the tile's last contributor: sum the partials in CTA order
-          __threadfence();
-#pragma unroll 1
-          for (int c = 0; c < NT / 32; ++c) {
-            const int m = c * 32 + lane;
-            float v[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = 0.f;
-            for (long long cc = c_lo; cc <= c_hi; ++cc) {
-              const long long first_unit = sk_first(cc, U, G);
-              if (sk_first(cc + 1, U, G) <= first_unit) continue;   // no units
-              const int sl = first_unit >= t0 ? 0 : 1;              // the tile holds its first unit?
-              const float4* p4 = reinterpret_cast<const float4*>(ws + ((cc * 2 + sl) * NT + m) * S_BM + ew * 32);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const float4 x = __ldcg(p4 + j);
-                v[4 * j] += x.x; v[4 * j + 1] += x.y; v[4 * j + 2] += x.z; v[4 * j + 3] += x.w;
-              }
-            }
-            epi_row32<KIND, T>(epi, m, f0, v);
-          }
-          if (threadIdx.x == 64) tickets[tile] = 0;
-        }
+        if (threadIdx.x == 64) atomicAdd(&counters[tile], 1);
       }
       if (++buf == 2) { buf = 0; acc_phase ^= 1; }
       u += n;
@@ -689,38 +685,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
-}
-
-// Apply the QKV/RoPE or SwiGLU epilogue to the summed fp32 staging rows
-// [M][N] left by the skinny GEMM, one (token, 32-feature chunk) per thread,
-// and zero the staging rows for the next GEMM.
-template <int KIND, typename T>
-__global__ void __launch_bounds__(128) skinny_finalize_kernel(EpiArgs epi, float* __restrict__ stg) {
-  pdl_trigger();
-  pdl_wait();
-  const int chunks = (epi.N + 31) / 32;
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= epi.M * chunks) return;
-  const int m = idx / chunks, n0 = (idx - m * chunks) * 32;
-  float* src = stg + (size_t)m * epi.N + n0;
-  float v[32];
-  if (n0 + 32 <= epi.N && (epi.N & 3) == 0) {
-    float4* p4 = reinterpret_cast<float4*>(src);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 x = __ldcg(p4 + j);
-      v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) __stcg(p4 + j, make_float4(0.f, 0.f, 0.f, 0.f));
-  } else {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      v[j] = n0 + j < epi.N ? __ldcg(src + j) : 0.f;
-      if (n0 + j < epi.N) src[j] = 0.f;
-    }
-  }
-  epi_row32<KIND, T>(epi, m, n0, v);
 }
 
 // -------------------------------------------------------------- host side
@@ -864,7 +828,7 @@ static int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, int M, int 
 
 template <int KIND, typename T, int NT>
 static int launch_skinny_nt(const CUtensorMap& tw, const CUtensorMap& tx, int M, int N, int K, const EpiArgs& e,
-                            float* ws, int* tickets, float* stg, int* status, cudaStream_t st) {
+                            float* ws, int* counters, int* status, cudaStream_t st) {
   using C = SkinnyCfg<NT>;
   auto kern = gemm_skinny_kernel<KIND, T, NT>;
   static bool attr = false;
@@ -873,23 +837,19 @@ static int launch_skinny_nt(const CUtensorMap& tw, const CUtensorMap& tx, int M,
       return LLAMA_ERR_CUDA;
     attr = true;
   }
-  cudaError_t err = launch_k(kern, dim3(num_sms()), dim3(kThreads), C::SMEM, st, tw, tx, M, N, K, e, ws, tickets,
-                             stg, status);
-  if (err == cudaSuccess && (KIND == EPI_QKV_ROPE || KIND == EPI_SWIGLU)) {
-    const int items = M * ((N + 31) / 32);
-    err = launch_k(skinny_finalize_kernel<KIND, T>, dim3((items + 127) / 128), dim3(128), 0, st, e, stg);
-  }
+  const cudaError_t err = launch_k(kern, dim3(num_sms()), dim3(kThreads), C::SMEM, st, tw, tx, M, N, K, e, ws,
+                                   counters, status);
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 template <int KIND, typename T>
 static int launch_skinny(const CUtensorMap& tw, const CUtensorMap& tx, int M, int N, int K, int NT, const EpiArgs& e,
-                         float* ws, int* tickets, float* stg, int* status, cudaStream_t st) {
+                         float* ws, int* counters, int* status, cudaStream_t st) {
   switch (NT) {
-    case 32: return launch_skinny_nt<KIND, T, 32>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
-    case 64: return launch_skinny_nt<KIND, T, 64>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
-    case 128: return launch_skinny_nt<KIND, T, 128>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
-    case 256: return launch_skinny_nt<KIND, T, 256>(tw, tx, M, N, K, e, ws, tickets, stg, status, st);
+    case 32: return launch_skinny_nt<KIND, T, 32>(tw, tx, M, N, K, e, ws, counters, status, st);
+    case 64: return launch_skinny_nt<KIND, T, 64>(tw, tx, M, N, K, e, ws, counters, status, st);
+    case 128: return launch_skinny_nt<KIND, T, 128>(tw, tx, M, N, K, e, ws, counters, status, st);
+    case 256: return launch_skinny_nt<KIND, T, 256>(tw, tx, M, N, K, e, ws, counters, status, st);
   }
   return LLAMA_ERR_INVALID_ARG;
 }
@@ -900,7 +860,7 @@ static int skinny_nt(int M) {
   return nt;
 }
 
-size_t skinny_workspace_floats(int M) { return (size_t)num_sms() * 2 * S_BM * skinny_nt(M); }
+size_t skinny_workspace_floats(int M) { return (size_t)num_sms() * S_BM * skinny_nt(M); }
 
 bool pdl_enabled() {
   static const bool on = getenv("LLAMA_NO_PDL") == nullptr;
@@ -945,18 +905,16 @@ static int gemm16_t(const void* A, int M, int K, int lda, const void* W, int N, 
   if (!scratch || !scratch->ws || scratch->ws_floats < skinny_workspace_floats(M) || !scratch->tickets ||
       scratch->n_tickets < tiles)
     return LLAMA_ERR_INVALID_ARG;
-  if ((kind == EPI_QKV_ROPE || kind == EPI_SWIGLU) && (!scratch->stg || scratch->stg_floats < (size_t)M * N))
-    return LLAMA_ERR_INVALID_ARG;
   CUtensorMap tw, tx;
   if ((rc = make_tmap_16(&tw, W, N, K, ldw, S_BM, F16)) != LLAMA_OK) return rc;
   if ((rc = make_tmap_16(&tx, A, M, K, lda, NT, F16)) != LLAMA_OK) return rc;
   float* ws = scratch->ws;
   int* tk = scratch->tickets;
   switch (kind) {
-    case EPI_STORE_F32: return launch_skinny<EPI_STORE_F32, T>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
-    case EPI_RESIDUAL: return launch_skinny<EPI_RESIDUAL, T>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
-    case EPI_SWIGLU: return launch_skinny<EPI_SWIGLU, T>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
-    case EPI_QKV_ROPE: return launch_skinny<EPI_QKV_ROPE, T>(tw, tx, M, N, K, NT, e, ws, tk, scratch->stg, status, st);
+    case EPI_STORE_F32: return launch_skinny<EPI_STORE_F32, T>(tw, tx, M, N, K, NT, e, ws, tk, status, st);
+    case EPI_RESIDUAL: return launch_skinny<EPI_RESIDUAL, T>(tw, tx, M, N, K, NT, e, ws, tk, status, st);
+    case EPI_SWIGLU: return launch_skinny<EPI_SWIGLU, T>(tw, tx, M, N, K, NT, e, ws, tk, status, st);
+    case EPI_QKV_ROPE: return launch_skinny<EPI_QKV_ROPE, T>(tw, tx, M, N, K, NT, e, ws, tk, status, st);
   }
   return LLAMA_ERR_INVALID_ARG;
 }

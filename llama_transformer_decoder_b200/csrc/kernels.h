@@ -36,16 +36,13 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
 
 enum GemmVariant { GEMM_AUTO = 0, GEMM_WIDE = 1, GEMM_SKINNY = 2 };
 
-// Scratch of the skinny GEMM: partial tiles, one ticket per 128-row weight
-// tile and the staging rows (tickets and staging must start at zero; the
-// kernels leave them zero).
+// Scratch of the split-tile fixups: one fp32 share slot per CTA and one
+// counter per split tile (counters start at zero; the kernels leave them zero).
 struct GemmScratch {
   float* ws;
   size_t ws_floats;
   int* tickets;
   int n_tickets;
-  float* stg;          // zeroed fp32 [M][N] staging for the skinny QKV/RoPE and SwiGLU epilogues (kept zero)
-  size_t stg_floats;
 };
 
 int num_sms();

@@ -575,12 +575,7 @@ int llama_create(const llama_config* cfg, llama_model** out) {
     if (grow_gemm_scratch(&m->gs, std::max<size_t>(ws, 1), tickets) != LLAMA_OK) { delete m; return LLAMA_ERR_OOM; }
     m->allocs.push_back(m->gs.ws);
     m->allocs.push_back(m->gs.tickets);
-    // staging rows for the skinny QKV / SwiGLU epilogues (M <= 128 rows)
-    const size_t stg = (size_t)std::min(128, m->Mmax) * std::max(m->qkv_n, 2 * m->F);
-    m->gs.stg = static_cast<float*>(m->alloc(stg * sizeof(float)));
-    if (!m->gs.stg) { delete m; return LLAMA_ERR_OOM; }
-    cudaMemset(m->gs.stg, 0, stg * sizeof(float));
-    m->gs.stg_floats = stg;
+
   }
   {
     size_t need = 0;
