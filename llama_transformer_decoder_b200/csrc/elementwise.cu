@@ -88,6 +88,36 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
   }
 }
 
+// Inputs of a GEMM with the RMSNorm folded in: y = x * g (16-bit, not yet
+// scaled by rsqrt(mean(x^2)+eps)) and the row's sum of squares in slot 0 of
+// its ss_n partial sums (the other slots 0).
+template <typename T>
+__global__ void __launch_bounds__(256) norm_prep_kernel(const float* __restrict__ x, const float* __restrict__ g,
+                                                        T* __restrict__ y, float* __restrict__ ss, int D, int ss_n) {
+  pdl_trigger();
+  pdl_wait();
+  const int r = blockIdx.x;
+  const float* xr = x + (size_t)r * D;
+  T* yr = y + (size_t)r * D;
+  __shared__ float red[8];
+  float acc = 0.f;
+  for (int i = threadIdx.x; i < D; i += 256) {
+    const float v = xr[i];
+    acc += v * v;
+    yr[i] = from_f<T>(v * g[i]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x < ss_n) {
+    float tot = 0.f;
+    if (threadIdx.x == 0)
+      for (int w = 0; w < 8; ++w) tot += red[w];
+    ss[(size_t)r * ss_n + threadIdx.x] = tot;
+  }
+}
+
 // ----------------------------------------------------------------- argmax
 // Greedy next token: largest logit, lowest index among equal maxima.
 __device__ __forceinline__ void better(float& bv, int& bi, float v, int i) {
@@ -265,6 +295,20 @@ int launch_rmsnorm(const float* x, const float* g, void* y, int rows, int D, flo
   else
     err = launch_k(rmsnorm_kernel<float>, dim3(rows), dim3(256), 0, st, x, g, static_cast<float*>(y), D, eps,
                    last_of_S);
+  return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+int launch_norm_prep(const float* x, const float* g, void* y, float* ss, int rows, int D, int ss_n, int dtype,
+                     cudaStream_t st) {
+  if (rows <= 0) return LLAMA_OK;
+  if (ss_n > 256) return LLAMA_ERR_INVALID_ARG;
+  cudaError_t err;
+  if (dtype == LLAMA_F16)
+    err = launch_k(norm_prep_kernel<f16>, dim3(rows), dim3(256), 0, st, x, g, static_cast<f16*>(y), ss, D, ss_n);
+  else if (dtype == LLAMA_BF16)
+    err = launch_k(norm_prep_kernel<bf16>, dim3(rows), dim3(256), 0, st, x, g, static_cast<bf16*>(y), ss, D, ss_n);
+  else
+    return LLAMA_ERR_INVALID_ARG;
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 

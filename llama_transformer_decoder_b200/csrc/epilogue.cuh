@@ -30,7 +30,27 @@ struct EpiArgs {
   int S, H, Hk, d, Smax;
   const int32_t* kv_table;  // paged cache block table (nullptr: contiguous)
   int kv_max_pages, kv_pages;
+  // RMSNorm folded into the GEMMs around it (prefill): rmsnorm(x) W^T equals
+  // r * ((x * g) W^T) with r = rsqrt(mean(x^2) + eps) per row. A RESIDUAL
+  // epilogue with g_next also writes y = x_new * g_next (16-bit, row pitch
+  // ldo) to y_out and the sum of x_new^2 over its 256-column tile to
+  // ss_out[m * ss_n + n0 / 256]; a QKV or SwiGLU epilogue with ss_in scales
+  // its accumulators by r = rsqrt(sum_t ss_in[m * ss_n + t] * norm_inv_d + norm_eps).
+  const float* g_next;
+  void* y_out;
+  float* ss_out;
+  const float* ss_in;
+  int ss_n;
+  float norm_inv_d, norm_eps;
 };
+
+// r of row m from its partial sums of squares (added in a fixed order).
+__device__ __forceinline__ float norm_row_scale(const EpiArgs& e, int m) {
+  const float* p = e.ss_in + (size_t)m * e.ss_n;
+  float t = 0.f;
+  for (int i = 0; i < e.ss_n; ++i) t += p[i];
+  return rsqrtf(t * e.norm_inv_d + e.norm_eps);
+}
 
 // Element offset of (sequence b, kv head g, position pos, dim 0) in a K/V cache.
 __device__ __forceinline__ size_t kv_elem(const EpiArgs& e, int b, int g, int pos) {
@@ -80,25 +100,43 @@ __device__ __forceinline__ void epi_elem(const EpiArgs& e, int m, int n, float v
 }
 
 // Row-chunk form: one thread holds 32 consecutive columns [n0, n0+32) of row m
-// (n0 % 32 == 0). Full chunks use 16-byte stores.
+// (n0 % 32 == 0). Full chunks use 16-byte stores. rs scales the accumulators
+// (the folded RMSNorm's r; 1 otherwise). Returns the chunk's sum of x_new^2
+// for a RESIDUAL epilogue with g_next, else 0.
 template <int KIND, typename T>
-__device__ __forceinline__ void epi_row32(const EpiArgs& e, int m, int n0, const float (&v)[32]) {
-  if (m >= e.M) return;
+__device__ __forceinline__ float epi_row32(const EpiArgs& e, int m, int n0, const float (&v)[32], float rs = 1.f) {
+  if (m >= e.M) return 0.f;
   const bool full = (n0 + 32 <= e.N);
+  float ssq = 0.f;
   if (KIND == EPI_STORE_F32 || KIND == EPI_RESIDUAL) {
+    const bool norm_out = KIND == EPI_RESIDUAL && e.g_next != nullptr;
     float* p = e.out + (size_t)m * e.ldo + n0;
-    if (full && ((e.ldo & 3) == 0) && ((reinterpret_cast<uintptr_t>(e.out) & 15) == 0)) {
+    T* yp = norm_out ? static_cast<T*>(e.y_out) + (size_t)m * e.ldo + n0 : nullptr;
+    if (full && ((e.ldo & 3) == 0) && ((reinterpret_cast<uintptr_t>(e.out) & 15) == 0) &&
+        (!norm_out || (sizeof(T) == 2 && (e.ldo & 7) == 0))) {
       float4* p4 = reinterpret_cast<float4*>(p);
       float4 x[8];
       if (KIND == EPI_RESIDUAL) {  // all loads before any store: they do not wait on one another
 #pragma unroll
         for (int j = 0; j < 8; ++j) x[j] = p4[j];
       }
+      uint32_t yw[16];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         float4 o = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
         if (KIND == EPI_RESIDUAL) { o.x += x[j].x; o.y += x[j].y; o.z += x[j].z; o.w += x[j].w; }
         p4[j] = o;
+        if (norm_out) {
+          const float4 gg = __ldg(reinterpret_cast<const float4*>(e.g_next + n0) + j);
+          ssq += o.x * o.x + o.y * o.y + o.z * o.z + o.w * o.w;
+          yw[2 * j] = pack2<T>(o.x * gg.x, o.y * gg.y);
+          yw[2 * j + 1] = pack2<T>(o.z * gg.z, o.w * gg.w);
+        }
+      }
+      if (norm_out) {
+        uint4* y4 = reinterpret_cast<uint4*>(yp);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) y4[j] = make_uint4(yw[4 * j], yw[4 * j + 1], yw[4 * j + 2], yw[4 * j + 3]);
       }
     } else {
 #pragma unroll
@@ -106,6 +144,10 @@ __device__ __forceinline__ void epi_row32(const EpiArgs& e, int m, int n0, const
         if (n0 + j < e.N) {
           if (KIND == EPI_RESIDUAL) p[j] += v[j];
           else p[j] = v[j];
+          if (norm_out) {
+            ssq += p[j] * p[j];
+            yp[j] = from_f<T>(p[j] * e.g_next[n0 + j]);
+          }
         }
       }
     }
@@ -114,21 +156,22 @@ __device__ __forceinline__ void epi_row32(const EpiArgs& e, int m, int n0, const
     if (sizeof(T) == 2 && full && ((e.ldg & 7) == 0)) {
       uint32_t w[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) w[j] = pack2<T>(silu_f(v[4 * j]) * v[4 * j + 1], silu_f(v[4 * j + 2]) * v[4 * j + 3]);
+      for (int j = 0; j < 8; ++j)
+        w[j] = pack2<T>(silu_f(rs * v[4 * j]) * (rs * v[4 * j + 1]), silu_f(rs * v[4 * j + 2]) * (rs * v[4 * j + 3]));
       uint4* p4 = reinterpret_cast<uint4*>(p);
       p4[0] = make_uint4(w[0], w[1], w[2], w[3]);
       p4[1] = make_uint4(w[4], w[5], w[6], w[7]);
     } else {
 #pragma unroll
       for (int j = 0; j < 16; ++j)
-        if (n0 + 2 * j + 1 < e.N) p[j] = from_f<T>(silu_f(v[2 * j]) * v[2 * j + 1]);
+        if (n0 + 2 * j + 1 < e.N) p[j] = from_f<T>(silu_f(rs * v[2 * j]) * (rs * v[2 * j + 1]));
     }
   } else {  // QKV_ROPE: a 32-column chunk never straddles a head when d % 32 == 0
     if (!full || (e.d & 31) != 0 || sizeof(T) != 2) {
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        if (n0 + j < e.N) qkv_store<T>(e, m, n0 + j, v[j], v[j ^ 1]);
-      return;
+        if (n0 + j < e.N) qkv_store<T>(e, m, n0 + j, rs * v[j], rs * v[j ^ 1]);
+      return 0.f;
     }
     const int b = m / e.S, s = m - b * e.S;
     const int pos = e.pos0[b] + s;
@@ -141,12 +184,13 @@ __device__ __forceinline__ void epi_row32(const EpiArgs& e, int m, int n0, const
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const float2 c = cs[j];
-        r[2 * j] = v[2 * j] * c.x - v[2 * j + 1] * c.y;
-        r[2 * j + 1] = v[2 * j] * c.y + v[2 * j + 1] * c.x;
+        const float a = rs * v[2 * j], b = rs * v[2 * j + 1];
+        r[2 * j] = a * c.x - b * c.y;
+        r[2 * j + 1] = a * c.y + b * c.x;
       }
     } else {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) r[j] = v[j];
+      for (int j = 0; j < 32; ++j) r[j] = rs * v[j];
     }
     if (n0 < hd) {
       const int h = n0 / e.d;
@@ -166,6 +210,7 @@ __device__ __forceinline__ void epi_row32(const EpiArgs& e, int m, int n0, const
 #pragma unroll
     for (int j = 0; j < 4; ++j) p4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
   }
+  return ssq;
 }
 
 // Column form for the swap-AB GEMM: one thread holds feature n for the 32

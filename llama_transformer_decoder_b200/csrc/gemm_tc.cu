@@ -244,6 +244,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + acc * W_BN;
       float4* mine = reinterpret_cast<float4*>(ws) + (size_t)blockIdx.x * (W_BM * W_BN / 4) + row;
+      const float rs = (KIND == EPI_QKV_ROPE || KIND == EPI_SWIGLU) && epi.ss_in && klo == 0 && m0 + row < M
+                           ? norm_row_scale(epi, m0 + row) : 1.f;
+      float ssq = 0.f;
 #pragma unroll 1
       for (int c = 0; c < W_BN / 32; ++c) {
         float v[32];
@@ -254,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(base + c * 32, v);
         }
         if (whole) {
-          if (!failed && n0 + c * 32 < N) epi_row32<KIND, T>(epi, m0 + row, n0 + c * 32, v);
+          if (!failed && n0 + c * 32 < N) ssq += epi_row32<KIND, T>(epi, m0 + row, n0 + c * 32, v, rs);
         } else if (klo != 0) {  // a share for the owner
 #pragma unroll
           for (int j = 0; j < 8; ++j)
@@ -270,9 +273,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               v[4 * j] += x[j].x; v[4 * j + 1] += x[j].y; v[4 * j + 2] += x[j].z; v[4 * j + 3] += x[j].w;
             }
           }
-          if (!failed && n0 + c * 32 < N) epi_row32<KIND, T>(epi, m0 + row, n0 + c * 32, v);
+          if (!failed && n0 + c * 32 < N) ssq += epi_row32<KIND, T>(epi, m0 + row, n0 + c * 32, v, rs);
         }
       }
+      if (KIND == EPI_RESIDUAL && epi.ss_out && klo == 0 && m0 + row < M)
+        epi.ss_out[(size_t)(m0 + row) * epi.ss_n + n0 / W_BN] = ssq;
       tc_fence_before();
       mbar_arrive(&acce[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
@@ -421,14 +426,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!failed) failed = !__all_sync(0xffffffffu, mbar_wait(&accf[acc], acc_phase, status));
       tc_fence_after();
       const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + acc * P_BN;
+      const float rs = (KIND == EPI_QKV_ROPE || KIND == EPI_SWIGLU) && epi.ss_in && m0 + row < M
+                           ? norm_row_scale(epi, m0 + row) : 1.f;
+      float ssq = 0.f;
 #pragma unroll 1
       for (int c = 0; c < P_BN / 32; ++c) {
         float v[32];
         if (!failed) {
           tmem_ld32(base + c * 32, v);
-          if (n0 + c * 32 < N) epi_row32<KIND, T>(epi, m0 + row, n0 + c * 32, v);
+          if (n0 + c * 32 < N) ssq += epi_row32<KIND, T>(epi, m0 + row, n0 + c * 32, v, rs);
         }
       }
+      if (KIND == EPI_RESIDUAL && epi.ss_out && m0 + row < M) epi.ss_out[(size_t)(m0 + row) * epi.ss_n + n0 / P_BN] = ssq;
       tc_fence_before();
       mbar_arrive_cluster(mapa_shared(smem_u32(&acce[acc]), 0));
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }

@@ -74,6 +74,10 @@ int launch_embed(const int32_t* tokens, int M, const void* table, int V, int D, 
 int launch_rmsnorm(const float* x, const float* g, void* y, int rows, int D, float eps, int last_of_S, int dtype,
                    cudaStream_t st);
 int launch_argmax(const float* logits, int32_t* out, int B, int V, cudaStream_t st);
+// y = x * g (16-bit) and ss[r*ss_n + 0] = sum of x[r]^2 (other slots 0): the
+// inputs of a GEMM that applies the RMSNorm in its epilogue.
+int launch_norm_prep(const float* x, const float* g, void* y, float* ss, int rows, int D, int ss_n, int dtype,
+                     cudaStream_t st);
 int launch_add_lengths(int32_t* len, int B, int add, cudaStream_t st);
 
 // Attention. q [B][H][S][d]; K/V cache [B][Hk][Smax][d] (this layer);

@@ -85,6 +85,8 @@ struct llama_model {
   std::vector<int32_t> h_len;
   float2* rope = nullptr;
   // workspace
+  float* ss = nullptr;        // [max_tokens][ceil(dim/256)] partial sums of squares (folded RMSNorm)
+  bool norm_ready = false;    // xn / ss already hold the next layer's attention-norm inputs
   float* x = nullptr;
   void* xn = nullptr;
   void* q = nullptr;
@@ -320,9 +322,37 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
   char* kc = static_cast<char*>(m->kcache) + (size_t)l * m->layer_cache_elems * m->esz;
   char* vc = static_cast<char*>(m->vcache) + (size_t)l * m->layer_cache_elems * m->esz;
 
-  mark(m, K_RMSNORM, st);
-  RC(launch_rmsnorm(m->x, w.attn_norm, m->xn, M, D, c.norm_eps, 0, m->adt, st));
+  // Prefill-sized GEMMs (M > 128) fold the RMSNorms in: the residual GEMMs'
+  // epilogues leave y = x * g and per-tile sums of squares for the next norm,
+  // and the QKV / w1-w3 epilogues scale by rsqrt(mean(x^2) + eps).
+  const bool fuse = m->adt != LLAMA_F32 && M > 128;
+  const int ss_n = (D + 255) / 256;
+  if (fuse) {
+    if (!m->norm_ready) {
+      mark(m, K_RMSNORM, st);
+      RC(launch_norm_prep(m->x, w.attn_norm, m->xn, m->ss, M, D, ss_n, m->adt, st));
+    }
+  } else {
+    mark(m, K_RMSNORM, st);
+    RC(launch_rmsnorm(m->x, w.attn_norm, m->xn, M, D, c.norm_eps, 0, m->adt, st));
+  }
+  m->norm_ready = false;
+  auto norm_in = [&](EpiArgs& a) {
+    if (!fuse) return;
+    a.ss_in = m->ss;
+    a.ss_n = ss_n;
+    a.norm_inv_d = 1.f / (float)D;
+    a.norm_eps = c.norm_eps;
+  };
+  auto norm_out = [&](EpiArgs& a, const float* g_next) {
+    if (!fuse || !g_next) return;
+    a.g_next = g_next;
+    a.y_out = m->xn;
+    a.ss_out = m->ss;
+    a.ss_n = ss_n;
+  };
   EpiArgs e = epi_base(M, m->qkv_n);
+  norm_in(e);
   e.q = m->q;
   e.kc = kc;
   e.vc = vc;
@@ -350,17 +380,28 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
   EpiArgs r = epi_base(M, D);
   r.out = m->x;
   r.ldo = D;
+  norm_out(r, w.ffn_norm);
   mark(m, K_GEMM_WO, st);
   RC(gemm(m, m->attn, M, H * d, w.wo, D, EPI_RESIDUAL, r, st));
-  mark(m, K_RMSNORM, st);
-  RC(launch_rmsnorm(m->x, w.ffn_norm, m->xn, M, D, c.norm_eps, 0, m->adt, st));
+  if (!fuse) {
+    mark(m, K_RMSNORM, st);
+    RC(launch_rmsnorm(m->x, w.ffn_norm, m->xn, M, D, c.norm_eps, 0, m->adt, st));
+  }
   EpiArgs sg = epi_base(M, 2 * m->F);
   sg.g = m->g;
   sg.ldg = m->F;
+  norm_in(sg);
   mark(m, K_GEMM_W13, st);
   RC(gemm(m, m->xn, M, D, w.w13, 2 * m->F, EPI_SWIGLU, sg, st));
+  EpiArgs r2 = epi_base(M, D);
+  r2.out = m->x;
+  r2.ldo = D;
+  if (l + 1 < c.n_layers) {   // the next layer's attention norm (the final norm takes the last rows only)
+    norm_out(r2, m->L[l + 1].attn_norm);
+    m->norm_ready = fuse;
+  }
   mark(m, K_GEMM_W2, st);
-  RC(gemm(m, m->g, M, m->F, w.w2, D, EPI_RESIDUAL, r, st));
+  RC(gemm(m, m->g, M, m->F, w.w2, D, EPI_RESIDUAL, r2, st));
   return LLAMA_OK;
 }
 
@@ -379,6 +420,7 @@ int run_head(llama_model* m, int B, int S, cudaStream_t st) {
 }
 
 int decode_body(llama_model* m, int B, int cmax, cudaStream_t st) {
+  m->norm_ready = false;
   mark(m, K_EMBED, st);
   RC(launch_embed(m->tok_buf, B, m->tok_emb, m->cfg.vocab_size, m->cfg.dim, m->adt, m->x, m->d_status, st));
   for (int l = 0; l < m->cfg.n_layers; ++l) RC(run_layer(m, l, B, 1, true, cmax, st));
@@ -528,6 +570,7 @@ int llama_create(const llama_config* cfg, llama_model** out) {
   // ---- workspace
   const size_t Mx = m->Mmax;
   m->x = static_cast<float*>(m->alloc(Mx * D * 4));
+  m->ss = static_cast<float*>(m->alloc(Mx * ((D + 255) / 256) * 4));
   m->xn = m->alloc(Mx * D * es);
   m->q = m->alloc(Mx * Hd * es);
   m->attn = m->alloc(Mx * Hd * es);
@@ -535,7 +578,7 @@ int llama_create(const llama_config* cfg, llama_model** out) {
   m->logits = static_cast<float*>(m->alloc((size_t)c.max_batch * V * 4));
   m->tok_buf = static_cast<int32_t*>(m->alloc(Mx * sizeof(int32_t)));
   m->d_status = static_cast<int*>(m->alloc(sizeof(int)));
-  if (!m->kcache || !m->vcache || !m->d_len || !m->rope || !m->x || !m->xn || !m->q || !m->attn || !m->g ||
+  if (!m->kcache || !m->vcache || !m->d_len || !m->rope || !m->x || !m->ss || !m->xn || !m->q || !m->attn || !m->g ||
       !m->logits || !m->tok_buf || !m->d_status) {
     delete m;
     return LLAMA_ERR_OOM;
@@ -684,6 +727,7 @@ int llama_prefill(llama_model* m, const int32_t* tokens, int32_t B, int32_t S, v
   cudaStream_t st = S_(stream);
   RC(fit_pages_all(m, B, S, st));
   const int M = B * S;
+  m->norm_ready = false;
   mark(m, K_EMBED, st);
   RC(launch_embed(tokens, M, m->tok_emb, m->cfg.vocab_size, m->cfg.dim, m->adt, m->x, m->d_status, st));
   for (int l = 0; l < m->cfg.n_layers; ++l) RC(run_layer(m, l, B, S, false, 0, st));
@@ -791,7 +835,9 @@ int llama_block_forward(llama_model* m, int32_t layer, const float* x, float* y,
   RC(fit_pages_all(m, B, S, st));
   const size_t bytes = (size_t)B * S * m->cfg.dim * sizeof(float);
   CK(cudaMemcpyAsync(m->x, x, bytes, cudaMemcpyDeviceToDevice, st));
+  m->norm_ready = false;
   RC(run_layer(m, layer, B, S, false, 0, st));
+  m->norm_ready = false;
   CK(cudaMemcpyAsync(y, m->x, bytes, cudaMemcpyDeviceToDevice, st));
   return LLAMA_OK;
 }
