@@ -182,7 +182,7 @@ D_, F_, H_, HK_, HD_, V_ = 4096, 14336, 32, 8, 128, 128256
 # Measured DRAM bytes per launch of the prefill projection GEMM (mean over a
 # layer's QKV, Wo, w1/w3, w2 launches at 2048 tokens; one ncu capture of the
 # current kernel). Set to None when the kernel changes until re-captured.
-PAIR_GEMM_TRAFFIC = 187.6e6
+PAIR_GEMM_TRAFFIC = 187.2e6
 
 
 def measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust, peak_src):
