@@ -343,7 +343,7 @@ def run_ours(args):
     max_seq = DECODE_CTX + DECODE_STEPS + max(args.warmup, 2) + 8
     cfg = make_config(LLAMA3_8B, dtype=L.LLAMA_BF16, max_batch=1 if args.no_decode else DECODE_B,
                       max_seq=PREFILL_S if args.no_decode else max_seq, max_tokens=PREFILL_B * PREFILL_S,
-                      n_layers=NL)
+                      n_layers=NL, kv_page_size=128 if args.paged else 0)
     st = torch.cuda.Stream()
     m = L.llama_create(cfg)
     L.llama_init_weights(m, 0, 0.02, st)
@@ -375,7 +375,8 @@ def run_ours(args):
                                        '+ argmax); decode: B=32, context 4096, 128 greedy steps',
                            'batch': PREFILL_B, 'seq_len': PREFILL_S, 'layers': NL,
                            'l2': 'inputs larger than L2 (16 GB of weights streamed per step)',
-                           'parallelism': f'replicas x{ws}'},
+                           'parallelism': f'replicas x{ws}',
+                           'kv_cache': 'paged (128-position pages)' if args.paged else 'contiguous'},
                 'roofline': roofline, 'cpu_baseline': cpu, 'e2e': e2e, 'gpu_launches': launches,
                 'clocks': clk, 'kernels': kernels, 'decode': decode}
         print(json.dumps(line), flush=True)
@@ -473,6 +474,7 @@ def main():
     ap.add_argument('--decode-only', action='store_true', help='skip the prefill and end-to-end legs (profiling)')
     ap.add_argument('--layers', type=int, default=32, help='decoder layers (32 = the 8B model)')
     ap.add_argument('--no-cpu-baseline', action='store_true')
+    ap.add_argument('--paged', action='store_true', help='run the model with the paged KV cache')
     ap.add_argument('--kernel', choices=['attention_prefill', 'attention_decode', 'linear'],
                     help='time one kernel alone on seeded inputs (profiling and sweeps)')
     ap.add_argument('--batch', default='1', help='--kernel attention_*: sequences (comma list)')
