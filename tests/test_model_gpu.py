@@ -362,3 +362,36 @@ def test_decode_is_repeatable():
         _check_status(m)
     finally:
         m.close()
+
+
+def test_long_context_chunked_prefill_on_pages():
+    """An 8192-token prompt prefilled in two 4096-token chunks over the paged
+    cache (64 pages), then one decode step: the last-token logits of both calls
+    against one float32 oracle pass over the same 8193 tokens."""
+    m = Model(dict(SMALL_BF16, kv_page_size=128), BF16, max_batch=1, max_seq=8200, max_tokens=4096)
+    try:
+        L.llama_init_weights(m.h, 12, 0.02)
+        toks = si.tokens(13, 8193, 3000)
+        L.llama_prefill(m.h, torch.from_numpy(np.ascontiguousarray(toks[:4096])).cuda(), 1, 4096)
+        L.llama_prefill(m.h, torch.from_numpy(np.ascontiguousarray(toks[4096:8192])).cuda(), 1, 4096)
+        got0 = m.logits(1).cpu().numpy()[0]
+        L.llama_decode_step(m.h, torch.from_numpy(np.ascontiguousarray(toks[8192:])).cuda(), 1)
+        got1 = m.logits(1).cpu().numpy()[0]
+        _check_status(m)
+        orc = Oracle(m.p, SeededWeights(m.p, 12, 0.02, BF16), dtype=np.float32)
+        _, hidden = orc.forward(toks, return_hidden=True)
+        ref = orc.logits(hidden[[8191, 8192]])
+        assert rel_l2(got0, ref[0]) < 2e-2
+        assert rel_l2(got1, ref[1]) < 2e-2
+    finally:
+        m.close()
+
+
+@pytest.mark.parametrize('over,status', [(dict(kv_page_size=64), 'UNSUPPORTED'), (dict(kv_page_size=128), 'F32')])
+def test_paged_config_validation(over, status):
+    """Pages are 128 positions and need a 16-bit model."""
+    dtype = F32 if status == 'F32' else BF16
+    cfg = make_config(dict(SMALL_BF16, **over), dtype=dtype, max_batch=1, max_seq=256)
+    with pytest.raises(L.LlamaError) as e:
+        L.llama_create(cfg)
+    assert e.value.status == L.LLAMA_ERR_UNSUPPORTED
