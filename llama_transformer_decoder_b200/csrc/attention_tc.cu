@@ -49,7 +49,7 @@ constexpr uint32_t FA_TMEM_P = 384;                   // P: 64 columns, keys 2c 
 constexpr float FA_RESCALE = 8.0f;                    // raise the running max only past +8 (log2)
 
 // 2^x with the hardware approximation (flushes results below 2^-126 to zero,
-// which only affects probabilities too small to matter in a bf16 P).
+// which only affects probabilities too small to matter in a 16-bit P).
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

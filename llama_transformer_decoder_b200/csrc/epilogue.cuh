@@ -213,69 +213,4 @@ __device__ __forceinline__ float epi_row32(const EpiArgs& e, int m, int n0, cons
   return ssq;
 }
 
-// Column form for the swap-AB GEMM: one thread holds feature n for the 32
-// consecutive tokens [m0, m0+32); partner[j] is feature n^1 of token m0+j
-// (from the neighbouring lane). Every global load is issued before the first
-// store, so the loads overlap instead of waiting behind possibly-aliasing stores.
-template <int KIND, typename T>
-__device__ __forceinline__ void epi_col32(const EpiArgs& e, int m0, int n, const float (&v)[32],
-                                          const float (&partner)[32]) {
-  if (n >= e.N) return;
-  const int mcount = e.M - m0 < 32 ? e.M - m0 : 32;
-  if (KIND == EPI_STORE_F32) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (j < mcount) e.out[(size_t)(m0 + j) * e.ldo + n] = v[j];
-  } else if (KIND == EPI_RESIDUAL) {
-    float x[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) x[j] = j < mcount ? e.out[(size_t)(m0 + j) * e.ldo + n] : 0.f;
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (j < mcount) e.out[(size_t)(m0 + j) * e.ldo + n] = x[j] + v[j];
-  } else if (KIND == EPI_SWIGLU) {
-    if ((n & 1) == 0) {
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (j < mcount) static_cast<T*>(e.g)[(size_t)(m0 + j) * e.ldg + (n >> 1)] = from_f<T>(silu_f(v[j]) * partner[j]);
-    }
-  } else {
-    const int hd = e.H * e.d;
-    const bool rot = n < hd + e.Hk * e.d;
-    const int i = (n % e.d) >> 1;
-    float2 cs[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      cs[j] = make_float2(1.f, 0.f);
-      if (rot && j < mcount) {
-        const int m = m0 + j, b = m / e.S;
-        cs[j] = e.rope[(size_t)(e.pos0[b] + m - b * e.S) * (e.d >> 1) + i];
-      }
-    }
-    int pos[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int m = m0 + j, b = m / e.S;
-      pos[j] = j < mcount ? e.pos0[b] + m - b * e.S : 0;
-    }
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (j >= mcount) continue;
-      const int m = m0 + j, b = m / e.S, s = m - b * e.S;
-      const float r = !rot ? v[j] : ((n & 1) ? (partner[j] * cs[j].y + v[j] * cs[j].x)
-                                             : (v[j] * cs[j].x - partner[j] * cs[j].y));
-      if (n < hd) {
-        const int h = n / e.d, dd = n - h * e.d;
-        static_cast<T*>(e.q)[(((size_t)b * e.H + h) * e.S + s) * e.d + dd] = from_f<T>(r);
-      } else {
-        const bool is_k = rot;
-        const int nn = n - hd - (is_k ? 0 : e.Hk * e.d);
-        const int g = nn / e.d, dd = nn - g * e.d;
-        T* dst = static_cast<T*>(is_k ? e.kc : e.vc);
-        dst[kv_elem(e, b, g, pos[j]) + dd] = from_f<T>(r);
-      }
-    }
-  }
-}
-
 }  // namespace llama

@@ -1,23 +1,26 @@
 // tcgen05 GEMMs for the 16-bit projections: acc = x W^T with x [M,K], W [N,K]
 // (bf16 or fp16 operands, fp32 accumulation).
 //
-// Two kernels share the same warp roles (warp 0: TMA producer, warp 1: MMA
+// Three kernels share the same warp roles (warp 0: TMA producer, warp 1: MMA
 // issuer and TMEM owner, warps 2-5: epilogue reading TMEM):
 //
-//  * gemm_wide  (M large, prefill): persistent, one CTA per SM, 128x256 output
-//    tiles (rows = tokens, cols = weight rows), 4-stage TMA ring of 48 KB,
-//    double-buffered fp32 accumulators in TMEM (2 x 256 columns) so the
-//    epilogue of tile i overlaps the main loop of tile i+1.
-//
+//  * gemm_pair (M large, at least one wave of tiles: prefill): clusters of two
+//    SMs, 256x256 output tiles; each CTA loads its 128 rows of x and its 128
+//    rows of W, the leader issues tcgen05.mma.cta_group::2 (M=256, N=256) and
+//    each CTA drains its 128 rows of the accumulator.
+//  * gemm_wide (M large, fewer tiles than SMs): persistent, one CTA per SM,
+//    128x256 output tiles, split stream-K over all SMs with an owner fixup.
+//    Both keep double-buffered fp32 accumulators in TMEM (2 x 256 columns) so
+//    the epilogue of one tile overlaps the main loop of the next.
 //  * gemm_skinny (M <= 256, decode and short prompts): the weight tile is the
 //    MMA's A operand (128 weight rows) and the tokens are its N side, so a
 //    decode step streams each weight byte exactly once at full MMA width.
 //    Persistent stream-K: every CTA streams an equal share of (tile, k-block)
-//    units. Tiles shared by several CTAs are reduced by their last
-//    contributor (atomic ticket, no spinning) in a fixed order, except for
-//    the residual epilogue, where each contributor adds into x atomically.
+//    units; a split tile is finished by the CTA holding its k-block 0, which
+//    waits (bounded) for the other shares and sums them in CTA order, except
+//    for the residual epilogue, where each share is added into x atomically.
 //
-// Both are launched with programmatic dependent launch: weight tiles are
+// All are launched with programmatic dependent launch: weight tiles are
 // requested before waiting for the previous kernel, activations after.
 #include <cudaTypedefs.h>
 
