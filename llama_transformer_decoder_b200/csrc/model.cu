@@ -12,6 +12,7 @@
 #include <map>
 #include <mutex>
 #include <string>
+#include <tuple>
 #include <vector>
 
 #include "epilogue.cuh"
@@ -51,6 +52,9 @@ struct LayerW {
 size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 }  // namespace
+
+using GraphKey = std::tuple<int, int, int>;
+enum GraphKind { G_PREFILL = 0, G_DECODE = 1 };
 
 struct llama_model {
   llama_config cfg{};
@@ -100,9 +104,11 @@ struct llama_model {
   GemmScratch gs{};
   DecodeScratch ds{};
   int* d_status = nullptr;
-  std::map<std::pair<int, int>, cudaGraphExec_t> graphs;
-  std::map<std::pair<int, int>, unsigned long long> graph_kernels;
-  std::map<std::pair<int, int>, int> seen;
+  // CUDA graphs of whole steps, keyed by (kind, B, S or cache bound): the
+  // executable, the kernels it launches, and how often the key has been seen.
+  std::map<GraphKey, cudaGraphExec_t> graphs;
+  std::map<GraphKey, unsigned long long> graph_kernels;
+  std::map<GraphKey, int> seen;
   size_t bytes = 0;
   std::vector<void*> allocs;
   // per-kernel profiling (eager runs only): an event before every launch
@@ -419,6 +425,17 @@ int run_head(llama_model* m, int B, int S, cudaStream_t st) {
   return LLAMA_OK;
 }
 
+int prefill_body(llama_model* m, int B, int S, cudaStream_t st) {
+  m->norm_ready = false;
+  mark(m, K_EMBED, st);
+  RC(launch_embed(m->tok_buf, B * S, m->tok_emb, m->cfg.vocab_size, m->cfg.dim, m->adt, m->x, m->d_status, st));
+  for (int l = 0; l < m->cfg.n_layers; ++l) RC(run_layer(m, l, B, S, false, 0, st));
+  RC(run_head(m, B, S, st));
+  mark(m, K_OTHER, st);
+  RC(launch_add_lengths(m->d_len, B, S, st));
+  return LLAMA_OK;
+}
+
 int decode_body(llama_model* m, int B, int cmax, cudaStream_t st) {
   m->norm_ready = false;
   mark(m, K_EMBED, st);
@@ -427,6 +444,45 @@ int decode_body(llama_model* m, int B, int cmax, cudaStream_t st) {
   RC(run_head(m, B, 1, st));
   mark(m, K_OTHER, st);
   RC(launch_add_lengths(m->d_len, B, 1, st));
+  return LLAMA_OK;
+}
+
+// Runs one step through a CUDA graph cached under `key`. The first call per key
+// runs eagerly (it also sets the kernels' attributes), the second captures the
+// step and replays it, later calls replay. A step only reads device state whose
+// addresses are fixed per model (tokens are staged in tok_buf; positions, lengths
+// and the block table are read from device memory), so a replay recomputes the
+// step for the current inputs. Profiling, the default stream and LLAMA_NO_GRAPH
+// keep every call eager.
+template <typename Body>
+int run_graphed(llama_model* m, const GraphKey& key, cudaStream_t st, Body&& body) {
+  static const bool no_graph = getenv("LLAMA_NO_GRAPH") != nullptr;
+  auto it = m->graphs.find(key);
+  if (it != m->graphs.end() && !m->prof_on) {
+    g_launches += m->graph_kernels[key];
+    CK(cudaGraphLaunch(it->second, st));
+    m->norm_ready = false;
+    return LLAMA_OK;
+  }
+  if (st == nullptr || no_graph || m->prof_on || m->seen[key]++ == 0) return body();
+  cudaGraph_t graph = nullptr;
+  CK(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
+  const unsigned long long before = g_launches.load();
+  const int rc = body();
+  const unsigned long long captured = g_launches.load() - before;
+  g_launches -= captured;  // counted again at every replay
+  const cudaError_t ce = cudaStreamEndCapture(st, &graph);
+  if (rc != LLAMA_OK) { if (graph) cudaGraphDestroy(graph); return rc; }
+  if (ce != cudaSuccess) { cudaGetLastError(); return LLAMA_ERR_CUDA; }
+  cudaGraphExec_t exec = nullptr;
+  const cudaError_t ie = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (ie != cudaSuccess) { cudaGetLastError(); return LLAMA_ERR_CUDA; }
+  m->graphs[key] = exec;
+  m->graph_kernels[key] = captured;
+  g_launches += captured;
+  CK(cudaGraphLaunch(exec, st));
+  m->norm_ready = false;
   return LLAMA_OK;
 }
 
@@ -611,8 +667,9 @@ int llama_create(const llama_config* cfg, llama_model** out) {
       ws = std::max(ws, skinny_workspace_floats(std::min(128, m->Mmax)));
       tickets = std::max(tickets, (sh[0] + 127) / 128);
     }
-    // the wide GEMM's stream-K tail has fewer than 1.5 waves of tiles
-    const int sk_max = m->Mmax > 128 ? 3 * num_sms() / 2 + 1 : 0;
+    // split tiles of the large-M GEMMs: fewer than 1.5 waves of 1-SM tiles, or
+    // fewer than two waves of pair tiles with a ticket per CTA of the pair
+    const int sk_max = m->Mmax > 128 ? 2 * num_sms() : 0;
     tickets = std::max(tickets, sk_max);
     if (sk_max) ws = std::max(ws, wide_workspace_floats());
     if (grow_gemm_scratch(&m->gs, std::max<size_t>(ws, 1), tickets) != LLAMA_OK) { delete m; return LLAMA_ERR_OOM; }
@@ -725,15 +782,10 @@ int llama_prefill(llama_model* m, const int32_t* tokens, int32_t B, int32_t S, v
   RC(check_lengths(m, B, S));
   if ((int64_t)B * S > m->Mmax) return LLAMA_ERR_SHAPE;
   cudaStream_t st = S_(stream);
-  RC(fit_pages_all(m, B, S, st));
-  const int M = B * S;
-  m->norm_ready = false;
-  mark(m, K_EMBED, st);
-  RC(launch_embed(tokens, M, m->tok_emb, m->cfg.vocab_size, m->cfg.dim, m->adt, m->x, m->d_status, st));
-  for (int l = 0; l < m->cfg.n_layers; ++l) RC(run_layer(m, l, B, S, false, 0, st));
-  RC(run_head(m, B, S, st));
-  mark(m, K_OTHER, st);
-  RC(launch_add_lengths(m->d_len, B, S, st));
+  RC(fit_pages_all(m, B, S, st));  // before the (possibly graph-replayed) step reads the table
+  CK(cudaMemcpyAsync(m->tok_buf, tokens, (size_t)B * S * sizeof(int32_t), cudaMemcpyDeviceToDevice, st));
+  RC(run_graphed(m, GraphKey(G_PREFILL, B, S), st, [&] { return prefill_body(m, B, S, st); }));
+  m->last_B = B;
   for (int b = 0; b < B; ++b) m->h_len[b] += S;
   return LLAMA_OK;
 }
@@ -747,33 +799,8 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t B, void* st
   for (int b = 0; b < B; ++b) maxlen = std::max(maxlen, m->h_len[b] + 1);
   const int cmax = std::min(m->cfg.max_seq, (maxlen + 511) / 512 * 512);
   CK(cudaMemcpyAsync(m->tok_buf, tokens, B * sizeof(int32_t), cudaMemcpyDeviceToDevice, st));
-  const auto key = std::make_pair(B, cmax);
-  static const bool no_graph = getenv("LLAMA_NO_GRAPH") != nullptr;
-  auto it = m->graphs.find(key);
-  if (it != m->graphs.end() && !m->prof_on) {
-    g_launches += m->graph_kernels[key];
-    CK(cudaGraphLaunch(it->second, st));
-  } else if (st == nullptr || no_graph || m->prof_on || m->seen[key]++ == 0) {
-    RC(decode_body(m, B, cmax, st));  // first call per shape runs eagerly (also sets kernel attributes)
-  } else {
-    cudaGraph_t graph = nullptr;
-    CK(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
-    const unsigned long long before = g_launches.load();
-    const int rc = decode_body(m, B, cmax, st);
-    const unsigned long long captured = g_launches.load() - before;
-    g_launches -= captured;  // counted again at every replay
-    const cudaError_t ce = cudaStreamEndCapture(st, &graph);
-    if (rc != LLAMA_OK) { if (graph) cudaGraphDestroy(graph); return rc; }
-    if (ce != cudaSuccess) { cudaGetLastError(); return LLAMA_ERR_CUDA; }
-    cudaGraphExec_t exec = nullptr;
-    const cudaError_t ie = cudaGraphInstantiate(&exec, graph, 0);
-    cudaGraphDestroy(graph);
-    if (ie != cudaSuccess) { cudaGetLastError(); return LLAMA_ERR_CUDA; }
-    m->graphs[key] = exec;
-    m->graph_kernels[key] = captured;
-    g_launches += captured;
-    CK(cudaGraphLaunch(exec, st));
-  }
+  RC(run_graphed(m, GraphKey(G_DECODE, B, cmax), st, [&] { return decode_body(m, B, cmax, st); }));
+  m->last_B = B;
   for (int b = 0; b < B; ++b) m->h_len[b] += 1;
   return LLAMA_OK;
 }
@@ -1050,7 +1077,7 @@ int llama_linear(const void* x, const void* w, float* y, int32_t M, int32_t N, i
     RC(grow_gemm_scratch(&c->gs, skinny_workspace_floats(M), (N + 127) / 128));
   } else {
     const WideSplit w = wide_split(M, N, K);
-    RC(grow_gemm_scratch(&c->gs, wide_workspace_floats(), std::max(w.sk_tiles, 1)));
+    RC(grow_gemm_scratch(&c->gs, wide_workspace_floats(), std::max(w.sk_tiles, 2 * num_sms())));
   }
   return gemm16(x, M, K, K, w, N, K, dtype, EPI_STORE_F32, e, variant, &c->gs, c->status, S_(stream));
 }

@@ -215,6 +215,43 @@ def test_chunked_prefill_continues_the_cache():
         m.close()
 
 
+@pytest.mark.parametrize('paged', [False, True])
+def test_graph_replayed_prefill_chunks(paged):
+    """Four equal prefill chunks on a stream: the first runs eagerly, the second
+    is captured into a CUDA graph, the others replay it. Each replay must take
+    its tokens, positions and (paged) block-table entries from the current
+    call, so the last-token logits after every chunk match one oracle pass over
+    the prompt so far; the logits of a replayed prompt equal the eager ones."""
+    params = dict(SMALL_BF16, kv_page_size=128) if paged else SMALL_BF16
+    m = Model(params, BF16, max_batch=2, max_seq=512)
+    try:
+        L.llama_init_weights(m.h, 14, 0.02)
+        orc = Oracle(m.p, SeededWeights(m.p, 14, 0.02, BF16))
+        B, C = 2, 96
+        toks = si.tokens(15, B * 4 * C, 3000).reshape(B, 4 * C)
+        st = torch.cuda.Stream()
+        with torch.cuda.stream(st):
+            for i in range(4):
+                chunk = torch.from_numpy(np.ascontiguousarray(toks[:, i * C:(i + 1) * C])).cuda()
+                L.llama_prefill(m.h, chunk, B, C, st)
+                got = m.logits(B, st).cpu().numpy()
+                ref = np.stack([orc.forward(toks[b, :(i + 1) * C]) for b in range(B)])
+                assert rel_l2(got, ref) < 2e-2, i
+                if i == 0:
+                    eager = got
+            first = torch.from_numpy(np.ascontiguousarray(toks[:, :C])).cuda()
+            outs = []
+            for _ in range(2):                    # graph replays from an empty cache
+                L.llama_reset(m.h, st)
+                L.llama_prefill(m.h, first, B, C, st)
+                outs.append(m.logits(B, st).cpu().numpy())
+            for out in outs:
+                assert rel_l2(out, eager) < 2e-3
+        _check_status(m)
+    finally:
+        m.close()
+
+
 def test_bf16_weights_and_cache_round_trip():
     """A bf16 model holds its weights as fp16: set/get return the caller's bf16
     bits wherever fp16 represents them exactly (|w| >= 2^-14), and within 2^-25
