@@ -667,9 +667,8 @@ int llama_create(const llama_config* cfg, llama_model** out) {
       ws = std::max(ws, skinny_workspace_floats(std::min(128, m->Mmax)));
       tickets = std::max(tickets, (sh[0] + 127) / 128);
     }
-    // split tiles of the large-M GEMMs: fewer than 1.5 waves of 1-SM tiles, or
-    // fewer than two waves of pair tiles with a ticket per CTA of the pair
-    const int sk_max = m->Mmax > 128 ? 2 * num_sms() : 0;
+    // the wide GEMM's stream-K tiles: fewer than 1.5 waves
+    const int sk_max = m->Mmax > 128 ? 3 * num_sms() / 2 + 1 : 0;
     tickets = std::max(tickets, sk_max);
     if (sk_max) ws = std::max(ws, wide_workspace_floats());
     if (grow_gemm_scratch(&m->gs, std::max<size_t>(ws, 1), tickets) != LLAMA_OK) { delete m; return LLAMA_ERR_OOM; }
@@ -1077,7 +1076,7 @@ int llama_linear(const void* x, const void* w, float* y, int32_t M, int32_t N, i
     RC(grow_gemm_scratch(&c->gs, skinny_workspace_floats(M), (N + 127) / 128));
   } else {
     const WideSplit w = wide_split(M, N, K);
-    RC(grow_gemm_scratch(&c->gs, wide_workspace_floats(), std::max(w.sk_tiles, 2 * num_sms())));
+    RC(grow_gemm_scratch(&c->gs, wide_workspace_floats(), std::max(w.sk_tiles, 1)));
   }
   return gemm16(x, M, K, K, w, N, K, dtype, EPI_STORE_F32, e, variant, &c->gs, c->status, S_(stream));
 }
