@@ -352,12 +352,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Make this thread's generic-proxy shared-memory writes visible to the async
-// proxy (TMA, tcgen05.mma operand reads).
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // 2-D tiled load into this CTA's shared memory whose completion bytes are
 // counted on an mbarrier given by its cluster address, which may be in the
 // peer CTA of a CTA pair (no multicast).
@@ -395,8 +389,6 @@ __device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t smem_addr, uint3
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
-
-__device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31) == 0; }
 
 // ------------------------------------------- programmatic dependent launch
 // A kernel launched with programmatic stream serialization may start before

@@ -251,13 +251,6 @@ __global__ void fill_const_kernel(float* dst, int64_t n, float v) {
     dst[i] = v;
 }
 
-__global__ void fill_tokens_kernel(int32_t* dst, int64_t n, uint64_t key, uint32_t vocab) {
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    const uint64_t d = mix64(key + ((uint64_t)i + 1) * SG);
-    dst[i] = (int32_t)(((d >> 32) * (uint64_t)vocab) >> 32);
-  }
-}
-
 int grid_for(int64_t n) {
   int64_t g = (n + 255) / 256;
   const int64_t cap = (int64_t)num_sms() * 16;
@@ -442,13 +435,6 @@ int launch_fill_const(float* dst, int64_t n, float v, cudaStream_t st) {
   if (n <= 0) return LLAMA_OK;
   count_launches(1);
   fill_const_kernel<<<grid_for(n), 256, 0, st>>>(dst, n, v);
-  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
-}
-
-int launch_fill_tokens(int32_t* dst, int64_t n, uint64_t seed, uint64_t stream_id, int vocab, cudaStream_t st) {
-  if (n <= 0) return LLAMA_OK;
-  count_launches(1);
-  fill_tokens_kernel<<<grid_for(n), 256, 0, st>>>(dst, n, stream_key(seed, stream_id), (uint32_t)vocab);
   return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 

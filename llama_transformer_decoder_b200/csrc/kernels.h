@@ -125,6 +125,5 @@ int launch_fill_kv(void* dst, const KvLayout& L, int B, int Hk, int c, int d, ui
 // Cache (through L) <- src [B][Hk][c][d], converting src_elt -> dst_elt.
 int launch_kv_scatter(void* dst, int dst_elt, const KvLayout& L, int B, int Hk, int c, int d, const void* src,
                       int src_elt, cudaStream_t st);
-int launch_fill_tokens(int32_t* dst, int64_t n, uint64_t seed, uint64_t stream_id, int vocab, cudaStream_t st);
 
 }  // namespace llama
