@@ -118,12 +118,19 @@ int llama_get_weight(llama_model* m, const char* name, void* dst, size_t nbytes,
 /* Prefill: tokens (device int32 [B][S]) are appended to sequences 0..B-1 at positions
  * len[b] .. len[b]+S-1, their post-RoPE K and V written to the cache, and the last token's
  * logits of each sequence kept ([W] 预测下一个输出: final norm once, final_embedding[-1] @
- * output^T). Requires B <= max_batch, B*S <= max_tokens, len[b]+S <= max_seq. len[b] += S. */
+ * output^T). Requires B <= max_batch, B*S <= max_tokens, len[b]+S <= max_seq. len[b] += S.
+ * On a non-default stream the step is replayed from a CUDA graph kept per (B, S): the first call
+ * for a shape runs eagerly, the second is captured, later calls replay it. Tokens are first
+ * copied into a model-owned buffer, and positions and the block table are read from device
+ * memory, so a replay always computes the current call. The default stream, profiling and the
+ * environment variable LLAMA_NO_GRAPH keep every call eager. A model must not be used from two
+ * host threads at once. */
 int llama_prefill(llama_model* m, const int32_t* tokens, int32_t B, int32_t S, void* stream);
 
 /* One decode step: token b (device int32 [B]) is processed at position len[b] of sequence b,
  * attending to keys 0..len[b] through the cache; len[b] += 1. Logits are kept as for prefill.
- * The step is replayed from a CUDA graph after its first call for a given B. */
+ * Replayed from CUDA graphs as for prefill, one graph per (B, cache bound), the cache bound
+ * being the longest sequence rounded up to 512 positions. */
 int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t B, void* stream);
 
 /* fp32 logits [B][vocab] (device) of the last prefill or decode step. */
