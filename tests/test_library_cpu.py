@@ -64,3 +64,37 @@ def test_binding_fails_loudly_without_library(tmp_path):
     r = subprocess.run(['python', '-c', f"import importlib.util as u; s=u.spec_from_file_location('b', {str(dst)!r});"
                         "m=u.module_from_spec(s); s.loader.exec_module(m)"], capture_output=True, text=True)
     assert r.returncode != 0 and 'ImportError' in r.stderr
+
+
+@pytest.mark.parametrize('over,dtype,status', [
+    (dict(n_heads=7), 'F32', 'SHAPE'),                     # heads do not divide dim
+    (dict(n_kv_heads=3), 'F32', 'SHAPE'),                  # kv heads do not divide heads
+    (dict(dim=0), 'F32', 'SHAPE'),
+    (dict(n_heads=32, n_kv_heads=2), 'F32', 'UNSUPPORTED'),  # more than 8 query heads per kv head
+    (dict(dim=2048, n_heads=32, n_kv_heads=8), 'BF16', 'UNSUPPORTED'),  # 16-bit kernels need head_dim 128
+    (dict(kv_page_size=64), 'BF16', 'UNSUPPORTED'),          # pages are 128 positions
+    (dict(kv_page_size=128), 'F32', 'UNSUPPORTED'),          # paged kernels are 16-bit
+    (dict(kv_page_size=128, kv_pages=-1), 'BF16', 'SHAPE'),
+    (dict(ffn_hidden=0, multiple_of=0), 'F32', 'SHAPE'),     # no hidden size and no rule to derive it
+    (dict(norm_eps=-1.0), 'F32', 'INVALID_ARG'),
+    (dict(rope_theta=0.0), 'F32', 'INVALID_ARG'),
+])
+def test_config_validation_on_host(over, dtype, status):
+    """llama_create rejects an invalid configuration before touching the
+    device, with the status the header documents."""
+    from llama_transformer_decoder_b200 import binding as b
+    from llama_transformer_decoder_b200.configs import make_config
+    base = dict(dim=4096, n_layers=1, n_heads=32, n_kv_heads=8, vocab_size=1000, ffn_hidden=14336,
+                multiple_of=1024, norm_eps=1e-5, rope_theta=500000.0)
+    cfg = make_config(base, dtype=getattr(b, 'LLAMA_' + dtype), max_batch=2, max_seq=256, **over)
+    with pytest.raises(b.LlamaError) as e:
+        b.llama_create(cfg)
+    assert e.value.status == getattr(b, 'LLAMA_ERR_' + status)
+
+
+def test_unknown_dtype_is_rejected_on_host():
+    from llama_transformer_decoder_b200 import binding as b
+    from llama_transformer_decoder_b200.configs import TINY, make_config
+    with pytest.raises(b.LlamaError) as e:
+        b.llama_create(make_config(TINY, dtype=7, max_batch=1, max_seq=16))
+    assert e.value.status == b.LLAMA_ERR_INVALID_ARG
