@@ -154,6 +154,16 @@ def oracle_prefill_sample(n_layers_model: int = 32, S: int = PREFILL_S):
     return tok_s, dt, f'oracle float32 numpy: 1 of {n_layers_model} layers of the 8B model at S={S}, x{n_layers_model}'
 
 
+def workload_config(ws, args, NL=32):
+    """The workload both arms report (the reference arm times a sample of it)."""
+    return {'workload': 'llama3-8b-shape full-model prefill, B=1, S=2048 (32 layers + LM head '
+                        '+ argmax); decode: B=32, context 4096, 128 greedy steps',
+            'batch': PREFILL_B, 'seq_len': PREFILL_S, 'layers': NL,
+            'l2': 'inputs larger than L2 (16 GB of weights streamed per step)',
+            'parallelism': f'replicas x{ws}',
+            'kv_cache': 'paged (128-position pages)' if args.paged else 'contiguous'}
+
+
 def run_reference(args):
     ws, rank, _ = _dist()
     if rank != 0:
@@ -170,7 +180,7 @@ def run_reference(args):
     line = {'impl': 'reference', 'metric': METRIC, 'value': value, 'unit': 'tokens/s', 'n_gpus': args.gpus,
             'steps': args.steps, 'warmup': args.warmup, 'ms_per_step': dt * 32 * 1e3, 'higher_is_better': True,
             'scaling': 'weak', 'vs_baseline': None, 'dtype': 'f32', 'data': 'synthetic (seeded)',
-            'config': {'workload': 'llama3-8b-shape prefill B=1 S=2048 (CPU oracle on a 1-layer sample)'},
+            'config': workload_config(ws, args),
             'cpu_baseline': {'value': value, 'unit': 'tokens/s', 'cores': cores, 'kind': 'oracle', 'sample': desc},
             'e2e': {'value': value, 'unit': 'tokens/s', 'h2d_bytes_per_step': 0, 'd2h_bytes_per_step': 0}}
     print(json.dumps(line), flush=True)
@@ -372,12 +382,7 @@ def run_ours(args):
                 'vs_baseline': None, 'dtype': 'f16',
                 'data': 'synthetic: seeded N(0,0.02) weights of the 8B shapes rounded to bf16 (held as fp16), '
                         'uniform token ids',
-                'config': {'workload': 'llama3-8b-shape full-model prefill, B=1, S=2048 (32 layers + LM head '
-                                       '+ argmax); decode: B=32, context 4096, 128 greedy steps',
-                           'batch': PREFILL_B, 'seq_len': PREFILL_S, 'layers': NL,
-                           'l2': 'inputs larger than L2 (16 GB of weights streamed per step)',
-                           'parallelism': f'replicas x{ws}',
-                           'kv_cache': 'paged (128-position pages)' if args.paged else 'contiguous'},
+                'config': workload_config(ws, args, NL),
                 'roofline': roofline, 'cpu_baseline': cpu, 'e2e': e2e, 'gpu_launches': launches,
                 'clocks': clk, 'kernels': kernels, 'decode': decode}
         print(json.dumps(line), flush=True)
