@@ -1,5 +1,5 @@
 // C-ABI host library: model handle, weights, KV cache, workspace, the layer
-// loop of prefill and decode, CUDA-graph replay of decode steps, and the
+// loop of prefill and decode, CUDA-graph replay of prefill and decode steps, and the
 // stateless entry points used by tests and benchmarks.
 #include <cuda_runtime.h>
 
