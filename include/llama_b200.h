@@ -123,8 +123,10 @@ int llama_get_weight(llama_model* m, const char* name, void* dst, size_t nbytes,
  * for a shape runs eagerly, the second is captured, later calls replay it. Tokens are first
  * copied into a model-owned buffer, and positions and the block table are read from device
  * memory, so a replay always computes the current call. The default stream, profiling and the
- * environment variable LLAMA_NO_GRAPH keep every call eager. A model must not be used from two
- * host threads at once. */
+ * environment variable LLAMA_NO_GRAPH keep every call eager. Graphs are kept until
+ * llama_destroy, one per shape seen twice: a workload with many distinct prompt lengths should
+ * prefill on the default stream (or set LLAMA_NO_GRAPH). A model must not be used from two host
+ * threads at once. */
 int llama_prefill(llama_model* m, const int32_t* tokens, int32_t B, int32_t S, void* stream);
 
 /* One decode step: token b (device int32 [B]) is processed at position len[b] of sequence b,
