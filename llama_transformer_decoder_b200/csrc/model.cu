@@ -11,6 +11,7 @@
 #include <atomic>
 #include <map>
 #include <mutex>
+#include <set>
 #include <string>
 #include <tuple>
 #include <vector>
@@ -109,6 +110,7 @@ struct llama_model {
   std::map<GraphKey, cudaGraphExec_t> graphs;
   std::map<GraphKey, unsigned long long> graph_kernels;
   std::map<GraphKey, int> seen;
+  std::set<GraphKey> eager_only;  // shapes whose capture failed: always run eagerly
   size_t bytes = 0;
   std::vector<void*> allocs;
   // per-kernel profiling (eager runs only): an event before every launch
@@ -453,7 +455,8 @@ int decode_body(llama_model* m, int B, int cmax, cudaStream_t st) {
 // addresses are fixed per model (tokens are staged in tok_buf; positions, lengths
 // and the block table are read from device memory), so a replay recomputes the
 // step for the current inputs. Profiling, the default stream and LLAMA_NO_GRAPH
-// keep every call eager.
+// keep every call eager. If a capture or its instantiation fails, the step
+// runs eagerly instead, and so does every later call with that key.
 template <typename Body>
 int run_graphed(llama_model* m, const GraphKey& key, cudaStream_t st, Body&& body) {
   static const bool no_graph = getenv("LLAMA_NO_GRAPH") != nullptr;
@@ -464,20 +467,28 @@ int run_graphed(llama_model* m, const GraphKey& key, cudaStream_t st, Body&& bod
     m->norm_ready = false;
     return LLAMA_OK;
   }
-  if (st == nullptr || no_graph || m->prof_on || m->seen[key]++ == 0) return body();
+  if (st == nullptr || no_graph || m->prof_on || m->eager_only.count(key) || m->seen[key]++ == 0) return body();
+  auto run_eagerly = [&] {
+    cudaGetLastError();
+    m->eager_only.insert(key);
+    return body();
+  };
+  if (cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return run_eagerly();
   cudaGraph_t graph = nullptr;
-  CK(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
   const unsigned long long before = g_launches.load();
   const int rc = body();
   const unsigned long long captured = g_launches.load() - before;
   g_launches -= captured;  // counted again at every replay
   const cudaError_t ce = cudaStreamEndCapture(st, &graph);
-  if (rc != LLAMA_OK) { if (graph) cudaGraphDestroy(graph); return rc; }
-  if (ce != cudaSuccess) { cudaGetLastError(); return LLAMA_ERR_CUDA; }
+  if (ce != cudaSuccess) {  // capture broken (launches inside it failed too): nothing ran
+    if (graph) cudaGraphDestroy(graph);
+    return run_eagerly();
+  }
+  if (rc != LLAMA_OK) { cudaGraphDestroy(graph); return rc; }
   cudaGraphExec_t exec = nullptr;
   const cudaError_t ie = cudaGraphInstantiate(&exec, graph, 0);
   cudaGraphDestroy(graph);
-  if (ie != cudaSuccess) { cudaGetLastError(); return LLAMA_ERR_CUDA; }
+  if (ie != cudaSuccess) return run_eagerly();
   m->graphs[key] = exec;
   m->graph_kernels[key] = captured;
   g_launches += captured;
