@@ -2,7 +2,7 @@
 ranks exchange nothing but the step time. These tests run that host logic as
 two gloo ranks on the CPU (rendezvous on 127.0.0.1): the max-over-ranks step
 time, the whole-job throughput, and the reference arm's non-zero ranks
-exiting without work."""
+exiting without work, and the reference arm's JSON line."""
 import json
 import os
 import socket
@@ -66,3 +66,26 @@ def test_reference_arm_other_ranks_exit_without_work():
                        text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ''
+
+
+def test_reference_arm_prints_the_contract_line():
+    """Rank 0 of the reference arm times the CPU oracle on a bounded sample and
+    prints one JSON line with the same metric and workload as the GPU arm."""
+    sys.path.insert(0, ROOT)
+    import bench
+    r = subprocess.run([sys.executable, os.path.join(ROOT, 'bench.py'), '--impl', 'reference', '--steps', '1',
+                        '--warmup', '0'], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.startswith('{')]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ('metric', 'value', 'unit', 'n_gpus', 'steps', 'warmup', 'ms_per_step', 'higher_is_better',
+                'scaling', 'vs_baseline', 'dtype', 'data', 'config', 'cpu_baseline', 'e2e'):
+        assert key in d, key
+    assert d['impl'] == 'reference' and d['metric'] == bench.METRIC and d['unit'] == 'tokens/s'
+    assert d['value'] > 0 and d['higher_is_better'] is True and d['steps'] == 1
+    import argparse
+    assert d['config'] == bench.workload_config(1, argparse.Namespace(paged=False))
+    cb = d['cpu_baseline']
+    assert cb['kind'] == 'oracle' and cb['value'] == d['value'] and cb['cores'] >= 1 and cb['sample']
+    assert d['e2e'] == {'value': d['value'], 'unit': 'tokens/s', 'h2d_bytes_per_step': 0, 'd2h_bytes_per_step': 0}
