@@ -38,6 +38,9 @@
  *    activations does not. llama_get_weight returns bf16 again.
  *  - A model and its buffers belong to the device that was current at
  *    llama_create; make that device current before every later call.
+ *    Kernel attributes and scratch of the stateless calls are kept per device.
+ *    cudaDeviceReset frees everything the library holds on that device:
+ *    models created before it must not be used after it.
  */
 #ifndef LLAMA_B200_H
 #define LLAMA_B200_H
@@ -200,7 +203,8 @@ int llama_attention_prefill(const void* q, const void* k, const void* v, void* o
 /* Single-query attention over a cache (decode): q [B][H][d]; kc, vc [B][Hk][cmax][d]; len
  * (device int32 [B], 1 <= len[b] <= cmax) = number of valid keys of sequence b; o [B][H*d].
  * Split over the key range, merged with the log-sum-exp rule. d in {64,128} (bf16, fp16) or
- * {32,64,128} (fp32); H/Hk <= 8. */
+ * {32,64,128} (fp32); H/Hk <= 8. A len[b] outside [1, cmax] gives a NaN row for sequence b (the
+ * other rows are computed normally) and latches LLAMA_ERR_DEVICE_BOUNDS for llama_status(). */
 int llama_attention_decode(const void* q, const void* kc, const void* vc, const int32_t* len, void* o, int32_t B,
                            int32_t cmax, int32_t H, int32_t Hk, int32_t d, int32_t dtype, void* stream);
 
@@ -210,17 +214,20 @@ int llama_attention_decode(const void* q, const void* kc, const void* vc, const 
  * the card): a cudaMalloc made behind their back can fail or fragment that pool, and a
  * cudaMalloc/cudaFree inside a latency-critical loop synchronizes the whole device. This call
  * never allocates or frees device memory; everything else is the same as
- * llama_attention_decode (arguments, layouts, results).
+ * llama_attention_decode (arguments, layouts, results, bit for bit).
  * Its split partials live in one static 4 MiB device array that every GPU which loads this
  * library keeps until the process exits. Calls needing more than 4 MiB of partials return
  * LLAMA_ERR_SHAPE: for bf16 or fp16 with d = 128 the partials take (B*Hk + 4*SMs) * (H/Hk) * (d+2) * 4
  * bytes (SMs = 148 on B200), so with H = 32, Hk = 8 every B up to 170 fits.
- * The first call on a device looks up the array's device address for that device
- * (cudaGetSymbolAddress); make that first call before any stream capture begins.
- * Every call uses the same array, so calls that may run at the same time on the GPU (e.g. on
- * two streams) race: order them. Nothing has to be cleared between calls, since every partial
- * is written before it is read. This call keeps no device status word: a len[b] outside
- * [1, cmax] gives NaN rows instead of an error code.
+ * Device-side errors of the call (a len[b] outside [1, cmax], which also gives a NaN row; a
+ * bounded wait that gave up) are latched in a static status word of its own, next to the
+ * array; llama_status() returns and clears it, and allocates nothing when only this call ran.
+ * The first call on a device looks up the array's and the status word's device addresses for
+ * that device (cudaGetSymbolAddress); make that first call before any stream capture begins.
+ * The lookup is repeated after the device's context changed (cudaDeviceReset).
+ * Every call uses the same array and status word, so calls that may run at the same time on
+ * the GPU (e.g. on two streams) race: order them. Nothing has to be cleared between calls,
+ * since every partial is written before it is read.
  * The pages have no counterpart of this entry point: it exists for deployment only. */
 int llama_attention_decode_noalloc(const void* q, const void* kc, const void* vc, const int32_t* len, void* o,
                                    int32_t B, int32_t cmax, int32_t H, int32_t Hk, int32_t d, int32_t dtype,
@@ -259,7 +266,8 @@ int llama_argmax_rows(const float* logits, int32_t* out, int32_t B, int32_t V, v
 int llama_fill_normal(void* dst, int64_t n, uint64_t seed, uint64_t stream_id, float std, int32_t dtype,
                       void* stream);
 
-/* Synchronizes `stream`, then returns and clears the status word of the stateless calls. */
+/* Synchronizes `stream`, then returns and clears the status word of the stateless calls on the
+ * current device (the first non-zero of theirs and llama_attention_decode_noalloc's). */
 int llama_status(void* stream);
 
 #ifdef __cplusplus

@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(128) attn_decode_part_kernel(const T* __restri
   const T* ksrc = kc + ((size_t)b * Hk + g) * Smax * D;
   const T* vsrc = vc + ((size_t)b * Hk + g) * Smax * D;
 
-  if (n > Smax && threadIdx.x == 0) set_status(status, LLAMA_ERR_DEVICE_BOUNDS);
+  if ((n < 1 || n > Smax) && split == 0 && threadIdx.x == 0) set_status(status, LLAMA_ERR_DEVICE_BOUNDS);
 
   // this lane's slice of the G query vectors, pre-scaled for exp2
   float qr[DEC_MAXG][DPL];
@@ -394,7 +394,8 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
 
   long long total = 0;
   for (int b = 0; b < B; ++b) {
-    if (nkeys[b] + add_keys > nmax && blockIdx.x == 0 && threadIdx.x == 0) set_status(status, LLAMA_ERR_DEVICE_BOUNDS);
+    const int nb = nkeys[b] + add_keys;
+    if ((nb < 1 || nb > nmax) && blockIdx.x == 0 && threadIdx.x == 0) set_status(status, LLAMA_ERR_DEVICE_BOUNDS);
     total += (long long)Hk * dm_tiles(dm_keys(nkeys, b, add_keys, nmax));
   }
   const long long W = (long long)gridDim.x * DM_WARPS;
@@ -556,7 +557,10 @@ __global__ void __launch_bounds__(128) attn_decode_combine_pieces_kernel(
   __syncthreads();
   const long long total = s_tot, t0 = s_t0;
   const int nt_b = s_nt;
-  if (nt_b == 0 || total == 0) {
+  const int nb = nkeys[b] + add_keys;
+  // no keys, or more keys than the cache holds (clamped for the other
+  // sequences' sake, latched by the decode kernel): NaN rows, as the split path
+  if (nt_b == 0 || total == 0 || nb < 1 || nb > nmax) {
     for (int dd = threadIdx.x; dd < D; dd += blockDim.x) o[((size_t)b * H + h) * D + dd] = from_f<T>(NAN);
     return;
   }
@@ -598,12 +602,7 @@ int decode_launch(const void* q, const void* kc, const void* vc, const int32_t* 
   constexpr int DEC_SUB = dec_sub<T, D>();
   constexpr int SMEM = DEC_STAGES * 2 * DEC_SUB * ROW + DEC_STAGES * 8 + 4 * DEC_MAXG * (D + 2) * 4;
   auto kern = attn_decode_part_kernel<T, D>;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
-      return LLAMA_ERR_CUDA;
-    attr = true;
-  }
+  if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), SMEM)) return rc;
   int chunk = (cmax + splits - 1) / splits;
   chunk = (chunk + 127) / 128 * 128;
   const float scale_log2 = kLog2e / sqrtf((float)D);
@@ -670,12 +669,7 @@ static int mma_decode_launch(const void* q, const void* kc, const void* vc, cons
                              DecodeScratch* scratch, int* status, cudaStream_t st) {
   const int grid = num_sms();
   auto kern = attn_decode_mma_kernel<T>;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DM_SMEM) != cudaSuccess)
-      return LLAMA_ERR_CUDA;
-    attr = true;
-  }
+  if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), DM_SMEM)) return rc;
   const float scale_log2 = kLog2e / sqrtf(128.f);
   const int nmax = cmax < Smax ? cmax : Smax;
   cudaError_t err = launch_k(kern, dim3(grid), dim3(DM_WARPS * 32), DM_SMEM, st, static_cast<const T*>(q),

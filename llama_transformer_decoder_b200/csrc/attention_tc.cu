@@ -677,15 +677,17 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
 
 // [outer][rows][128] 16-bit -> 3-D map with boxes of 64 x 128 x 1, 128-byte swizzle.
 int make_tmap_3d(CUtensorMap* map, const void* base, int64_t outer, int64_t rows, bool is_f16) {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return LLAMA_ERR_CUDA;
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+    }
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  if (!fn) return LLAMA_ERR_CUDA;
   if (reinterpret_cast<uintptr_t>(base) & 15) return LLAMA_ERR_INVALID_ARG;
   cuuint64_t gdim[3] = {(cuuint64_t)FA_D, (cuuint64_t)rows, (cuuint64_t)outer};
   cuuint64_t gstride[2] = {(cuuint64_t)FA_D * 2, (cuuint64_t)rows * FA_D * 2};
@@ -723,12 +725,7 @@ static int attention_prefill_tc_t(const void* q, const void* kc, const void* vc,
   static const bool per_tile = getenv("LLAMA_ATTN_PER_TILE") != nullptr;
   if (!per_tile && S <= kPersistentMaxS) {
     auto kern = attn_prefill_tc_persistent_kernel<T>;
-    static bool attr = false;
-    if (!attr) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FP_SMEM) != cudaSuccess)
-        return LLAMA_ERR_CUDA;
-      attr = true;
-    }
+    if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), FP_SMEM)) return rc;
     const long long items = (long long)((S + FA_BM - 1) / FA_BM) * H * B;
     const int grid = (int)std::min<long long>(items, num_sms());
     const cudaError_t err = launch_k(kern, dim3(grid), dim3(FP_THREADS), FP_SMEM, st, tq, tk, tv, static_cast<T*>(o),
@@ -736,12 +733,7 @@ static int attention_prefill_tc_t(const void* q, const void* kc, const void* vc,
     return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
   }
   auto kern = attn_prefill_tc_kernel<T>;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM) != cudaSuccess)
-      return LLAMA_ERR_CUDA;
-    attr = true;
-  }
+  if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), FA_SMEM)) return rc;
   const cudaError_t err = launch_k(kern, dim3(((S + FA_BM - 1) / FA_BM) * H * B), dim3(FA_THREADS), FA_SMEM, st, tq,
                                    tk, tv,
                                    static_cast<T*>(o), pos0, S, H, Hk, scale_log2, kv_table, kv_max_pages, kv_pages,

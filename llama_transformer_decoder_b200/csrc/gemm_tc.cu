@@ -29,6 +29,7 @@
 #include <mutex>
 #include <type_traits>
 
+#include "device_cache.h"
 #include "epilogue.cuh"
 #include "kernels.h"
 
@@ -733,15 +734,67 @@ int make_tmap_16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
   return r == CUDA_SUCCESS ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
-int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+namespace {
+PerDeviceValue<int> g_sm_count;
+OncePerDevice g_smem_attr;
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
   }
-  return n;
+  return dev;
+}
+}  // namespace
+
+uint64_t context_key() {
+  typedef CUresult (*GetCurrent)(CUcontext*);
+  typedef CUresult (*GetId)(CUcontext, unsigned long long*);
+  struct Fns {
+    GetCurrent cur = nullptr;
+    GetId id = nullptr;
+  };
+  static const Fns fns = [] {
+    Fns f;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.cur = reinterpret_cast<GetCurrent>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.id = reinterpret_cast<GetId>(p);
+    cudaGetLastError();
+    return f;
+  }();
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (fns.cur && fns.id && fns.cur(&c) == CUDA_SUCCESS && c != nullptr && fns.id(c, &id) == CUDA_SUCCESS)
+    return id;
+  return (1ull << 63) | (uint64_t)(uint32_t)current_device();
+}
+
+int num_sms() {
+  const int dev = current_device();
+  return g_sm_count.get(dev, [dev] {
+    int n = 0;
+    if (dev < 0 || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    return n;
+  }, 148);
+}
+
+int ensure_smem_attr(const void* kern, int bytes) {
+  // Attributes belong to a context: key by the current one, so that a device
+  // reset (new context) sets them again.
+  const uint64_t key = context_key();
+  return g_smem_attr.run(key, kern, [&] {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess) return 0;
+    cudaGetLastError();
+    return (int)LLAMA_ERR_CUDA;
+  });
 }
 
 bool streamk_enabled() {
@@ -776,12 +829,7 @@ template <int KIND, typename T>
 static int launch_wide(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, const EpiArgs& e,
                        GemmScratch* scratch, int* status, cudaStream_t st) {
   auto kern = gemm_wide_kernel<KIND, T>;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, W_SMEM) != cudaSuccess)
-      return LLAMA_ERR_CUDA;
-    attr = true;
-  }
+  if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), W_SMEM)) return rc;
   WideSplit w = wide_split(M, N, K);
   float* ws = nullptr;
   int* tickets = nullptr;
@@ -811,12 +859,7 @@ template <int KIND, typename T>
 static int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, const EpiArgs& e,
                        int* status, cudaStream_t st) {
   auto kern = gemm_pair_kernel<KIND, T>;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM) != cudaSuccess)
-      return LLAMA_ERR_CUDA;
-    attr = true;
-  }
+  if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), P_SMEM)) return rc;
   const int tiles = ((M + 2 * P_BM - 1) / (2 * P_BM)) * ((N + P_BN - 1) / P_BN);
   const int pairs = std::min(tiles, num_sms() / 2);
   cudaLaunchConfig_t cfg = {};
@@ -843,12 +886,7 @@ static int launch_skinny_nt(const CUtensorMap& tw, const CUtensorMap& tx, int M,
                             float* ws, int* counters, int* status, cudaStream_t st) {
   using C = SkinnyCfg<NT>;
   auto kern = gemm_skinny_kernel<KIND, T, NT>;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
-      return LLAMA_ERR_CUDA;
-    attr = true;
-  }
+  if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return rc;
   const cudaError_t err = launch_k(kern, dim3(num_sms()), dim3(kThreads), C::SMEM, st, tw, tx, M, N, K, e, ws,
                                    counters, status);
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;

@@ -45,7 +45,15 @@ struct GemmScratch {
   int n_tickets;
 };
 
+// Identity of the calling thread's current CUDA context (unique over the
+// process lifetime; a device reset gives a new one). Falls back to a key of
+// the device ordinal when no context is current.
+uint64_t context_key();
+// SM count of the current device (cached per device).
 int num_sms();
+// Raises the dynamic shared-memory limit of `kern` to `bytes` on the current
+// device, once per device (thread-safe). LLAMA_OK or LLAMA_ERR_CUDA.
+int ensure_smem_attr(const void* kern, int bytes);
 
 // How a wide (prefill) GEMM is spread over the SMs: tiles [0, T_dp) in
 // data-parallel waves, the rest stream-K over G_sk CTAs (see gemm_tc.cu).
@@ -102,6 +110,10 @@ int attention_decode(const void* q, const void* kc, const void* vc, const int32_
                      int B, int cmax, int H, int Hk, int d, int Smax, int dtype, DecodeScratch* scratch,
                      int* status, cudaStream_t st, const int32_t* kv_table = nullptr, int kv_max_pages = 0,
                      int kv_pages = 0);
+
+// Status word of llama_attention_decode_noalloc on the current device: read
+// and cleared (0 when that call never ran on the device). Allocates nothing.
+int noalloc_take_status(int* out);
 
 // Seeded generator: SplitMix64 counter streams + Box-Muller from IEEE basic ops.
 // Logical element i = ((o * rows + r) * cols + c) of a [outer][rows][cols]

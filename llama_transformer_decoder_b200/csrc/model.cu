@@ -236,12 +236,19 @@ struct DevCtx {
   DecodeScratch ds{};
 };
 std::mutex g_mu;
-std::map<int, DevCtx> g_ctx;
+std::map<uint64_t, DevCtx> g_ctx;
 
-DevCtx* dev_ctx() {
-  int dev = 0;
-  cudaGetDevice(&dev);
+// The stateless context of the current device, created on first use
+// (create == false: nullptr if it does not exist yet).
+// Keyed by the current context, so that the scratch of a context destroyed by
+// a device reset (whose memory went with it) is not reused.
+DevCtx* dev_ctx(bool create = true) {
+  const uint64_t dev = context_key();
   std::lock_guard<std::mutex> lk(g_mu);
+  if (!create) {
+    auto it = g_ctx.find(dev);
+    return it == g_ctx.end() || !it->second.status ? nullptr : &it->second;
+  }
   DevCtx& c = g_ctx[dev];
   if (!c.status) {
     if (cudaMalloc(&c.status, sizeof(int)) != cudaSuccess) { cudaGetLastError(); c.status = nullptr; return nullptr; }
@@ -997,13 +1004,15 @@ int llama_sync_status(llama_model* m, void* stream) {
 
 // ------------------------------------------------------------- stateless
 int llama_status(void* stream) {
-  DevCtx* c = dev_ctx();
-  if (!c) return LLAMA_ERR_OOM;
   if (cudaStreamSynchronize(S_(stream)) != cudaSuccess) { cudaGetLastError(); return LLAMA_ERR_CUDA; }
   int s = 0;
-  CK(cudaMemcpy(&s, c->status, sizeof(int), cudaMemcpyDeviceToHost));
-  CK(cudaMemset(c->status, 0, sizeof(int)));
-  return s;
+  if (DevCtx* c = dev_ctx(false)) {   // no context yet: no stateless call has run, nothing to allocate
+    CK(cudaMemcpy(&s, c->status, sizeof(int), cudaMemcpyDeviceToHost));
+    CK(cudaMemset(c->status, 0, sizeof(int)));
+  }
+  int s2 = 0;
+  RC(noalloc_take_status(&s2));
+  return s != 0 ? s : s2;
 }
 
 int llama_attention_prefill(const void* q, const void* k, const void* v, void* o, int32_t B, int32_t S, int32_t H,
