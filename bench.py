@@ -29,6 +29,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = 'tokens/s: 8B-shape prefill & batch-32 decode; % tensor/HBM roofline'
 PREFILL_B, PREFILL_S = 1, 2048
+PREFILL_B8 = 8
 DECODE_B, DECODE_CTX, DECODE_STEPS = 32, 4096, 128
 
 
@@ -133,35 +134,103 @@ def oracle_threads() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_prefill_sample(n_layers_model: int = 32, S: int = PREFILL_S):
-    """Time the CPU oracle (float32 numpy, as it stands) on one of the 32 layers
-    of the 8B model at S tokens; returns (tokens/s scaled to the full model,
-    seconds, description)."""
-    import numpy as np
-    from oracle import Oracle, Params
-    import seeded_inputs as si
-    p = Params(4096, n_layers_model, 32, 8, 128256, 14336)
+class OracleSample:
+    """The float32 CPU oracle, as it stands, on bounded samples of the 8B
+    workloads. Weights of layer 0 and the output matrix are generated once,
+    outside every timed region. Samples:
 
-    class W(dict):
-        def __missing__(self, name):
-            if name.endswith('norm.weight'):
-                v = np.ones(4096, np.float32)
-            else:
-                shape = si.weight_shape(name, 4096, 32, 8, 14336, 128256)
-                v = si.bf16_bits_to_f32(si.weight(0, name, shape, n_layers_model, 0.02, 'bf16'))
-            self[name] = v
-            return v
+    * layer(S): one of the 32 decoder layers over S prompt tokens;
+    * head(): embedding of the prompt, final norm and LM head of the last row;
+    * decode_layer(ctx): one layer of one decode step (B = 1) over a cache of
+      ctx positions of N(0,1) K/V entries.
 
-    w = W()
-    for k in si.LAYER_KEYS:                      # inputs are prepared outside the timed region
-        w[f'layers.0.{k}.weight']
-    x = si.bf16_bits_to_f32(si.normal(2, si.STREAM_HIDDEN, S * 4096, 1.0)).reshape(S, 4096)
-    orc = Oracle(p, w, dtype=np.float32)
-    t0 = time.perf_counter()
-    orc.layer(0, x, None, 0)
-    dt = time.perf_counter() - t0
-    tok_s = S / (dt * n_layers_model)
-    return tok_s, dt, f'oracle float32 numpy: 1 of {n_layers_model} layers of the 8B model at S={S}, x{n_layers_model}'
+    Full-model figures are derived from the timed samples as
+    tokens / (32 x layer time + head time); every sample that enters one was
+    timed in the same run."""
+
+    def __init__(self):
+        import numpy as np
+        from oracle import Oracle, Params, SequenceCache
+        import seeded_inputs as si
+        self.np, self.si = np, si
+        self.p = Params(4096, 32, 32, 8, 128256, 14336)
+
+        class W(dict):
+            def __missing__(self, name):
+                if name.endswith('norm.weight'):
+                    v = np.ones(4096, np.float32)
+                else:
+                    shape = si.weight_shape(name, 4096, 32, 8, 14336, 128256)
+                    v = si.bf16_bits_to_f32(si.weight(0, name, shape, 32, 0.02, 'bf16'))
+                self[name] = v
+                return v
+
+        self.w = W()
+        for name in ['tok_embeddings.weight', 'output.weight', 'norm.weight'] + \
+                [f'layers.0.{k}.weight' for k in si.LAYER_KEYS]:
+            self.w[name]
+        self.orc = Oracle(self.p, self.w, dtype=np.float32)
+        self.SequenceCache = SequenceCache
+        self._x = {}
+        self._cache = None
+
+    def _hidden(self, S):
+        if S not in self._x:
+            si = self.si
+            self._x[S] = si.bf16_bits_to_f32(si.normal(2, si.STREAM_HIDDEN, S * 4096, 1.0)).reshape(S, 4096)
+        return self._x[S]
+
+    def layer(self, S=PREFILL_S):
+        x = self._hidden(S)
+        t0 = time.perf_counter()
+        self.orc.layer(0, x, None, 0)
+        return time.perf_counter() - t0
+
+    def head(self, S=PREFILL_S):
+        toks = self.si.tokens(1, S, 128256)
+        x = self._hidden(S)
+        t0 = time.perf_counter()
+        self.orc.embed(toks)
+        self.orc.logits(x[-1])
+        return time.perf_counter() - t0
+
+    def decode_layer(self, ctx=DECODE_CTX):
+        si = self.si
+        if self._cache is None:
+            n = 8 * ctx * 128
+            k = si.bf16_bits_to_f32(si.normal(3, si.STREAM_KV_BASE, n, 1.0, 'bf16')).reshape(8, ctx, 128)
+            v = si.bf16_bits_to_f32(si.normal(3, si.STREAM_KV_BASE + 1, n, 1.0, 'bf16')).reshape(8, ctx, 128)
+            self._cache = (k, v)
+        c = self.SequenceCache(k=[self._cache[0]], v=[self._cache[1]])
+        x = self._hidden(1)
+        t0 = time.perf_counter()
+        self.orc.layer(0, x, c, ctx)
+        return time.perf_counter() - t0
+
+
+def cpu_baseline(samples: OracleSample, layer_reps: int = 3) -> dict:
+    """The oracle on the host cores (all BLAS threads, then one thread) for the
+    prefill workload and for one decode step; about 20 s of CPU work."""
+    from threadpoolctl import threadpool_limits
+    cores = oracle_threads()
+    t_layer = min(samples.layer() for _ in range(layer_reps))
+    t_head = min(samples.head() for _ in range(2))
+    t_dec = min(samples.decode_layer() for _ in range(5))
+    t_dhead = min(samples.head(1) for _ in range(3))
+    with threadpool_limits(limits=1, user_api='blas'):
+        t1_layer = samples.layer(256)
+        t1_head = samples.head(256)
+    return {'value': PREFILL_S / (32 * t_layer + t_head), 'unit': 'tokens/s', 'cores': cores, 'kind': 'oracle',
+            'sample': f'float32 numpy oracle, prefill B=1: one of the 32 layers at S={PREFILL_S} '
+                      f'({t_layer:.3f} s, best of {layer_reps}) and the embedding + final norm + LM head of the '
+                      f'last row ({t_head:.3f} s), each timed; value = {PREFILL_S} / (32 x layer + head)',
+            'one_thread': {'value': 256 / (32 * t1_layer + t1_head), 'unit': 'tokens/s', 'cores': 1,
+                           'sample': f'the same at S=256 with one BLAS thread (layer {t1_layer:.3f} s, '
+                                     f'head {t1_head:.3f} s)'},
+            'decode': {'value': 1.0 / (32 * t_dec + t_dhead), 'unit': 'tokens/s', 'cores': cores,
+                       'sample': f'one decode step, B=1, context {DECODE_CTX} (N(0,1) cache): one layer '
+                                 f'({t_dec * 1e3:.1f} ms, best of 5) x 32 plus the LM head of the row '
+                                 f'({t_dhead * 1e3:.1f} ms)'}}
 
 
 def workload_config(ws, args, NL=32):
@@ -175,20 +244,28 @@ def workload_config(ws, args, NL=32):
 
 
 def run_reference(args):
+    """The oracle as the reference arm (the pages hold no implementation to
+    install). Every step is one bounded sample: one of the 32 decoder layers
+    of the 8B model over the B=1, S=2048 prompt; steps and ms_per_step describe
+    exactly those timed samples. The line's value is the full-model prefill
+    throughput derived from them and from the embedding + final norm + LM head
+    of the last row, timed once in the same run."""
     ws, rank, _ = _dist()
     if rank != 0:
         return 0
-    times = []
-    desc = ''
-    for i in range(args.warmup + args.steps):
-        tok_s, dt, desc = oracle_prefill_sample()
-        if i >= args.warmup:
-            times.append(dt)
+    samples = OracleSample()
+    for _ in range(args.warmup):
+        samples.layer()
+    times = [samples.layer() for _ in range(args.steps)]
+    t_head = samples.head()
     dt = statistics.mean(times)
     cores = oracle_threads()
-    value = PREFILL_S / (dt * 32)
+    value = PREFILL_S / (32 * dt + t_head)
+    desc = (f'float32 numpy oracle; each step: one of the 32 layers of the 8B model at S={PREFILL_S} '
+            f'(mean {dt:.3f} s); value = {PREFILL_S} / (32 x step + embedding/final-norm/LM-head time '
+            f'{t_head:.3f} s)')
     line = {'impl': 'reference', 'metric': METRIC, 'value': value, 'unit': 'tokens/s', 'n_gpus': args.gpus,
-            'steps': args.steps, 'warmup': args.warmup, 'ms_per_step': dt * 32 * 1e3, 'higher_is_better': True,
+            'steps': args.steps, 'warmup': args.warmup, 'ms_per_step': dt * 1e3, 'higher_is_better': True,
             'scaling': 'weak', 'vs_baseline': None, 'dtype': 'f32', 'data': 'synthetic (seeded)',
             'config': workload_config(ws, args),
             'cpu_baseline': {'value': value, 'unit': 'tokens/s', 'cores': cores, 'kind': 'oracle', 'sample': desc},
@@ -205,14 +282,15 @@ D_, F_, H_, HK_, HD_, V_ = 4096, 14336, 32, 8, 128, 128256
 PAIR_GEMM_TRAFFIC = 187.2e6
 
 
-def measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust, peak_src):
-    """Timed prefill steps (no per-launch events), then the same steps with
-    the library's per-launch events for the kernel breakdown and roofline."""
+def measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust, peak_src, B=PREFILL_B):
+    """Timed prefill steps of B sequences (no per-launch events), then the
+    same steps with the library's per-launch events for the kernel breakdown
+    and roofline."""
     import torch
 
     def prefill_step():
         L.llama_reset(m, st)
-        L.llama_prefill(m, toks, PREFILL_B, PREFILL_S, st)
+        L.llama_prefill(m, toks, B, PREFILL_S, st)
         L.llama_argmax(m, arg, st)
 
     for _ in range(args.warmup):
@@ -243,7 +321,7 @@ def measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust, peak_src)
     L.llama_profile(m, 0)
     prof_ms = p0.elapsed_time(p1) / args.steps
     _barrier(ws)
-    M = PREFILL_B * PREFILL_S
+    M = B * PREFILL_S
     flops_layer = 2.0 * M * D_ * ((H_ + 2 * HK_) * HD_ + H_ * HD_ + 2 * F_ + F_)
     gemm_kinds = ['gemm_qkv_rope', 'gemm_wo_residual', 'gemm_w13_swiglu', 'gemm_w2_residual']
     gemm_ms = sum(prof[k][0] for k in gemm_kinds)
@@ -252,7 +330,7 @@ def measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust, peak_src)
     total_prof = max(sum(x[0] for x in prof.values()), 1e-9)
     kernels = {k: {'ms_per_step': v[0] / args.steps, 'launches_per_step': v[1] / args.steps,
                    'share': v[0] / total_prof} for k, v in prof.items() if v[1]}
-    attn_flops = 4.0 * PREFILL_B * H_ * HD_ * PREFILL_S * (PREFILL_S + 1) / 2 * NL
+    attn_flops = 4.0 * B * H_ * HD_ * PREFILL_S * (PREFILL_S + 1) / 2 * NL
     attn = prof.get('attention_prefill', (0, 0))
     roofline = {'kernel': 'gemm_pair_kernel (tcgen05 cta_group::2, 4 projections)', 'bound': 'tensor',
                 'achieved': achieved, 'peak': tf_sust, 'unit': 'TFLOP/s',
@@ -348,6 +426,46 @@ def measure_decode(L, m, st, arg, args, ws, local, NL, hbm_peak, peak_src):
             'clocks': clk.summary()}
 
 
+def measure_block(L, m, st, S, args, hbm_peak, tf_burst, tf_sust, peak_src):
+    """One 8B-shaped decoder block (layer 0 of the model) on N(0,1) hidden
+    states of one sequence of S tokens at positions 0..S-1: S = 17 is bound by
+    streaming the block's 436 MB of weights, S = 2048 by the tensor cores.
+    Weights (436 MB) exceed L2, so every call streams them from HBM."""
+    import torch
+    x = torch.empty((1, S, D_), dtype=torch.float32, device='cuda')
+    L.llama_fill_normal(x, x.numel(), 2, (1 << 20) + 1, 1.0, L.LLAMA_F32, st)
+    y = torch.empty_like(x)
+    lens = __import__('numpy').zeros(DECODE_B, __import__('numpy').int32)
+    L.llama_set_lengths(m, lens, DECODE_B, st)
+    for _ in range(max(args.warmup, 3)):
+        L.llama_block_forward(m, 0, x, y, 1, S, st)
+    torch.cuda.synchronize()
+    reps = max(args.steps, 10)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(reps):
+        L.llama_block_forward(m, 0, x, y, 1, S, st)
+    e1.record(st)
+    torch.cuda.synchronize()
+    assert L.llama_sync_status(m, st) == 0
+    ms = e0.elapsed_time(e1) / reps
+    w_bytes = 2.0 * (D_ * (H_ + 2 * HK_) * HD_ + D_ * H_ * HD_ + 3 * D_ * F_)
+    flops = 2.0 * S * w_bytes / 2 + 4.0 * H_ * HD_ * S * (S + 1) / 2
+    out = {'value': S / (ms / 1e3), 'unit': 'tokens/s', 'ms_per_call': ms, 'calls': reps,
+           'workload': f'one 8B-shaped decoder block, B=1, S={S}, positions 0..{S - 1}, N(0,1) hidden states'}
+    if S <= 128:
+        gbs = w_bytes / (ms / 1e3) / 1e9
+        out['roofline'] = {'bound': 'hbm', 'achieved': gbs, 'peak': hbm_peak, 'unit': 'GB/s',
+                           'frac': gbs / hbm_peak, 'work': 'weight bytes per call (activations negligible)',
+                           'peak_kind': f'hbm copy ({peak_src})'}
+    else:
+        tf = flops / (ms / 1e3) / 1e12
+        out['roofline'] = {'bound': 'tensor', 'achieved': tf, 'peak': tf_burst, 'unit': 'TFLOP/s',
+                           'frac': tf / tf_burst, 'work': 'linear + causal attention flops per call',
+                           'peak_kind': f'bf16 burst ({peak_src}): the block is timed alone'}
+    return out
+
+
 def run_ours(args):
     import torch
     ws, rank, local = _dist()
@@ -362,9 +480,8 @@ def run_ours(args):
 
     NL = args.layers
     max_seq = DECODE_CTX + DECODE_STEPS + max(args.warmup, 2) + 8
-    cfg = make_config(LLAMA3_8B, dtype=L.LLAMA_BF16, max_batch=1 if args.no_decode else DECODE_B,
-                      max_seq=PREFILL_S if args.no_decode else max_seq, max_tokens=PREFILL_B * PREFILL_S,
-                      n_layers=NL, kv_page_size=128 if args.paged else 0)
+    cfg = make_config(LLAMA3_8B, dtype=L.LLAMA_BF16, max_batch=DECODE_B, max_seq=max_seq,
+                      max_tokens=PREFILL_B8 * PREFILL_S, n_layers=NL, kv_page_size=128 if args.paged else 0)
     st = torch.cuda.Stream()
     m = L.llama_create(cfg)
     L.llama_init_weights(m, 0, 0.02, st)
@@ -374,16 +491,24 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     ms = launches = clk = roofline = kernels = e2e = None
+    prefill_b8 = blocks = None
     if not args.decode_only:
         ms, launches, clk, roofline, kernels = measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust,
                                                                peak_src)
         e2e = measure_e2e(L, m, st, toks_h, args, ws)
+        if not args.no_extra:
+            toks8 = torch.from_numpy(si.tokens(1, PREFILL_B8 * PREFILL_S, V_).reshape(PREFILL_B8, PREFILL_S)).cuda()
+            ms8, _, clk8, roof8, _ = measure_prefill(L, m, st, toks8, arg, args, ws, local, NL, tf_sust, peak_src,
+                                                     B=PREFILL_B8)
+            v8, _ = replica_throughput(PREFILL_B8 * PREFILL_S, ms8, ws)
+            prefill_b8 = {'value': v8, 'unit': 'tokens/s', 'ms_per_step': ms8, 'batch': PREFILL_B8,
+                          'seq_len': PREFILL_S, 'roofline': roof8, 'clocks': clk8}
+            blocks = {f's{S}': measure_block(L, m, st, S, args, hbm_peak, tf_burst, tf_sust, peak_src)
+                      for S in (17, 2048)}
     decode = None if args.no_decode else measure_decode(L, m, st, arg, args, ws, local, NL, hbm_peak, peak_src)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and NL == 32 and not args.decode_only:
-        tok_s, dt, desc = oracle_prefill_sample()
-        cpu = {'value': tok_s, 'unit': 'tokens/s', 'cores': oracle_threads(), 'kind': 'oracle', 'sample': desc,
-               'seconds': dt}
+        cpu = cpu_baseline(OracleSample())
     L.llama_destroy(m)
     if rank == 0:
         value = ws * PREFILL_B * PREFILL_S / (ms / 1e3) if ms else None
@@ -394,7 +519,8 @@ def run_ours(args):
                         'uniform token ids',
                 'config': workload_config(ws, args, NL),
                 'roofline': roofline, 'cpu_baseline': cpu, 'e2e': e2e, 'gpu_launches': launches,
-                'clocks': clk, 'kernels': kernels, 'decode': decode}
+                'clocks': clk, 'kernels': kernels, 'decode': decode, 'prefill_b8': prefill_b8,
+                'block_8b': blocks}
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist
@@ -490,6 +616,7 @@ def main():
     ap.add_argument('--decode-only', action='store_true', help='skip the prefill and end-to-end legs (profiling)')
     ap.add_argument('--layers', type=int, default=32, help='decoder layers (32 = the 8B model)')
     ap.add_argument('--no-cpu-baseline', action='store_true')
+    ap.add_argument('--no-extra', action='store_true', help='skip the B=8 prefill and single-block legs')
     ap.add_argument('--paged', action='store_true', help='run the model with the paged KV cache')
     ap.add_argument('--kernel', choices=['attention_prefill', 'attention_decode', 'linear'],
                     help='time one kernel alone on seeded inputs (profiling and sweeps)')

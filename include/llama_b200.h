@@ -60,6 +60,8 @@ extern "C" {
 #define LLAMA_ERR_DEVICE_TIMEOUT (-5)/* a bounded device-side wait gave up */
 #define LLAMA_ERR_DEVICE_BOUNDS (-6) /* an index checked on the device was out of range */
 #define LLAMA_ERR_UNSUPPORTED (-7)   /* combination not implemented (e.g. 16-bit model with head_dim != 128) */
+#define LLAMA_ERR_RANGE (-8)         /* a 16-bit activation was not finite after rounding (fp16 overflows above
+                                        65504): latched by the kernel that rounded it; the outputs are garbage */
 
 typedef enum { LLAMA_F32 = 0, LLAMA_BF16 = 1, LLAMA_F16 = 2 } llama_dtype;
 
@@ -85,6 +87,10 @@ typedef struct llama_config {
                                  table (16-bit models; pages are taken from a pool as sequences grow and
                                  returned by llama_reset / llama_set_lengths) */
   int32_t kv_pages;           /* paged: pages in the pool; 0 = max_batch * ceil(max_seq / 128) */
+  int32_t act_dtype;          /* 16-bit models: element type of activations, KV cache and P. 0 = LLAMA_F16
+                                 (the default policy described above); LLAMA_BF16 (bf16 models only) keeps
+                                 weights, activations, cache and P in bf16 as the pages compute (logits of a
+                                 deep stack drift further from the exact result: see the dtype note) */
 } llama_config;
 
 typedef struct llama_model llama_model; /* opaque: weights, KV cache, lengths, workspace */
@@ -265,6 +271,15 @@ int llama_argmax_rows(const float* logits, int32_t* out, int32_t B, int32_t V, v
  * (device, dtype; fp16 rounds the fp32 draw to fp16 directly). */
 int llama_fill_normal(void* dst, int64_t n, uint64_t seed, uint64_t stream_id, float std, int32_t dtype,
                       void* stream);
+
+/* Failure-detection self test. Every spin-wait of the library's kernels (on an mbarrier, or on a
+ * counter other CTAs increment) is bounded: after its limit (2 s in the kernels) it latches
+ * LLAMA_ERR_DEVICE_TIMEOUT in the status word and the kernel returns, so a stuck wait never hangs
+ * the GPU and the context stays usable. This call runs one such wait that can never complete
+ * (kind 0: the first phase of an mbarrier nobody arrives on; kind 1: a device counter nobody
+ * increments) with the limit limit_ns (1 .. 10^10); llama_status() then returns
+ * LLAMA_ERR_DEVICE_TIMEOUT. Not part of the pages' method: it tests the library's failure handling. */
+int llama_wait_selftest(int32_t kind, uint64_t limit_ns, void* stream);
 
 /* Synchronizes `stream`, then returns and clears the status word of the stateless calls on the
  * current device (the first non-zero of theirs and llama_attention_decode_noalloc's). */

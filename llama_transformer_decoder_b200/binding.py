@@ -22,6 +22,7 @@ LLAMA_ERR_CUDA = -4
 LLAMA_ERR_DEVICE_TIMEOUT = -5
 LLAMA_ERR_DEVICE_BOUNDS = -6
 LLAMA_ERR_UNSUPPORTED = -7
+LLAMA_ERR_RANGE = -8
 LLAMA_F32 = 0
 LLAMA_BF16 = 1
 LLAMA_F16 = 2
@@ -39,7 +40,7 @@ class llama_config(ctypes.Structure):
                 ('multiple_of', ctypes.c_int32), ('ffn_dim_multiplier', ctypes.c_float),
                 ('norm_eps', ctypes.c_float), ('rope_theta', ctypes.c_float), ('max_batch', ctypes.c_int32),
                 ('max_seq', ctypes.c_int32), ('max_tokens', ctypes.c_int32), ('dtype', ctypes.c_int32),
-                ('kv_page_size', ctypes.c_int32), ('kv_pages', ctypes.c_int32)]
+                ('kv_page_size', ctypes.c_int32), ('kv_pages', ctypes.c_int32), ('act_dtype', ctypes.c_int32)]
 
 
 if not os.path.exists(LIB_PATH):
@@ -89,6 +90,7 @@ _SIGS = {
     'llama_argmax_rows': (ctypes.c_int, [_P, _P, _I32, _I32, _P]),
     'llama_fill_normal': (ctypes.c_int, [_P, _I64, _U64, _U64, _F, _I32, _P]),
     'llama_status': (ctypes.c_int, [_P]),
+    'llama_wait_selftest': (ctypes.c_int, [_I32, _U64, _P]),
     'llama_profile': (ctypes.c_int, [_P, ctypes.c_int]),
     'llama_profile_read': (ctypes.c_int, [_P, _P, _P, ctypes.c_int]),
     'llama_profile_kind_name': (ctypes.c_char_p, [ctypes.c_int]),
@@ -271,6 +273,10 @@ def llama_fill_normal(dst, n, seed, stream_id, std, dtype, stream=None):
 
 def llama_status(stream=None) -> int:
     return _lib.llama_status(_stream(stream))
+
+
+def llama_wait_selftest(kind, limit_ns, stream=None):
+    _check(_lib.llama_wait_selftest(int(kind), int(limit_ns), _stream(stream)), 'llama_wait_selftest')
 
 
 def llama_status_string(status: int) -> str:

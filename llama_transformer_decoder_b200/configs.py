@@ -20,4 +20,4 @@ def make_config(params: dict, *, dtype: int, max_batch: int, max_seq: int, max_t
                         multiple_of=p.get('multiple_of', 256), ffn_dim_multiplier=p.get('ffn_dim_multiplier', 0.0),
                         norm_eps=p['norm_eps'], rope_theta=p['rope_theta'], max_batch=max_batch, max_seq=max_seq,
                         max_tokens=max_tokens, dtype=dtype, kv_page_size=p.get('kv_page_size', 0),
-                        kv_pages=p.get('kv_pages', 0))
+                        kv_pages=p.get('kv_pages', 0), act_dtype=p.get('act_dtype', 0))

@@ -6,12 +6,11 @@
 // items, for short chunks; described above its definition).
 //
 // One CTA computes 128 queries of one head. Warp roles: warp 0 issues TMA
-// loads (Q once, then K and V tiles of 128 keys into a 2-stage ring), warp 1
-// allocates TMEM and issues tcgen05.mma, warps 2-9 run the softmax: query row
-// r belongs to two threads, one in warps 2-5 (keys 0-63 of each tile, output
-// columns 0-63) and one in warps 6-9 (keys 64-127, columns 64-127), which
-// exchange their row maxima through shared memory once per tile and their
-// partial row sums once at the end.
+// loads (Q once, then K and V tiles of 128 keys into 2-stage rings), warp 1
+// allocates TMEM and issues tcgen05.mma, warps 2-5 run the softmax: query row
+// r (TMEM lane r) belongs to one thread of the warp that may read that lane
+// quarter, which keeps the row's running maximum and sum in registers, so no
+// value is exchanged between threads inside the key loop.
 //
 //   S_j = Q K_j^T      -> TMEM (two 128-column buffers, so S_{j+1} is computed
 //                         while the softmax works on S_j)
@@ -47,8 +46,7 @@ constexpr int FA_STAGES = 2;
 constexpr int FA_OFF_Q = 0;
 constexpr int FA_OFF_K = FA_OFF_Q + FA_Q_BYTES;
 constexpr int FA_OFF_V = FA_OFF_K + FA_STAGES * FA_KV_BYTES;
-constexpr int FA_OFF_RED = FA_OFF_V + FA_STAGES * FA_KV_BYTES;  // row maxima [2 slots][2 halves][128], sums [2][128]
-constexpr int FA_OFF_BAR = FA_OFF_RED + 6 * 128 * 4;
+constexpr int FA_OFF_BAR = FA_OFF_V + FA_STAGES * FA_KV_BYTES;
 constexpr int FA_SMEM = FA_OFF_BAR + 256 + 1024;
 constexpr uint32_t FA_TMEM_O = 0, FA_TMEM_S = 128;   // S buffers at columns 128 and 256
 constexpr uint32_t FA_TMEM_P = 384;                   // P: 64 columns, keys 2c and 2c+1 in column c
@@ -72,7 +70,110 @@ __device__ __forceinline__ uint8_t* fa_align(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-constexpr int FA_THREADS = 320;
+constexpr int FA_THREADS = 192;
+
+// The softmax of one 128-key tile for the query row this thread owns: the
+// row's 128 scores of S buffer `s_tmem` (TMEM lane base in lane_off), keys
+// past qpos masked on diagonal tiles (kbase = the tile's first key), the
+// running maximum m_used raised only past +FA_RESCALE (first tile: set), the
+// 64 packed probabilities in pk and the tile's row sum returned. corr is the
+// factor O and l must be multiplied by (1 unless the maximum was raised).
+template <typename T>
+__device__ __forceinline__ float fa_tile_softmax(uint32_t s_tmem, bool ok, bool masked, int kbase, int qpos,
+                                                 float scale_log2, bool first, float& m_used, float& corr,
+                                                 uint32_t (&pk)[64]) {
+  float sv[128];
+  if (ok) {
+    uint32_t u0[32], u1[32], u2[32], u3[32];
+    tmem_ld32_nowait(s_tmem, u0);
+    tmem_ld32_nowait(s_tmem + 32, u1);
+    tmem_ld32_nowait(s_tmem + 64, u2);
+    tmem_ld32_nowait(s_tmem + 96, u3);
+    tmem_ld_wait();
+#pragma unroll
+    for (int x = 0; x < 32; ++x) {
+      sv[x] = __uint_as_float(u0[x]);
+      sv[32 + x] = __uint_as_float(u1[x]);
+      sv[64 + x] = __uint_as_float(u2[x]);
+      sv[96 + x] = __uint_as_float(u3[x]);
+    }
+  } else {
+#pragma unroll
+    for (int x = 0; x < 128; ++x) sv[x] = 0.f;
+  }
+  if (masked) {
+#pragma unroll
+    for (int x = 0; x < 128; ++x)
+      if (kbase + x > qpos) sv[x] = -INFINITY;
+  }
+  float mx8[8];
+#pragma unroll
+  for (int x = 0; x < 8; ++x) mx8[x] = sv[x];
+#pragma unroll
+  for (int x = 8; x < 128; ++x) mx8[x & 7] = fmaxf(mx8[x & 7], sv[x]);
+  const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
+  corr = 1.f;
+  if (first) {
+    m_used = mx;
+  } else if (mx > m_used + FA_RESCALE) {
+    corr = fast_exp2(m_used - mx);
+    m_used = mx;
+  }
+  float sum8[8];
+#pragma unroll
+  for (int x = 0; x < 8; ++x) sum8[x] = 0.f;
+#pragma unroll
+  for (int x = 0; x < 64; ++x) {
+    const float a = fast_exp2(fmaf(sv[2 * x], scale_log2, -m_used));
+    const float b = fast_exp2(fmaf(sv[2 * x + 1], scale_log2, -m_used));
+    sum8[x & 7] += a + b;
+    pk[x] = pack2<T>(a, b);
+  }
+  return ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+}
+
+// O *= corr for this thread's row (all 128 columns).
+__device__ __forceinline__ void fa_rescale_o(uint32_t o_tmem, float corr) {
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    float t[32];
+    tmem_ld32(o_tmem + c * 32, t);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) t[i] *= corr;
+    tmem_st32(o_tmem + c * 32, t);
+  }
+  tmem_st_wait();
+}
+
+// P of this thread's row into the 64 P columns.
+__device__ __forceinline__ void fa_store_p(uint32_t p_tmem, const uint32_t (&pk)[64]) {
+  tmem_st32_u(p_tmem, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+  tmem_st32_u(p_tmem + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+  tmem_st_wait();
+}
+
+// O / l of this thread's row (128 columns) to dst, 16-byte stores.
+template <typename T>
+__device__ __forceinline__ void fa_store_o(uint32_t o_tmem, bool ok, float inv, T* dst, bool valid) {
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    float t[32];
+    if (ok) tmem_ld32(o_tmem + c * 32, t);
+    else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) t[i] = 0.f;
+    }
+    if (valid) {
+      uint32_t w[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) w[i] = pack2<T>(t[2 * i] * inv, t[2 * i + 1] * inv);
+      uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    }
+  }
+}
 
 template <typename T>
 __global__ void __launch_bounds__(FA_THREADS, 1)
@@ -113,7 +214,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
     }
-    mbar_init(p_full, 256);
+    mbar_init(p_full, 128);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -208,121 +309,39 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     }
   } else if (warp >= 2) {
     const int quarter = warp & 3;                       // TMEM lanes this warp may read
-    const int half = (warp - 2) >> 2;                   // 0: keys / columns 0-63, 1: 64-127
     const int r = quarter * 32 + lane;                  // query row in the tile
     const int qpos = p0 + q0 + r;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t col0 = (uint32_t)half * 64;
-    float* red_max = reinterpret_cast<float*>(smem + FA_OFF_RED);       // [slot][half][row]
-    float* red_sum = red_max + 4 * 128;                                  // [half][row]
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kt; ++j) {
       const int st = j & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[st], (j >> 1) & 1, status)) && ok;
       tc_fence_after();
-      float sv[64];
-      if (ok) {
-        uint32_t t0[32], t1[32];
-        tmem_ld32_nowait(tmem + lane_off + FA_TMEM_S + (uint32_t)st * 128 + col0, t0);
-        tmem_ld32_nowait(tmem + lane_off + FA_TMEM_S + (uint32_t)st * 128 + col0 + 32, t1);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) { sv[i] = __uint_as_float(t0[i]); sv[32 + i] = __uint_as_float(t1[i]); }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) sv[i] = 0.f;
-      }
-      const int kbase = j * FA_BN + (int)col0;
-      // masked tiles: the last one or two of a causal row block
-      if (j * FA_BN + FA_BN - 1 > p0 + q0) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (kbase + i > qpos) sv[i] = -INFINITY;
-      }
-      float mx8[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) mx8[c] = sv[c];
-#pragma unroll
-      for (int i = 8; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
-      float mloc = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      red_max[(st * 2 + half) * 128 + r] = mloc;
-      named_bar_sync(1, 256);
-      // both threads of the row see the same maximum and take the same decisions
-      const float mx = fmaxf(mloc, red_max[(st * 2 + (half ^ 1)) * 128 + r]) * scale_log2;
-      float corr = 1.f;
-      bool rescale = false;
-      if (j == 0) {
-        m_used = mx;
-      } else if (mx > m_used + FA_RESCALE) {
-        corr = fast_exp2(m_used - mx);
-        m_used = mx;
-        rescale = true;
-      }
-      float sum8[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) sum8[c] = 0.f;
-      uint32_t pk[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float a = fast_exp2(fmaf(sv[2 * i], scale_log2, -m_used));
-        const float c2 = fast_exp2(fmaf(sv[2 * i + 1], scale_log2, -m_used));
-        sum8[i & 7] += a + c2;
-        pk[i] = pack2<T>(a, c2);
-      }
-      const float rowsum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      uint32_t pk[64];
+      float corr;
+      const float rowsum = fa_tile_softmax<T>(tmem + lane_off + FA_TMEM_S + (uint32_t)st * 128, ok,
+                                              j * FA_BN + FA_BN - 1 > p0 + q0, j * FA_BN, qpos, scale_log2, j == 0,
+                                              m_used, corr, pk);
       l = l * corr + rowsum;
       // P and O may be touched only once the previous P V product has finished
       if (j > 0) {
         ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, status)) && ok;
         tc_fence_after();
       }
-      if (__any_sync(0xffffffffu, rescale) && ok) {
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          float t[32];
-          tmem_ld32(tmem + lane_off + FA_TMEM_O + col0 + c * 32, t);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) t[i] *= corr;
-          tmem_st32(tmem + lane_off + FA_TMEM_O + col0 + c * 32, t);
-        }
-        tmem_st_wait();
-      }
-      // this thread's 64 keys: P columns 32*half .. 32*half+31 of its lane
-      tmem_st32_u(tmem + lane_off + FA_TMEM_P + col0 / 2, pk);
-      tmem_st_wait();
+      if (__any_sync(0xffffffffu, corr != 1.f) && ok) fa_rescale_o(tmem + lane_off + FA_TMEM_O, corr);
+      if (ok) fa_store_p(tmem + lane_off + FA_TMEM_P, pk);
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    // final: O / l to global memory, each thread its 64 columns
+    // final: O / l to global memory
     if (n_kt > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait(o_done, (n_kt - 1) & 1, status)) && ok;
       tc_fence_after();
     }
-    red_sum[half * 128 + r] = l;
-    named_bar_sync(1, 256);
-    const float ltot = l + red_sum[(half ^ 1) * 128 + r];
     const int qi = q0 + r;
-    const float inv = 1.f / ltot;
-    T* dst = o + ((size_t)b * S + (qi < S ? qi : 0)) * H * FA_D + (size_t)h * FA_D + col0;
-#pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
-      float t[32];
-      if (ok) tmem_ld32(tmem + lane_off + FA_TMEM_O + col0 + c * 32, t);
-      else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) t[i] = 0.f;
-      }
-      if (qi < S) {
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = pack2<T>(t[2 * i] * inv, t[2 * i + 1] * inv);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-      }
-    }
+    T* dst = o + ((size_t)b * S + (qi < S ? qi : 0)) * H * FA_D + (size_t)h * FA_D;
+    fa_store_o<T>(tmem + lane_off + FA_TMEM_O, ok, 1.f / l, dst, qi < S);
   }
   tc_fence_before();
   __syncthreads();
@@ -337,8 +356,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
 // sequence) items, so that the start of one item overlaps the end of the
 // previous one: Q is double-buffered and loaded while the previous item runs,
 // the K/V rings, the S buffers and the P/O barriers run on across items, and
-// four extra warps (10-13) move O / l to global memory while the softmax warps
-// already work on the next item's first tile. The next item's first P V
+// four extra warps (6-9) move O / l to global memory while the softmax warps
+// (2-5) already work on the next item's first tile. The next item's first P V
 // product waits only until those warps have read O out of TMEM.
 //
 // Items are taken in the longest-first order of the per-tile kernel, dealt
@@ -350,13 +369,13 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
 // wait is bounded; after a failed wait a role stops waiting (and issuing)
 // but walks its loops to the end, so the named barrier of the softmax warps
 // stays matched.
-constexpr int FP_THREADS = 448;
+constexpr int FP_THREADS = 320;
 constexpr int kPersistentMaxS = 4096;
 constexpr int FP_OFF_Q = 0;                                      // two Q buffers
 constexpr int FP_OFF_K = FP_OFF_Q + 2 * FA_Q_BYTES;
 constexpr int FP_OFF_V = FP_OFF_K + FA_STAGES * FA_KV_BYTES;
-constexpr int FP_OFF_RED = FP_OFF_V + FA_STAGES * FA_KV_BYTES;  // maxima [2][2][128], sums [2 items][2][128]
-constexpr int FP_OFF_BAR = FP_OFF_RED + 8 * 128 * 4;
+constexpr int FP_OFF_RED = FP_OFF_V + FA_STAGES * FA_KV_BYTES;  // row sums [2 item slots][128]
+constexpr int FP_OFF_BAR = FP_OFF_RED + 2 * 128 * 4;
 constexpr int FP_SMEM = FP_OFF_BAR + 256 + 1024;
 
 __device__ __forceinline__ int fp_item(int c, int G, int i) { return i * G + ((i & 1) ? G - 1 - c : c); }
@@ -397,9 +416,9 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
   uint64_t* v_full = bars + 8;     // [2]
   uint64_t* v_empty = bars + 10;   // [2]
   uint64_t* s_full = bars + 12;    // [2]
-  uint64_t* p_full = bars + 14;    // softmax threads stored P (256 arrivals)
+  uint64_t* p_full = bars + 14;    // softmax threads stored P (128 arrivals)
   uint64_t* o_done = bars + 15;    // O += P V finished
-  uint64_t* l_ready = bars + 16;   // softmax threads stored the item's row sums (256 arrivals)
+  uint64_t* l_ready = bars + 16;   // softmax threads stored the item's row sums (128 arrivals)
   uint64_t* o_free = bars + 17;    // the O warps have read O out of TMEM (128 arrivals)
   uint64_t* drain = bars + 18;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
@@ -416,9 +435,9 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
       mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
     }
-    mbar_init(p_full, 256);
+    mbar_init(p_full, 128);
     mbar_init(o_done, 1);
-    mbar_init(l_ready, 256);
+    mbar_init(l_ready, 128);
     mbar_init(o_free, 128);
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -429,8 +448,7 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_wait();
-  float* red_max = reinterpret_cast<float*>(smem + FP_OFF_RED);   // [slot][half][row]
-  float* red_sum = red_max + 4 * 128;                              // [item slot][half][row]
+  float* red_sum = reinterpret_cast<float*>(smem + FP_OFF_RED);   // [item slot][row]
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmQ);
@@ -531,12 +549,10 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
       umma_commit(drain);
       mbar_wait(drain, 0, status);
     }
-  } else if (warp >= 2 && warp < 10) {
+  } else if (warp >= 2 && warp < 6) {
     const int quarter = warp & 3;                       // TMEM lanes this warp may read
-    const int half = (warp - 2) >> 2;                   // 0: keys / columns 0-63, 1: 64-127
     const int r = quarter * 32 + lane;                  // query row in the tile
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t col0 = (uint32_t)half * 64;
     bool ok = true;
     int t = 0;
     for (int i = 0;; ++i) {
@@ -549,87 +565,28 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
         const int st = t & 1;
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s_full[st], (t >> 1) & 1, status));
         tc_fence_after();
-        float sv[64];
-        if (ok) {
-          uint32_t t0[32], t1[32];
-          tmem_ld32_nowait(tmem + lane_off + FA_TMEM_S + (uint32_t)st * 128 + col0, t0);
-          tmem_ld32_nowait(tmem + lane_off + FA_TMEM_S + (uint32_t)st * 128 + col0 + 32, t1);
-          tmem_ld_wait();
-#pragma unroll
-          for (int x = 0; x < 32; ++x) { sv[x] = __uint_as_float(t0[x]); sv[32 + x] = __uint_as_float(t1[x]); }
-        } else {
-#pragma unroll
-          for (int x = 0; x < 64; ++x) sv[x] = 0.f;
-        }
-        const int kbase = j * FA_BN + (int)col0;
-        if (j * FA_BN + FA_BN - 1 > it.p0 + it.q0) {  // masked tiles: the last one or two of a causal row block
-#pragma unroll
-          for (int x = 0; x < 64; ++x)
-            if (kbase + x > qpos) sv[x] = -INFINITY;
-        }
-        float mx8[8];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) mx8[x] = sv[x];
-#pragma unroll
-        for (int x = 8; x < 64; ++x) mx8[x & 7] = fmaxf(mx8[x & 7], sv[x]);
-        const float mloc = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        red_max[(st * 2 + half) * 128 + r] = mloc;
-        named_bar_sync(1, 256);
-        // both threads of the row see the same maximum and take the same decisions
-        const float mx = fmaxf(mloc, red_max[(st * 2 + (half ^ 1)) * 128 + r]) * scale_log2;
-        float corr = 1.f;
-        bool rescale = false;
-        if (j == 0) {
-          m_used = mx;
-        } else if (mx > m_used + FA_RESCALE) {
-          corr = fast_exp2(m_used - mx);
-          m_used = mx;
-          rescale = true;
-        }
-        float sum8[8];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) sum8[x] = 0.f;
-        uint32_t pk[32];
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const float a = fast_exp2(fmaf(sv[2 * x], scale_log2, -m_used));
-          const float c2 = fast_exp2(fmaf(sv[2 * x + 1], scale_log2, -m_used));
-          sum8[x & 7] += a + c2;
-          pk[x] = pack2<T>(a, c2);
-        }
-        const float rowsum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+        uint32_t pk[64];
+        float corr;
+        const float rowsum = fa_tile_softmax<T>(tmem + lane_off + FA_TMEM_S + (uint32_t)st * 128, ok,
+                                                j * FA_BN + FA_BN - 1 > it.p0 + it.q0, j * FA_BN, qpos, scale_log2,
+                                                j == 0, m_used, corr, pk);
         l = l * corr + rowsum;
         // P (and O) may be touched only once the previous P V product has finished
         if (t > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (t - 1) & 1, status));
         tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale) && ok) {
-#pragma unroll 1
-          for (int cc = 0; cc < 2; ++cc) {
-            float v[32];
-            tmem_ld32(tmem + lane_off + FA_TMEM_O + col0 + cc * 32, v);
-#pragma unroll
-            for (int x = 0; x < 32; ++x) v[x] *= corr;
-            tmem_st32(tmem + lane_off + FA_TMEM_O + col0 + cc * 32, v);
-          }
-          tmem_st_wait();
-        }
-        // this thread's 64 keys: P columns 32*half .. 32*half+31 of its lane
-        if (ok) {
-          tmem_st32_u(tmem + lane_off + FA_TMEM_P + col0 / 2, pk);
-          tmem_st_wait();
-        }
+        if (__any_sync(0xffffffffu, corr != 1.f) && ok) fa_rescale_o(tmem + lane_off + FA_TMEM_O, corr);
+        if (ok) fa_store_p(tmem + lane_off + FA_TMEM_P, pk);
         tc_fence_before();
         mbar_arrive(p_full);
       }
       // hand the row sums to the O warps; slot i&1 was last read for item
       // i-2, and those warps have finished item i-1 once o_free says so
       if (i > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(o_free, (i - 1) & 1, status));
-      red_sum[((i & 1) * 2 + half) * 128 + r] = l;
+      red_sum[(i & 1) * 128 + r] = l;
       mbar_arrive(l_ready);
     }
-  } else if (warp >= 10) {
-    const int quarter = warp & 3;                       // warps 10-13: lanes 64-95, 96-127, 0-31, 32-63
+  } else if (warp >= 6) {
+    const int quarter = warp & 3;                       // warps 6-9: lanes 64-95, 96-127, 0-31, 32-63
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     bool ok = true;
@@ -642,27 +599,10 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(l_ready, i & 1, status));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (t - 1) & 1, status));
       tc_fence_after();
-      const float ltot = red_sum[((i & 1) * 2) * 128 + r] + red_sum[((i & 1) * 2 + 1) * 128 + r];
-      const float inv = 1.f / ltot;
+      const float inv = 1.f / red_sum[(i & 1) * 128 + r];
       const int qi = it.q0 + r;
       T* dst = o + ((size_t)it.b * S + (qi < S ? qi : 0)) * H * FA_D + (size_t)it.h * FA_D;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        float v[32];
-        if (ok) tmem_ld32(tmem + lane_off + FA_TMEM_O + cc * 32, v);
-        else {
-#pragma unroll
-          for (int x = 0; x < 32; ++x) v[x] = 0.f;
-        }
-        if (qi < S) {
-          uint32_t pw[16];
-#pragma unroll
-          for (int x = 0; x < 16; ++x) pw[x] = pack2<T>(v[2 * x] * inv, v[2 * x + 1] * inv);
-          uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-          for (int x = 0; x < 4; ++x) d4[x] = make_uint4(pw[4 * x], pw[4 * x + 1], pw[4 * x + 2], pw[4 * x + 3]);
-        }
-      }
+      fa_store_o<T>(tmem + lane_off + FA_TMEM_O, ok, inv, dst, qi < S);
       tc_fence_before();
       mbar_arrive(o_free);
     }

@@ -113,13 +113,14 @@ __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_
 }
 
 // Bounded wait: returns false (and latches a timeout) when the phase with the
-// given parity has not completed within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+// given parity has not completed within limit_ns (kWaitLimitNs by default).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((it & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) {
       set_status(status, LLAMA_ERR_DEVICE_TIMEOUT);
       return false;
     }
@@ -147,13 +148,14 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ __forceinline__ bool counter_wait_geq(const int* p, int target, int* status) {
+__device__ __forceinline__ bool counter_wait_geq(const int* p, int target, int* status,
+                                                 uint64_t limit_ns = kWaitLimitNs) {
   if (ld_acquire_gpu(p) >= target) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
     __nanosleep(64);
     if (ld_acquire_gpu(p) >= target) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       set_status(status, LLAMA_ERR_DEVICE_TIMEOUT);
       return false;
     }
@@ -444,6 +446,34 @@ template <>
 __device__ __forceinline__ uint32_t pack2<f16>(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Range checks of 16-bit activations. A value that rounds to +-inf in the
+// 16-bit type (fp16 overflows above 65504), or is NaN, cannot be represented;
+// the kernels that round activations latch LLAMA_ERR_RANGE when they meet one.
+// fp32 outputs are not checked.
+template <typename T>
+__device__ __forceinline__ bool nonfinite16(float v) {
+  return !isfinite(to_f<T>(from_f<T>(v)));
+}
+template <>
+__device__ __forceinline__ bool nonfinite16<float>(float) {
+  return false;
+}
+// Either half of a packed pair has an all-ones exponent (inf or NaN).
+template <typename T>
+__device__ __forceinline__ bool packed_nonfinite(uint32_t w);
+template <>
+__device__ __forceinline__ bool packed_nonfinite<f16>(uint32_t w) {
+  return (w & 0x7c00u) == 0x7c00u || (w & 0x7c000000u) == 0x7c000000u;
+}
+template <>
+__device__ __forceinline__ bool packed_nonfinite<bf16>(uint32_t w) {
+  return (w & 0x7f80u) == 0x7f80u || (w & 0x7f800000u) == 0x7f800000u;
+}
+template <>
+__device__ __forceinline__ bool packed_nonfinite<float>(uint32_t) {
+  return false;
 }
 
 // tcgen05 operand format code of a 16-bit element type (kind::f16).

@@ -43,7 +43,8 @@ __device__ __forceinline__ void store4(T* p, float a, float b, float c, float d)
 // are written with 8- or 16-byte stores.
 template <typename T>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ g,
-                                                      T* __restrict__ y, int D, float eps, int last_of_S) {
+                                                      T* __restrict__ y, int D, float eps, int last_of_S,
+                                                      int* status) {
   pdl_trigger();
   pdl_wait();
   const int r = blockIdx.x;
@@ -74,18 +75,26 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
 #pragma unroll
   for (int w = 0; w < 8; ++w) tot += red[w];
   const float inv = rsqrtf(tot / (float)D + eps);
+  bool bad = false;
   if (vec) {
 #pragma unroll
     for (int k = 0; k < NV; ++k) {
       const int i = (threadIdx.x + k * 256) * 4;
       if (i < D) {
         const float4 w = __ldg(reinterpret_cast<const float4*>(g + i));
-        store4<T>(yr + i, v[k].x * inv * w.x, v[k].y * inv * w.y, v[k].z * inv * w.z, v[k].w * inv * w.w);
+        const float4 o = make_float4(v[k].x * inv * w.x, v[k].y * inv * w.y, v[k].z * inv * w.z, v[k].w * inv * w.w);
+        bad |= nonfinite16<T>(o.x) | nonfinite16<T>(o.y) | nonfinite16<T>(o.z) | nonfinite16<T>(o.w);
+        store4<T>(yr + i, o.x, o.y, o.z, o.w);
       }
     }
   } else {
-    for (int i = threadIdx.x; i < D; i += 256) yr[i] = from_f<T>(xr[i] * inv * g[i]);
+    for (int i = threadIdx.x; i < D; i += 256) {
+      const float o = xr[i] * inv * g[i];
+      bad |= nonfinite16<T>(o);
+      yr[i] = from_f<T>(o);
+    }
   }
+  if (bad) set_status(status, LLAMA_ERR_RANGE);
 }
 
 // Inputs of a GEMM with the RMSNorm folded in: y = x * g (16-bit, not yet
@@ -93,7 +102,8 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
 // its ss_n partial sums (the other slots 0).
 template <typename T>
 __global__ void __launch_bounds__(256) norm_prep_kernel(const float* __restrict__ x, const float* __restrict__ g,
-                                                        T* __restrict__ y, float* __restrict__ ss, int D, int ss_n) {
+                                                        T* __restrict__ y, float* __restrict__ ss, int D, int ss_n,
+                                                        int* status) {
   pdl_trigger();
   pdl_wait();
   const int r = blockIdx.x;
@@ -101,11 +111,14 @@ __global__ void __launch_bounds__(256) norm_prep_kernel(const float* __restrict_
   T* yr = y + (size_t)r * D;
   __shared__ float red[8];
   float acc = 0.f;
+  bool bad = false;
   for (int i = threadIdx.x; i < D; i += 256) {
     const float v = xr[i];
     acc += v * v;
+    bad |= nonfinite16<T>(v * g[i]);
     yr[i] = from_f<T>(v * g[i]);
   }
+  if (bad) set_status(status, LLAMA_ERR_RANGE);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
@@ -278,28 +291,32 @@ int launch_embed(const int32_t* tokens, int M, const void* table, int V, int D, 
 }
 
 int launch_rmsnorm(const float* x, const float* g, void* y, int rows, int D, float eps, int last_of_S, int dtype,
-                   cudaStream_t st) {
+                   cudaStream_t st, int* status) {
   if (rows <= 0) return LLAMA_OK;
   cudaError_t err;
   if (dtype == LLAMA_F16)
-    err = launch_k(rmsnorm_kernel<f16>, dim3(rows), dim3(256), 0, st, x, g, static_cast<f16*>(y), D, eps, last_of_S);
+    err = launch_k(rmsnorm_kernel<f16>, dim3(rows), dim3(256), 0, st, x, g, static_cast<f16*>(y), D, eps, last_of_S,
+                   status);
   else if (dtype == LLAMA_BF16)
-    err = launch_k(rmsnorm_kernel<bf16>, dim3(rows), dim3(256), 0, st, x, g, static_cast<bf16*>(y), D, eps, last_of_S);
+    err = launch_k(rmsnorm_kernel<bf16>, dim3(rows), dim3(256), 0, st, x, g, static_cast<bf16*>(y), D, eps,
+                   last_of_S, status);
   else
     err = launch_k(rmsnorm_kernel<float>, dim3(rows), dim3(256), 0, st, x, g, static_cast<float*>(y), D, eps,
-                   last_of_S);
+                   last_of_S, status);
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
 int launch_norm_prep(const float* x, const float* g, void* y, float* ss, int rows, int D, int ss_n, int dtype,
-                     cudaStream_t st) {
+                     cudaStream_t st, int* status) {
   if (rows <= 0) return LLAMA_OK;
   if (ss_n > 256) return LLAMA_ERR_INVALID_ARG;
   cudaError_t err;
   if (dtype == LLAMA_F16)
-    err = launch_k(norm_prep_kernel<f16>, dim3(rows), dim3(256), 0, st, x, g, static_cast<f16*>(y), ss, D, ss_n);
+    err = launch_k(norm_prep_kernel<f16>, dim3(rows), dim3(256), 0, st, x, g, static_cast<f16*>(y), ss, D, ss_n,
+                   status);
   else if (dtype == LLAMA_BF16)
-    err = launch_k(norm_prep_kernel<bf16>, dim3(rows), dim3(256), 0, st, x, g, static_cast<bf16*>(y), ss, D, ss_n);
+    err = launch_k(norm_prep_kernel<bf16>, dim3(rows), dim3(256), 0, st, x, g, static_cast<bf16*>(y), ss, D, ss_n,
+                   status);
   else
     return LLAMA_ERR_INVALID_ARG;
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
@@ -428,6 +445,34 @@ int launch_kv_scatter(void* dst, int dst_elt, const KvLayout& L, int B, int Hk, 
   else if (dst_elt == LLAMA_F32 && src_elt == LLAMA_F32) LLAMA_SCATTER(float, float);
   else return LLAMA_ERR_INVALID_ARG;
 #undef LLAMA_SCATTER
+  return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+}
+
+namespace {
+// A counter nothing ever increments (the target of the counter self test).
+__device__ int g_never_set = 0;
+
+// Failure-detection self test: one thread waits for something that never
+// happens (kind 0: the first phase of an mbarrier nobody arrives on; kind 1:
+// a device counter nobody increments), through the same bounded waits as the
+// kernels use, with the given limit. The wait gives up, latches
+// LLAMA_ERR_DEVICE_TIMEOUT and the kernel returns.
+__global__ void wait_selftest_kernel(int kind, uint64_t limit_ns, int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  if (kind == 0) mbar_wait(&bar, 0, status, limit_ns);
+  else counter_wait_geq(&g_never_set, 1, status, limit_ns);
+}
+}  // namespace
+
+int launch_wait_selftest(int kind, uint64_t limit_ns, int* status, cudaStream_t st) {
+  count_launches(1);
+  wait_selftest_kernel<<<1, 32, 0, st>>>(kind, limit_ns, status);
   return cudaGetLastError() == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 

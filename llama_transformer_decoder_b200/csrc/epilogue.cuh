@@ -42,6 +42,9 @@ struct EpiArgs {
   const float* ss_in;
   int ss_n;
   float norm_inv_d, norm_eps;
+  // Status word for LLAMA_ERR_RANGE: a 16-bit output (q/k/v, the SwiGLU
+  // product, y = x * g) that is not finite after rounding (nullptr: unchecked).
+  int* status;
 };
 
 // r of row m from its partial sums of squares (added in a fixed order).
@@ -71,6 +74,7 @@ __device__ __forceinline__ void qkv_store(const EpiArgs& e, int m, int n, float 
     const float2 cs = e.rope[(size_t)pos * (e.d >> 1) + i];
     r = (n & 1) ? (partner * cs.y + v * cs.x) : (v * cs.x - partner * cs.y);
   }
+  if (nonfinite16<T>(r)) set_status(e.status, LLAMA_ERR_RANGE);
   if (n < hd) {
     const int h = n / e.d, dd = n - h * e.d;
     static_cast<T*>(e.q)[(((size_t)b * e.H + h) * e.S + s) * e.d + dd] = from_f<T>(r);
@@ -93,7 +97,11 @@ __device__ __forceinline__ void epi_elem(const EpiArgs& e, int m, int n, float v
     float* p = e.out + (size_t)m * e.ldo + n;
     *p = *p + v;
   } else if (KIND == EPI_SWIGLU) {
-    if ((n & 1) == 0) static_cast<T*>(e.g)[(size_t)m * e.ldg + (n >> 1)] = from_f<T>(silu_f(v) * partner);
+    if ((n & 1) == 0) {
+      const float r = silu_f(v) * partner;
+      if (nonfinite16<T>(r)) set_status(e.status, LLAMA_ERR_RANGE);
+      static_cast<T*>(e.g)[(size_t)m * e.ldg + (n >> 1)] = from_f<T>(r);
+    }
   } else {
     qkv_store<T>(e, m, n, v, partner);
   }
@@ -108,6 +116,7 @@ __device__ __forceinline__ float epi_row32(const EpiArgs& e, int m, int n0, cons
   if (m >= e.M) return 0.f;
   const bool full = (n0 + 32 <= e.N);
   float ssq = 0.f;
+  bool bad = false;   // a 16-bit output of this chunk is not finite
   if (KIND == EPI_STORE_F32 || KIND == EPI_RESIDUAL) {
     const bool norm_out = KIND == EPI_RESIDUAL && e.g_next != nullptr;
     float* p = e.out + (size_t)m * e.ldo + n0;
@@ -137,6 +146,10 @@ __device__ __forceinline__ float epi_row32(const EpiArgs& e, int m, int n0, cons
         uint4* y4 = reinterpret_cast<uint4*>(yp);
 #pragma unroll
         for (int j = 0; j < 4; ++j) y4[j] = make_uint4(yw[4 * j], yw[4 * j + 1], yw[4 * j + 2], yw[4 * j + 3]);
+        if (sizeof(T) == 2) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) bad |= packed_nonfinite<T>(yw[j]);
+        }
       }
     } else {
 #pragma unroll
@@ -146,7 +159,9 @@ __device__ __forceinline__ float epi_row32(const EpiArgs& e, int m, int n0, cons
           else p[j] = v[j];
           if (norm_out) {
             ssq += p[j] * p[j];
-            yp[j] = from_f<T>(p[j] * e.g_next[n0 + j]);
+            const float y = p[j] * e.g_next[n0 + j];
+            bad |= nonfinite16<T>(y);
+            yp[j] = from_f<T>(y);
           }
         }
       }
@@ -161,10 +176,16 @@ __device__ __forceinline__ float epi_row32(const EpiArgs& e, int m, int n0, cons
       uint4* p4 = reinterpret_cast<uint4*>(p);
       p4[0] = make_uint4(w[0], w[1], w[2], w[3]);
       p4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) bad |= packed_nonfinite<T>(w[j]);
     } else {
 #pragma unroll
       for (int j = 0; j < 16; ++j)
-        if (n0 + 2 * j + 1 < e.N) p[j] = from_f<T>(silu_f(rs * v[2 * j]) * (rs * v[2 * j + 1]));
+        if (n0 + 2 * j + 1 < e.N) {
+          const float r = silu_f(rs * v[2 * j]) * (rs * v[2 * j + 1]);
+          bad |= nonfinite16<T>(r);
+          p[j] = from_f<T>(r);
+        }
     }
   } else {  // QKV_ROPE: a 32-column chunk never straddles a head when d % 32 == 0
     if (!full || (e.d & 31) != 0 || sizeof(T) != 2) {
@@ -209,7 +230,10 @@ __device__ __forceinline__ float epi_row32(const EpiArgs& e, int m, int n0, cons
     uint4* p4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
     for (int j = 0; j < 4; ++j) p4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) bad |= packed_nonfinite<T>(w[j]);
   }
+  if (bad) set_status(e.status, LLAMA_ERR_RANGE);
   return ssq;
 }
 

@@ -79,13 +79,14 @@ int gemm_f32(const float* A, int M, int K, int lda, const float* W, int N, int l
 int launch_embed(const int32_t* tokens, int M, const void* table, int V, int D, int dtype, float* x, int* status,
                  cudaStream_t st);
 // y[r] = rmsnorm(x[row(r)]) * g; row(r) = r, or (r+1)*S-1 when last_of_S > 0.
+// 16-bit outputs that are not finite latch LLAMA_ERR_RANGE in *status (if given).
 int launch_rmsnorm(const float* x, const float* g, void* y, int rows, int D, float eps, int last_of_S, int dtype,
-                   cudaStream_t st);
+                   cudaStream_t st, int* status = nullptr);
 int launch_argmax(const float* logits, int32_t* out, int B, int V, cudaStream_t st);
 // y = x * g (16-bit) and ss[r*ss_n + 0] = sum of x[r]^2 (other slots 0): the
 // inputs of a GEMM that applies the RMSNorm in its epilogue.
 int launch_norm_prep(const float* x, const float* g, void* y, float* ss, int rows, int D, int ss_n, int dtype,
-                     cudaStream_t st);
+                     cudaStream_t st, int* status = nullptr);
 int launch_add_lengths(int32_t* len, int B, int add, cudaStream_t st);
 
 // Attention. q [B][H][S][d]; K/V cache [B][Hk][Smax][d] (this layer);
@@ -130,6 +131,9 @@ int launch_fill_normal(void* dst, const FillLayout& L, uint64_t seed, uint64_t s
 int launch_convert_2d(void* dst, int64_t dpitch, int dst_elt, const void* src, int64_t spitch, int src_elt,
                       int64_t rows, int64_t cols, cudaStream_t st);
 int launch_fill_const(float* dst, int64_t n, float v, cudaStream_t st);
+// One kernel whose bounded wait can never complete (kind 0: mbarrier, 1:
+// device counter); it gives up after limit_ns and latches a timeout.
+int launch_wait_selftest(int kind, uint64_t limit_ns, int* status, cudaStream_t st);
 // N(0, std^2) draws of stream `stream_id` in the logical order [B][Hk][c][d]
 // (the cache generator's order), written through a cache layout.
 int launch_fill_kv(void* dst, const KvLayout& L, int B, int Hk, int c, int d, uint64_t seed, uint64_t stream_id,

@@ -62,10 +62,11 @@ struct llama_model {
   int dev = 0;
   int d = 0, F = 0, qkv_n = 0, Mmax = 0;
   size_t esz = 2;
-  // Element type of weights, activations and cache on the device. A bf16
-  // model keeps its bf16 weight values in fp16 storage and computes with fp16
-  // activations: fp16 has 3 more mantissa bits, which holds the logits of a
-  // 32-layer stack within 2e-2 of the exact result where bf16 activations do not.
+  // Element type of weights, activations and cache on the device. By default
+  // a bf16 model keeps its bf16 weight values in fp16 storage and computes with
+  // fp16 activations: fp16 has 3 more mantissa bits, which holds the logits of
+  // a 32-layer stack within 2e-2 of the exact result where bf16 activations do
+  // not. act_dtype = LLAMA_BF16 keeps everything in bf16 instead.
   int adt = LLAMA_F16;
   // weights
   void* wbase = nullptr;
@@ -169,6 +170,10 @@ int resolve(const llama_config* in, llama_config* c) {
   } else {
     c->kv_pages = 0;
   }
+  if (c->act_dtype != 0 && c->act_dtype != LLAMA_F16 && c->act_dtype != LLAMA_BF16) return LLAMA_ERR_INVALID_ARG;
+  if (c->act_dtype == LLAMA_BF16 && c->dtype != LLAMA_BF16) return LLAMA_ERR_UNSUPPORTED;
+  if (c->act_dtype == LLAMA_F16 && c->dtype == LLAMA_F32) return LLAMA_ERR_UNSUPPORTED;
+  if (c->dtype != LLAMA_F32 && c->act_dtype == 0) c->act_dtype = LLAMA_F16;
   if (c->max_tokens <= 0) {
     const int64_t mt = (int64_t)c->max_batch * c->max_seq;
     c->max_tokens = (int32_t)std::min<int64_t>(mt, 16384);
@@ -319,11 +324,12 @@ int gemm(llama_model* m, const void* A, int M, int K, const void* W, int N, int 
                   st);
 }
 
-EpiArgs epi_base(int M, int N) {
+EpiArgs epi_base(int M, int N, int* status = nullptr) {
   EpiArgs e;
   memset(&e, 0, sizeof(e));
   e.M = M;
   e.N = N;
+  e.status = status;
   return e;
 }
 
@@ -345,11 +351,11 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
   if (fuse) {
     if (!m->norm_ready) {
       mark(m, K_RMSNORM, st);
-      RC(launch_norm_prep(m->x, w.attn_norm, m->xn, m->ss, M, D, ss_n, m->adt, st));
+      RC(launch_norm_prep(m->x, w.attn_norm, m->xn, m->ss, M, D, ss_n, m->adt, st, m->d_status));
     }
   } else {
     mark(m, K_RMSNORM, st);
-    RC(launch_rmsnorm(m->x, w.attn_norm, m->xn, M, D, c.norm_eps, 0, m->adt, st));
+    RC(launch_rmsnorm(m->x, w.attn_norm, m->xn, M, D, c.norm_eps, 0, m->adt, st, m->d_status));
   }
   m->norm_ready = false;
   auto norm_in = [&](EpiArgs& a) {
@@ -366,7 +372,7 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
     a.ss_out = m->ss;
     a.ss_n = ss_n;
   };
-  EpiArgs e = epi_base(M, m->qkv_n);
+  EpiArgs e = epi_base(M, m->qkv_n, m->d_status);
   norm_in(e);
   e.q = m->q;
   e.kc = kc;
@@ -392,7 +398,7 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
     RC(attention_prefill(m->q, kc, vc, m->attn, m->d_len, B, S, H, Hk, d, c.max_seq, m->adt, m->d_status, st,
                          e.kv_table, m->max_pages, m->n_pages));
   }
-  EpiArgs r = epi_base(M, D);
+  EpiArgs r = epi_base(M, D, m->d_status);
   r.out = m->x;
   r.ldo = D;
   norm_out(r, w.ffn_norm);
@@ -400,15 +406,15 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
   RC(gemm(m, m->attn, M, H * d, w.wo, D, EPI_RESIDUAL, r, st));
   if (!fuse) {
     mark(m, K_RMSNORM, st);
-    RC(launch_rmsnorm(m->x, w.ffn_norm, m->xn, M, D, c.norm_eps, 0, m->adt, st));
+    RC(launch_rmsnorm(m->x, w.ffn_norm, m->xn, M, D, c.norm_eps, 0, m->adt, st, m->d_status));
   }
-  EpiArgs sg = epi_base(M, 2 * m->F);
+  EpiArgs sg = epi_base(M, 2 * m->F, m->d_status);
   sg.g = m->g;
   sg.ldg = m->F;
   norm_in(sg);
   mark(m, K_GEMM_W13, st);
   RC(gemm(m, m->xn, M, D, w.w13, 2 * m->F, EPI_SWIGLU, sg, st));
-  EpiArgs r2 = epi_base(M, D);
+  EpiArgs r2 = epi_base(M, D, m->d_status);
   r2.out = m->x;
   r2.ldo = D;
   if (l + 1 < c.n_layers) {   // the next layer's attention norm (the final norm takes the last rows only)
@@ -424,8 +430,8 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
 int run_head(llama_model* m, int B, int S, cudaStream_t st) {
   const llama_config& c = m->cfg;
   mark(m, K_RMSNORM, st);
-  RC(launch_rmsnorm(m->x, m->norm_w, m->xn, B, c.dim, c.norm_eps, S, m->adt, st));
-  EpiArgs e = epi_base(B, c.vocab_size);
+  RC(launch_rmsnorm(m->x, m->norm_w, m->xn, B, c.dim, c.norm_eps, S, m->adt, st, m->d_status));
+  EpiArgs e = epi_base(B, c.vocab_size, m->d_status);
   e.out = m->logits;
   e.ldo = c.vocab_size;
   mark(m, K_GEMM_LMHEAD, st);
@@ -572,6 +578,7 @@ const char* llama_status_string(int status) {
     case LLAMA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
     case LLAMA_ERR_DEVICE_BOUNDS: return "device-side index out of range";
     case LLAMA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LLAMA_ERR_RANGE: return "16-bit activation out of range (not finite after rounding)";
   }
   return "unknown status";
 }
@@ -586,7 +593,7 @@ int llama_create(const llama_config* cfg, llama_model** out) {
   m->cfg = c;
   cudaGetDevice(&m->dev);
   m->esz = c.dtype == LLAMA_F32 ? 4 : 2;
-  m->adt = c.dtype == LLAMA_F32 ? LLAMA_F32 : LLAMA_F16;
+  m->adt = c.dtype == LLAMA_F32 ? LLAMA_F32 : c.act_dtype;
   m->d = c.dim / c.n_heads;
   m->F = c.ffn_hidden;
   m->qkv_n = (c.n_heads + 2 * c.n_kv_heads) * m->d;
@@ -754,7 +761,7 @@ static int copy_weight(llama_model* m, const char* name, void* host_or_dev, size
   if (nbytes != row_bytes * (size_t)p.rows) return LLAMA_ERR_SHAPE;
   const size_t model_pitch = row_bytes * p.row_mult;
   cudaStream_t st = S_(stream);
-  if (m->cfg.dtype == LLAMA_BF16 && !p.is_norm) {
+  if (m->cfg.dtype == LLAMA_BF16 && m->adt == LLAMA_F16 && !p.is_norm) {
     // bf16 in the caller's buffer, fp16 in the model: convert on the device.
     void* dev = host_or_dev;
     if (!on_device) {
@@ -1106,13 +1113,23 @@ int llama_rmsnorm(const float* x, const float* g, void* y, int32_t M, int32_t D,
   if (!x || !g || !y) return LLAMA_ERR_INVALID_ARG;
   if (M <= 0 || D <= 0) return LLAMA_ERR_SHAPE;
   if (dtype != LLAMA_F32 && dtype != LLAMA_BF16 && dtype != LLAMA_F16) return LLAMA_ERR_INVALID_ARG;
-  return launch_rmsnorm(x, g, y, M, D, eps, 0, dtype, S_(stream));
+  DevCtx* c = dev_ctx();
+  if (!c) return LLAMA_ERR_OOM;
+  return launch_rmsnorm(x, g, y, M, D, eps, 0, dtype, S_(stream), c->status);
 }
 
 int llama_argmax_rows(const float* logits, int32_t* out, int32_t B, int32_t V, void* stream) {
   if (!logits || !out) return LLAMA_ERR_INVALID_ARG;
   if (B <= 0 || V <= 0) return LLAMA_ERR_SHAPE;
   return launch_argmax(logits, out, B, V, S_(stream));
+}
+
+int llama_wait_selftest(int32_t kind, uint64_t limit_ns, void* stream) {
+  if (kind != 0 && kind != 1) return LLAMA_ERR_INVALID_ARG;
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return LLAMA_ERR_INVALID_ARG;
+  DevCtx* c = dev_ctx();
+  if (!c) return LLAMA_ERR_OOM;
+  return launch_wait_selftest(kind, limit_ns, c->status, S_(stream));
 }
 
 int llama_fill_normal(void* dst, int64_t n, uint64_t seed, uint64_t stream_id, float std, int32_t dtype,

@@ -4,13 +4,16 @@
   last-token logits of sequences 0 and 7 against the float32 oracle (the
   sequences are independent, so checking two of them is exact for those two);
   B = 1 on the same tokens must agree with sequence 0 of the batch.
-* Batch-32 decode over a 4096-token cache of N(0,1) K/V entries, 128 greedy
-  steps replayed from a CUDA graph on a stream: sequences 0 and 31 are
-  teacher-forced through the oracle (one causal pass over the tokens the GPU
-  chose, after the same cache).
+* Batch-32 decode over a 4096-token cache of N(0,1) K/V entries, 128 steps
+  replayed from a CUDA graph on a stream. Every step consumes seeded token
+  ids (the same ones on both sides, so nothing the GPU computed enters the
+  oracle); sequences 0 and 31 are checked against one causal oracle pass over
+  their 128 tokens after the same cache (row i of that pass is decode step i).
 
-Tolerances: rel-L2 <= 2e-2 on logits; the GPU's greedy token must be the
-oracle's argmax or within the observed logit error of its maximum.
+Tolerances: rel-L2 <= 2e-2 on every checked logits row. Every step also
+yields a greedy decision (the GPU's argmax of its logits, the oracle's of
+its own); the last test reports strict top-1 agreement over all of them
+(2 prefill + 2 x 128 decode) and asserts it (see that test for the bound).
 The oracle runs in float32 here (its float64 twin agrees to ~1e-6, far inside
 the tolerance) to keep the 32-layer passes within about a minute each.
 """
@@ -19,7 +22,7 @@ import pytest
 
 import seeded_inputs as si
 from oracle import Oracle, SequenceCache
-from tests.helpers import BF16, SeededWeights, near_tie_ok, params_from, rel_l2
+from tests.helpers import BF16, SeededWeights, Top1, params_from, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -33,6 +36,7 @@ from llama_transformer_decoder_b200.configs import LLAMA3_8B, make_config  # noq
 S_PREFILL, B_PREFILL = 2048, 8
 B_DEC, CTX, STEPS = 32, 4096, 128
 V = 128256
+TOP1 = Top1()          # every greedy decision of this module
 
 
 @pytest.fixture(scope='module')
@@ -75,7 +79,7 @@ def test_8b_prefill_batch8_s2048(model8b):
         err = rel_l2(got8[b], ref)
         print(f'sequence {b}: rel-L2 {err:.3e}, gpu argmax {arg8[b]}, oracle argmax {int(np.argmax(ref))}')
         assert err < 2e-2
-        assert near_tie_ok(int(arg8[b]), ref, 2 * float(np.max(np.abs(got8[b] - ref))) + 1e-6)
+        TOP1.add(int(arg8[b]), ref, got8[b])
     assert rel_l2(got1[0], got8[0]) < 5e-3          # batch size does not change a sequence's result
 
 
@@ -84,24 +88,26 @@ def test_8b_decode_batch32_ctx4096_graph(model8b):
     st = torch.cuda.Stream()
     watch = (0, B_DEC - 1)
     toks, rows = [], []
+    seeded = si.tokens(1, STEPS * B_DEC, V, start=B_PREFILL * S_PREFILL).reshape(STEPS, B_DEC)
+    args = []
     with torch.cuda.stream(st):       # torch's reads of lg / arg are ordered after the library's writes
         L.llama_fill_kv_random(h, 3, CTX, st)
-        cur = torch.from_numpy(si.tokens(1, B_DEC, V, start=B_PREFILL * S_PREFILL)).cuda()
+        dev_toks = torch.from_numpy(seeded).cuda()
         arg = torch.empty(B_DEC, dtype=torch.int32, device='cuda')
         lg = torch.empty((B_DEC, V), device='cuda')
         for step in range(STEPS):
-            toks.append(cur.cpu().numpy().copy())
-            L.llama_decode_step(h, cur, B_DEC, st)
+            toks.append(seeded[step])
+            L.llama_decode_step(h, dev_toks[step], B_DEC, st)
             L.llama_logits(h, lg, st)
             L.llama_argmax(h, arg, st)
             rows.append(lg[list(watch)].cpu().numpy())
-            cur = arg.clone()
+            args.append(arg[list(watch)].cpu().numpy())
     torch.cuda.synchronize()
     assert L.llama_sync_status(h, st) == 0
     lens = np.zeros(B_DEC, np.int32)
     L.llama_get_lengths(h, lens, B_DEC)
     assert np.all(lens == CTX + STEPS)
-    # oracle: the same N(0,1) cache slices for the watched sequences, then teacher forcing
+    # oracle: the same N(0,1) cache slices for the watched sequences, then the same tokens
     orc = Oracle(p, w, dtype=np.float32)
     d, Hk = p.head_dim, p.n_kv_heads
     n = Hk * CTX * d
@@ -113,8 +119,8 @@ def test_8b_decode_batch32_ctx4096_graph(model8b):
             v = si.normal(3, si.STREAM_KV_BASE + 2 * layer + 1, n, 1.0, 'bf16', start=b * n)
             cache.k.append(si.bf16_bits_to_f32(k).reshape(Hk, CTX, d))
             cache.v.append(si.bf16_bits_to_f32(v).reshape(Hk, CTX, d))
-        # Teacher forcing = one causal pass over the 128 tokens the GPU consumed:
-        # row i of that pass sees the cache plus tokens 0..i, exactly decode step i.
+        # One causal pass over the 128 seeded tokens: row i of that pass sees
+        # the cache plus tokens 0..i, exactly decode step i.
         seq = np.array([toks[step][b] for step in range(STEPS)])
         _, hidden = orc.forward(seq, cache, return_hidden=True)
         refs = orc.logits(hidden)
@@ -123,6 +129,13 @@ def test_8b_decode_batch32_ctx4096_graph(model8b):
             err = rel_l2(got, ref)
             worst = max(worst, err)
             assert err < 2e-2, (b, step, err)
-            if step + 1 < STEPS:
-                assert near_tie_ok(int(toks[step + 1][b]), ref, 2 * float(np.max(np.abs(got - ref))) + 1e-6)
+            TOP1.add(int(args[step][wi]), ref, got)
     print(f'decode: worst logits rel-L2 over {STEPS} steps x {len(watch)} sequences: {worst:.3e}')
+
+
+def test_8b_top1_agreement():
+    """At least 99% strict top-1 agreement over the greedy decisions above."""
+    if TOP1.total < 2 + 2 * STEPS:
+        pytest.skip('the prefill and decode tests of this module did not run')
+    print(TOP1.summary())
+    assert TOP1.fraction() >= 0.99, TOP1.summary()
