@@ -60,6 +60,13 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Largest of three (one instruction on sm_100a).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Page j of sequence b (page 0 for an index outside the pool).
 __device__ __forceinline__ int kv_page(const int32_t* table, int max_pages, int n_pages, int b, int j) {
   const int p = table[(size_t)b * max_pages + j];
@@ -110,9 +117,14 @@ __device__ __forceinline__ float fa_tile_softmax(uint32_t s_tmem, bool ok, bool 
 #pragma unroll
   for (int x = 0; x < 8; ++x) mx8[x] = sv[x];
 #pragma unroll
-  for (int x = 8; x < 128; ++x) mx8[x & 7] = fmaxf(mx8[x & 7], sv[x]);
-  const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
+  for (int x = 8; x < 120; x += 16) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) mx8[c] = fmax3(mx8[c], sv[x + c], sv[x + 8 + c]);
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) mx8[c] = fmaxf(mx8[c], sv[120 + c]);
+  const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])) *
+                   scale_log2;
   corr = 1.f;
   if (first) {
     m_used = mx;
@@ -355,27 +367,26 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
 // The same computation with one CTA per SM looping over (query tile, head,
 // sequence) items, so that the start of one item overlaps the end of the
 // previous one: Q is double-buffered and loaded while the previous item runs,
-// the K/V rings, the S buffers and the P/O barriers run on across items, and
-// four extra warps (6-9) move O / l to global memory while the softmax warps
-// (2-5) already work on the next item's first tile. The next item's first P V
-// product waits only until those warps have read O out of TMEM.
+// and the K/V rings, the S buffers and the P/O barriers run on across items.
+// At the end of an item the softmax warps read O out of TMEM and store O / l;
+// meanwhile the tensor cores already compute the next item's first S. The
+// next item's first P V product needs that item's first P, which the same
+// threads store only after reading O, so O is never overwritten early.
 //
 // Items are taken in the longest-first order of the per-tile kernel, dealt
 // to the CTAs in a snake (round r goes to CTAs 0..G-1 for even r and G-1..0
 // for odd r), which balances the decreasing causal lengths.
 //
 // Barrier phases are counted per CTA over all items: global tile t uses K/V
-// and S stage t&1; item i uses Q buffer i&1 and row-sum slot i&1. Every
-// wait is bounded; after a failed wait a role stops waiting (and issuing)
-// but walks its loops to the end, so the named barrier of the softmax warps
-// stays matched.
-constexpr int FP_THREADS = 320;
+// and S stage t&1; item i uses Q buffer i&1. Every wait is bounded; after a
+// failed wait a role stops waiting (and issuing) but walks its loops to the
+// end.
+constexpr int FP_THREADS = 192;
 constexpr int kPersistentMaxS = 4096;
 constexpr int FP_OFF_Q = 0;                                      // two Q buffers
 constexpr int FP_OFF_K = FP_OFF_Q + 2 * FA_Q_BYTES;
 constexpr int FP_OFF_V = FP_OFF_K + FA_STAGES * FA_KV_BYTES;
-constexpr int FP_OFF_RED = FP_OFF_V + FA_STAGES * FA_KV_BYTES;  // row sums [2 item slots][128]
-constexpr int FP_OFF_BAR = FP_OFF_RED + 2 * 128 * 4;
+constexpr int FP_OFF_BAR = FP_OFF_V + FA_STAGES * FA_KV_BYTES;
 constexpr int FP_SMEM = FP_OFF_BAR + 256 + 1024;
 
 __device__ __forceinline__ int fp_item(int c, int G, int i) { return i * G + ((i & 1) ? G - 1 - c : c); }
@@ -418,10 +429,8 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
   uint64_t* s_full = bars + 12;    // [2]
   uint64_t* p_full = bars + 14;    // softmax threads stored P (128 arrivals)
   uint64_t* o_done = bars + 15;    // O += P V finished
-  uint64_t* l_ready = bars + 16;   // softmax threads stored the item's row sums (128 arrivals)
-  uint64_t* o_free = bars + 17;    // the O warps have read O out of TMEM (128 arrivals)
-  uint64_t* drain = bars + 18;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  uint64_t* drain = bars + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = ((S + FA_BM - 1) / FA_BM) * H * B;
@@ -437,8 +446,6 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
     }
     mbar_init(p_full, 128);
     mbar_init(o_done, 1);
-    mbar_init(l_ready, 128);
-    mbar_init(o_free, 128);
     mbar_init(drain, 1);
     fence_barrier_init();
   }
@@ -448,7 +455,6 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_wait();
-  float* red_sum = reinterpret_cast<float*>(smem + FP_OFF_RED);   // [item slot][row]
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmQ);
@@ -531,9 +537,8 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
         if (!(ok = mbar_wait(p_full, tj & 1, status))) break;
         const int st = tj & 1;
         if (!(ok = mbar_wait(&v_full[st], (tj >> 1) & 1, status))) break;
-        // the first product of an item overwrites O: the previous item's O
-        // must have been read out of TMEM
-        if (j == 0 && i > 0 && !(ok = mbar_wait(o_free, (i - 1) & 1, status))) break;
+        // (the first product of an item overwrites O: the softmax threads read
+        // the previous item's O out before they stored this item's first P)
         tc_fence_after();
         const uint32_t v_addr = smem_u32(smem + FP_OFF_V + st * FA_KV_BYTES);
 #pragma unroll
@@ -549,7 +554,7 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
       umma_commit(drain);
       mbar_wait(drain, 0, status);
     }
-  } else if (warp >= 2 && warp < 6) {
+  } else if (warp >= 2) {
     const int quarter = warp & 3;                       // TMEM lanes this warp may read
     const int r = quarter * 32 + lane;                  // query row in the tile
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -579,32 +584,14 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
         tc_fence_before();
         mbar_arrive(p_full);
       }
-      // hand the row sums to the O warps; slot i&1 was last read for item
-      // i-2, and those warps have finished item i-1 once o_free says so
-      if (i > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(o_free, (i - 1) & 1, status));
-      red_sum[(i & 1) * 128 + r] = l;
-      mbar_arrive(l_ready);
-    }
-  } else if (warp >= 6) {
-    const int quarter = warp & 3;                       // warps 6-9: lanes 64-95, 96-127, 0-31, 32-63
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    bool ok = true;
-    int t = 0;
-    for (int i = 0;; ++i) {
-      const int w = fp_item(c, G, i);
-      if (w >= total) break;
-      const FpItem it = fp_decode(w, S, H, Hk, B, pos0);
-      t += it.n_kt;
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(l_ready, i & 1, status));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (t - 1) & 1, status));
+      // the item's last P V product, then O / l out of TMEM (the next item's
+      // first P V product, which overwrites O, waits for this thread's next P)
+      if (it.n_kt > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (t - 1) & 1, status));
       tc_fence_after();
-      const float inv = 1.f / red_sum[(i & 1) * 128 + r];
       const int qi = it.q0 + r;
       T* dst = o + ((size_t)it.b * S + (qi < S ? qi : 0)) * H * FA_D + (size_t)it.h * FA_D;
-      fa_store_o<T>(tmem + lane_off + FA_TMEM_O, ok, inv, dst, qi < S);
+      fa_store_o<T>(tmem + lane_off + FA_TMEM_O, ok, 1.f / l, dst, qi < S);
       tc_fence_before();
-      mbar_arrive(o_free);
     }
   }
   tc_fence_before();

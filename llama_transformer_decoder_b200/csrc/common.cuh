@@ -162,6 +162,13 @@ __device__ __forceinline__ bool counter_wait_geq(const int* p, int target, int* 
   }
 }
 
+// Orders this thread's earlier generic-proxy accesses (and what it acquired
+// from other threads) before its later async-proxy (TMA) accesses of global
+// memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // --------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -45,6 +45,17 @@ struct EpiArgs {
   // Status word for LLAMA_ERR_RANGE: a 16-bit output (q/k/v, the SwiGLU
   // product, y = x * g) that is not finite after rounding (nullptr: unchecked).
   int* status;
+  // Row-block readiness between consecutive CTA-pair GEMMs (prefill). With
+  // ready_out, every CTA adds 1 to ready_out[r] after its epilogue has written
+  // the 128 rows r*128 .. r*128+127 of an output tile. With ready_in, the
+  // kernel does not wait for the previous kernel to finish: before reading
+  // rows of block r it waits (bounded) until ready_in[r] >= ready_target.
+  // Tiles are taken in groups of m_group 256-row blocks (column by column
+  // inside a group), so the first groups' rows are complete early.
+  int* ready_out;
+  const int* ready_in;
+  int ready_target;
+  int m_group;
 };
 
 // r of row m from its partial sums of squares (added in a fixed order).

@@ -318,6 +318,19 @@ constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
 constexpr int P_STAGES = 6;
 constexpr int P_SMEM = P_STAGES * P_STAGE_BYTES + 1024 + 256;
 
+// Tile t of the pair grid as (256-row block m, 256-column block n): groups of
+// G row blocks, each group taken column by column with its row blocks
+// innermost (G = m_tiles is plain column-major order).
+__device__ __forceinline__ void pair_tile(int t, int m_tiles, int G, int& m, int& n, int n_tiles) {
+  const int per = G * n_tiles;
+  const int g = t / per;
+  const int r = t - g * per;
+  const int m0 = g * G;
+  const int gm = min(G, m_tiles - m0);
+  n = r / gm;
+  m = m0 + (r - n * gm);
+}
+
 template <int KIND, typename T>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
@@ -352,30 +365,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  const int G = epi.m_group > 0 ? min(epi.m_group, m_tiles) : m_tiles;
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     const uint64_t pol_a = l2_policy_evict_last(), pol_b = l2_policy_evict_last();
     const int first = pair < tiles ? pair : -1;
     const int pre = first >= 0 ? (kb < P_STAGES ? kb : P_STAGES) : 0;
+    // this CTA's 128 rows of tile t may be read once the previous kernel (or
+    // only its tiles of those rows, with ready_in) has written them
+    auto rows_ready = [&](int mb) -> bool {
+      if (!epi.ready_in) return true;
+      const bool r = counter_wait_geq(epi.ready_in + 2 * mb + (int)rank, epi.ready_target, status);
+      fence_proxy_async_global();
+      return r;
+    };
+    bool ok = true;
     {  // weight halves of the first stages before waiting for the previous kernel
-      const int n0 = first >= 0 ? (first / m_tiles) * P_BN + (int)rank * (P_BN / 2) : 0;
+      int fm = 0, fn = 0;
+      if (first >= 0) pair_tile(first, m_tiles, G, fm, fn, n_tiles);
+      const int n0 = fn * P_BN + (int)rank * (P_BN / 2);
       for (int k = 0; k < pre; ++k) {
         if (leader) mbar_arrive_expect_tx(&full[k], 2 * P_STAGE_BYTES);
         tma_load_2d_pair(smem + k * P_STAGE_BYTES + P_A_BYTES, &tmB, mapa_shared(smem_u32(&full[k]), 0), k * BK, n0,
                          pol_b);
       }
-      pdl_wait();
-      const int m0 = first >= 0 ? (first % m_tiles) * 2 * P_BM + (int)rank * P_BM : 0;
-      for (int k = 0; k < pre; ++k)
+      if (!epi.ready_in) pdl_wait();
+      else if (first >= 0) ok = rows_ready(fm);
+      const int m0 = fm * 2 * P_BM + (int)rank * P_BM;
+      for (int k = 0; k < pre; ++k)   // issued even after a failed wait: the barriers expect these bytes
         tma_load_2d_pair(smem + k * P_STAGE_BYTES, &tmA, mapa_shared(smem_u32(&full[k]), 0), k * BK, m0, pol_a);
     }
     int stage = pre % P_STAGES, issued = pre;
     uint32_t phase = pre == P_STAGES ? 1u : 0u;
-    bool ok = true;
     for (int t = pair; t < tiles && ok; t += pairs) {
-      const int m0 = (t % m_tiles) * 2 * P_BM + (int)rank * P_BM;
-      const int n0 = (t / m_tiles) * P_BN + (int)rank * (P_BN / 2);
+      int tm, tn;
+      pair_tile(t, m_tiles, G, tm, tn, n_tiles);
+      if (t != pair && !(ok = rows_ready(tm))) break;
+      const int m0 = tm * 2 * P_BM + (int)rank * P_BM;
+      const int n0 = tn * P_BN + (int)rank * (P_BN / 2);
       for (int k = (t == pair ? pre : 0); k < kb; ++k) {
         if (!mbar_wait(&empty[stage], phase ^ 1, status)) { ok = false; break; }
         uint8_t* sa = smem + stage * P_STAGE_BYTES;
@@ -419,15 +447,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(drain, 0, status);
     }
   } else if (warp >= 2) {
-    pdl_wait();  // the epilogue reads and writes memory owned by earlier kernels
+    // The epilogue reads and writes memory owned by earlier kernels: all of
+    // the previous kernel's output, or (ready_in) the rows of the tile.
+    if (!epi.ready_in) pdl_wait();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool failed = false;  // after a timed-out wait the MMA has stopped: no further waits
     for (int t = pair; t < tiles; t += pairs) {
-      const int m0 = (t % m_tiles) * 2 * P_BM + (int)rank * P_BM, n0 = (t / m_tiles) * P_BN;
+      int tm, tn;
+      pair_tile(t, m_tiles, G, tm, tn, n_tiles);
+      const int m0 = tm * 2 * P_BM + (int)rank * P_BM, n0 = tn * P_BN;
       if (!failed) failed = !__all_sync(0xffffffffu, mbar_wait(&accf[acc], acc_phase, status));
+      if (!failed && epi.ready_in)   // already complete (the producer warp waited): acquires its rows' writes
+        failed = !__all_sync(0xffffffffu, counter_wait_geq(epi.ready_in + 2 * tm + (int)rank, epi.ready_target, status));
       tc_fence_after();
       const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + acc * P_BN;
       const float rs = (KIND == EPI_QKV_ROPE || KIND == EPI_SWIGLU) && epi.ss_in && m0 + row < M
@@ -445,6 +479,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive_cluster(mapa_shared(smem_u32(&acce[acc]), 0));
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      if (epi.ready_out) {   // this CTA's 128 rows of the tile are written: publish them
+        named_bar_sync(1, 128);
+        if (warp == 2 && lane == 0) {
+          __threadfence();
+          atomicAdd(epi.ready_out + 2 * tm + (int)rank, 1);
+        }
+      }
     }
   }
   tc_fence_before();
@@ -855,6 +896,8 @@ bool pair_gemm_enabled() {
   return on;
 }
 
+bool gemm16_uses_pair(int M, int N, int K) { return M > 128 && pair_gemm_enabled() && wide_split(M, N, K).sk_tiles == 0; }
+
 template <int KIND, typename T>
 static int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, const EpiArgs& e,
                        int* status, cudaStream_t st) {
@@ -927,7 +970,7 @@ static int gemm16_t(const void* A, int M, int K, int lda, const void* W, int N, 
   int rc;
   if (!skinny) {
     CUtensorMap ta, tb;
-    if (pair_gemm_enabled() && wide_split(M, N, K).sk_tiles == 0) {
+    if (gemm16_uses_pair(M, N, K)) {
       // at least one full wave of 128x256 tiles: CTA pairs on 256x256 tiles
       if ((rc = make_tmap_16(&ta, A, M, K, lda, P_BM, F16)) != LLAMA_OK) return rc;
       if ((rc = make_tmap_16(&tb, W, N, K, ldw, P_BN / 2, F16)) != LLAMA_OK) return rc;

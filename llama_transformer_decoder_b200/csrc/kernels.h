@@ -69,6 +69,9 @@ int make_tmap_16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
 // Scratch of the stream-K skinny GEMM for M rows: two partial tiles per CTA.
 size_t skinny_workspace_floats(int M);
 
+// True when an automatic 16-bit GEMM of this shape runs the CTA-pair kernel
+// (the only one that honours EpiArgs::ready_in / ready_out / m_group).
+bool gemm16_uses_pair(int M, int N, int K);
 // 16-bit GEMM; elt = LLAMA_BF16 or LLAMA_F16 (element type of A, W and 16-bit outputs).
 int gemm16(const void* A, int M, int K, int lda, const void* W, int N, int ldw, int elt, int kind, const EpiArgs& e,
            int variant, GemmScratch* scratch, int* status, cudaStream_t st);

@@ -93,6 +93,13 @@ struct llama_model {
   // workspace
   float* ss = nullptr;        // [max_tokens][ceil(dim/256)] partial sums of squares (folded RMSNorm)
   bool norm_ready = false;    // xn / ss already hold the next layer's attention-norm inputs
+  // Row-block readiness counters of the prefill GEMMs (16-bit models): per
+  // layer three sets (Wo, w1/w3, w2 outputs) of one counter per 128 rows,
+  // zeroed at the start of every prefill step. last_signal_layer: layer whose
+  // w2 GEMM published its rows last (-1: the last GEMM published nothing).
+  int* ready = nullptr;
+  int ready_rb = 0;
+  int last_signal_layer = -1;
   float* x = nullptr;
   void* xn = nullptr;
   void* q = nullptr;
@@ -348,6 +355,8 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
   // and the QKV / w1-w3 epilogues scale by rsqrt(mean(x^2) + eps).
   const bool fuse = m->adt != LLAMA_F32 && M > 128;
   const int ss_n = (D + 255) / 256;
+  // QKV directly after the previous layer's w2 that published its row blocks
+  const bool after_w2 = fuse && m->norm_ready && m->last_signal_layer == l - 1 && l > 0;
   if (fuse) {
     if (!m->norm_ready) {
       mark(m, K_RMSNORM, st);
@@ -358,6 +367,24 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
     RC(launch_rmsnorm(m->x, w.attn_norm, m->xn, M, D, c.norm_eps, 0, m->adt, st, m->d_status));
   }
   m->norm_ready = false;
+  m->last_signal_layer = -1;
+  // Consecutive CTA-pair GEMMs overlap: a producer publishes each 128-row
+  // block of its output (ready_out), and its consumer, launched early, waits
+  // only for the blocks it reads (ready_in) instead of the whole kernel, so
+  // the consumer's first tiles run on the SMs the producer's last, partial
+  // wave leaves idle. Producers whose consumer follows take their tiles in
+  // row-block order (m_group 1: early blocks complete early); w1/w3 keeps two
+  // groups so its 235 MB of weights are streamed twice, not once per block.
+  const bool ov = fuse && m->ready != nullptr;
+  const int m_tiles = (M + 255) / 256;
+  auto ready_set = [&](int layer, int which) { return m->ready + ((size_t)layer * 3 + which) * m->ready_rb; };
+  auto link = [&](EpiArgs& a, int* in_set, bool producer_pair, int producer_n, bool consumer_pair) {
+    if (!ov || !in_set || !producer_pair || !consumer_pair) return;
+    a.ready_in = in_set;
+    a.ready_target = (producer_n + 255) / 256;
+  };
+  const bool qkv_pair = ov && gemm16_uses_pair(M, m->qkv_n, D), wo_pair = ov && gemm16_uses_pair(M, D, H * d);
+  const bool w13_pair = ov && gemm16_uses_pair(M, 2 * m->F, D), w2_pair = ov && gemm16_uses_pair(M, D, m->F);
   auto norm_in = [&](EpiArgs& a) {
     if (!fuse) return;
     a.ss_in = m->ss;
@@ -387,6 +414,8 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
   e.kv_table = m->paged ? m->d_table : nullptr;
   e.kv_max_pages = m->max_pages;
   e.kv_pages = m->n_pages;
+  if (after_w2) link(e, ready_set(l - 1, 2), gemm16_uses_pair(M, D, m->F), D, qkv_pair);
+  e.m_group = 1;
   mark(m, K_GEMM_QKV, st);
   RC(gemm(m, m->xn, M, D, w.wqkv, m->qkv_n, EPI_QKV_ROPE, e, st));
   if (decode) {
@@ -402,6 +431,8 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
   r.out = m->x;
   r.ldo = D;
   norm_out(r, w.ffn_norm);
+  if (ov && wo_pair) r.ready_out = ready_set(l, 0);
+  r.m_group = 1;
   mark(m, K_GEMM_WO, st);
   RC(gemm(m, m->attn, M, H * d, w.wo, D, EPI_RESIDUAL, r, st));
   if (!fuse) {
@@ -412,17 +443,24 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
   sg.g = m->g;
   sg.ldg = m->F;
   norm_in(sg);
+  link(sg, ready_set(l, 0), wo_pair, D, w13_pair);
+  if (ov && w13_pair) sg.ready_out = ready_set(l, 1);
+  sg.m_group = (m_tiles + 1) / 2;
   mark(m, K_GEMM_W13, st);
   RC(gemm(m, m->xn, M, D, w.w13, 2 * m->F, EPI_SWIGLU, sg, st));
   EpiArgs r2 = epi_base(M, D, m->d_status);
   r2.out = m->x;
   r2.ldo = D;
+  link(r2, ready_set(l, 1), w13_pair, 2 * m->F, w2_pair);
+  r2.m_group = 1;
   if (l + 1 < c.n_layers) {   // the next layer's attention norm (the final norm takes the last rows only)
     norm_out(r2, m->L[l + 1].attn_norm);
     m->norm_ready = fuse;
+    if (ov && w2_pair) r2.ready_out = ready_set(l, 2);
   }
   mark(m, K_GEMM_W2, st);
   RC(gemm(m, m->g, M, m->F, w.w2, D, EPI_RESIDUAL, r2, st));
+  if (r2.ready_out) m->last_signal_layer = l;
   return LLAMA_OK;
 }
 
@@ -440,8 +478,18 @@ int run_head(llama_model* m, int B, int S, cudaStream_t st) {
   return LLAMA_OK;
 }
 
+// Zeroes the row-block counters of the prefill GEMMs (part of the step, so a
+// graph replay zeroes them too).
+int reset_ready(llama_model* m, int M, cudaStream_t st) {
+  m->last_signal_layer = -1;
+  if (!m->ready || M <= 128) return LLAMA_OK;
+  CK(cudaMemsetAsync(m->ready, 0, (size_t)3 * m->cfg.n_layers * m->ready_rb * sizeof(int), st));
+  return LLAMA_OK;
+}
+
 int prefill_body(llama_model* m, int B, int S, cudaStream_t st) {
   m->norm_ready = false;
+  RC(reset_ready(m, B * S, st));
   mark(m, K_EMBED, st);
   RC(launch_embed(m->tok_buf, B * S, m->tok_emb, m->cfg.vocab_size, m->cfg.dim, m->adt, m->x, m->d_status, st));
   for (int l = 0; l < m->cfg.n_layers; ++l) RC(run_layer(m, l, B, S, false, 0, st));
@@ -453,6 +501,7 @@ int prefill_body(llama_model* m, int B, int S, cudaStream_t st) {
 
 int decode_body(llama_model* m, int B, int cmax, cudaStream_t st) {
   m->norm_ready = false;
+  m->last_signal_layer = -1;
   mark(m, K_EMBED, st);
   RC(launch_embed(m->tok_buf, B, m->tok_emb, m->cfg.vocab_size, m->cfg.dim, m->adt, m->x, m->d_status, st));
   for (int l = 0; l < m->cfg.n_layers; ++l) RC(run_layer(m, l, B, 1, true, cmax, st));
@@ -659,6 +708,12 @@ int llama_create(const llama_config* cfg, llama_model** out) {
   m->logits = static_cast<float*>(m->alloc((size_t)c.max_batch * V * 4));
   m->tok_buf = static_cast<int32_t*>(m->alloc(Mx * sizeof(int32_t)));
   m->d_status = static_cast<int*>(m->alloc(sizeof(int)));
+  if (m->adt != LLAMA_F32 && Mx > 128 && getenv("LLAMA_NO_GEMM_OVERLAP") == nullptr) {
+    m->ready_rb = (int)(2 * ((Mx + 255) / 256));
+    m->ready = static_cast<int*>(m->alloc((size_t)3 * c.n_layers * m->ready_rb * sizeof(int)));
+    if (!m->ready) { delete m; return LLAMA_ERR_OOM; }
+    cudaMemset(m->ready, 0, (size_t)3 * c.n_layers * m->ready_rb * sizeof(int));
+  }
   if (!m->kcache || !m->vcache || !m->d_len || !m->rope || !m->x || !m->ss || !m->xn || !m->q || !m->attn || !m->g ||
       !m->logits || !m->tok_buf || !m->d_status) {
     delete m;
@@ -887,6 +942,7 @@ int llama_block_forward(llama_model* m, int32_t layer, const float* x, float* y,
   const size_t bytes = (size_t)B * S * m->cfg.dim * sizeof(float);
   CK(cudaMemcpyAsync(m->x, x, bytes, cudaMemcpyDeviceToDevice, st));
   m->norm_ready = false;
+  RC(reset_ready(m, B * S, st));
   RC(run_layer(m, layer, B, S, false, 0, st));
   m->norm_ready = false;
   CK(cudaMemcpyAsync(y, m->x, bytes, cudaMemcpyDeviceToDevice, st));

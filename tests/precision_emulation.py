@@ -121,3 +121,49 @@ def last_token_logits(seed: int, p: Params, tokens, variants: dict, std: float =
         xf = rnd(rms_norm(xs[name][-1], np.ones(p.dim, dt), p.norm_eps))
         res[name] = np.asarray(xf, np.float64) @ np.asarray(out_w, np.float64).T
     return res
+
+
+def _attention_rounded_at(q, k, v, q_pos, rnd, dtype):
+    """_attention_rounded for queries at absolute positions q_pos over keys
+    0 .. T-1 (key j visible to query i iff j <= q_pos[i])."""
+    H, S, d = q.shape
+    group = H // k.shape[0]
+    mask = np.arange(k.shape[1])[None, :] > np.asarray(q_pos)[:, None]
+    out = np.empty((S, H * d), dtype)
+    for h in range(H):
+        s = (q[h] @ k[h // group].T) * (1.0 / np.sqrt(d))
+        s = np.where(mask, -np.inf, s)
+        e = np.exp(s - s.max(axis=1, keepdims=True))
+        out[:, h * d:(h + 1) * d] = (rnd(e) @ v[h // group]) / e.sum(axis=1, keepdims=True)
+    return out
+
+
+def pass_after_cache_rounded(p: Params, w, cache_k, cache_v, tokens, rnd, dtype=np.float32):
+    """Last-token logits of every row of one causal pass over `tokens` placed
+    after a cache (cache_k[l], cache_v[l]: [Hk, c, d], exact values, taken as
+    already rotated), with the 16-bit roundings `rnd` at the GPU path's
+    rounding points (decode shapes: the normalised activations are rounded
+    after the scale). Row i is the decode step that consumes tokens[i]."""
+    d, H, Hk = p.head_dim, p.n_heads, p.n_kv_heads
+    c = cache_k[0].shape[1]
+    T = len(tokens)
+    pos = c + np.arange(T)
+    x = rnd(np.asarray(w['tok_embeddings.weight'][np.asarray(tokens)], dtype))
+    for i in range(p.n_layers):
+        pre = f'layers.{i}.'
+        W = lambda n: np.asarray(w[pre + n], dtype)
+        xn = rnd(rms_norm(x, W('attention_norm.weight'), p.norm_eps))
+        q = (xn @ W('attention.wq.weight').T).reshape(T, H, d).transpose(1, 0, 2)
+        k = (xn @ W('attention.wk.weight').T).reshape(T, Hk, d).transpose(1, 0, 2)
+        v = rnd((xn @ W('attention.wv.weight').T).reshape(T, Hk, d).transpose(1, 0, 2))
+        q = rnd(apply_rope(q, pos, p.rope_theta).astype(dtype))
+        k = rnd(apply_rope(k, pos, p.rope_theta).astype(dtype))
+        kall = np.concatenate([np.asarray(cache_k[i], dtype), k], axis=1)
+        vall = np.concatenate([np.asarray(cache_v[i], dtype), v], axis=1)
+        o = rnd(_attention_rounded_at(q, kall, vall, pos, rnd, dtype))
+        h = x + o @ W('attention.wo.weight').T
+        hn = rnd(rms_norm(h, W('ffn_norm.weight'), p.norm_eps))
+        g = rnd(silu(hn @ W('feed_forward.w1.weight').T) * (hn @ W('feed_forward.w3.weight').T))
+        x = (h + g @ W('feed_forward.w2.weight').T).astype(dtype)
+    xf = rnd(rms_norm(x, np.asarray(w['norm.weight'], dtype), p.norm_eps))
+    return np.asarray(xf, np.float64) @ np.asarray(w['output.weight'], np.float64).T

@@ -1,17 +1,17 @@
 """Model check of the persistent prefill attention kernel's barrier protocol
 (attention_tc.cu, attn_prefill_tc_persistent_kernel), run on the CPU.
 
-Six actors are simulated under random interleavings: the TMA producer, the
-MMA issuer, the softmax warps, the O warps, and the two asynchronous engines
-(TMA copies and tensor-core operations, each completing in issue order).
-mbarriers follow their parity semantics: a wait for parity p returns once the
-phase with that parity has completed, so a waiter two phases behind would
-pass wrongly. The model checks, at every wait, that the completed phase is
-exactly the one meant, and at every buffer access that the data is the
-intended version (Q per item, K/V per tile, S per tile, P per tile, O per
-item, row-sum slot per item). The waits mirror the kernel's; the kernel and
-this model are kept in step by hand. Dropping any of the protocol's
-cross-item waits must make the model fail."""
+Five actors are simulated under random interleavings: the TMA producer, the
+MMA issuer, the softmax warps (which also read O out at the end of every
+item), and the two asynchronous engines (TMA copies and tensor-core
+operations, each completing in issue order). mbarriers follow their parity
+semantics: a wait for parity p returns once the phase with that parity has
+completed, so a waiter two phases behind would pass wrongly. The model
+checks, at every wait, that the completed phase is exactly the one meant,
+and at every buffer access that the data is the intended version (Q per
+item, K/V per tile, S per tile, P per tile, O per item). The waits mirror
+the kernel's; the kernel and this model are kept in step by hand. Dropping
+any of the protocol's cross-item waits must make the model fail."""
 import random
 
 import pytest
@@ -41,10 +41,10 @@ def simulate(nkts, seed, drop=()):
     for i in range(2):
         for n in ('q_full', 'q_empty', 'k_full', 'k_empty', 'v_full', 'v_empty', 's_full'):
             bars[f'{n}{i}'] = Bar()
-    for n in ('p_full', 'o_done', 'l_ready', 'o_free'):
+    for n in ('p_full', 'o_done'):
         bars[n] = Bar()
     st = dict(Q=[None, None], K=[None, None], V=[None, None], S=[None, None], P=None, O_item=None, O_tiles=set(),
-              slot=[None, None], s_read=set(), o_read=set(), pv_done=set(), s_done=set())
+              s_read=set(), o_read=set(), pv_done=set(), s_done=set())
     tma, tc = [], []
     first = [sum(nkts[:i]) for i in range(len(nkts))]
 
@@ -98,8 +98,6 @@ def simulate(nkts, seed, drop=()):
                     tc.append(('commit', f'q_empty{qs}'))
                 yield from wait('p_full', tj)
                 yield from wait(f'v_full{tj & 1}', tj >> 1)
-                if j == 0 and i > 0 and 'mma_o_free' not in drop:
-                    yield from wait('o_free', i - 1)
                 tc.extend([('PV', tj, i, j), ('commit', f'v_empty{tj & 1}'), ('commit', 'o_done')])
                 yield 'step'
             t += n
@@ -122,27 +120,16 @@ def simulate(nkts, seed, drop=()):
                 st['P'] = t
                 bars['p_full'].arrive()
                 t += 1
-            if i > 0 and 'softmax_o_free' not in drop:
-                yield from wait('o_free', i - 1)
-            if i >= 2 and i - 2 not in st['o_read']:
-                raise ProtocolError('row-sum slot overwritten before it was read')
-            st['slot'][i & 1] = i
-            bars['l_ready'].arrive()
-
-    def o_warps():
-        t = 0
-        for i, n in enumerate(nkts):
-            t += n
-            yield from wait('l_ready', i)
-            yield from wait('o_done', t - 1)
+            # O / l of item i out of TMEM
+            if 'softmax_o_final' not in drop:
+                yield from wait('o_done', t - 1)
             want = set(range(t - n, t))
-            if st['slot'][i & 1] != i or st['O_item'] != i or st['O_tiles'] != want:
-                raise ProtocolError('O warps read the wrong O or row sums')
+            if st['O_item'] != i or st['O_tiles'] != want:
+                raise ProtocolError('read the wrong O')
             yield 'step'
             if st['O_item'] != i or st['O_tiles'] != want:
                 raise ProtocolError('O changed while being read')
             st['o_read'].add(i)
-            bars['o_free'].arrive()
 
     def run_tma():
         kind, s, x = tma.pop(0)
@@ -172,7 +159,7 @@ def simulate(nkts, seed, drop=()):
         else:
             bars[op[1]].arrive()
 
-    actors = {'producer': producer(), 'mma': mma(), 'softmax': softmax(), 'o': o_warps()}
+    actors = {'producer': producer(), 'mma': mma(), 'softmax': softmax()}
     # each actor and engine runs at its own random rate, so some schedules
     # starve one of them for long stretches
     rate = {a: rng.choice([0.05, 0.3, 1.0]) for a in list(actors) + ['tma', 'tc']}
@@ -215,7 +202,7 @@ def test_protocol_holds_under_random_schedules():
         simulate(nkts, seed)
 
 
-@pytest.mark.parametrize('drop', ['mma_o_free', 'softmax_o_free', 'softmax_o_done', 'q_empty'])
+@pytest.mark.parametrize('drop', ['softmax_o_final', 'softmax_o_done', 'q_empty'])
 def test_dropping_a_wait_is_caught(drop):
     with pytest.raises(ProtocolError):
         for nkts, seed in _cases(400):

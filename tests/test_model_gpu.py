@@ -163,6 +163,70 @@ def test_block_8b_bf16(block8b, B, S):
         assert rel_l2(got[b][rows], ref) < 2e-2
 
 
+def test_block_8b_bf16_activations():
+    """act_dtype = LLAMA_BF16: weights, activations, cache and P all in bf16,
+    as the pages compute. One 8B-shaped block at S = 2048 (pair GEMMs and the
+    persistent attention kernel) and S = 17 (skinny GEMMs) against the
+    oracle, rel-L2 <= 2e-2 (one layer of bf16 roundings is about 1.5e-3)."""
+    m = Model(dict(BLOCK_8B, act_dtype=BF16), BF16, max_batch=1, max_seq=2048, max_tokens=2048)
+    try:
+        assert m.rc.act_dtype == BF16
+        L.llama_init_weights(m.h, 0, 0.02)
+        w = SeededWeights(m.p, 0, 0.02, BF16)
+        orc = Oracle(m.p, w)
+        for S in (2048, 17):
+            L.llama_reset(m.h)
+            xv, _ = normal_values(2, si.STREAM_HIDDEN, (1, S, 4096), BF16)
+            x = torch.from_numpy(np.ascontiguousarray(xv)).cuda()
+            y = torch.empty_like(x)
+            L.llama_block_forward(m.h, 0, x, y, 1, S)
+            _check_status(m)
+            rows = np.arange(S) if S <= 300 else np.unique(np.r_[np.arange(0, S, 97), S - 1])
+            ref = orc.layer(0, xv[0].astype(np.float64), None, 0, rows=rows)
+            err = rel_l2(y.cpu().numpy()[0][rows], ref)
+            print(f'bf16 activations, S={S}: rel-L2 {err:.3e}')
+            assert err < 2e-2
+    finally:
+        m.close()
+
+
+def test_fp16_range_overflow_is_latched_and_model_stays_usable():
+    """A residual stream beyond the fp16 range entering the folded norm of a
+    prefill (y = x * g is stored in fp16), and a SwiGLU product beyond it in
+    decode, each latch LLAMA_ERR_RANGE; after fresh weights and a reset the
+    same model computes correct logits again."""
+    m = Model(SMALL_BF16, BF16, max_batch=2, max_seq=256)
+    try:
+        L.llama_init_weights(m.h, 18, 0.02)
+        xv, _ = normal_values(19, si.STREAM_HIDDEN, (1, 200, 512), BF16)
+        xv = xv.copy()
+        xv[0, 5, 7] = 1.0e5
+        x = torch.from_numpy(np.ascontiguousarray(xv)).cuda()
+        y = torch.empty_like(x)
+        L.llama_block_forward(m.h, 0, x, y, 1, 200)              # 200 rows: folded-norm path
+        assert L.llama_sync_status(m.h) == L.LLAMA_ERR_RANGE
+        assert L.llama_sync_status(m.h) == 0
+        F = m.rc.ffn_hidden
+        big = np.where(np.arange(F)[:, None] % 2 == 0, 256.0, -256.0).astype(np.float32) * np.ones((1, 512), np.float32)
+        bits = si.f32_to_bf16_bits(big)
+        for name in ('layers.0.feed_forward.w1.weight', 'layers.0.feed_forward.w3.weight'):
+            L.llama_set_weight(m.h, name, bits, bits.nbytes, 0)
+        L.llama_set_lengths(m.h, np.array([0, 0], np.int32), 2)          # attend to the new token only
+        L.llama_decode_step(m.h, torch.tensor([5, 9], dtype=torch.int32, device='cuda'), 2)
+        assert L.llama_sync_status(m.h) == L.LLAMA_ERR_RANGE
+        L.llama_init_weights(m.h, 18, 0.02)
+        L.llama_reset(m.h)
+        toks = si.tokens(20, 2 * 30, 3000).reshape(2, 30)
+        L.llama_prefill(m.h, torch.from_numpy(toks).cuda(), 2, 30)
+        got = m.logits(2).cpu().numpy()
+        _check_status(m)
+        orc = Oracle(m.p, SeededWeights(m.p, 18, 0.02, BF16))
+        ref = np.stack([orc.forward(toks[b]) for b in range(2)])
+        assert rel_l2(got, ref) < 2e-2
+    finally:
+        m.close()
+
+
 # --------------------------------------------- bf16 multi-layer end to end
 SMALL_BF16 = dict(dim=512, n_layers=3, n_heads=4, n_kv_heads=2, vocab_size=3000, ffn_hidden=1536,
                   norm_eps=1e-5, rope_theta=500000.0)
@@ -493,6 +557,70 @@ def test_generate_graph_replayed_matches_oracle():
                     print(f'call {call} sequence {b}: chains part at step {k}, oracle margin {margins[b, k]:.2e}')
                     assert margins[b, k] < bound[b, k], (b, k, margins[b, k], bound[b, k])
             assert parted <= 1
+    finally:
+        m.close()
+
+
+# ------------------------------------------------------------ long context
+LONG_8B = dict(LLAMA3_8B, n_layers=1, vocab_size=512, kv_page_size=128)
+
+
+def test_long_context_8b_prefill_tokens_to_32k():
+    """One 8B-shaped layer (H = 32, Hk = 8, d = 128, F = 14336) on the paged
+    cache: a prompt of 32768 + 300 seeded tokens prefilled in 4096-token
+    chunks (each chunk's queries start at the cached length), then the
+    last-token logits against one float32 oracle pass over the whole prompt."""
+    S_total, chunk = 32768 + 300, 4096
+    m = Model(LONG_8B, BF16, max_batch=1, max_seq=S_total + 8, max_tokens=chunk)
+    try:
+        L.llama_init_weights(m.h, 21, 0.02)
+        toks = si.tokens(22, S_total, 512)
+        for a in range(0, S_total, chunk):
+            part = np.ascontiguousarray(toks[a:a + chunk])
+            L.llama_prefill(m.h, torch.from_numpy(part).cuda(), 1, len(part))
+        got = m.logits(1).cpu().numpy()[0]
+        arg = int(m.argmax(1).cpu().numpy()[0])
+        _check_status(m)
+        orc = Oracle(m.p, SeededWeights(m.p, 21, 0.02, BF16), dtype=np.float32)
+        ref = orc.forward(toks)
+        err = rel_l2(got, ref)
+        print(f'32k-token prompt, last-token logits rel-L2 {err:.3e}')
+        assert err < 2e-2
+        TOP1.add(arg, ref, got)
+    finally:
+        m.close()
+
+
+@pytest.mark.parametrize('S_total,chunk', [(32768 + 300, 4096), (131072, 8192)])
+def test_long_context_8b_block_chunks_sampled_rows(S_total, chunk):
+    """The same layer on N(0,1) hidden states, fed chunk by chunk through
+    llama_block_forward with the cached length advanced between chunks (the
+    cache holds every earlier chunk's keys and values; 8192-token chunks run
+    the per-tile attention kernel, 4096-token chunks the persistent one). 64
+    sampled rows of the last chunk plus its last row are checked against the
+    oracle's layer over the whole sequence (rel-L2 <= 2e-2)."""
+    m = Model(LONG_8B, BF16, max_batch=1, max_seq=S_total + 8, max_tokens=chunk)
+    try:
+        L.llama_init_weights(m.h, 23, 0.02)
+        xv = si.bf16_bits_to_f32(si.normal(24, si.STREAM_HIDDEN, S_total * 4096, 1.0)).reshape(S_total, 4096)
+        last = None
+        for a in range(0, S_total, chunk):
+            n = min(chunk, S_total - a)
+            L.llama_set_lengths(m.h, np.array([a], np.int32), 1)
+            x = torch.from_numpy(np.ascontiguousarray(xv[a:a + n])).cuda()[None]
+            y = torch.empty_like(x)
+            L.llama_block_forward(m.h, 0, x, y, 1, n)
+            last = (a, n, y)
+        _check_status(m)
+        a, n, y = last
+        rng = np.random.RandomState(S_total)
+        rows = np.unique(np.r_[rng.choice(n, 64, replace=False), n - 1])
+        got = y[0][torch.from_numpy(rows).cuda()].cpu().numpy()
+        orc = Oracle(m.p, SeededWeights(m.p, 23, 0.02, BF16), dtype=np.float32)
+        ref = orc.layer(0, xv, None, 0, rows=a + rows)
+        err = rel_l2(got, ref)
+        print(f'{S_total} tokens in {chunk}-token chunks: sampled rows of the last chunk rel-L2 {err:.3e}')
+        assert err < 2e-2
     finally:
         m.close()
 
