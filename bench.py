@@ -276,10 +276,10 @@ def run_reference(args):
 
 # ---------------------------------------------------------------- our arm
 D_, F_, H_, HK_, HD_, V_ = 4096, 14336, 32, 8, 128, 128256
-# Measured DRAM bytes per launch of the prefill projection GEMM (mean over a
-# layer's QKV, Wo, w1/w3, w2 launches at 2048 tokens; one ncu capture of the
-# current kernel). Set to None when the kernel changes until re-captured.
-PAIR_GEMM_TRAFFIC = 187.2e6
+# Measured DRAM bytes per launch of the chained prefill projection GEMM (one
+# layer's Wo, w1/w3, w2 and the next QKV at 2048 tokens; one ncu capture of
+# the current kernel). None until captured for the current kernel.
+PAIR_GEMM_TRAFFIC = None
 
 
 def measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust, peak_src, B=PREFILL_B):
@@ -323,7 +323,7 @@ def measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust, peak_src,
     _barrier(ws)
     M = B * PREFILL_S
     flops_layer = 2.0 * M * D_ * ((H_ + 2 * HK_) * HD_ + H_ * HD_ + 2 * F_ + F_)
-    gemm_kinds = ['gemm_qkv_rope', 'gemm_wo_residual', 'gemm_w13_swiglu', 'gemm_w2_residual']
+    gemm_kinds = ['gemm_qkv_rope', 'gemm_wo_residual', 'gemm_w13_swiglu', 'gemm_w2_residual', 'gemm_chain']
     gemm_ms = sum(prof[k][0] for k in gemm_kinds)
     gemm_launches = sum(prof[k][1] for k in gemm_kinds)
     achieved = flops_layer * NL * args.steps / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
@@ -332,11 +332,12 @@ def measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust, peak_src,
                    'share': v[0] / total_prof} for k, v in prof.items() if v[1]}
     attn_flops = 4.0 * B * H_ * HD_ * PREFILL_S * (PREFILL_S + 1) / 2 * NL
     attn = prof.get('attention_prefill', (0, 0))
-    roofline = {'kernel': 'gemm_pair_kernel (tcgen05 cta_group::2, 4 projections)', 'bound': 'tensor',
+    roofline = {'kernel': 'gemm_chain_kernel (tcgen05 cta_group::2; per layer one launch of Wo, w1/w3, w2 and the '
+                          'next layer\'s QKV, plus layer 0\'s QKV)', 'bound': 'tensor',
                 'achieved': achieved, 'peak': tf_sust, 'unit': 'TFLOP/s',
                 'frac': achieved / tf_sust if achieved else None, 'traffic': PAIR_GEMM_TRAFFIC,
-                'traffic_note': 'DRAM read+write bytes per launch, mean of one layer\'s four launches, '
-                                'ncu (profiles/gemm_pair_kernel_llama3_8b_prefill_s2048.md)',
+                'traffic_note': 'DRAM read+write bytes per chained launch from one ncu capture (null: not yet '
+                                'captured for this kernel)',
                 'peak_kind': f'bf16 sustained ({peak_src}); fp16 has the same nominal tensor rate',
                 'launches': gemm_launches // max(args.steps, 1),
                 'attention_tflops': attn_flops * args.steps / (attn[0] / 1e3) / 1e12 if attn[0] else None,

@@ -183,7 +183,8 @@ int llama_reset(llama_model* m, void* stream);
  * bypassed). llama_profile_read synchronizes, then fills ms[k] (summed time from the launch's
  * event to the next one) and launches[k] for kinds k < n_kinds, clears the record and returns
  * the number of kinds (embed, rmsnorm, gemm_qkv_rope, attention_prefill, attention_decode,
- * gemm_wo_residual, gemm_w13_swiglu, gemm_w2_residual, gemm_lm_head, other). */
+ * gemm_wo_residual, gemm_w13_swiglu, gemm_w2_residual, gemm_lm_head, other, gemm_chain: one prefill
+ * launch running a layer's Wo, w1/w3 and w2 projections and the next layer's QKV projection). */
 int llama_profile(llama_model* m, int enable);
 int llama_profile_read(llama_model* m, double* ms, int64_t* launches, int n_kinds);
 const char* llama_profile_kind_name(int kind);

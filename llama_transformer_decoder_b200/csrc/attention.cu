@@ -315,6 +315,9 @@ constexpr int DM_WARPS = 4;
 constexpr int DM_TILE = DM_KEYS * 256;             // one K (or V) tile: 32 rows x 256 B
 constexpr int DM_STAGE = 2 * DM_TILE;
 constexpr int DM_SMEM = DM_WARPS * DM_STAGES * DM_STAGE;
+// Decoding warps of the grid (SMs x DM_WARPS) the combine can merge for one
+// (sequence, kv head): every warp of the grid may hold a piece of it.
+constexpr int kMaxDecodeWarps = 1024;
 
 __device__ __forceinline__ int dm_keys(const int32_t* nkeys, int b, int add, int nmax) {
   return min(nkeys[b] + add, nmax);
@@ -540,8 +543,7 @@ __global__ void __launch_bounds__(128) attn_decode_combine_pieces_kernel(
   pdl_wait();
   __shared__ long long s_tot, s_t0;
   __shared__ int s_nt, s_cnt;
-  __shared__ int s_w[256];
-  __shared__ float s_f[256];
+  __shared__ int s_w[kMaxDecodeWarps];
   const int h = blockIdx.x, b = blockIdx.y;
   const int G = H / Hk, g = h / G, row = h - g * G;
   if (threadIdx.x == 0) {
@@ -564,34 +566,71 @@ __global__ void __launch_bounds__(128) attn_decode_combine_pieces_kernel(
     for (int dd = threadIdx.x; dd < D; dd += blockDim.x) o[((size_t)b * H + h) * D + dd] = from_f<T>(NAN);
     return;
   }
-  // warps owning tiles of (b, g): owner(t0) .. owner(t0 + nt_b - 1), skipping warps with empty ranges
+  // warps owning tiles of (b, g): owner(t0) .. owner(t0 + nt_b - 1), skipping
+  // warps with empty ranges, listed in warp order (a fixed merge order, so
+  // results do not depend on timing)
   const long long w_lo = ((t0 + 1) * W - 1) / total, w_hi = ((t0 + nt_b) * W - 1) / total;
+  __shared__ int s_warp_cnt[4];
   if (threadIdx.x == 0) s_cnt = 0;
   __syncthreads();
-  for (long long w = w_lo + threadIdx.x; w <= w_hi; w += blockDim.x)
-    if (total * (w + 1) / W > total * w / W) {
-      const int k = atomicAdd(&s_cnt, 1);
-      if (k < 256) s_w[k] = (int)w;
+  for (long long base = w_lo; base <= w_hi; base += blockDim.x) {
+    const long long w = base + threadIdx.x;
+    const bool has = w <= w_hi && total * (w + 1) / W > total * w / W;
+    const unsigned bal = __ballot_sync(0xffffffffu, has);
+    if ((threadIdx.x & 31) == 0) s_warp_cnt[threadIdx.x >> 5] = __popc(bal);
+    __syncthreads();
+    int off = s_cnt;
+    for (int q = 0; q < (int)(threadIdx.x >> 5); ++q) off += s_warp_cnt[q];
+    if (has) {
+      const int k = off + __popc(bal & ((1u << (threadIdx.x & 31)) - 1u));
+      if (k < kMaxDecodeWarps) s_w[k] = (int)w;
     }
-  __syncthreads();
-  const int cnt = s_cnt < 256 ? s_cnt : 256;
-  const size_t bg = (size_t)b * Hk + g;
-  if (threadIdx.x < 32) {  // merge weights exp2(m_w - M) per piece (order does not matter here)
-    float M = -INFINITY;
-    for (int k = threadIdx.x; k < cnt; k += 32) M = fmaxf(M, part[((bg + s_w[k]) * G + row) * (D + 2) + D]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    for (int k = threadIdx.x; k < cnt; k += 32) s_f[k] = exp2f(part[((bg + s_w[k]) * G + row) * (D + 2) + D] - M);
+    __syncthreads();
+    if (threadIdx.x == 0) s_cnt += s_warp_cnt[0] + s_warp_cnt[1] + s_warp_cnt[2] + s_warp_cnt[3];
+    __syncthreads();
   }
+  const int cnt = s_cnt < kMaxDecodeWarps ? s_cnt : kMaxDecodeWarps;   // the host keeps W <= kMaxDecodeWarps
+  const size_t bg = (size_t)b * Hk + g;
+  // M = the largest piece maximum
+  __shared__ float s_red[4];
+  float M = -INFINITY;
+  for (int k = threadIdx.x; k < cnt; k += blockDim.x) M = fmaxf(M, part[((bg + s_w[k]) * G + row) * (D + 2) + D]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = M;
   __syncthreads();
+  M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
+  // warp q merges pieces [cnt*q/4, cnt*(q+1)/4), lane i dims 4i .. 4i+3 (loads
+  // of consecutive lanes are contiguous); the four warps' sums are then added
+  // in warp order, so the merge order is fixed
+  static_assert(D == 128, "one 4-dim slice per lane");
+  const int q = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k0 = cnt * q / 4, k1 = cnt * (q + 1) / 4;
+  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f, L = 0.f;
+#pragma unroll 4
+  for (int k = k0; k < k1; ++k) {
+    const float* r = part + ((bg + s_w[k]) * G + row) * (D + 2);
+    const float f = exp2f(r[D] - M);
+    const float2 a = *reinterpret_cast<const float2*>(r + 4 * lane);
+    const float2 c = *reinterpret_cast<const float2*>(r + 4 * lane + 2);
+    L += r[D + 1] * f;
+    acc0 += a.x * f;
+    acc1 += a.y * f;
+    acc2 += c.x * f;
+    acc3 += c.y * f;
+  }
+  __shared__ float s_acc[4][D];
+  __shared__ float s_l[4];
+  s_acc[q][4 * lane] = acc0;
+  s_acc[q][4 * lane + 1] = acc1;
+  s_acc[q][4 * lane + 2] = acc2;
+  s_acc[q][4 * lane + 3] = acc3;
+  if (lane == 0) s_l[q] = L;
+  __syncthreads();
+  const float Lt = ((s_l[0] + s_l[1]) + s_l[2]) + s_l[3];
   for (int dd = threadIdx.x; dd < D; dd += blockDim.x) {
-    float L = 0.f, O = 0.f;
-    for (int k = 0; k < cnt; ++k) {
-      const float* r = part + ((bg + s_w[k]) * G + row) * (D + 2);
-      L += r[D + 1] * s_f[k];
-      O += r[dd] * s_f[k];
-    }
-    o[((size_t)b * H + h) * D + dd] = from_f<T>(O / L);
+    const float O = ((s_acc[0][dd] + s_acc[1][dd]) + s_acc[2][dd]) + s_acc[3][dd];
+    o[((size_t)b * H + h) * D + dd] = from_f<T>(O / Lt);
   }
 }
 
@@ -668,6 +707,7 @@ static int mma_decode_launch(const void* q, const void* kc, const void* vc, cons
                              void* o, int B, int cmax, int H, int Hk, int Smax, const KvLayout& L,
                              DecodeScratch* scratch, int* status, cudaStream_t st) {
   const int grid = num_sms();
+  if (grid * DM_WARPS > kMaxDecodeWarps) return LLAMA_ERR_UNSUPPORTED;
   auto kern = attn_decode_mma_kernel<T>;
   if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), DM_SMEM)) return rc;
   const float scale_log2 = kLog2e / sqrtf(128.f);

@@ -602,6 +602,302 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
   }
 }
 
+// ------------------------------------------------------- two CTAs per SM
+// The persistent computation with two CTAs resident on every SM, each with
+// half of the SM's TMEM (O: 128 columns, one S buffer of 128 columns whose
+// upper 64 columns take P) and single-stage Q, K and V buffers (96 KB of
+// shared memory). Inside a CTA the steps of a tile are serial (S, softmax,
+// P V, then the next S into the same buffer); the two CTAs of an SM
+// interleave, so one CTA's softmax overlaps the other's products and the
+// serial parts of the two softmaxes overlap each other. Items and their
+// snake order over 2 x SMs CTAs are those of the one-CTA persistent kernel.
+//
+// Per tile t (counted over the CTA's items): K(t) is loaded once S(t-1) has
+// read the K buffer, V(t) once P(t-1) V(t-1) has read the V buffer; S(t) is
+// issued once P(t-1) V(t-1) has completed (S overwrites the P it read); the
+// softmax threads load the row's 128 scores in two halves of 64 (registers),
+// store P over the upper half of S after both halves are loaded, and may
+// rescale O at once (the commit that signalled S(t) follows P(t-1) V(t-1)).
+// After an item's last product they read O out; the next item's first
+// product, which overwrites O, needs their next P. Every wait is bounded.
+constexpr int F2_THREADS = 192;
+constexpr int F2_OFF_Q = 0;
+constexpr int F2_OFF_K = F2_OFF_Q + FA_Q_BYTES;
+constexpr int F2_OFF_V = F2_OFF_K + FA_KV_BYTES;
+constexpr int F2_OFF_BAR = F2_OFF_V + FA_KV_BYTES;
+constexpr int F2_SMEM = F2_OFF_BAR + 256 + 1024;
+constexpr uint32_t F2_TMEM_O = 0, F2_TMEM_S = 128, F2_TMEM_P = 192;   // P: upper half of S
+
+// Softmax of one 128-key tile for this thread's row with the scores loaded
+// in two halves (fewer live registers): the upper half (keys 64-127) stays
+// in registers while the maximum is formed; O is rescaled if the running
+// maximum rises; the upper half's P is stored at once (over scores already
+// loaded), then the lower half is loaded again for its exponentials and its
+// P stored. Returns the tile's row sum; corr as for fa_tile_softmax.
+template <typename T>
+__device__ __forceinline__ float f2_tile_softmax(uint32_t s_tmem, uint32_t o_tmem, uint32_t p_tmem, bool ok,
+                                                 bool masked, int kbase, int qpos, float scale_log2, bool first,
+                                                 float& m_used, float& corr) {
+  float hi[64];
+  float mlo = -INFINITY;
+  if (ok) {
+    uint32_t u0[32], u1[32];
+    tmem_ld32_nowait(s_tmem, u0);
+    tmem_ld32_nowait(s_tmem + 32, u1);
+    tmem_ld_wait();
+    float m8[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) m8[c] = -INFINITY;
+#pragma unroll
+    for (int x = 0; x < 32; x += 8) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float a = masked && kbase + x + c > qpos ? -INFINITY : __uint_as_float(u0[x + c]);
+        const float b = masked && kbase + 32 + x + c > qpos ? -INFINITY : __uint_as_float(u1[x + c]);
+        m8[c] = fmax3(m8[c], a, b);
+      }
+    }
+    mlo = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+    tmem_ld32_nowait(s_tmem + 64, u0);
+    tmem_ld32_nowait(s_tmem + 96, u1);
+    tmem_ld_wait();
+#pragma unroll
+    for (int x = 0; x < 32; ++x) {
+      hi[x] = __uint_as_float(u0[x]);
+      hi[32 + x] = __uint_as_float(u1[x]);
+    }
+  } else {
+#pragma unroll
+    for (int x = 0; x < 64; ++x) hi[x] = 0.f;
+  }
+  if (masked) {
+#pragma unroll
+    for (int x = 0; x < 64; ++x)
+      if (kbase + 64 + x > qpos) hi[x] = -INFINITY;
+  }
+  float m8[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) m8[c] = hi[c];
+#pragma unroll
+  for (int x = 8; x < 56; x += 16) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) m8[c] = fmax3(m8[c], hi[x + c], hi[x + 8 + c]);
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) m8[c] = fmaxf(m8[c], hi[56 + c]);
+  const float mx = fmaxf(mlo, fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
+                   scale_log2;
+  corr = 1.f;
+  if (first) {
+    m_used = mx;
+  } else if (mx > m_used + FA_RESCALE) {
+    corr = fast_exp2(m_used - mx);
+    m_used = mx;
+  }
+  if (__any_sync(0xffffffffu, corr != 1.f) && ok) fa_rescale_o(o_tmem, corr);
+  float sum8[8];
+#pragma unroll
+  for (int x = 0; x < 8; ++x) sum8[x] = 0.f;
+  {
+    uint32_t pk[32];
+#pragma unroll
+    for (int x = 0; x < 32; ++x) {
+      const float a = fast_exp2(fmaf(hi[2 * x], scale_log2, -m_used));
+      const float b = fast_exp2(fmaf(hi[2 * x + 1], scale_log2, -m_used));
+      sum8[x & 7] += a + b;
+      pk[x] = pack2<T>(a, b);
+    }
+    if (ok) tmem_st32_u(p_tmem + 32, pk);        // keys 64-127: over scores 96-127, already loaded
+  }
+  if (ok) {
+    uint32_t u0[32], u1[32], pk[32];
+    tmem_ld32_nowait(s_tmem, u0);
+    tmem_ld32_nowait(s_tmem + 32, u1);
+    tmem_ld_wait();
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+      float a = __uint_as_float(u0[2 * x]), b = __uint_as_float(u0[2 * x + 1]);
+      if (masked && kbase + 2 * x > qpos) a = -INFINITY;
+      if (masked && kbase + 2 * x + 1 > qpos) b = -INFINITY;
+      a = fast_exp2(fmaf(a, scale_log2, -m_used));
+      b = fast_exp2(fmaf(b, scale_log2, -m_used));
+      sum8[x & 7] += a + b;
+      pk[x] = pack2<T>(a, b);
+      float c = __uint_as_float(u1[2 * x]), d = __uint_as_float(u1[2 * x + 1]);
+      if (masked && kbase + 32 + 2 * x > qpos) c = -INFINITY;
+      if (masked && kbase + 33 + 2 * x > qpos) d = -INFINITY;
+      c = fast_exp2(fmaf(c, scale_log2, -m_used));
+      d = fast_exp2(fmaf(d, scale_log2, -m_used));
+      sum8[(x + 4) & 7] += c + d;
+      pk[16 + x] = pack2<T>(c, d);
+    }
+    tmem_st32_u(p_tmem, pk);                    // keys 0-63: over scores 64-95, already loaded
+  }
+  tmem_st_wait();
+  return ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+}
+
+template <typename T>
+__global__ void __launch_bounds__(F2_THREADS, 2)
+    attn_prefill_tc_2cta_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                                const __grid_constant__ CUtensorMap tmV, T* __restrict__ o,
+                                const int32_t* __restrict__ pos0, int B, int S, int H, int Hk, float scale_log2,
+                                const int32_t* __restrict__ kv_table, int kv_max_pages, int kv_pages, int* status) {
+  extern __shared__ uint8_t fa_smem_raw[];
+  uint8_t* smem = fa_align(fa_smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + F2_OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;    // the item's last S = Q K^T has read Q
+  uint64_t* k_full = bars + 2;
+  uint64_t* k_empty = bars + 3;    // S has read K
+  uint64_t* v_full = bars + 4;
+  uint64_t* v_empty = bars + 5;    // P V has read V
+  uint64_t* s_full = bars + 6;     // S written (and every earlier product complete)
+  uint64_t* p_full = bars + 7;     // softmax threads stored P (128 arrivals)
+  uint64_t* o_done = bars + 8;     // P V complete
+  uint64_t* drain = bars + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total = ((S + FA_BM - 1) / FA_BM) * H * B;
+  const int c = blockIdx.x, G = gridDim.x;
+
+  pdl_trigger();
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1); mbar_init(q_empty, 1);
+    mbar_init(k_full, 1); mbar_init(k_empty, 1);
+    mbar_init(v_full, 1); mbar_init(v_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    int t = 0, q_issued = 0, k_issued = 0, v_issued = 0;
+    bool ok = true;
+    for (int i = 0; ok; ++i) {
+      const int w = fp_item(c, G, i);
+      if (w >= total) break;
+      const FpItem it = fp_decode(w, S, H, Hk, B, pos0);
+      if (i > 0 && !(ok = mbar_wait(q_empty, (i - 1) & 1, status))) break;
+      mbar_arrive_expect_tx(q_full, FA_Q_BYTES);
+      tma_load_3d(smem + F2_OFF_Q, &tmQ, q_full, 0, it.q0, it.b * H + it.h);
+      tma_load_3d(smem + F2_OFF_Q + FA_HALF, &tmQ, q_full, 64, it.q0, it.b * H + it.h);
+      ++q_issued;
+      for (int j = 0; j < it.n_kt; ++j, ++t) {
+        const int kv_y = kv_table ? 0 : j * FA_BN;
+        const int kv_z = kv_table ? kv_page(kv_table, kv_max_pages, kv_pages, it.b, j) * Hk + it.g : it.b * Hk + it.g;
+        if (t > 0 && !(ok = mbar_wait(k_empty, (t - 1) & 1, status))) break;
+        mbar_arrive_expect_tx(k_full, FA_KV_BYTES);
+        tma_load_3d(smem + F2_OFF_K, &tmK, k_full, 0, kv_y, kv_z);
+        tma_load_3d(smem + F2_OFF_K + FA_HALF, &tmK, k_full, 64, kv_y, kv_z);
+        ++k_issued;
+        if (t > 0 && !(ok = mbar_wait(v_empty, (t - 1) & 1, status))) break;
+        mbar_arrive_expect_tx(v_full, FA_KV_BYTES);
+        tma_load_3d(smem + F2_OFF_V, &tmV, v_full, 0, kv_y, kv_z);
+        tma_load_3d(smem + F2_OFF_V + FA_HALF, &tmV, v_full, 64, kv_y, kv_z);
+        ++v_issued;
+      }
+    }
+    if (!ok) {  // let issued copies land before the CTA can exit
+      if (q_issued > 0) mbar_wait(q_full, (q_issued - 1) & 1, status);
+      if (k_issued > 0) mbar_wait(k_full, (k_issued - 1) & 1, status);
+      if (v_issued > 0) mbar_wait(v_full, (v_issued - 1) & 1, status);
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc_s = umma_idesc_16(UmmaFmt<T>::value, FA_BM, FA_BN, false);
+    constexpr uint32_t idesc_o = umma_idesc_16(UmmaFmt<T>::value, FA_BM, FA_D, true);
+    const uint32_t q_addr = smem_u32(smem + F2_OFF_Q);
+    const uint32_t k_addr = smem_u32(smem + F2_OFF_K);
+    const uint32_t v_addr = smem_u32(smem + F2_OFF_V);
+    bool ok = true, any = false;
+    int t = 0;
+    for (int i = 0; ok; ++i) {
+      const int w = fp_item(c, G, i);
+      if (w >= total) break;
+      const int n_kt = fp_decode(w, S, H, Hk, B, pos0).n_kt;
+      if (!(ok = mbar_wait(q_full, i & 1, status))) break;
+      for (int j = 0; j < n_kt; ++j, ++t) {
+        // S overwrites the P that the previous product read: that product first
+        if (t > 0 && !(ok = mbar_wait(o_done, (t - 1) & 1, status))) break;
+        if (!(ok = mbar_wait(k_full, t & 1, status))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < FA_D / 16; ++ks) {
+          const uint32_t off = (uint32_t)(ks >> 2) * FA_HALF + (uint32_t)(ks & 3) * 32;
+          umma_bf16(tmem + F2_TMEM_S, umma_desc_sw128(q_addr + off), umma_desc_sw128(k_addr + off), idesc_s, ks != 0);
+        }
+        umma_commit(s_full);
+        umma_commit(k_empty);
+        if (j + 1 == n_kt) umma_commit(q_empty);
+        any = true;
+        if (!(ok = mbar_wait(p_full, t & 1, status))) break;
+        if (!(ok = mbar_wait(v_full, t & 1, status))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < FA_BN / 16; ++ks)
+          umma_ts(tmem + F2_TMEM_O, tmem + F2_TMEM_P + ks * 8, umma_desc_sw128_mn(v_addr + ks * 2048, FA_HALF), idesc_o,
+                  (j | ks) != 0);
+        umma_commit(v_empty);
+        umma_commit(o_done);
+      }
+    }
+    if (!ok && any) {
+      umma_commit(drain);
+      mbar_wait(drain, 0, status);
+    }
+  } else if (warp >= 2) {
+    const int quarter = warp & 3;                       // TMEM lanes this warp may read
+    const int r = quarter * 32 + lane;                  // query row in the tile
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    bool ok = true;
+    int t = 0;
+    for (int i = 0;; ++i) {
+      const int w = fp_item(c, G, i);
+      if (w >= total) break;
+      const FpItem it = fp_decode(w, S, H, Hk, B, pos0);
+      const int qpos = it.p0 + it.q0 + r;
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < it.n_kt; ++j, ++t) {
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full, t & 1, status));
+        tc_fence_after();
+        // O is complete up to the previous product (its commit came before S's),
+        // so the softmax may rescale it at once
+        float corr;
+        const float rowsum = f2_tile_softmax<T>(tmem + lane_off + F2_TMEM_S, tmem + lane_off + F2_TMEM_O,
+                                                tmem + lane_off + F2_TMEM_P, ok, j * FA_BN + FA_BN - 1 > it.p0 + it.q0,
+                                                j * FA_BN, qpos, scale_log2, j == 0, m_used, corr);
+        l = l * corr + rowsum;
+        tc_fence_before();
+        mbar_arrive(p_full);
+      }
+      if (it.n_kt > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (t - 1) & 1, status));
+      tc_fence_after();
+      const int qi = it.q0 + r;
+      T* dst = o + ((size_t)it.b * S + (qi < S ? qi : 0)) * H * FA_D + (size_t)it.h * FA_D;
+      fa_store_o<T>(tmem + lane_off + F2_TMEM_O, ok, 1.f / l, dst, qi < S);
+      tc_fence_before();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
 // [outer][rows][128] 16-bit -> 3-D map with boxes of 64 x 128 x 1, 128-byte swizzle.
 int make_tmap_3d(CUtensorMap* map, const void* base, int64_t outer, int64_t rows, bool is_f16) {
   static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
@@ -650,6 +946,16 @@ static int attention_prefill_tc_t(const void* q, const void* kc, const void* vc,
   // CTA's fixed cost is small against its key loop. LLAMA_ATTN_PER_TILE
   // selects the per-tile kernel for every length.
   static const bool per_tile = getenv("LLAMA_ATTN_PER_TILE") != nullptr;
+  static const bool two_cta = getenv("LLAMA_ATTN_2CTA") != nullptr;
+  if (two_cta) {
+    auto kern = attn_prefill_tc_2cta_kernel<T>;
+    if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), F2_SMEM)) return rc;
+    const long long items = (long long)((S + FA_BM - 1) / FA_BM) * H * B;
+    const int grid = (int)std::min<long long>(items, 2LL * num_sms());
+    const cudaError_t err = launch_k(kern, dim3(grid), dim3(F2_THREADS), F2_SMEM, st, tq, tk, tv, static_cast<T*>(o),
+                                     pos0, B, S, H, Hk, scale_log2, kv_table, kv_max_pages, kv_pages, status);
+    return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
+  }
   if (!per_tile && S <= kPersistentMaxS) {
     auto kern = attn_prefill_tc_persistent_kernel<T>;
     if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), FP_SMEM)) return rc;

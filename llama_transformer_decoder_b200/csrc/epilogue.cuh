@@ -45,17 +45,24 @@ struct EpiArgs {
   // Status word for LLAMA_ERR_RANGE: a 16-bit output (q/k/v, the SwiGLU
   // product, y = x * g) that is not finite after rounding (nullptr: unchecked).
   int* status;
-  // Row-block readiness between consecutive CTA-pair GEMMs (prefill). With
-  // ready_out, every CTA adds 1 to ready_out[r] after its epilogue has written
-  // the 128 rows r*128 .. r*128+127 of an output tile. With ready_in, the
-  // kernel does not wait for the previous kernel to finish: before reading
-  // rows of block r it waits (bounded) until ready_in[r] >= ready_target.
-  // Tiles are taken in groups of m_group 256-row blocks (column by column
-  // inside a group), so the first groups' rows are complete early.
-  int* ready_out;
-  const int* ready_in;
-  int ready_target;
-  int m_group;
+};
+
+// One GEMM of a chain of CTA-pair GEMMs run by one persistent launch
+// (gemm16_chain): acc = A W^T with A [M][K] (row pitch lda), W [N][K] (ldw),
+// epilogue `kind` with `epi`. Tiles are taken in groups of m_group 256-row
+// blocks (column by column inside a group; 0 = all blocks in one group).
+// With `ready`, every CTA adds 1 to ready[r] once it has written the 128
+// output rows r*128 .. r*128+127 of a tile (zero before the launch). A job
+// with dep = d reads rows that job d writes: before touching rows of block r
+// it waits until job d has published all of its column tiles of r.
+struct ChainJobDesc {
+  const void* A;
+  int lda;
+  const void* W;
+  int ldw;
+  int M, N, K, kind, m_group, dep;
+  int* ready;
+  EpiArgs epi;
 };
 
 // r of row m from its partial sums of squares (added in a fixed order).

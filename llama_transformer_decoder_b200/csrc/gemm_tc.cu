@@ -25,6 +25,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstring>
 #include <cstdlib>
 #include <mutex>
 #include <type_traits>
@@ -331,10 +332,50 @@ __device__ __forceinline__ void pair_tile(int t, int m_tiles, int G, int& m, int
   m = m0 + (r - n * gm);
 }
 
+// A chain runs up to kMaxJobs CTA-pair GEMMs in one persistent launch (one
+// layer's Wo, w1/w3, w2 and the next layer's QKV projections). The tiles of all
+// jobs form one list, job after job, each job's tiles in its own order
+// (pair_tile with its m_group); pair p takes positions p, p + pairs, ... in
+// order. A job may read rows another job of the chain writes (dep): before
+// reading the 128 rows of block r of its A operand, and before its epilogue
+// touches rows of r, a CTA waits (bounded) until the dep job has published
+// all of its tiles of r (ready counter == the dep job's column tiles). A tile
+// only waits for tiles earlier in the list, every pair handles its
+// positions in order, and all pairs are resident at once, so every wait ends.
+// The first job reads what earlier kernels wrote (programmatic dependent
+// launch: its weight tiles are requested before griddepcontrol.wait).
+constexpr int kMaxJobs = 4;
+struct ChainJob {
+  int M, N, K, kind, m_group;
+  int m_tiles, n_tiles, kb, G, tile0;  // tile0: first list position of the job
+  int dep;                             // job whose output rows it reads (-1: none)
+  int* ready;                          // per-128-row counters this job publishes (nullptr: none)
+  EpiArgs epi;
+};
+struct ChainArgs {
+  CUtensorMap tmA[kMaxJobs];
+  CUtensorMap tmB[kMaxJobs];
+  ChainJob job[kMaxJobs];
+  int n_jobs, total;
+};
+
+// List position t -> job j, 256-row block m and 256-column block n.
+__device__ __forceinline__ int chain_tile(const ChainArgs& c, int t, int& m, int& n) {
+  int j = 0;
+  while (j + 1 < c.n_jobs && t >= c.job[j + 1].tile0) ++j;
+  const ChainJob& J = c.job[j];
+  pair_tile(t - J.tile0, J.m_tiles, J.G, m, n, J.n_tiles);
+  return j;
+}
+
 template <int KIND, typename T>
+__device__ __forceinline__ float chain_epi_row32(const EpiArgs& e, int m, int n0, const float (&v)[32], float rs) {
+  return epi_row32<KIND, T>(e, m, n0, v, rs);
+}
+
+template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
-                     int K, EpiArgs epi, int* status) {
+    gemm_chain_kernel(const __grid_constant__ ChainArgs args, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES);
@@ -348,9 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, pairs = gridDim.x >> 1;
-  const int m_tiles = (M + 2 * P_BM - 1) / (2 * P_BM), n_tiles = (N + P_BN - 1) / P_BN;
-  const int tiles = m_tiles * n_tiles;
-  const int kb = (K + BK - 1) / BK;
+  const int tiles = args.total;
 
   pdl_trigger();
   if (threadIdx.x == 0) {
@@ -365,56 +404,65 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int G = epi.m_group > 0 ? min(epi.m_group, m_tiles) : m_tiles;
+  // rows of block mb of job j's A operand (and output) are complete in its dep job
+  auto rows_ready = [&](int j, int mb) -> bool {
+    const int d = args.job[j].dep;
+    if (d < 0) return true;
+    return counter_wait_geq(args.job[d].ready + 2 * mb + (int)rank, args.job[d].n_tiles, status);
+  };
+
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-    const uint64_t pol_a = l2_policy_evict_last(), pol_b = l2_policy_evict_last();
-    const int first = pair < tiles ? pair : -1;
-    const int pre = first >= 0 ? (kb < P_STAGES ? kb : P_STAGES) : 0;
-    // this CTA's 128 rows of tile t may be read once the previous kernel (or
-    // only its tiles of those rows, with ready_in) has written them
-    auto rows_ready = [&](int mb) -> bool {
-      if (!epi.ready_in) return true;
-      const bool r = counter_wait_geq(epi.ready_in + 2 * mb + (int)rank, epi.ready_target, status);
-      fence_proxy_async_global();
-      return r;
-    };
-    bool ok = true;
-    {  // weight halves of the first stages before waiting for the previous kernel
-      int fm = 0, fn = 0;
-      if (first >= 0) pair_tile(first, m_tiles, G, fm, fn, n_tiles);
-      const int n0 = fn * P_BN + (int)rank * (P_BN / 2);
-      for (int k = 0; k < pre; ++k) {
-        if (leader) mbar_arrive_expect_tx(&full[k], 2 * P_STAGE_BYTES);
-        tma_load_2d_pair(smem + k * P_STAGE_BYTES + P_A_BYTES, &tmB, mapa_shared(smem_u32(&full[k]), 0), k * BK, n0,
-                         pol_b);
-      }
-      if (!epi.ready_in) pdl_wait();
-      else if (first >= 0) ok = rows_ready(fm);
-      const int m0 = fm * 2 * P_BM + (int)rank * P_BM;
-      for (int k = 0; k < pre; ++k)   // issued even after a failed wait: the barriers expect these bytes
-        tma_load_2d_pair(smem + k * P_STAGE_BYTES, &tmA, mapa_shared(smem_u32(&full[k]), 0), k * BK, m0, pol_a);
+    for (int j = 0; j < args.n_jobs; ++j) {
+      tma_prefetch_desc(&args.tmA[j]);
+      tma_prefetch_desc(&args.tmB[j]);
     }
-    int stage = pre % P_STAGES, issued = pre;
-    uint32_t phase = pre == P_STAGES ? 1u : 0u;
+    const uint64_t pol_a = l2_policy_evict_last(), pol_b = l2_policy_evict_last();
+    int stage = 0, issued = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    bool waited = false;   // griddepcontrol.wait done (before the first A operand)
     for (int t = pair; t < tiles && ok; t += pairs) {
       int tm, tn;
-      pair_tile(t, m_tiles, G, tm, tn, n_tiles);
-      if (t != pair && !(ok = rows_ready(tm))) break;
+      const int j = chain_tile(args, t, tm, tn);
+      const ChainJob& J = args.job[j];
+      const CUtensorMap* ta = &args.tmA[j];
+      const CUtensorMap* tb = &args.tmB[j];
       const int m0 = tm * 2 * P_BM + (int)rank * P_BM;
       const int n0 = tn * P_BN + (int)rank * (P_BN / 2);
-      for (int k = (t == pair ? pre : 0); k < kb; ++k) {
+      int k = 0;
+      if (!waited) {  // weight halves of the first stages before waiting for the previous kernel
+        const int pre = J.kb < P_STAGES ? J.kb : P_STAGES;
+        for (; k < pre; ++k) {
+          if (leader) mbar_arrive_expect_tx(&full[k], 2 * P_STAGE_BYTES);
+          tma_load_2d_pair(smem + k * P_STAGE_BYTES + P_A_BYTES, tb, mapa_shared(smem_u32(&full[k]), 0), k * BK, n0,
+                           pol_b);
+        }
+        pdl_wait();
+        waited = true;
+        ok = rows_ready(j, tm);
+        fence_proxy_async_global();
+        for (int kk = 0; kk < pre; ++kk)   // issued even after a failed wait: the barriers expect these bytes
+          tma_load_2d_pair(smem + kk * P_STAGE_BYTES, ta, mapa_shared(smem_u32(&full[kk]), 0), kk * BK, m0, pol_a);
+        issued = pre;
+        stage = pre % P_STAGES;
+        phase = pre == P_STAGES ? 1u : 0u;
+        if (!ok) break;
+      } else {
+        if (!(ok = rows_ready(j, tm))) break;
+        fence_proxy_async_global();
+      }
+      for (; k < J.kb; ++k) {
         if (!mbar_wait(&empty[stage], phase ^ 1, status)) { ok = false; break; }
         uint8_t* sa = smem + stage * P_STAGE_BYTES;
         const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
         if (leader) mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
-        tma_load_2d_pair(sa, &tmA, fb, k * BK, m0, pol_a);
-        tma_load_2d_pair(sa + P_A_BYTES, &tmB, fb, k * BK, n0, pol_b);
+        tma_load_2d_pair(sa, ta, fb, k * BK, m0, pol_a);
+        tma_load_2d_pair(sa + P_A_BYTES, tb, fb, k * BK, n0, pol_b);
         ++issued;
         if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
       }
     }
+    if (!waited) pdl_wait();
     if (!ok && leader) drain_loads(full, stage, phase, issued, P_STAGES, status);
   } else if (warp == 1 && lane == 0 && leader) {
     constexpr uint32_t idesc = umma_idesc_16(UmmaFmt<T>::value, 2 * P_BM, P_BN);
@@ -422,6 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0, acc_phase = 0;
     bool ok = true, any = false;
     for (int t = pair; t < tiles && ok; t += pairs) {
+      int tm, tn;
+      const int kb = args.job[chain_tile(args, t, tm, tn)].kb;
       if (!mbar_wait_cluster(&acce[acc], acc_phase ^ 1, status)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem + acc * P_BN;
@@ -447,9 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(drain, 0, status);
     }
   } else if (warp >= 2) {
-    // The epilogue reads and writes memory owned by earlier kernels: all of
-    // the previous kernel's output, or (ready_in) the rows of the tile.
-    if (!epi.ready_in) pdl_wait();
+    pdl_wait();  // the epilogue reads and writes memory owned by earlier kernels
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     int acc = 0;
@@ -457,14 +505,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool failed = false;  // after a timed-out wait the MMA has stopped: no further waits
     for (int t = pair; t < tiles; t += pairs) {
       int tm, tn;
-      pair_tile(t, m_tiles, G, tm, tn, n_tiles);
+      const int j = chain_tile(args, t, tm, tn);
+      const ChainJob& J = args.job[j];
+      const EpiArgs& epi = J.epi;
       const int m0 = tm * 2 * P_BM + (int)rank * P_BM, n0 = tn * P_BN;
       if (!failed) failed = !__all_sync(0xffffffffu, mbar_wait(&accf[acc], acc_phase, status));
-      if (!failed && epi.ready_in)   // already complete (the producer warp waited): acquires its rows' writes
-        failed = !__all_sync(0xffffffffu, counter_wait_geq(epi.ready_in + 2 * tm + (int)rank, epi.ready_target, status));
+      // already complete (the producer warp waited for it): acquires those rows' writes for this thread
+      if (!failed && J.dep >= 0) failed = !__all_sync(0xffffffffu, rows_ready(j, tm));
       tc_fence_after();
       const uint32_t base = tmem + ((uint32_t)(quarter * 32) << 16) + acc * P_BN;
-      const float rs = (KIND == EPI_QKV_ROPE || KIND == EPI_SWIGLU) && epi.ss_in && m0 + row < M
+      const int kind = J.kind;
+      const float rs = (kind == EPI_QKV_ROPE || kind == EPI_SWIGLU) && epi.ss_in && m0 + row < J.M
                            ? norm_row_scale(epi, m0 + row) : 1.f;
       float ssq = 0.f;
 #pragma unroll 1
@@ -472,18 +523,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         float v[32];
         if (!failed) {
           tmem_ld32(base + c * 32, v);
-          if (n0 + c * 32 < N) ssq += epi_row32<KIND, T>(epi, m0 + row, n0 + c * 32, v, rs);
+          if (n0 + c * 32 < J.N) {
+            switch (kind) {
+              case EPI_STORE_F32: ssq += chain_epi_row32<EPI_STORE_F32, T>(epi, m0 + row, n0 + c * 32, v, rs); break;
+              case EPI_RESIDUAL: ssq += chain_epi_row32<EPI_RESIDUAL, T>(epi, m0 + row, n0 + c * 32, v, rs); break;
+              case EPI_SWIGLU: ssq += chain_epi_row32<EPI_SWIGLU, T>(epi, m0 + row, n0 + c * 32, v, rs); break;
+              default: ssq += chain_epi_row32<EPI_QKV_ROPE, T>(epi, m0 + row, n0 + c * 32, v, rs); break;
+            }
+          }
         }
       }
-      if (KIND == EPI_RESIDUAL && epi.ss_out && m0 + row < M) epi.ss_out[(size_t)(m0 + row) * epi.ss_n + n0 / P_BN] = ssq;
+      if (kind == EPI_RESIDUAL && epi.ss_out && m0 + row < J.M) epi.ss_out[(size_t)(m0 + row) * epi.ss_n + n0 / P_BN] = ssq;
       tc_fence_before();
       mbar_arrive_cluster(mapa_shared(smem_u32(&acce[acc]), 0));
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
-      if (epi.ready_out) {   // this CTA's 128 rows of the tile are written: publish them
+      if (J.ready) {   // this CTA's 128 rows of the tile are written: publish them
         named_bar_sync(1, 128);
         if (warp == 2 && lane == 0) {
           __threadfence();
-          atomicAdd(epi.ready_out + 2 * tm + (int)rank, 1);
+          atomicAdd(J.ready + 2 * tm + (int)rank, 1);
         }
       }
     }
@@ -898,13 +956,40 @@ bool pair_gemm_enabled() {
 
 bool gemm16_uses_pair(int M, int N, int K) { return M > 128 && pair_gemm_enabled() && wide_split(M, N, K).sk_tiles == 0; }
 
-template <int KIND, typename T>
-static int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, int M, int N, int K, const EpiArgs& e,
-                       int* status, cudaStream_t st) {
-  auto kern = gemm_pair_kernel<KIND, T>;
+// One persistent launch of the CTA-pair kernel over the jobs' tiles.
+template <typename T>
+static int launch_chain(const ChainJobDesc* jobs, int n, int* status, cudaStream_t st) {
+  constexpr bool F16 = std::is_same<T, f16>::value;
+  if (n <= 0 || n > kMaxJobs) return LLAMA_ERR_INVALID_ARG;
+  ChainArgs args;
+  memset(&args, 0, sizeof(args));
+  int total = 0;
+  for (int j = 0; j < n; ++j) {
+    const ChainJobDesc& d = jobs[j];
+    if (d.M <= 0 || d.N <= 0 || d.K <= 0) return LLAMA_ERR_SHAPE;
+    if (d.K % 8 != 0 || d.lda % 8 != 0 || d.ldw % 8 != 0) return LLAMA_ERR_SHAPE;
+    if (d.dep >= j || (d.dep >= 0 && !jobs[d.dep].ready)) return LLAMA_ERR_INVALID_ARG;
+    int rc;
+    if ((rc = make_tmap_16(&args.tmA[j], d.A, d.M, d.K, d.lda, P_BM, F16)) != LLAMA_OK) return rc;
+    if ((rc = make_tmap_16(&args.tmB[j], d.W, d.N, d.K, d.ldw, P_BN / 2, F16)) != LLAMA_OK) return rc;
+    ChainJob& J = args.job[j];
+    J.M = d.M; J.N = d.N; J.K = d.K; J.kind = d.kind;
+    J.m_tiles = (d.M + 2 * P_BM - 1) / (2 * P_BM);
+    J.n_tiles = (d.N + P_BN - 1) / P_BN;
+    J.kb = (d.K + BK - 1) / BK;
+    J.G = d.m_group > 0 ? std::min(d.m_group, J.m_tiles) : J.m_tiles;
+    J.m_group = J.G;
+    J.tile0 = total;
+    J.dep = d.dep;
+    J.ready = d.ready;
+    J.epi = d.epi;
+    total += J.m_tiles * J.n_tiles;
+  }
+  args.n_jobs = n;
+  args.total = total;
+  auto kern = gemm_chain_kernel<T>;
   if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), P_SMEM)) return rc;
-  const int tiles = ((M + 2 * P_BM - 1) / (2 * P_BM)) * ((N + P_BN - 1) / P_BN);
-  const int pairs = std::min(tiles, num_sms() / 2);
+  const int pairs = std::min(total, num_sms() / 2);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
   cfg.blockDim = dim3(kThreads);
@@ -920,7 +1005,7 @@ static int launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, int M, int 
   cfg.attrs = at;
   cfg.numAttrs = pdl_enabled() ? 2 : 1;
   count_launches(1);
-  const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, ta, tb, M, N, K, e, status);
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, args, status);
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
@@ -971,16 +1056,10 @@ static int gemm16_t(const void* A, int M, int K, int lda, const void* W, int N, 
   if (!skinny) {
     CUtensorMap ta, tb;
     if (gemm16_uses_pair(M, N, K)) {
-      // at least one full wave of 128x256 tiles: CTA pairs on 256x256 tiles
-      if ((rc = make_tmap_16(&ta, A, M, K, lda, P_BM, F16)) != LLAMA_OK) return rc;
-      if ((rc = make_tmap_16(&tb, W, N, K, ldw, P_BN / 2, F16)) != LLAMA_OK) return rc;
-      switch (kind) {
-        case EPI_STORE_F32: return launch_pair<EPI_STORE_F32, T>(ta, tb, M, N, K, e, status, st);
-        case EPI_RESIDUAL: return launch_pair<EPI_RESIDUAL, T>(ta, tb, M, N, K, e, status, st);
-        case EPI_SWIGLU: return launch_pair<EPI_SWIGLU, T>(ta, tb, M, N, K, e, status, st);
-        case EPI_QKV_ROPE: return launch_pair<EPI_QKV_ROPE, T>(ta, tb, M, N, K, e, status, st);
-      }
-      return LLAMA_ERR_INVALID_ARG;
+      // at least one full wave of 128x256 tiles: CTA pairs on 256x256 tiles (a chain of one job)
+      if (kind < EPI_STORE_F32 || kind > EPI_QKV_ROPE) return LLAMA_ERR_INVALID_ARG;
+      ChainJobDesc d{A, lda, W, ldw, M, N, K, kind, 0, -1, nullptr, e};
+      return launch_chain<T>(&d, 1, status, st);
     }
     if ((rc = make_tmap_16(&ta, A, M, K, lda, W_BM, F16)) != LLAMA_OK) return rc;
     if ((rc = make_tmap_16(&tb, W, N, K, ldw, W_BN, F16)) != LLAMA_OK) return rc;
@@ -1009,6 +1088,14 @@ static int gemm16_t(const void* A, int M, int K, int lda, const void* W, int N, 
     case EPI_SWIGLU: return launch_skinny<EPI_SWIGLU, T>(tw, tx, M, N, K, NT, e, ws, tk, status, st);
     case EPI_QKV_ROPE: return launch_skinny<EPI_QKV_ROPE, T>(tw, tx, M, N, K, NT, e, ws, tk, status, st);
   }
+  return LLAMA_ERR_INVALID_ARG;
+}
+
+int gemm16_chain(const ChainJobDesc* jobs, int n, int elt, int* status, cudaStream_t st) {
+  for (int j = 0; j < n; ++j)
+    if (!gemm16_uses_pair(jobs[j].M, jobs[j].N, jobs[j].K)) return LLAMA_ERR_UNSUPPORTED;
+  if (elt == LLAMA_F16) return launch_chain<f16>(jobs, n, status, st);
+  if (elt == LLAMA_BF16) return launch_chain<bf16>(jobs, n, status, st);
   return LLAMA_ERR_INVALID_ARG;
 }
 

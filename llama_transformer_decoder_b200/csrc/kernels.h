@@ -11,6 +11,7 @@ namespace llama {
 
 struct EpiArgs;
 struct KvLayout;
+struct ChainJobDesc;
 
 // Launch with programmatic stream serialization (the kernel must call
 // pdl_wait() before reading its predecessor's output). Disabled when the
@@ -69,9 +70,12 @@ int make_tmap_16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
 // Scratch of the stream-K skinny GEMM for M rows: two partial tiles per CTA.
 size_t skinny_workspace_floats(int M);
 
-// True when an automatic 16-bit GEMM of this shape runs the CTA-pair kernel
-// (the only one that honours EpiArgs::ready_in / ready_out / m_group).
+// True when an automatic 16-bit GEMM of this shape runs the CTA-pair kernel.
 bool gemm16_uses_pair(int M, int N, int K);
+// Up to four CTA-pair GEMMs (each gemm16_uses_pair) in one persistent launch,
+// later jobs waiting only for the row blocks of earlier jobs they read (see
+// ChainJobDesc in epilogue.cuh). elt = LLAMA_BF16 or LLAMA_F16.
+int gemm16_chain(const ChainJobDesc* jobs, int n, int elt, int* status, cudaStream_t st);
 // 16-bit GEMM; elt = LLAMA_BF16 or LLAMA_F16 (element type of A, W and 16-bit outputs).
 int gemm16(const void* A, int M, int K, int lda, const void* W, int N, int ldw, int elt, int kind, const EpiArgs& e,
            int variant, GemmScratch* scratch, int* status, cudaStream_t st);

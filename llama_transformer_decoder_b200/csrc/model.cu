@@ -93,13 +93,13 @@ struct llama_model {
   // workspace
   float* ss = nullptr;        // [max_tokens][ceil(dim/256)] partial sums of squares (folded RMSNorm)
   bool norm_ready = false;    // xn / ss already hold the next layer's attention-norm inputs
-  // Row-block readiness counters of the prefill GEMMs (16-bit models): per
-  // layer three sets (Wo, w1/w3, w2 outputs) of one counter per 128 rows,
-  // zeroed at the start of every prefill step. last_signal_layer: layer whose
-  // w2 GEMM published its rows last (-1: the last GEMM published nothing).
+  // Row-block readiness counters of the chained prefill GEMMs (16-bit
+  // models): per layer three sets (Wo, w1/w3, w2 outputs) of one counter per
+  // 128 rows, zeroed at the start of every prefill step. qkv_ready_layer: the
+  // layer whose QKV projection the previous chain already ran (-1: none).
   int* ready = nullptr;
   int ready_rb = 0;
-  int last_signal_layer = -1;
+  int qkv_ready_layer = -1;
   float* x = nullptr;
   void* xn = nullptr;
   void* q = nullptr;
@@ -303,10 +303,10 @@ int grow_decode_scratch(DecodeScratch* ds, size_t floats) {
 
 // ------------------------------------------------------------ profiling
 enum ProfKind { K_EMBED = 0, K_RMSNORM, K_GEMM_QKV, K_ATTN_PREFILL, K_ATTN_DECODE, K_GEMM_WO, K_GEMM_W13, K_GEMM_W2,
-                K_GEMM_LMHEAD, K_OTHER, K_END, K_COUNT };
+                K_GEMM_LMHEAD, K_OTHER, K_GEMM_CHAIN, K_END, K_COUNT };
 const char* kProfNames[K_COUNT] = {"embed", "rmsnorm", "gemm_qkv_rope", "attention_prefill", "attention_decode",
                                    "gemm_wo_residual", "gemm_w13_swiglu", "gemm_w2_residual", "gemm_lm_head",
-                                   "other", "end"};
+                                   "other", "gemm_chain", "end"};
 std::atomic<unsigned long long> g_launches{0};
 
 void mark(llama_model* m, int kind, cudaStream_t st) {
@@ -343,48 +343,28 @@ EpiArgs epi_base(int M, int N, int* status = nullptr) {
 // One decoder block on m->x ([M][D], M = B*S) for sequences 0..B-1 whose
 // first new token sits at position d_len[b]. decode: S == 1 and attention
 // reads keys 0..d_len[b] through the split-K kernel.
-int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaStream_t st) {
+//
+// Prefill-sized GEMMs (M > 128) fold the RMSNorms in: the residual GEMMs'
+// epilogues leave y = x * g and per-tile sums of squares for the next norm,
+// and the QKV / w1-w3 epilogues scale by rsqrt(mean(x^2) + eps). When all
+// four projections run on the CTA-pair kernel, the layer's Wo, w1/w3 and w2
+// and the next layer's QKV run as one chained launch (gemm16_chain): each
+// projection's tiles wait only for the 128-row blocks of the previous one
+// they read, so the partial last waves of one projection fill with the next
+// one's tiles and three launches per layer disappear. The next layer then
+// starts at its attention.
+int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaStream_t st, bool alone = false) {
   const llama_config& c = m->cfg;
   const int D = c.dim, H = c.n_heads, Hk = c.n_kv_heads, d = m->d, M = B * S;
   const LayerW& w = m->L[l];
   char* kc = static_cast<char*>(m->kcache) + (size_t)l * m->layer_cache_elems * m->esz;
   char* vc = static_cast<char*>(m->vcache) + (size_t)l * m->layer_cache_elems * m->esz;
 
-  // Prefill-sized GEMMs (M > 128) fold the RMSNorms in: the residual GEMMs'
-  // epilogues leave y = x * g and per-tile sums of squares for the next norm,
-  // and the QKV / w1-w3 epilogues scale by rsqrt(mean(x^2) + eps).
   const bool fuse = m->adt != LLAMA_F32 && M > 128;
   const int ss_n = (D + 255) / 256;
-  // QKV directly after the previous layer's w2 that published its row blocks
-  const bool after_w2 = fuse && m->norm_ready && m->last_signal_layer == l - 1 && l > 0;
-  if (fuse) {
-    if (!m->norm_ready) {
-      mark(m, K_RMSNORM, st);
-      RC(launch_norm_prep(m->x, w.attn_norm, m->xn, m->ss, M, D, ss_n, m->adt, st, m->d_status));
-    }
-  } else {
-    mark(m, K_RMSNORM, st);
-    RC(launch_rmsnorm(m->x, w.attn_norm, m->xn, M, D, c.norm_eps, 0, m->adt, st, m->d_status));
-  }
-  m->norm_ready = false;
-  m->last_signal_layer = -1;
-  // Consecutive CTA-pair GEMMs overlap: a producer publishes each 128-row
-  // block of its output (ready_out), and its consumer, launched early, waits
-  // only for the blocks it reads (ready_in) instead of the whole kernel, so
-  // the consumer's first tiles run on the SMs the producer's last, partial
-  // wave leaves idle. Producers whose consumer follows take their tiles in
-  // row-block order (m_group 1: early blocks complete early); w1/w3 keeps two
-  // groups so its 235 MB of weights are streamed twice, not once per block.
-  const bool ov = fuse && m->ready != nullptr;
-  const int m_tiles = (M + 255) / 256;
-  auto ready_set = [&](int layer, int which) { return m->ready + ((size_t)layer * 3 + which) * m->ready_rb; };
-  auto link = [&](EpiArgs& a, int* in_set, bool producer_pair, int producer_n, bool consumer_pair) {
-    if (!ov || !in_set || !producer_pair || !consumer_pair) return;
-    a.ready_in = in_set;
-    a.ready_target = (producer_n + 255) / 256;
-  };
-  const bool qkv_pair = ov && gemm16_uses_pair(M, m->qkv_n, D), wo_pair = ov && gemm16_uses_pair(M, D, H * d);
-  const bool w13_pair = ov && gemm16_uses_pair(M, 2 * m->F, D), w2_pair = ov && gemm16_uses_pair(M, D, m->F);
+  const bool chain = fuse && m->ready != nullptr && gemm16_uses_pair(M, m->qkv_n, D) &&
+                     gemm16_uses_pair(M, D, H * d) && gemm16_uses_pair(M, 2 * m->F, D) &&
+                     gemm16_uses_pair(M, D, m->F);
   auto norm_in = [&](EpiArgs& a) {
     if (!fuse) return;
     a.ss_in = m->ss;
@@ -399,68 +379,96 @@ int run_layer(llama_model* m, int l, int B, int S, bool decode, int cmax, cudaSt
     a.ss_out = m->ss;
     a.ss_n = ss_n;
   };
-  EpiArgs e = epi_base(M, m->qkv_n, m->d_status);
-  norm_in(e);
-  e.q = m->q;
-  e.kc = kc;
-  e.vc = vc;
-  e.rope = m->rope;
-  e.pos0 = m->d_len;
-  e.S = S;
-  e.H = H;
-  e.Hk = Hk;
-  e.d = d;
-  e.Smax = c.max_seq;
-  e.kv_table = m->paged ? m->d_table : nullptr;
-  e.kv_max_pages = m->max_pages;
-  e.kv_pages = m->n_pages;
-  if (after_w2) link(e, ready_set(l - 1, 2), gemm16_uses_pair(M, D, m->F), D, qkv_pair);
-  e.m_group = 1;
-  mark(m, K_GEMM_QKV, st);
-  RC(gemm(m, m->xn, M, D, w.wqkv, m->qkv_n, EPI_QKV_ROPE, e, st));
+  auto qkv_args = [&](int layer) {
+    EpiArgs e = epi_base(M, m->qkv_n, m->d_status);
+    norm_in(e);
+    e.q = m->q;
+    e.kc = static_cast<char*>(m->kcache) + (size_t)layer * m->layer_cache_elems * m->esz;
+    e.vc = static_cast<char*>(m->vcache) + (size_t)layer * m->layer_cache_elems * m->esz;
+    e.rope = m->rope;
+    e.pos0 = m->d_len;
+    e.S = S;
+    e.H = H;
+    e.Hk = Hk;
+    e.d = d;
+    e.Smax = c.max_seq;
+    e.kv_table = m->paged ? m->d_table : nullptr;
+    e.kv_max_pages = m->max_pages;
+    e.kv_pages = m->n_pages;
+    return e;
+  };
+
+  // ---- attention norm and QKV (unless the previous layer's chain ran it)
+  if (!(chain && m->qkv_ready_layer == l)) {
+    if (fuse) {
+      if (!m->norm_ready) {
+        mark(m, K_RMSNORM, st);
+        RC(launch_norm_prep(m->x, w.attn_norm, m->xn, m->ss, M, D, ss_n, m->adt, st, m->d_status));
+      }
+    } else {
+      mark(m, K_RMSNORM, st);
+      RC(launch_rmsnorm(m->x, w.attn_norm, m->xn, M, D, c.norm_eps, 0, m->adt, st, m->d_status));
+    }
+    const EpiArgs e = qkv_args(l);
+    mark(m, K_GEMM_QKV, st);
+    RC(gemm(m, m->xn, M, D, w.wqkv, m->qkv_n, EPI_QKV_ROPE, e, st));
+  }
+  m->norm_ready = false;
+  m->qkv_ready_layer = -1;
+  const int32_t* kv_table = m->paged ? m->d_table : nullptr;
   if (decode) {
     mark(m, K_ATTN_DECODE, st);
     RC(attention_decode(m->q, kc, vc, m->d_len, 1, m->attn, B, cmax, H, Hk, d, c.max_seq, m->adt, &m->ds,
-                        m->d_status, st, e.kv_table, m->max_pages, m->n_pages));
+                        m->d_status, st, kv_table, m->max_pages, m->n_pages));
   } else {
     mark(m, K_ATTN_PREFILL, st);
     RC(attention_prefill(m->q, kc, vc, m->attn, m->d_len, B, S, H, Hk, d, c.max_seq, m->adt, m->d_status, st,
-                         e.kv_table, m->max_pages, m->n_pages));
+                         kv_table, m->max_pages, m->n_pages));
   }
+  const bool has_next = !alone && l + 1 < c.n_layers;   // alone: one block on its own (no next layer)
   EpiArgs r = epi_base(M, D, m->d_status);
   r.out = m->x;
   r.ldo = D;
   norm_out(r, w.ffn_norm);
-  if (ov && wo_pair) r.ready_out = ready_set(l, 0);
-  r.m_group = 1;
+  EpiArgs sg = epi_base(M, 2 * m->F, m->d_status);
+  sg.g = m->g;
+  sg.ldg = m->F;
+  norm_in(sg);
+  EpiArgs r2 = epi_base(M, D, m->d_status);
+  r2.out = m->x;
+  r2.ldo = D;
+  if (has_next) norm_out(r2, m->L[l + 1].attn_norm);   // the final norm takes the last rows only
+
+  if (chain) {
+    const int m_tiles = (M + 255) / 256;
+    int* rs = m->ready + (size_t)l * 3 * m->ready_rb;
+    ChainJobDesc jobs[4] = {
+        {m->attn, H * d, w.wo, H * d, M, D, H * d, EPI_RESIDUAL, 1, -1, rs, r},
+        {m->xn, D, w.w13, D, M, 2 * m->F, D, EPI_SWIGLU, (m_tiles + 1) / 2, 0, rs + m->ready_rb, sg},
+        {m->g, m->F, w.w2, m->F, M, D, m->F, EPI_RESIDUAL, 1, 1, has_next ? rs + 2 * m->ready_rb : nullptr, r2},
+        {}};
+    int n = 3;
+    if (has_next) {
+      jobs[3] = ChainJobDesc{m->xn, D, m->L[l + 1].wqkv, D, M, m->qkv_n, D, EPI_QKV_ROPE, 1, 2, nullptr, qkv_args(l + 1)};
+      n = 4;
+      m->qkv_ready_layer = l + 1;
+    }
+    mark(m, K_GEMM_CHAIN, st);
+    RC(gemm16_chain(jobs, n, m->adt, m->d_status, st));
+    m->norm_ready = has_next;
+    return LLAMA_OK;
+  }
   mark(m, K_GEMM_WO, st);
   RC(gemm(m, m->attn, M, H * d, w.wo, D, EPI_RESIDUAL, r, st));
   if (!fuse) {
     mark(m, K_RMSNORM, st);
     RC(launch_rmsnorm(m->x, w.ffn_norm, m->xn, M, D, c.norm_eps, 0, m->adt, st, m->d_status));
   }
-  EpiArgs sg = epi_base(M, 2 * m->F, m->d_status);
-  sg.g = m->g;
-  sg.ldg = m->F;
-  norm_in(sg);
-  link(sg, ready_set(l, 0), wo_pair, D, w13_pair);
-  if (ov && w13_pair) sg.ready_out = ready_set(l, 1);
-  sg.m_group = (m_tiles + 1) / 2;
   mark(m, K_GEMM_W13, st);
   RC(gemm(m, m->xn, M, D, w.w13, 2 * m->F, EPI_SWIGLU, sg, st));
-  EpiArgs r2 = epi_base(M, D, m->d_status);
-  r2.out = m->x;
-  r2.ldo = D;
-  link(r2, ready_set(l, 1), w13_pair, 2 * m->F, w2_pair);
-  r2.m_group = 1;
-  if (l + 1 < c.n_layers) {   // the next layer's attention norm (the final norm takes the last rows only)
-    norm_out(r2, m->L[l + 1].attn_norm);
-    m->norm_ready = fuse;
-    if (ov && w2_pair) r2.ready_out = ready_set(l, 2);
-  }
   mark(m, K_GEMM_W2, st);
   RC(gemm(m, m->g, M, m->F, w.w2, D, EPI_RESIDUAL, r2, st));
-  if (r2.ready_out) m->last_signal_layer = l;
+  m->norm_ready = fuse && has_next;
   return LLAMA_OK;
 }
 
@@ -481,7 +489,7 @@ int run_head(llama_model* m, int B, int S, cudaStream_t st) {
 // Zeroes the row-block counters of the prefill GEMMs (part of the step, so a
 // graph replay zeroes them too).
 int reset_ready(llama_model* m, int M, cudaStream_t st) {
-  m->last_signal_layer = -1;
+  m->qkv_ready_layer = -1;
   if (!m->ready || M <= 128) return LLAMA_OK;
   CK(cudaMemsetAsync(m->ready, 0, (size_t)3 * m->cfg.n_layers * m->ready_rb * sizeof(int), st));
   return LLAMA_OK;
@@ -501,7 +509,7 @@ int prefill_body(llama_model* m, int B, int S, cudaStream_t st) {
 
 int decode_body(llama_model* m, int B, int cmax, cudaStream_t st) {
   m->norm_ready = false;
-  m->last_signal_layer = -1;
+  m->qkv_ready_layer = -1;
   mark(m, K_EMBED, st);
   RC(launch_embed(m->tok_buf, B, m->tok_emb, m->cfg.vocab_size, m->cfg.dim, m->adt, m->x, m->d_status, st));
   for (int l = 0; l < m->cfg.n_layers; ++l) RC(run_layer(m, l, B, 1, true, cmax, st));
@@ -708,7 +716,7 @@ int llama_create(const llama_config* cfg, llama_model** out) {
   m->logits = static_cast<float*>(m->alloc((size_t)c.max_batch * V * 4));
   m->tok_buf = static_cast<int32_t*>(m->alloc(Mx * sizeof(int32_t)));
   m->d_status = static_cast<int*>(m->alloc(sizeof(int)));
-  if (m->adt != LLAMA_F32 && Mx > 128 && getenv("LLAMA_NO_GEMM_OVERLAP") == nullptr) {
+  if (m->adt != LLAMA_F32 && Mx > 128 && getenv("LLAMA_NO_GEMM_CHAIN") == nullptr) {
     m->ready_rb = (int)(2 * ((Mx + 255) / 256));
     m->ready = static_cast<int*>(m->alloc((size_t)3 * c.n_layers * m->ready_rb * sizeof(int)));
     if (!m->ready) { delete m; return LLAMA_ERR_OOM; }
@@ -943,7 +951,7 @@ int llama_block_forward(llama_model* m, int32_t layer, const float* x, float* y,
   CK(cudaMemcpyAsync(m->x, x, bytes, cudaMemcpyDeviceToDevice, st));
   m->norm_ready = false;
   RC(reset_ready(m, B * S, st));
-  RC(run_layer(m, layer, B, S, false, 0, st));
+  RC(run_layer(m, layer, B, S, false, 0, st, true));
   m->norm_ready = false;
   CK(cudaMemcpyAsync(y, m->x, bytes, cudaMemcpyDeviceToDevice, st));
   return LLAMA_OK;

@@ -123,11 +123,14 @@ def test_8b_decode_batch32_ctx4096_graph(model8b):
             cache.k.append(si.bf16_bits_to_f32(k).reshape(Hk, CTX, d))
             cache.v.append(si.bf16_bits_to_f32(v).reshape(Hk, CTX, d))
         # One causal pass over the 128 seeded tokens: row i of that pass sees
-        # the cache plus tokens 0..i, exactly decode step i.
+        # the cache plus tokens 0..i, exactly decode step i. (The oracle
+        # appends to the cache it is given, so the replay below gets the
+        # cache as it was before the pass.)
         seq = np.array([toks[step][b] for step in range(STEPS)])
+        ck, cv = list(cache.k), list(cache.v)
         _, hidden = orc.forward(seq, cache, return_hidden=True)
         refs = orc.logits(hidden)
-        emu = pass_after_cache_rounded(p, w, cache.k, cache.v, seq, round_fp16)
+        emu = pass_after_cache_rounded(p, w, ck, cv, seq, round_fp16)
         for step in range(STEPS):
             ref, got = refs[step], rows[step][wi]
             err = rel_l2(got, ref)

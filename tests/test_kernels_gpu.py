@@ -181,6 +181,7 @@ def test_attention_prefill_f32(d):
     (BF16, 128, 32, 32, 8, 4224, [4097 + 4 * i for i in range(32)]),   # batch-32 decode shape
     (BF16, 128, 1, 32, 8, 131072, [131072]),                 # longest cache of the sweep
     (BF16, 128, 64, 32, 8, 1024, [1 + 16 * i for i in range(64)]),
+    (F16, 128, 1, 8, 1, 65536, [65536]),                   # one kv head: every decoding warp holds a piece of it
     (BF16, 64, 2, 8, 2, 300, [17, 300]),
     (F16, 128, 3, 32, 8, 1000, [1, 517, 1000]),
     (F16, 128, 32, 32, 8, 4224, [4097 + 4 * i for i in range(32)]),
