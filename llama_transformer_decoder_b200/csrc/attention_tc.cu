@@ -1,9 +1,10 @@
 // Causal GQA prefill attention on the 5th-generation tensor cores (16-bit
 // q/k/v, bf16 or fp16, head_dim 128).
 //
-// Two kernels share the arithmetic below: a per-tile one (one CTA per 128
-// queries of one head) and a persistent one (one CTA per SM looping over such
-// items, for short chunks; described above its definition).
+// Three kernels share the arithmetic below: a per-tile one (one CTA per 128
+// queries of one head), a persistent one (one CTA per SM looping over such
+// items) and a persistent one whose items are the same 128 queries of two
+// heads of one GQA group (each described above its definition).
 //
 // One CTA computes 128 queries of one head. Warp roles: warp 0 issues TMA
 // loads (Q once, then K and V tiles of 128 keys into 2-stage rings), warp 1
@@ -29,6 +30,7 @@
 
 #include <algorithm>
 #include <cstdlib>
+#include <mutex>
 #include <type_traits>
 
 #include "common.cuh"
@@ -602,299 +604,308 @@ __global__ void __launch_bounds__(FP_THREADS, 1)
   }
 }
 
-// ------------------------------------------------------- two CTAs per SM
-// The persistent computation with two CTAs resident on every SM, each with
-// half of the SM's TMEM (O: 128 columns, one S buffer of 128 columns whose
-// upper 64 columns take P) and single-stage Q, K and V buffers (96 KB of
-// shared memory). Inside a CTA the steps of a tile are serial (S, softmax,
-// P V, then the next S into the same buffer); the two CTAs of an SM
-// interleave, so one CTA's softmax overlaps the other's products and the
-// serial parts of the two softmaxes overlap each other. Items and their
-// snake order over 2 x SMs CTAs are those of the one-CTA persistent kernel.
+// ------------------------------------------------------- two heads per item
+// The persistent computation on items of two query tiles: the same 128
+// queries of two heads of one GQA group (h0 = 2p and h0 + 1, which read the
+// same K and V). Every K and V tile loaded serves both tiles, and two softmax
+// warpgroups work on different tiles (A: head h0, B: head h0 + 1), so one
+// group's exponentials overlap the other's TMEM
+// loads, maxima, stores and waits while the tensor pipe alternates between
+// the two. Per key tile t the MMA issuer runs P_A(t) V(t), S_A(t+1),
+// P_B(t) V(t), S_B(t+1) (S_A(t0), S_B(t0) at the start of an item).
 //
-// Per tile t (counted over the CTA's items): K(t) is loaded once S(t-1) has
-// read the K buffer, V(t) once P(t-1) V(t-1) has read the V buffer; S(t) is
-// issued once P(t-1) V(t-1) has completed (S overwrites the P it read); the
-// softmax threads load the row's 128 scores in two halves of 64 (registers),
-// store P over the upper half of S after both halves are loaded, and may
-// rescale O at once (the commit that signalled S(t) follows P(t-1) V(t-1)).
-// After an item's last product they read O out; the next item's first
-// product, which overwrites O, needs their next P. Every wait is bounded.
-constexpr int F2_THREADS = 192;
-constexpr int F2_OFF_Q = 0;
-constexpr int F2_OFF_K = F2_OFF_Q + FA_Q_BYTES;
-constexpr int F2_OFF_V = F2_OFF_K + FA_KV_BYTES;
-constexpr int F2_OFF_BAR = F2_OFF_V + FA_KV_BYTES;
-constexpr int F2_SMEM = F2_OFF_BAR + 256 + 1024;
-constexpr uint32_t F2_TMEM_O = 0, F2_TMEM_S = 128, F2_TMEM_P = 192;   // P: upper half of S
+// 384 threads in three warpgroups: warp 0 issues TMA loads, warp 1 the
+// products (warps 2-3 idle); warps 4-7 run the softmax of tile A and warps
+// 8-11 that of tile B (thread = query row = TMEM lane). The first warpgroup
+// hands registers to the other two (setmaxnreg): it drops to FD_REGS_LOW and
+// the softmax groups rise to FD_REGS_HIGH, 128 x 96 + 256 x 192 = 61440
+// registers, what the launch holds at 160 per thread. The host launches the
+// kernel only when its compiled register count is at least that (else the
+// raise would wait for registers that never come) and runs the one-tile
+// kernel otherwise.
+//
+// TMEM: O_A [0,128), O_B [128,256), S_A [256,384), S_B [384,512). A tile's P
+// (64 columns, keys 2c and 2c+1 in column c) is written over the first half
+// of its own S, which the softmax thread has read by then. S_X(t+1) overwrites
+// P_X(t), so it is issued only once P_X(t) V(t) has completed (o_done[X]);
+// this also makes O_X final up to tile t whenever the softmax sees S_X(t+1),
+// so a rescale of O needs no wait. Q: one buffer per tile, reloaded once the
+// item's last S of that tile has completed (q_empty[X]); K and V: 2-stage
+// rings, released by commits after S_B(t) and P_B(t) V(t) (a commit covers
+// every product issued before it, the A products included).
+//
+// Needs an even number of query heads per KV head; otherwise the one-tile
+// persistent kernel runs.
+constexpr int FD_THREADS = 384;
+constexpr int FD_REGS_LOW = 96, FD_REGS_HIGH = 192;
+static_assert(128 * FD_REGS_LOW + 256 * FD_REGS_HIGH <= FD_THREADS * 160, "register split exceeds the launch");
+constexpr int FD_OFF_Q = 0;                                      // Q_A, Q_B
+constexpr int FD_OFF_K = FD_OFF_Q + 2 * FA_Q_BYTES;
+constexpr int FD_OFF_V = FD_OFF_K + FA_STAGES * FA_KV_BYTES;
+constexpr int FD_OFF_BAR = FD_OFF_V + FA_STAGES * FA_KV_BYTES;
+constexpr int FD_SMEM = FD_OFF_BAR + 256 + 1024;
+constexpr uint32_t FD_TMEM_O = 0, FD_TMEM_S = 256;   // O_X at 128 X, S_X at 256 + 128 X
 
-// Softmax of one 128-key tile for this thread's row with the scores loaded
-// in two halves (fewer live registers): the upper half (keys 64-127) stays
-// in registers while the maximum is formed; O is rescaled if the running
-// maximum rises; the upper half's P is stored at once (over scores already
-// loaded), then the lower half is loaded again for its exponentials and its
-// P stored. Returns the tile's row sum; corr as for fa_tile_softmax.
+struct FdItem {
+  int b, h0, g, q0, p0, n_kt;
+};
+
+// Item w in longest-first order: query tile (from the last), then head pair
+// and sequence.
+__device__ __forceinline__ FdItem fd_decode(int w, int S, int H, int Hk, int B, const int32_t* pos0) {
+  const int nqt = (S + FA_BM - 1) / FA_BM;
+  const int HP = (H / 2) * B;
+  FdItem it;
+  const int hb = w % HP;
+  it.q0 = (nqt - 1 - w / HP) * FA_BM;
+  it.h0 = 2 * (hb % (H / 2));
+  it.b = hb / (H / 2);
+  it.g = it.h0 / (H / Hk);
+  it.p0 = pos0 ? pos0[it.b] : 0;
+  const int k_end = min(it.p0 + S, it.p0 + it.q0 + FA_BM);
+  it.n_kt = (k_end + FA_BN - 1) / FA_BN;
+  return it;
+}
+
+// The dual kernel's barriers, in shared memory after the K and V rings.
+struct FdBars {
+  uint64_t *q_full, *q_empty, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_done, *drain;
+  __device__ explicit FdBars(uint8_t* smem) {
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + FD_OFF_BAR);
+    q_full = bars + 0;     // [tile]
+    q_empty = bars + 2;    // [tile] the item's last S of that tile has read Q
+    k_full = bars + 4;     // [stage]
+    k_empty = bars + 6;    // [stage] S_B (and the S_A before it) has read K
+    v_full = bars + 8;     // [stage]
+    v_empty = bars + 10;   // [stage] P_B V (and P_A V) has read V
+    s_full = bars + 12;    // [tile]
+    p_full = bars + 14;    // [tile] the tile's 128 softmax threads stored P
+    o_done = bars + 16;    // [tile] P V of the tile finished
+    drain = bars + 18;
+  }
+};
+
+// Warps 0-3 of the dual kernel: warp 0 lane 0 issues the TMA loads, warp 1
+// lane 0 the products.
 template <typename T>
-__device__ __forceinline__ float f2_tile_softmax(uint32_t s_tmem, uint32_t o_tmem, uint32_t p_tmem, bool ok,
-                                                 bool masked, int kbase, int qpos, float scale_log2, bool first,
-                                                 float& m_used, float& corr) {
-  float hi[64];
-  float mlo = -INFINITY;
-  if (ok) {
-    uint32_t u0[32], u1[32];
-    tmem_ld32_nowait(s_tmem, u0);
-    tmem_ld32_nowait(s_tmem + 32, u1);
-    tmem_ld_wait();
-    float m8[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) m8[c] = -INFINITY;
-#pragma unroll
-    for (int x = 0; x < 32; x += 8) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float a = masked && kbase + x + c > qpos ? -INFINITY : __uint_as_float(u0[x + c]);
-        const float b = masked && kbase + 32 + x + c > qpos ? -INFINITY : __uint_as_float(u1[x + c]);
-        m8[c] = fmax3(m8[c], a, b);
+__device__ __forceinline__ void fd_loads_and_products(uint8_t* smem, uint32_t tmem, int warp, int lane,
+                                                      const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                                      const CUtensorMap& tmV, const int32_t* __restrict__ pos0,
+                                                      int B, int S, int H, int Hk,
+                                                      const int32_t* __restrict__ kv_table, int kv_max_pages,
+                                                      int kv_pages, int* status) {
+  FdBars fb(smem);
+  uint64_t *q_full = fb.q_full, *q_empty = fb.q_empty, *k_full = fb.k_full, *k_empty = fb.k_empty;
+  uint64_t *v_full = fb.v_full, *v_empty = fb.v_empty, *s_full = fb.s_full, *p_full = fb.p_full;
+  uint64_t *o_done = fb.o_done, *drain = fb.drain;
+  const int total = ((S + FA_BM - 1) / FA_BM) * (H / 2) * B;
+  const int c = blockIdx.x, G = gridDim.x;
+  if (warp == 0 && lane == 0) {
+
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    int t = 0, qa_issued = 0, qb_issued = 0, k_issued = 0, v_issued = 0;
+    bool ok = true;
+    for (int i = 0; ok; ++i) {
+      const int w = fp_item(c, G, i);
+      if (w >= total) break;
+      const FdItem it = fd_decode(w, S, H, Hk, B, pos0);
+      for (int j = 0; j < it.n_kt; ++j, ++t) {
+        const int st = t & 1;
+        const uint32_t ph = (t >> 1) & 1;
+        if (!(ok = mbar_wait(&k_empty[st], ph ^ 1, status))) break;
+        const int kv_y = kv_table ? 0 : j * FA_BN;
+        const int kv_z = kv_table ? kv_page(kv_table, kv_max_pages, kv_pages, it.b, j) * Hk + it.g : it.b * Hk + it.g;
+        mbar_arrive_expect_tx(&k_full[st], FA_KV_BYTES);
+        uint8_t* kd = smem + FD_OFF_K + st * FA_KV_BYTES;
+        tma_load_3d(kd, &tmK, &k_full[st], 0, kv_y, kv_z);
+        tma_load_3d(kd + FA_HALF, &tmK, &k_full[st], 64, kv_y, kv_z);
+        ++k_issued;
+        if (j == 0) {   // the item's Q tiles, after its first K (which does not wait for the last item's S)
+          for (int x = 0; x < 2 && ok; ++x) {
+            if (!(ok = mbar_wait(&q_empty[x], (i & 1) ^ 1, status))) break;
+            mbar_arrive_expect_tx(&q_full[x], FA_Q_BYTES);
+            uint8_t* qd = smem + FD_OFF_Q + x * FA_Q_BYTES;
+            tma_load_3d(qd, &tmQ, &q_full[x], 0, it.q0, it.b * H + it.h0 + x);
+            tma_load_3d(qd + FA_HALF, &tmQ, &q_full[x], 64, it.q0, it.b * H + it.h0 + x);
+            ++(x ? qb_issued : qa_issued);
+          }
+          if (!ok) break;
+        }
+        if (!(ok = mbar_wait(&v_empty[st], ph ^ 1, status))) break;
+        mbar_arrive_expect_tx(&v_full[st], FA_KV_BYTES);
+        uint8_t* vd = smem + FD_OFF_V + st * FA_KV_BYTES;
+        tma_load_3d(vd, &tmV, &v_full[st], 0, kv_y, kv_z);
+        tma_load_3d(vd + FA_HALF, &tmV, &v_full[st], 64, kv_y, kv_z);
+        ++v_issued;
       }
     }
-    mlo = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-    tmem_ld32_nowait(s_tmem + 64, u0);
-    tmem_ld32_nowait(s_tmem + 96, u1);
-    tmem_ld_wait();
-#pragma unroll
-    for (int x = 0; x < 32; ++x) {
-      hi[x] = __uint_as_float(u0[x]);
-      hi[32 + x] = __uint_as_float(u1[x]);
+    if (!ok) {  // let issued copies land before the CTA can exit
+      if (qa_issued > 0) mbar_wait(&q_full[0], (qa_issued - 1) & 1, status);
+      if (qb_issued > 0) mbar_wait(&q_full[1], (qb_issued - 1) & 1, status);
+      for (int j = k_issued - 1; j >= 0 && j >= k_issued - 2; --j) mbar_wait(&k_full[j & 1], (j >> 1) & 1, status);
+      for (int j = v_issued - 1; j >= 0 && j >= v_issued - 2; --j) mbar_wait(&v_full[j & 1], (j >> 1) & 1, status);
     }
-  } else {
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc_s = umma_idesc_16(UmmaFmt<T>::value, FA_BM, FA_BN, false);
+    constexpr uint32_t idesc_o = umma_idesc_16(UmmaFmt<T>::value, FA_BM, FA_D, true);
+    bool any = false;
+    // S_x(t) = Q_x K(t)^T over P_x(t-1), once P_x(t-1) V(t-1) has completed;
+    // `last`: the item's last S of tile x, after which Q_x may be reloaded
+    auto issue_s = [&](int x, int t, bool last) -> bool {
+      const int st = t & 1;
+      if (t > 0 && !mbar_wait(&o_done[x], (t - 1) & 1, status)) return false;
+      if (x == 0 && !mbar_wait(&k_full[st], (t >> 1) & 1, status)) return false;
+      tc_fence_after();
+      const uint32_t q_addr = smem_u32(smem + FD_OFF_Q + x * FA_Q_BYTES);
+      const uint32_t k_addr = smem_u32(smem + FD_OFF_K + st * FA_KV_BYTES);
+      const uint32_t d_tmem = tmem + FD_TMEM_S + (uint32_t)x * 128;
 #pragma unroll
-    for (int x = 0; x < 64; ++x) hi[x] = 0.f;
+      for (int ks = 0; ks < FA_D / 16; ++ks) {
+        const uint32_t off = (uint32_t)(ks >> 2) * FA_HALF + (uint32_t)(ks & 3) * 32;
+        umma_bf16(d_tmem, umma_desc_sw128(q_addr + off), umma_desc_sw128(k_addr + off), idesc_s, ks != 0);
+      }
+      umma_commit(&s_full[x]);
+      if (x == 1) umma_commit(&k_empty[st]);
+      if (last) umma_commit(&q_empty[x]);
+      any = true;
+      return true;
+    };
+    // O_x (+)= P_x(t) V(t); j == 0 starts the item's O
+    auto issue_pv = [&](int x, int t, int j) -> bool {
+      const int st = t & 1;
+      if (!mbar_wait(&p_full[x], t & 1, status)) return false;
+      if (x == 0 && !mbar_wait(&v_full[st], (t >> 1) & 1, status)) return false;
+      tc_fence_after();
+      const uint32_t v_addr = smem_u32(smem + FD_OFF_V + st * FA_KV_BYTES);
+      const uint32_t p_tmem = tmem + FD_TMEM_S + (uint32_t)x * 128;
+#pragma unroll
+      for (int ks = 0; ks < FA_BN / 16; ++ks)
+        umma_ts(tmem + FD_TMEM_O + (uint32_t)x * 128, p_tmem + ks * 8,
+                umma_desc_sw128_mn(v_addr + ks * 2048, FA_HALF), idesc_o, (j | ks) != 0);
+      if (x == 1) umma_commit(&v_empty[st]);
+      umma_commit(&o_done[x]);
+      return true;
+    };
+    bool ok = true;
+    int t = 0;
+    for (int i = 0; ok; ++i) {
+      const int w = fp_item(c, G, i);
+      if (w >= total) break;
+      const int n_kt = fd_decode(w, S, H, Hk, B, pos0).n_kt;
+      for (int x = 0; x < 2 && ok; ++x) ok = mbar_wait(&q_full[x], i & 1, status);
+      if (!ok || !(ok = issue_s(0, t, n_kt == 1)) || !(ok = issue_s(1, t, n_kt == 1))) break;
+      for (int j = 0; j < n_kt && ok; ++j) {
+        const int tj = t + j;
+        const bool more = j + 1 < n_kt, last_next = j + 2 == n_kt;
+        ok = issue_pv(0, tj, j) && (!more || issue_s(0, tj + 1, last_next)) && issue_pv(1, tj, j) &&
+             (!more || issue_s(1, tj + 1, last_next));
+      }
+      t += n_kt;
+    }
+    if (!ok && any) {
+      umma_commit(drain);
+      mbar_wait(drain, 0, status);
+    }
   }
-  if (masked) {
-#pragma unroll
-    for (int x = 0; x < 64; ++x)
-      if (kbase + 64 + x > qpos) hi[x] = -INFINITY;
-  }
-  float m8[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) m8[c] = hi[c];
-#pragma unroll
-  for (int x = 8; x < 56; x += 16) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) m8[c] = fmax3(m8[c], hi[x + c], hi[x + 8 + c]);
-  }
-#pragma unroll
-  for (int c = 0; c < 8; ++c) m8[c] = fmaxf(m8[c], hi[56 + c]);
-  const float mx = fmaxf(mlo, fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
-                   scale_log2;
-  corr = 1.f;
-  if (first) {
-    m_used = mx;
-  } else if (mx > m_used + FA_RESCALE) {
-    corr = fast_exp2(m_used - mx);
-    m_used = mx;
-  }
-  if (__any_sync(0xffffffffu, corr != 1.f) && ok) fa_rescale_o(o_tmem, corr);
-  float sum8[8];
-#pragma unroll
-  for (int x = 0; x < 8; ++x) sum8[x] = 0.f;
+}
+
+// Warps 4-11 of the dual kernel: the softmax of tile A (warps 4-7) or B (8-11).
+template <typename T>
+__device__ __forceinline__ void fd_softmax(uint8_t* smem, uint32_t tmem, int warp, int lane, T* __restrict__ o,
+                                           const int32_t* __restrict__ pos0, int B, int S, int H, int Hk,
+                                           float scale_log2, int* status) {
+  const FdBars fb(smem);
+  uint64_t *s_full = fb.s_full, *p_full = fb.p_full, *o_done = fb.o_done;
+  const int total = ((S + FA_BM - 1) / FA_BM) * (H / 2) * B;
+  const int c = blockIdx.x, G = gridDim.x;
   {
-    uint32_t pk[32];
-#pragma unroll
-    for (int x = 0; x < 32; ++x) {
-      const float a = fast_exp2(fmaf(hi[2 * x], scale_log2, -m_used));
-      const float b = fast_exp2(fmaf(hi[2 * x + 1], scale_log2, -m_used));
-      sum8[x & 7] += a + b;
-      pk[x] = pack2<T>(a, b);
+    const int x = (warp - 4) >> 2;                      // 0: tile A (head h0), 1: tile B (head h0 + 1)
+    const int quarter = warp & 3;                       // TMEM lanes this warp may read
+    const int r = quarter * 32 + lane;                  // query row in the tile
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t s_tm = tmem + lane_off + FD_TMEM_S + (uint32_t)x * 128;
+    const uint32_t o_tm = tmem + lane_off + FD_TMEM_O + (uint32_t)x * 128;
+    bool ok = true;
+    int t = 0;
+    for (int i = 0;; ++i) {
+      const int w = fp_item(c, G, i);
+      if (w >= total) break;
+      const FdItem it = fd_decode(w, S, H, Hk, B, pos0);
+      const int qpos = it.p0 + it.q0 + r;
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < it.n_kt; ++j, ++t) {
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s_full[x], t & 1, status));
+        tc_fence_after();
+        uint32_t pk[64];
+        float corr;
+        const float rowsum = fa_tile_softmax<T>(s_tm, ok, j * FA_BN + FA_BN - 1 > it.p0 + it.q0, j * FA_BN, qpos,
+                                                scale_log2, j == 0, m_used, corr, pk);
+        l = l * corr + rowsum;
+        // O_x is final up to tile t-1: S_x(t) was issued after P_x(t-1) V(t-1) completed
+        if (__any_sync(0xffffffffu, corr != 1.f) && ok) fa_rescale_o(o_tm, corr);
+        if (ok) fa_store_p(s_tm, pk);
+        tc_fence_before();
+        mbar_arrive(&p_full[x]);
+      }
+      // the item's last product, then O / l out of TMEM (the next item's first
+      // product, which overwrites O, waits for this thread's next P)
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[x], (t - 1) & 1, status));
+      tc_fence_after();
+      const int qi = it.q0 + r;
+      T* dst = o + ((size_t)it.b * S + (qi < S ? qi : 0)) * H * FA_D + (size_t)(it.h0 + x) * FA_D;
+      fa_store_o<T>(o_tm, ok, 1.f / l, dst, qi < S);
+      tc_fence_before();
     }
-    if (ok) tmem_st32_u(p_tmem + 32, pk);        // keys 64-127: over scores 96-127, already loaded
   }
-  if (ok) {
-    uint32_t u0[32], u1[32], pk[32];
-    tmem_ld32_nowait(s_tmem, u0);
-    tmem_ld32_nowait(s_tmem + 32, u1);
-    tmem_ld_wait();
-#pragma unroll
-    for (int x = 0; x < 16; ++x) {
-      float a = __uint_as_float(u0[2 * x]), b = __uint_as_float(u0[2 * x + 1]);
-      if (masked && kbase + 2 * x > qpos) a = -INFINITY;
-      if (masked && kbase + 2 * x + 1 > qpos) b = -INFINITY;
-      a = fast_exp2(fmaf(a, scale_log2, -m_used));
-      b = fast_exp2(fmaf(b, scale_log2, -m_used));
-      sum8[x & 7] += a + b;
-      pk[x] = pack2<T>(a, b);
-      float c = __uint_as_float(u1[2 * x]), d = __uint_as_float(u1[2 * x + 1]);
-      if (masked && kbase + 32 + 2 * x > qpos) c = -INFINITY;
-      if (masked && kbase + 33 + 2 * x > qpos) d = -INFINITY;
-      c = fast_exp2(fmaf(c, scale_log2, -m_used));
-      d = fast_exp2(fmaf(d, scale_log2, -m_used));
-      sum8[(x + 4) & 7] += c + d;
-      pk[16 + x] = pack2<T>(c, d);
-    }
-    tmem_st32_u(p_tmem, pk);                    // keys 0-63: over scores 64-95, already loaded
-  }
-  tmem_st_wait();
-  return ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
 }
 
 template <typename T>
-__global__ void __launch_bounds__(F2_THREADS, 2)
-    attn_prefill_tc_2cta_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(FD_THREADS, 1)
+    attn_prefill_tc_dual_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                                 const __grid_constant__ CUtensorMap tmV, T* __restrict__ o,
                                 const int32_t* __restrict__ pos0, int B, int S, int H, int Hk, float scale_log2,
                                 const int32_t* __restrict__ kv_table, int kv_max_pages, int kv_pages, int* status) {
   extern __shared__ uint8_t fa_smem_raw[];
   uint8_t* smem = fa_align(fa_smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + F2_OFF_BAR);
-  uint64_t* q_full = bars + 0;
-  uint64_t* q_empty = bars + 1;    // the item's last S = Q K^T has read Q
-  uint64_t* k_full = bars + 2;
-  uint64_t* k_empty = bars + 3;    // S has read K
-  uint64_t* v_full = bars + 4;
-  uint64_t* v_empty = bars + 5;    // P V has read V
-  uint64_t* s_full = bars + 6;     // S written (and every earlier product complete)
-  uint64_t* p_full = bars + 7;     // softmax threads stored P (128 arrivals)
-  uint64_t* o_done = bars + 8;     // P V complete
-  uint64_t* drain = bars + 9;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
-
+  const FdBars fb(smem);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fb.drain + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int total = ((S + FA_BM - 1) / FA_BM) * H * B;
-  const int c = blockIdx.x, G = gridDim.x;
 
   pdl_trigger();
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1); mbar_init(q_empty, 1);
-    mbar_init(k_full, 1); mbar_init(k_empty, 1);
-    mbar_init(v_full, 1); mbar_init(v_empty, 1);
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
-    mbar_init(drain, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&fb.q_full[i], 1); mbar_init(&fb.q_empty[i], 1);
+      mbar_init(&fb.k_full[i], 1); mbar_init(&fb.k_empty[i], 1);
+      mbar_init(&fb.v_full[i], 1); mbar_init(&fb.v_empty[i], 1);
+      mbar_init(&fb.s_full[i], 1);
+      mbar_init(&fb.p_full[i], 128);
+      mbar_init(&fb.o_done[i], 1);
+    }
+    mbar_init(fb.drain, 1);
     fence_barrier_init();
   }
-  if (warp == 1) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
+  if (warp == 1) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_wait();
 
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmK);
-    tma_prefetch_desc(&tmV);
-    int t = 0, q_issued = 0, k_issued = 0, v_issued = 0;
-    bool ok = true;
-    for (int i = 0; ok; ++i) {
-      const int w = fp_item(c, G, i);
-      if (w >= total) break;
-      const FpItem it = fp_decode(w, S, H, Hk, B, pos0);
-      if (i > 0 && !(ok = mbar_wait(q_empty, (i - 1) & 1, status))) break;
-      mbar_arrive_expect_tx(q_full, FA_Q_BYTES);
-      tma_load_3d(smem + F2_OFF_Q, &tmQ, q_full, 0, it.q0, it.b * H + it.h);
-      tma_load_3d(smem + F2_OFF_Q + FA_HALF, &tmQ, q_full, 64, it.q0, it.b * H + it.h);
-      ++q_issued;
-      for (int j = 0; j < it.n_kt; ++j, ++t) {
-        const int kv_y = kv_table ? 0 : j * FA_BN;
-        const int kv_z = kv_table ? kv_page(kv_table, kv_max_pages, kv_pages, it.b, j) * Hk + it.g : it.b * Hk + it.g;
-        if (t > 0 && !(ok = mbar_wait(k_empty, (t - 1) & 1, status))) break;
-        mbar_arrive_expect_tx(k_full, FA_KV_BYTES);
-        tma_load_3d(smem + F2_OFF_K, &tmK, k_full, 0, kv_y, kv_z);
-        tma_load_3d(smem + F2_OFF_K + FA_HALF, &tmK, k_full, 64, kv_y, kv_z);
-        ++k_issued;
-        if (t > 0 && !(ok = mbar_wait(v_empty, (t - 1) & 1, status))) break;
-        mbar_arrive_expect_tx(v_full, FA_KV_BYTES);
-        tma_load_3d(smem + F2_OFF_V, &tmV, v_full, 0, kv_y, kv_z);
-        tma_load_3d(smem + F2_OFF_V + FA_HALF, &tmV, v_full, 64, kv_y, kv_z);
-        ++v_issued;
-      }
-    }
-    if (!ok) {  // let issued copies land before the CTA can exit
-      if (q_issued > 0) mbar_wait(q_full, (q_issued - 1) & 1, status);
-      if (k_issued > 0) mbar_wait(k_full, (k_issued - 1) & 1, status);
-      if (v_issued > 0) mbar_wait(v_full, (v_issued - 1) & 1, status);
-    }
-  } else if (warp == 1 && lane == 0) {
-    constexpr uint32_t idesc_s = umma_idesc_16(UmmaFmt<T>::value, FA_BM, FA_BN, false);
-    constexpr uint32_t idesc_o = umma_idesc_16(UmmaFmt<T>::value, FA_BM, FA_D, true);
-    const uint32_t q_addr = smem_u32(smem + F2_OFF_Q);
-    const uint32_t k_addr = smem_u32(smem + F2_OFF_K);
-    const uint32_t v_addr = smem_u32(smem + F2_OFF_V);
-    bool ok = true, any = false;
-    int t = 0;
-    for (int i = 0; ok; ++i) {
-      const int w = fp_item(c, G, i);
-      if (w >= total) break;
-      const int n_kt = fp_decode(w, S, H, Hk, B, pos0).n_kt;
-      if (!(ok = mbar_wait(q_full, i & 1, status))) break;
-      for (int j = 0; j < n_kt; ++j, ++t) {
-        // S overwrites the P that the previous product read: that product first
-        if (t > 0 && !(ok = mbar_wait(o_done, (t - 1) & 1, status))) break;
-        if (!(ok = mbar_wait(k_full, t & 1, status))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < FA_D / 16; ++ks) {
-          const uint32_t off = (uint32_t)(ks >> 2) * FA_HALF + (uint32_t)(ks & 3) * 32;
-          umma_bf16(tmem + F2_TMEM_S, umma_desc_sw128(q_addr + off), umma_desc_sw128(k_addr + off), idesc_s, ks != 0);
-        }
-        umma_commit(s_full);
-        umma_commit(k_empty);
-        if (j + 1 == n_kt) umma_commit(q_empty);
-        any = true;
-        if (!(ok = mbar_wait(p_full, t & 1, status))) break;
-        if (!(ok = mbar_wait(v_full, t & 1, status))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < FA_BN / 16; ++ks)
-          umma_ts(tmem + F2_TMEM_O, tmem + F2_TMEM_P + ks * 8, umma_desc_sw128_mn(v_addr + ks * 2048, FA_HALF), idesc_o,
-                  (j | ks) != 0);
-        umma_commit(v_empty);
-        umma_commit(o_done);
-      }
-    }
-    if (!ok && any) {
-      umma_commit(drain);
-      mbar_wait(drain, 0, status);
-    }
-  } else if (warp >= 2) {
-    const int quarter = warp & 3;                       // TMEM lanes this warp may read
-    const int r = quarter * 32 + lane;                  // query row in the tile
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    bool ok = true;
-    int t = 0;
-    for (int i = 0;; ++i) {
-      const int w = fp_item(c, G, i);
-      if (w >= total) break;
-      const FpItem it = fp_decode(w, S, H, Hk, B, pos0);
-      const int qpos = it.p0 + it.q0 + r;
-      float m_used = -INFINITY, l = 0.f;
-      for (int j = 0; j < it.n_kt; ++j, ++t) {
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full, t & 1, status));
-        tc_fence_after();
-        // O is complete up to the previous product (its commit came before S's),
-        // so the softmax may rescale it at once
-        float corr;
-        const float rowsum = f2_tile_softmax<T>(tmem + lane_off + F2_TMEM_S, tmem + lane_off + F2_TMEM_O,
-                                                tmem + lane_off + F2_TMEM_P, ok, j * FA_BN + FA_BN - 1 > it.p0 + it.q0,
-                                                j * FA_BN, qpos, scale_log2, j == 0, m_used, corr);
-        l = l * corr + rowsum;
-        tc_fence_before();
-        mbar_arrive(p_full);
-      }
-      if (it.n_kt > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (t - 1) & 1, status));
-      tc_fence_after();
-      const int qi = it.q0 + r;
-      T* dst = o + ((size_t)it.b * S + (qi < S ? qi : 0)) * H * FA_D + (size_t)it.h * FA_D;
-      fa_store_o<T>(tmem + lane_off + F2_TMEM_O, ok, 1.f / l, dst, qi < S);
-      tc_fence_before();
-    }
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(FD_REGS_LOW) : "memory");
+    fd_loads_and_products<T>(smem, tmem, warp, lane, tmQ, tmK, tmV, pos0, B, S, H, Hk, kv_table, kv_max_pages,
+                             kv_pages, status);
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(FD_REGS_HIGH) : "memory");
+    fd_softmax<T>(smem, tmem, warp, lane, o, pos0, B, S, H, Hk, scale_log2, status);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -925,6 +936,22 @@ int make_tmap_3d(CUtensorMap* map, const void* base, int64_t outer, int64_t rows
 
 }  // namespace
 
+// The dual kernel's register hand-off fits the registers its launch holds
+// (compiled count x threads); checked once per instantiation.
+template <typename T>
+bool dual_regs_ok() {
+  static std::once_flag once;
+  static bool ok = false;
+  std::call_once(once, [] {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(attn_prefill_tc_dual_kernel<T>)) == cudaSuccess)
+      ok = fa.numRegs * FD_THREADS >= 128 * FD_REGS_LOW + 256 * FD_REGS_HIGH;
+    else
+      cudaGetLastError();
+  });
+  return ok;
+}
+
 template <typename T>
 static int attention_prefill_tc_t(const void* q, const void* kc, const void* vc, void* o, const int32_t* pos0, int B,
                                   int S, int H, int Hk, int Smax, int* status, cudaStream_t st,
@@ -940,19 +967,22 @@ static int attention_prefill_tc_t(const void* q, const void* kc, const void* vc,
   if ((rc = make_tmap_3d(&tk, kc, kv_outer, kv_rows, F16)) != LLAMA_OK) return rc;
   if ((rc = make_tmap_3d(&tv, vc, kv_outer, kv_rows, F16)) != LLAMA_OK) return rc;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)FA_D);
-  // Short chunks (few key tiles per item) run the persistent kernel, which
-  // hides each item's start and end behind its neighbours: measured 10%
-  // faster at 2048 queries (B = 1 and 4), but 6-8% slower at 32768, where a
-  // CTA's fixed cost is small against its key loop. LLAMA_ATTN_PER_TILE
-  // selects the per-tile kernel for every length.
+  // Two heads per item (the dual kernel) wherever the heads of a GQA group
+  // pair up: measured 11-18% faster than the one-head persistent kernel at
+  // 2048 queries (B = 1, 4, 16) and 12-14% faster than the per-tile kernel at
+  // 8192 and 32768. Otherwise short chunks (few key tiles per item) run the
+  // one-head persistent kernel, which hides each item's start and end behind
+  // its neighbours (10% faster than the per-tile kernel at 2048 queries, 6-8%
+  // slower at 32768). LLAMA_ATTN_NO_DUAL and LLAMA_ATTN_PER_TILE select the
+  // other kernels, for comparisons.
   static const bool per_tile = getenv("LLAMA_ATTN_PER_TILE") != nullptr;
-  static const bool two_cta = getenv("LLAMA_ATTN_2CTA") != nullptr;
-  if (two_cta) {
-    auto kern = attn_prefill_tc_2cta_kernel<T>;
-    if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), F2_SMEM)) return rc;
-    const long long items = (long long)((S + FA_BM - 1) / FA_BM) * H * B;
-    const int grid = (int)std::min<long long>(items, 2LL * num_sms());
-    const cudaError_t err = launch_k(kern, dim3(grid), dim3(F2_THREADS), F2_SMEM, st, tq, tk, tv, static_cast<T*>(o),
+  static const bool no_dual = getenv("LLAMA_ATTN_NO_DUAL") != nullptr;
+  if (!no_dual && !per_tile && (H / Hk) % 2 == 0 && dual_regs_ok<T>()) {
+    auto kern = attn_prefill_tc_dual_kernel<T>;
+    if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), FD_SMEM)) return rc;
+    const long long items = (long long)((S + FA_BM - 1) / FA_BM) * (H / 2) * B;
+    const int grid = (int)std::min<long long>(items, num_sms());
+    const cudaError_t err = launch_k(kern, dim3(grid), dim3(FD_THREADS), FD_SMEM, st, tq, tk, tv, static_cast<T*>(o),
                                      pos0, B, S, H, Hk, scale_log2, kv_table, kv_max_pages, kv_pages, status);
     return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
   }

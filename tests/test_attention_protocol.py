@@ -1,5 +1,7 @@
-"""Model check of the persistent prefill attention kernel's barrier protocol
-(attention_tc.cu, attn_prefill_tc_persistent_kernel), run on the CPU.
+"""Model check of the persistent prefill attention kernels' barrier protocols
+(attention_tc.cu: attn_prefill_tc_persistent_kernel, one head per item, and
+attn_prefill_tc_dual_kernel, two heads of a GQA group per item), run on the
+CPU.
 
 Five actors are simulated under random interleavings: the TMA producer, the
 MMA issuer, the softmax warps (which also read O out at the end of every
@@ -210,15 +212,23 @@ def test_dropping_a_wait_is_caught(drop):
 
 
 # ------------------------------------------------------- two CTAs per SM
-def simulate_2cta(nkts, seed, drop=()):
-    """The barrier protocol of attn_prefill_tc_2cta_kernel: single-stage Q, K
-    and V buffers; one S buffer whose upper half takes P; the MMA issuer waits
-    for the previous P V product before the next S overwrites that P."""
+def simulate_dual(nkts, seed, drop=()):
+    """The barrier protocol of attn_prefill_tc_dual_kernel: items of two query
+    tiles (A, B) that share every K and V tile; one Q buffer per tile; S_X
+    single-buffered per tile with P_X written over it; per key tile the
+    products run P_A V, S_A(t+1), P_B V, S_B(t+1). Products writing different
+    accumulators need not run in issue order on the hardware, so the model
+    checks at issue time that S_X(t+1) follows the completion of P_X(t) V(t)
+    (the wait on o_done[X]) instead of relying on the in-order queue."""
     rng = random.Random(seed)
-    bars = {n: Bar() for n in ('q_full', 'q_empty', 'k_full', 'k_empty', 'v_full', 'v_empty', 's_full', 'p_full',
-                               'o_done')}
-    st = dict(Q=None, K=None, V=None, S=None, P=None, O_item=None, O_tiles=set(), o_read=set(), pv_done=set(),
-              s_done=set(), s_read=set())
+    bars = {}
+    for i in range(2):
+        for n in ('q_full', 'q_empty', 'k_full', 'k_empty', 'v_full', 'v_empty', 's_full', 'o_done'):
+            bars[f'{n}{i}'] = Bar()
+        bars[f'p_full{i}'] = Bar()
+    st = dict(Q=[None, None], K=[None, None], V=[None, None], S=[None, None], P=[None, None],
+              O=[None, None], O_tiles=[set(), set()], o_read=[set(), set()], pv_done=set(), s_done=set(),
+              s_read=[set(), set()])
     tma, tc = [], []
     first = [sum(nkts[:i]) for i in range(len(nkts))]
 
@@ -232,102 +242,127 @@ def simulate_2cta(nkts, seed, drop=()):
     def producer():
         t = 0
         for i, n in enumerate(nkts):
-            if i > 0 and 'q_empty' not in drop:
-                yield from wait('q_empty', i - 1)
-            tma.append(('Q', i))
-            for _ in range(n):
-                if t > 0:
-                    yield from wait('k_empty', t - 1)
-                tma.append(('K', t))
-                if t > 0:
-                    yield from wait('v_empty', t - 1)
-                tma.append(('V', t))
+            for j in range(n):
+                s = t & 1
+                if t >= 2 and 'k_empty' not in drop:
+                    yield from wait(f'k_empty{s}', (t >> 1) - 1)
+                if t >= 2 and not {(0, t - 2), (1, t - 2)} <= st['s_done']:
+                    raise ProtocolError('K stage reloaded while still read')
+                tma.append(('K', s, t))
+                if j == 0:
+                    for x in range(2):
+                        if i >= 1:
+                            if 'q_empty' not in drop:
+                                yield from wait(f'q_empty{x}', i - 1)
+                            last = first[i - 1] + nkts[i - 1] - 1
+                            if (x, last) not in st['s_done']:
+                                raise ProtocolError('Q buffer reloaded while still read')
+                        tma.append(('Q', x, i))
+                if t >= 2:
+                    yield from wait(f'v_empty{s}', (t >> 1) - 1)
+                    if not {(0, t - 2), (1, t - 2)} <= st['pv_done']:
+                        raise ProtocolError('V stage reloaded while still read')
+                tma.append(('V', s, t))
                 t += 1
                 yield 'step'
 
     def mma():
         t = 0
         for i, n in enumerate(nkts):
-            yield from wait('q_full', i)
-            for j in range(n):
-                if t > 0 and 'mma_o_done' not in drop:
-                    yield from wait('o_done', t - 1)
-                yield from wait('k_full', t)
-                tc.extend([('S', t, i), ('commit', 's_full'), ('commit', 'k_empty')])
-                if j + 1 == n:
-                    tc.append(('commit', 'q_empty'))
-                yield from wait('p_full', t)
-                yield from wait('v_full', t)
-                tc.extend([('PV', t, i, j), ('commit', 'v_empty'), ('commit', 'o_done')])
-                t += 1
-                yield 'step'
+            for x in range(2):
+                yield from wait(f'q_full{x}', i)
 
-    def softmax():
+            def issue_s(x, tt, last):
+                if tt > 0 and 'o_done_before_s' not in drop:
+                    yield from wait(f'o_done{x}', tt - 1)
+                if tt > 0 and (x, tt - 1) not in st['pv_done']:
+                    raise ProtocolError('S overwrites a P whose product has not run')
+                if x == 0:
+                    yield from wait(f'k_full{tt & 1}', tt >> 1)
+                tc.append(('S', x, tt, i))
+                tc.append(('commit', f's_full{x}'))
+                if x == 1:
+                    tc.append(('commit', f'k_empty{tt & 1}'))
+                if last:
+                    tc.append(('commit', f'q_empty{x}'))
+
+            def issue_pv(x, tt, j):
+                yield from wait(f'p_full{x}', tt)
+                if x == 0:
+                    yield from wait(f'v_full{tt & 1}', tt >> 1)
+                tc.append(('PV', x, tt, i, j))
+                if x == 1:
+                    tc.append(('commit', f'v_empty{tt & 1}'))
+                tc.append(('commit', f'o_done{x}'))
+
+            yield from issue_s(0, t, n == 1)
+            yield from issue_s(1, t, n == 1)
+            for j in range(n):
+                tj = t + j
+                more, last_next = j + 1 < n, j + 2 == n
+                yield from issue_pv(0, tj, j)
+                if more:
+                    yield from issue_s(0, tj + 1, last_next)
+                yield from issue_pv(1, tj, j)
+                if more:
+                    yield from issue_s(1, tj + 1, last_next)
+                yield 'step'
+            t += n
+
+    def softmax(x):
         t = 0
         for i, n in enumerate(nkts):
             for j in range(n):
-                yield from wait('s_full', t)
-                if st['S'] != t:
+                yield from wait(f's_full{x}', t)
+                if st['S'][x] != t:
                     raise ProtocolError('softmax read a stale S')
-                if j > 0 and (st['O_item'] != i or t - 1 not in st['pv_done']):
-                    raise ProtocolError('rescaled an O that is not up to date')
                 yield 'step'
-                if st['S'] != t:
-                    raise ProtocolError('S overwritten while the softmax read it')
-                st['s_read'].add(t)
-                st['P'] = t
-                bars['p_full'].arrive()
+                if rng.random() < 0.3 and j > 0:   # a rescale of O: no wait
+                    if st['O'][x] != i or (x, t - 1) not in st['pv_done']:
+                        raise ProtocolError('rescaled an O that is not up to date')
+                if st['S'][x] != t:
+                    raise ProtocolError('S overwritten before P was stored')
+                st['P'][x] = t
+                bars[f'p_full{x}'].arrive()
                 t += 1
             if 'softmax_o_final' not in drop:
-                yield from wait('o_done', t - 1)
+                yield from wait(f'o_done{x}', t - 1)
             want = set(range(t - n, t))
-            if st['O_item'] != i or st['O_tiles'] != want:
+            if st['O'][x] != i or st['O_tiles'][x] != want:
                 raise ProtocolError('read the wrong O')
             yield 'step'
-            if st['O_item'] != i or st['O_tiles'] != want:
+            if st['O'][x] != i or st['O_tiles'][x] != want:
                 raise ProtocolError('O changed while being read')
-            st['o_read'].add(i)
+            st['o_read'][x].add(i)
 
     def run_tma():
-        op = tma.pop(0)
-        kind, x = op
-        if kind == 'Q':
-            if x > 0 and not set(range(first[x - 1], first[x - 1] + nkts[x - 1])) <= st['s_done']:
-                raise ProtocolError('Q reloaded while still read')
-        elif kind == 'K':
-            if x > 0 and x - 1 not in st['s_done']:
-                raise ProtocolError('K reloaded while still read')
-        elif x > 0 and x - 1 not in st['pv_done']:
-            raise ProtocolError('V reloaded while still read')
-        st[kind] = x
-        bars[f'{kind.lower()}_full'].arrive()
+        kind, s, v = tma.pop(0)
+        st[kind][s] = v
+        bars[f'{kind.lower()}_full{s}'].arrive()
 
     def run_tc():
         op = tc.pop(0)
         if op[0] == 'S':
-            _, t, i = op
-            if st['Q'] != i or st['K'] != t:
+            _, x, tt, i = op
+            if st['Q'][x] != i or st['K'][tt & 1] != tt:
                 raise ProtocolError('S product read a stale Q or K')
-            if t > 0 and t - 1 not in st['pv_done']:
-                raise ProtocolError('S overwrote a P before its product ran')
-            if t > 0 and t - 1 not in st['s_read']:
-                raise ProtocolError('S overwritten before it was read')
-            st['S'] = t
-            st['s_done'].add(t)
+            st['S'][x] = tt
+            st['P'][x] = None
+            st['s_done'].add((x, tt))
         elif op[0] == 'PV':
-            _, t, i, j = op
-            if st['P'] != t or st['V'] != t:
+            _, x, tt, i, j = op
+            if st['P'][x] != tt or st['V'][tt & 1] != tt:
                 raise ProtocolError('P V product read a stale P or V')
             if j == 0:
-                if i > 0 and i - 1 not in st['o_read']:
+                if i > 0 and i - 1 not in st['o_read'][x]:
                     raise ProtocolError('O overwritten before it was read')
-                st['O_item'], st['O_tiles'] = i, set()
-            st['O_tiles'].add(t)
-            st['pv_done'].add(t)
+                st['O'][x], st['O_tiles'][x] = i, set()
+            st['O_tiles'][x].add(tt)
+            st['pv_done'].add((x, tt))
         else:
             bars[op[1]].arrive()
 
-    actors = {'producer': producer(), 'mma': mma(), 'softmax': softmax()}
+    actors = {'producer': producer(), 'mma': mma(), 'a': softmax(0), 'b': softmax(1)}
     rate = {a: rng.choice([0.05, 0.3, 1.0]) for a in list(actors) + ['tma', 'tc']}
     finished, idle = set(), 0
     while len(finished) < len(actors):
@@ -353,21 +388,17 @@ def simulate_2cta(nkts, seed, drop=()):
             raise ProtocolError(f'deadlock; finished: {sorted(finished)}')
     while tc:
         run_tc()
-    if len(st['o_read']) != len(nkts):
+    if any(len(r) != len(nkts) for r in st['o_read']):
         raise ProtocolError('an item was never written out')
 
 
-def test_2cta_protocol_holds_under_random_schedules():
+def test_dual_protocol_holds_under_random_schedules():
     for nkts, seed in _cases(400):
-        simulate_2cta(nkts, seed)
+        simulate_dual(nkts, seed)
 
 
-# (The MMA issuer's wait for the previous P V product before the next S is
-# not in this list: the model's tensor engine completes operations in issue
-# order, which already keeps S behind that product; the wait keeps the kernel
-# correct without relying on that order.)
-@pytest.mark.parametrize('drop', ['softmax_o_final', 'q_empty'])
-def test_2cta_dropping_a_wait_is_caught(drop):
+@pytest.mark.parametrize('drop', ['o_done_before_s', 'softmax_o_final', 'q_empty', 'k_empty'])
+def test_dual_dropping_a_wait_is_caught(drop):
     with pytest.raises(ProtocolError):
         for nkts, seed in _cases(400):
-            simulate_2cta(nkts, seed, drop=(drop,))
+            simulate_dual(nkts, seed, drop=(drop,))
