@@ -130,10 +130,14 @@ def test_argmax_rows_exact_with_ties():
 
 
 # ----------------------------------------------------- prefill attention
+# Even query heads per KV head run the two-heads-per-item kernel at every
+# length; otherwise up to 4096 queries run the one-head persistent kernel and
+# longer chunks the per-tile kernel (the group-1 and group-3 cases below).
 PREFILL_CASES = [(BF16, 2, 200, 8, 2), (BF16, 1, 1, 4, 1), (BF16, 1, 64, 4, 4), (BF16, 1, 65, 8, 2),
                  (BF16, 1, 2048, 32, 8), (BF16, 2, 300, 32, 8), (BF16, 1, 4097, 8, 2), (BF16, 3, 129, 4, 1),
                  (F16, 2, 200, 8, 2), (F16, 1, 1, 4, 1), (F16, 1, 2048, 32, 8), (F16, 1, 4097, 8, 2),
-                 (F16, 3, 129, 4, 1)]
+                 (F16, 3, 129, 4, 1), (F16, 2, 300, 6, 2), (BF16, 1, 4200, 6, 2), (F16, 1, 4097, 3, 3),
+                 (BF16, 1, 1000, 2, 2)]
 
 
 @pytest.mark.parametrize('dtype,B,S,H,Hk', PREFILL_CASES)
