@@ -409,6 +409,20 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
   TileCursor ld, cp;
   tc_seek(ld, x0, x1 - x0, nkeys, add_keys, nmax, B, Hk);
   cp = ld;
+  const int row = lane >> 2, tq = lane & 3;   // fragment row (query head within the group), column pair
+  const bool real = row < G;
+  uint32_t qa[8][2];
+  // the first piece's query rows before the ring fills, so that they do not
+  // queue behind every warp's first K/V tiles
+  auto load_q = [&](const TileCursor& c) {
+    const T* qr = q + ((size_t)c.b * H + c.g * G + (real ? row : 0)) * 128;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      qa[ks][0] = real ? *reinterpret_cast<const uint32_t*>(qr + ks * 16 + 2 * tq) : 0u;
+      qa[ks][1] = real ? *reinterpret_cast<const uint32_t*>(qr + ks * 16 + 8 + 2 * tq) : 0u;
+    }
+  };
+  if (cp.left > 0) load_q(cp);
   int issued = 0;
   bool ld_done = ld.left <= 0;
   for (int i = 0; i < DM_STAGES - 1; ++i) {
@@ -421,21 +435,14 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
     cp_async_commit();
   }
 
-  const int row = lane >> 2, tq = lane & 3;   // fragment row (query head within the group), column pair
-  const bool real = row < G;
-  uint32_t qa[8][2];
   float oacc[16][2];
   float m_r = -INFINITY, l_r = 0.f;
   int consumed = 0;
-  bool start = true;
+  bool start = true, first_piece = true;
   while (cp.left > 0) {
     if (start) {   // new piece: reset the state and fetch the G query rows of (b, g)
-      const T* qr = q + ((size_t)cp.b * H + cp.g * G + (real ? row : 0)) * 128;
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        qa[ks][0] = real ? *reinterpret_cast<const uint32_t*>(qr + ks * 16 + 2 * tq) : 0u;
-        qa[ks][1] = real ? *reinterpret_cast<const uint32_t*>(qr + ks * 16 + 8 + 2 * tq) : 0u;
-      }
+      if (!first_piece) load_q(cp);
+      first_piece = false;
 #pragma unroll
       for (int n = 0; n < 16; ++n) oacc[n][0] = oacc[n][1] = 0.f;
       m_r = -INFINITY;
@@ -591,33 +598,53 @@ __global__ void __launch_bounds__(128) attn_decode_combine_pieces_kernel(
   }
   const int cnt = s_cnt < kMaxDecodeWarps ? s_cnt : kMaxDecodeWarps;   // the host keeps W <= kMaxDecodeWarps
   const size_t bg = (size_t)b * Hk + g;
-  // M = the largest piece maximum
+  // every piece's (maximum, sum), one thread per piece, and M = the largest maximum
   __shared__ float s_red[4];
+  __shared__ float s_m[kMaxDecodeWarps], s_ls[kMaxDecodeWarps];
   float M = -INFINITY;
-  for (int k = threadIdx.x; k < cnt; k += blockDim.x) M = fmaxf(M, part[((bg + s_w[k]) * G + row) * (D + 2) + D]);
+  for (int k = threadIdx.x; k < cnt; k += blockDim.x) {
+    const float* r = part + ((bg + s_w[k]) * G + row) * (D + 2);
+    s_m[k] = r[D];
+    s_ls[k] = r[D + 1];
+    M = fmaxf(M, s_m[k]);
+  }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = M;
   __syncthreads();
   M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
+  for (int k = threadIdx.x; k < cnt; k += blockDim.x) s_m[k] = exp2f(s_m[k] - M);   // the piece's weight
+  __syncthreads();
   // warp q merges pieces [cnt*q/4, cnt*(q+1)/4), lane i dims 4i .. 4i+3 (loads
-  // of consecutive lanes are contiguous); the four warps' sums are then added
-  // in warp order, so the merge order is fixed
+  // of consecutive lanes are contiguous), eight pieces' loads in flight; the
+  // four warps' sums are then added in warp order, so the merge order is fixed
   static_assert(D == 128, "one 4-dim slice per lane");
   const int q = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k0 = cnt * q / 4, k1 = cnt * (q + 1) / 4;
   float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f, L = 0.f;
-#pragma unroll 4
-  for (int k = k0; k < k1; ++k) {
-    const float* r = part + ((bg + s_w[k]) * G + row) * (D + 2);
-    const float f = exp2f(r[D] - M);
-    const float2 a = *reinterpret_cast<const float2*>(r + 4 * lane);
-    const float2 c = *reinterpret_cast<const float2*>(r + 4 * lane + 2);
-    L += r[D + 1] * f;
-    acc0 += a.x * f;
-    acc1 += a.y * f;
-    acc2 += c.x * f;
-    acc3 += c.y * f;
+  for (int kb = k0; kb < k1; kb += 8) {
+    float2 a[8], c[8];   // rows are D + 2 floats apart: 8-byte aligned
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (kb + u < k1) {
+        const float* r = part + ((bg + s_w[kb + u]) * G + row) * (D + 2) + 4 * lane;
+        a[u] = *reinterpret_cast<const float2*>(r);
+        c[u] = *reinterpret_cast<const float2*>(r + 2);
+      } else {
+        a[u] = c[u] = make_float2(0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (kb + u < k1) {
+        const float f = s_m[kb + u];
+        L += s_ls[kb + u] * f;
+        acc0 += a[u].x * f;
+        acc1 += a[u].y * f;
+        acc2 += c[u].x * f;
+        acc3 += c[u].y * f;
+      }
+    }
   }
   __shared__ float s_acc[4][D];
   __shared__ float s_l[4];

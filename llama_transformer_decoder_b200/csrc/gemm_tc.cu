@@ -767,16 +767,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             __stcg(p4 + (c * 8 + j) * 128, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
           continue;
         }
-        if (owner) {  // add the other shares in CTA order
-          for (long long cc = c_own + 1; cc <= c_hi; ++cc) {
-            if (sk_first(cc + 1, U, G) <= sk_first(cc, U, G)) continue;   // no units
-            const float4* p4 = reinterpret_cast<const float4*>(ws) + (size_t)cc * (NT * S_BM / 4) + tid;
-            float4 x[8];
+        if (owner) {  // add the other shares in CTA order, four shares' loads in flight at a time
+          for (long long c0 = c_own + 1; c0 <= c_hi; c0 += 4) {
+            float4 x[4][8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) x[j] = __ldcg(p4 + (c * 8 + j) * 128);
+            for (int q = 0; q < 4; ++q) {
+              const long long cc = c0 + q;
+              if (cc <= c_hi && sk_first(cc + 1, U, G) > sk_first(cc, U, G)) {   // a CTA with units
+                const float4* p4 = reinterpret_cast<const float4*>(ws) + (size_t)cc * (NT * S_BM / 4) + tid;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              v[4 * j] += x[j].x; v[4 * j + 1] += x[j].y; v[4 * j + 2] += x[j].z; v[4 * j + 3] += x[j].w;
+                for (int j = 0; j < 8; ++j) x[q][j] = __ldcg(p4 + (c * 8 + j) * 128);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) x[q][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+              }
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                v[4 * j] += x[q][j].x; v[4 * j + 1] += x[q][j].y; v[4 * j + 2] += x[q][j].z; v[4 * j + 3] += x[q][j].w;
+              }
             }
           }
         }

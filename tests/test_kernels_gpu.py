@@ -183,6 +183,7 @@ def test_attention_prefill_f32(d):
     (BF16, 128, 2, 8, 8, 4097, [4097, 130]),
     (BF16, 128, 2, 16, 2, 300, [300, 45]),                   # 8 query heads per kv head
     (BF16, 128, 32, 32, 8, 4224, [4097 + 4 * i for i in range(32)]),   # batch-32 decode shape
+    (BF16, 128, 24, 32, 8, 8192, [1 + 341 * i for i in range(24)]),      # ragged lengths, 1 to 7844
     (BF16, 128, 1, 32, 8, 131072, [131072]),                 # longest cache of the sweep
     (BF16, 128, 64, 32, 8, 1024, [1 + 16 * i for i in range(64)]),
     (F16, 128, 1, 8, 1, 65536, [65536]),                   # one kv head: every decoding warp holds a piece of it
@@ -205,7 +206,7 @@ def test_attention_decode(dtype, d, B, H, Hk, cmax, lens):
     torch.cuda.synchronize()
     _sync_ok()
     got = o.float().cpu().numpy()
-    for b in (range(B) if B <= 8 else [0, 1, B // 2, B - 1]):
+    for b in (range(B) if B <= 32 else [0, 1, B // 2, B - 1]):
         n = lens[b]
         worst, err = attention_row_errors(got[b][None], qv[b][:, None, :].astype(np.float64),
                                           kv[b][:, :n].astype(np.float64), vv[b][:, :n].astype(np.float64),
