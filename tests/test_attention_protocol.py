@@ -211,7 +211,7 @@ def test_dropping_a_wait_is_caught(drop):
             simulate(nkts, seed, drop=(drop,))
 
 
-# ------------------------------------------------------- two CTAs per SM
+# ------------------------------------------------ two heads of a group per item
 def simulate_dual(nkts, seed, drop=()):
     """The barrier protocol of attn_prefill_tc_dual_kernel: items of two query
     tiles (A, B) that share every K and V tile; one Q buffer per tile; S_X
