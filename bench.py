@@ -279,7 +279,9 @@ D_, F_, H_, HK_, HD_, V_ = 4096, 14336, 32, 8, 128, 128256
 # Measured DRAM bytes per launch of the chained prefill projection GEMM (one
 # layer's Wo, w1/w3, w2 and the next QKV at 2048 tokens; one ncu capture of
 # the current kernel). None until captured for the current kernel.
-PAIR_GEMM_TRAFFIC = None
+# DRAM read + write bytes of one middle layer's chained launch (Wo, w1/w3,
+# w2, next QKV) from an ncu capture (profiles/gemm_chain_kernel_dram_llama3_8b_layer.md)
+PAIR_GEMM_TRAFFIC = 1096.8e6 + 163.6e6
 
 
 def measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust, peak_src, B=PREFILL_B):
@@ -336,8 +338,9 @@ def measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust, peak_src,
                           'next layer\'s QKV, plus layer 0\'s QKV)', 'bound': 'tensor',
                 'achieved': achieved, 'peak': tf_sust, 'unit': 'TFLOP/s',
                 'frac': achieved / tf_sust if achieved else None, 'traffic': PAIR_GEMM_TRAFFIC,
-                'traffic_note': 'DRAM read+write bytes per chained launch from one ncu capture (null: not yet '
-                                'captured for this kernel)',
+                'traffic_note': 'DRAM read+write bytes of a middle layer\'s chained launch from one ncu capture '
+                                '(1.3x its operand bytes: w1/w3 weights stream twice by design, w2\'s weight is '
+                                'partly re-read per row block)',
                 'peak_kind': f'bf16 sustained ({peak_src}); fp16 has the same nominal tensor rate',
                 'launches': gemm_launches // max(args.steps, 1),
                 'attention_tflops': attn_flops * args.steps / (attn[0] / 1e3) / 1e12 if attn[0] else None,
