@@ -280,7 +280,7 @@ D_, F_, H_, HK_, HD_, V_ = 4096, 14336, 32, 8, 128, 128256
 # layer's Wo, w1/w3, w2 and the next QKV at 2048 tokens; one ncu capture of
 # the current kernel). None until captured for the current kernel.
 # DRAM read + write bytes of one middle layer's chained launch (Wo, w1/w3,
-# w2, next QKV) from an ncu capture (profiles/gemm_chain_kernel_dram_llama3_8b_layer.md)
+# w2, next QKV), from an ncu capture of a 2-layer model of the 8B shapes
 PAIR_GEMM_TRAFFIC = 1096.8e6 + 163.6e6
 
 
