@@ -30,6 +30,7 @@ sys.path.insert(0, ROOT)
 METRIC = 'tokens/s: 8B-shape prefill & batch-32 decode; % tensor/HBM roofline'
 PREFILL_B, PREFILL_S = 1, 2048
 PREFILL_B8 = 8
+LONG_S, LONG_CHUNK = 32768, 4096       # long-context leg: one layer, chunked prefill
 DECODE_B, DECODE_CTX, DECODE_STEPS = 32, 4096, 128
 
 
@@ -470,6 +471,55 @@ def measure_block(L, m, st, S, args, hbm_peak, tf_burst, tf_sust, peak_src):
     return out
 
 
+def measure_long(L, st, args, tf_burst, peak_src):
+    """Long-context prefill through one 8B-shaped decoder layer: 32768
+    positions of one sequence fed through llama_block_forward in 4096-token
+    chunks, each chunk's queries attending to every earlier chunk's keys in
+    the cache (N(0,1) hidden states; a separate one-layer model with a
+    32768-position cache). Causal attention is ~38% of the flops here against
+    ~4% at 2048 tokens."""
+    import numpy as np
+    import torch
+    from llama_transformer_decoder_b200.configs import LLAMA3_8B, make_config
+    cfg = make_config(LLAMA3_8B, dtype=L.LLAMA_BF16, max_batch=1, max_seq=LONG_S, max_tokens=LONG_CHUNK, n_layers=1)
+    m2 = L.llama_create(cfg)
+    try:
+        L.llama_init_weights(m2, 0, 0.02, st)
+        x = torch.empty((1, LONG_CHUNK, D_), dtype=torch.float32, device='cuda')
+        L.llama_fill_normal(x, x.numel(), 2, (1 << 20) + 2, 1.0, L.LLAMA_F32, st)
+        y = torch.empty_like(x)
+
+        def one_pass():
+            for a in range(0, LONG_S, LONG_CHUNK):
+                L.llama_set_lengths(m2, np.array([a], np.int32), 1, st)
+                L.llama_block_forward(m2, 0, x, y, 1, LONG_CHUNK, st)
+
+        one_pass()
+        torch.cuda.synchronize()
+        reps = max(2, min(args.steps, 5))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(reps):
+            one_pass()
+        e1.record(st)
+        torch.cuda.synchronize()
+        assert L.llama_sync_status(m2, st) == 0
+        ms = e0.elapsed_time(e1) / reps
+    finally:
+        L.llama_destroy(m2)
+    w_elems = D_ * (H_ + 2 * HK_) * HD_ + D_ * H_ * HD_ + 3 * D_ * F_
+    lin = 2.0 * LONG_S * w_elems
+    attn = 4.0 * H_ * HD_ * LONG_S * (LONG_S + 1) / 2
+    tf = (lin + attn) / (ms / 1e3) / 1e12
+    return {'value': LONG_S / (ms / 1e3), 'unit': 'tokens/s', 'ms_per_pass': ms, 'passes': reps,
+            'workload': f'one 8B-shaped decoder layer, B=1, {LONG_S} positions in {LONG_CHUNK}-token chunks '
+                        '(chunked prefill over the cache), N(0,1) hidden states',
+            'attention_share_of_flops': attn / (lin + attn),
+            'roofline': {'bound': 'tensor', 'achieved': tf, 'peak': tf_burst, 'unit': 'TFLOP/s', 'frac': tf / tf_burst,
+                         'work': 'linear + causal attention flops per pass',
+                         'peak_kind': f'bf16 burst ({peak_src}): one layer timed alone'}}
+
+
 def run_ours(args):
     import torch
     ws, rank, local = _dist()
@@ -495,7 +545,7 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     ms = launches = clk = roofline = kernels = e2e = None
-    prefill_b8 = blocks = None
+    prefill_b8 = blocks = long_prefill = None
     if not args.decode_only:
         ms, launches, clk, roofline, kernels = measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust,
                                                                peak_src)
@@ -509,6 +559,7 @@ def run_ours(args):
                           'seq_len': PREFILL_S, 'roofline': roof8, 'clocks': clk8}
             blocks = {f's{S}': measure_block(L, m, st, S, args, hbm_peak, tf_burst, tf_sust, peak_src)
                       for S in (17, 2048)}
+            long_prefill = measure_long(L, st, args, tf_burst, peak_src)
     decode = None if args.no_decode else measure_decode(L, m, st, arg, args, ws, local, NL, hbm_peak, peak_src)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and NL == 32 and not args.decode_only:
@@ -524,7 +575,7 @@ def run_ours(args):
                 'config': workload_config(ws, args, NL),
                 'roofline': roofline, 'cpu_baseline': cpu, 'e2e': e2e, 'gpu_launches': launches,
                 'clocks': clk, 'kernels': kernels, 'decode': decode, 'prefill_b8': prefill_b8,
-                'block_8b': blocks}
+                'block_8b': blocks, 'long_prefill': long_prefill}
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist

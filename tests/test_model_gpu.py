@@ -165,8 +165,8 @@ def test_block_8b_bf16(block8b, B, S):
 
 def test_block_8b_bf16_activations():
     """act_dtype = LLAMA_BF16: weights, activations, cache and P all in bf16,
-    as the pages compute. One 8B-shaped block at S = 2048 (pair GEMMs and the
-    persistent attention kernel) and S = 17 (skinny GEMMs) against the
+    as the pages compute. One 8B-shaped block at S = 2048 (CTA-pair GEMMs and
+    the two-heads-per-item attention kernel) and S = 17 (skinny GEMMs) against the
     oracle, rel-L2 <= 2e-2 (one layer of bf16 roundings is about 1.5e-3)."""
     m = Model(dict(BLOCK_8B, act_dtype=BF16), BF16, max_batch=1, max_seq=2048, max_tokens=2048)
     try:
@@ -595,8 +595,8 @@ def test_long_context_8b_prefill_tokens_to_32k():
 def test_long_context_8b_block_chunks_sampled_rows(S_total, chunk):
     """The same layer on N(0,1) hidden states, fed chunk by chunk through
     llama_block_forward with the cached length advanced between chunks (the
-    cache holds every earlier chunk's keys and values; 8192-token chunks run
-    the per-tile attention kernel, 4096-token chunks the persistent one). 64
+    cache holds every earlier chunk's keys and values; chunks of either size
+    run the two-heads-per-item attention kernel). 64
     sampled rows of the last chunk plus its last row are checked against the
     oracle's layer over the whole sequence (rel-L2 <= 2e-2)."""
     m = Model(LONG_8B, BF16, max_batch=1, max_seq=S_total + 8, max_tokens=chunk)
