@@ -315,9 +315,6 @@ constexpr int DM_WARPS = 4;
 constexpr int DM_TILE = DM_KEYS * 256;             // one K (or V) tile: 32 rows x 256 B
 constexpr int DM_STAGE = 2 * DM_TILE;
 constexpr int DM_SMEM = DM_WARPS * DM_STAGES * DM_STAGE;
-// Decoding warps of the grid (SMs x DM_WARPS) the combine can merge for one
-// (sequence, kv head): every warp of the grid may hold a piece of it.
-constexpr int kMaxDecodeWarps = 1024;
 
 __device__ __forceinline__ int dm_keys(const int32_t* nkeys, int b, int add, int nmax) {
   return min(nkeys[b] + add, nmax);
@@ -540,124 +537,126 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
   cp_async_wait<0>();
 }
 
-// Merge the pieces of every (b, h): the warps holding tiles of (b, g) are
-// owner(T0) .. owner(T1-1), owner(x) = ((x+1)W - 1) / T.
-template <typename T, int D>
-__global__ void __launch_bounds__(128) attn_decode_combine_pieces_kernel(
+// Merge the pieces of every (b, h). The warps holding tiles of (b, g) are
+// owner(t0) .. owner(t0 + nt - 1), owner(x) = ((x+1)W - 1) / T: when T >= W
+// every warp's range is non-empty, so the pieces are all the warps between
+// those two; when T < W every warp holds at most one tile, so piece k is the
+// owner of tile t0 + k. A block of CW warps serves CW / wh heads (flattened
+// b*H + h), wh warps each: warp j of a head merges its pieces
+// [cnt j / wh, cnt (j+1) / wh), loading CB pieces at a time with every load in
+// flight and keeping a running (max, sum, o) rescaled as the maximum grows;
+// the wh warps' results are then merged in warp order. The order is fixed, so
+// results do not depend on timing. wh (1, 2, 4 or 8) and CB are chosen on
+// the host from the pieces a head is expected to have: many pieces per head
+// when B * Hk is small, few when it is large (a smaller CB then holds fewer
+// registers, leaving room on the SM for the next kernel's early blocks).
+constexpr int CW = 8;        // warps of a combine block
+constexpr int CB_MAX = 12;   // pieces a warp loads per round, at most
+
+template <typename T, int D, int CB>
+__global__ void __launch_bounds__(CW * 32) attn_decode_combine_pieces_kernel(
     const float* __restrict__ part, const int32_t* __restrict__ nkeys, int add_keys, int nmax, T* __restrict__ o,
-    int B, int H, int Hk, long long W) {
+    int B, int H, int Hk, long long W, int wh) {
+  static_assert(D == 128, "one 4-dim slice per lane");
   pdl_trigger();
   pdl_wait();
-  __shared__ long long s_tot, s_t0;
-  __shared__ int s_nt, s_cnt;
-  __shared__ int s_w[kMaxDecodeWarps];
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int G = H / Hk, g = h / G, row = h - g * G;
-  if (threadIdx.x == 0) {
-    long long total = 0, t0 = 0;
-    int nt_b = 0;
-    for (int bb = 0; bb < B; ++bb) {
-      const int nt = dm_tiles(dm_keys(nkeys, bb, add_keys, nmax));
-      if (bb == b) { t0 = total + (long long)g * nt; nt_b = nt; }
-      total += (long long)Hk * nt;
-    }
-    s_tot = total; s_t0 = t0; s_nt = nt_b;
-  }
-  __syncthreads();
-  const long long total = s_tot, t0 = s_t0;
-  const int nt_b = s_nt;
-  const int nb = nkeys[b] + add_keys;
-  // no keys, or more keys than the cache holds (clamped for the other
-  // sequences' sake, latched by the decode kernel): NaN rows, as the split path
-  if (nt_b == 0 || total == 0 || nb < 1 || nb > nmax) {
-    for (int dd = threadIdx.x; dd < D; dd += blockDim.x) o[((size_t)b * H + h) * D + dd] = from_f<T>(NAN);
-    return;
-  }
-  // warps owning tiles of (b, g): owner(t0) .. owner(t0 + nt_b - 1), skipping
-  // warps with empty ranges, listed in warp order (a fixed merge order, so
-  // results do not depend on timing)
-  const long long w_lo = ((t0 + 1) * W - 1) / total, w_hi = ((t0 + nt_b) * W - 1) / total;
-  __shared__ int s_warp_cnt[4];
-  if (threadIdx.x == 0) s_cnt = 0;
-  __syncthreads();
-  for (long long base = w_lo; base <= w_hi; base += blockDim.x) {
-    const long long w = base + threadIdx.x;
-    const bool has = w <= w_hi && total * (w + 1) / W > total * w / W;
-    const unsigned bal = __ballot_sync(0xffffffffu, has);
-    if ((threadIdx.x & 31) == 0) s_warp_cnt[threadIdx.x >> 5] = __popc(bal);
-    __syncthreads();
-    int off = s_cnt;
-    for (int q = 0; q < (int)(threadIdx.x >> 5); ++q) off += s_warp_cnt[q];
-    if (has) {
-      const int k = off + __popc(bal & ((1u << (threadIdx.x & 31)) - 1u));
-      if (k < kMaxDecodeWarps) s_w[k] = (int)w;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) s_cnt += s_warp_cnt[0] + s_warp_cnt[1] + s_warp_cnt[2] + s_warp_cnt[3];
-    __syncthreads();
-  }
-  const int cnt = s_cnt < kMaxDecodeWarps ? s_cnt : kMaxDecodeWarps;   // the host keeps W <= kMaxDecodeWarps
-  const size_t bg = (size_t)b * Hk + g;
-  // every piece's (maximum, sum), one thread per piece, and M = the largest maximum
-  __shared__ float s_red[4];
-  __shared__ float s_m[kMaxDecodeWarps], s_ls[kMaxDecodeWarps];
-  float M = -INFINITY;
-  for (int k = threadIdx.x; k < cnt; k += blockDim.x) {
-    const float* r = part + ((bg + s_w[k]) * G + row) * (D + 2);
-    s_m[k] = r[D];
-    s_ls[k] = r[D + 1];
-    M = fmaxf(M, s_m[k]);
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = M;
-  __syncthreads();
-  M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
-  for (int k = threadIdx.x; k < cnt; k += blockDim.x) s_m[k] = exp2f(s_m[k] - M);   // the piece's weight
-  __syncthreads();
-  // warp q merges pieces [cnt*q/4, cnt*(q+1)/4), lane i dims 4i .. 4i+3 (loads
-  // of consecutive lanes are contiguous), eight pieces' loads in flight; the
-  // four warps' sums are then added in warp order, so the merge order is fixed
-  static_assert(D == 128, "one 4-dim slice per lane");
+  __shared__ float s_mq[CW], s_lq[CW];
+  __shared__ float s_acc[CW][D];
+  __shared__ int s_bad[CW];
   const int q = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int k0 = cnt * q / 4, k1 = cnt * (q + 1) / 4;
-  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f, L = 0.f;
-  for (int kb = k0; kb < k1; kb += 8) {
-    float2 a[8], c[8];   // rows are D + 2 floats apart: 8-byte aligned
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (kb + u < k1) {
-        const float* r = part + ((bg + s_w[kb + u]) * G + row) * (D + 2) + 4 * lane;
-        a[u] = *reinterpret_cast<const float2*>(r);
-        c[u] = *reinterpret_cast<const float2*>(r + 2);
-      } else {
-        a[u] = c[u] = make_float2(0.f, 0.f);
-      }
+  const int hpb = CW / wh;   // heads per block
+  const long long bh = (long long)blockIdx.x * hpb + q / wh;
+  const int j = q % wh;
+  const int G = H / Hk;
+  float M = -INFINITY, L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (bh < (long long)B * H) {
+    const int b = (int)(bh / H), h = (int)(bh - (long long)b * H);
+    const int g = h / G, row = h - g * G;
+    // T and the tiles of the sequences before b, the lengths loaded 32 at a time
+    long long total = 0, t0 = 0;
+    for (int bb = lane; bb < B; bb += 32) {
+      const long long c = (long long)Hk * dm_tiles(dm_keys(nkeys, bb, add_keys, nmax));
+      total += c;
+      if (bb < b) t0 += c;
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (kb + u < k1) {
-        const float f = s_m[kb + u];
-        L += s_ls[kb + u] * f;
-        acc0 += a[u].x * f;
-        acc1 += a[u].y * f;
-        acc2 += c[u].x * f;
-        acc3 += c[u].y * f;
+    for (int off = 16; off > 0; off >>= 1) {
+      total += __shfl_xor_sync(0xffffffffu, total, off);
+      t0 += __shfl_xor_sync(0xffffffffu, t0, off);
+    }
+    const int nb = nkeys[b] + add_keys;
+    const int nt_b = dm_tiles(dm_keys(nkeys, b, add_keys, nmax));
+    t0 += (long long)g * nt_b;
+    // no keys, or more keys than the cache holds (clamped for the other
+    // sequences' sake, latched by the decode kernel): NaN rows, as the split path
+    const bool bad = nt_b == 0 || total == 0 || nb < 1 || nb > nmax;
+    if (j == 0 && lane == 0) s_bad[q / wh] = bad;
+    if (!bad) {
+      const long long w_lo = ((t0 + 1) * W - 1) / total;
+      const bool dense = total >= W;
+      const int cnt = dense ? (int)(((t0 + nt_b) * W - 1) / total - w_lo + 1) : nt_b;
+      const size_t bg = (size_t)b * Hk + g;
+      const int k0 = cnt * j / wh, k1 = cnt * (j + 1) / wh;
+      for (int kb = k0; kb < k1; kb += CB) {
+        float2 a[CB], c[CB], ml[CB];   // rows are D + 2 floats apart: 8-byte aligned
+#pragma unroll
+        for (int u = 0; u < CB; ++u) {
+          if (kb + u < k1) {
+            const long long k = kb + u;
+            const long long w = dense ? w_lo + k : ((t0 + k + 1) * W - 1) / total;
+            const float* r = part + ((bg + w) * G + row) * (D + 2);
+            a[u] = *reinterpret_cast<const float2*>(r + 4 * lane);
+            c[u] = *reinterpret_cast<const float2*>(r + 4 * lane + 2);
+            ml[u] = *reinterpret_cast<const float2*>(r + D);
+          } else {
+            a[u] = c[u] = make_float2(0.f, 0.f);
+            ml[u] = make_float2(-INFINITY, 0.f);
+          }
+        }
+        float Mc = M;
+#pragma unroll
+        for (int u = 0; u < CB; ++u) Mc = fmaxf(Mc, ml[u].x);
+        const float s = M == -INFINITY ? 0.f : exp2f(M - Mc);
+        L *= s;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] *= s;
+#pragma unroll
+        for (int u = 0; u < CB; ++u) {
+          const float f = exp2f(ml[u].x - Mc);   // 0 for the padding
+          L += ml[u].y * f;
+          acc[0] += a[u].x * f;
+          acc[1] += a[u].y * f;
+          acc[2] += c[u].x * f;
+          acc[3] += c[u].y * f;
+        }
+        M = Mc;
       }
     }
   }
-  __shared__ float s_acc[4][D];
-  __shared__ float s_l[4];
-  s_acc[q][4 * lane] = acc0;
-  s_acc[q][4 * lane + 1] = acc1;
-  s_acc[q][4 * lane + 2] = acc2;
-  s_acc[q][4 * lane + 3] = acc3;
-  if (lane == 0) s_l[q] = L;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) s_acc[q][4 * lane + i] = acc[i];
+  if (lane == 0) { s_mq[q] = M; s_lq[q] = L; }
   __syncthreads();
-  const float Lt = ((s_l[0] + s_l[1]) + s_l[2]) + s_l[3];
-  for (int dd = threadIdx.x; dd < D; dd += blockDim.x) {
-    const float O = ((s_acc[0][dd] + s_acc[1][dd]) + s_acc[2][dd]) + s_acc[3][dd];
-    o[((size_t)b * H + h) * D + dd] = from_f<T>(O / Lt);
+  for (int idx = threadIdx.x; idx < hpb * D; idx += blockDim.x) {
+    const int hh = idx / D, dd = idx - hh * D;
+    const long long bh2 = (long long)blockIdx.x * hpb + hh;
+    if (bh2 >= (long long)B * H) break;
+    float r;
+    if (s_bad[hh]) {
+      r = NAN;
+    } else {
+      const int q0 = hh * wh;
+      float Mt = -INFINITY;
+      for (int i = 0; i < wh; ++i) Mt = fmaxf(Mt, s_mq[q0 + i]);
+      float O = 0.f, Lt = 0.f;
+      for (int i = 0; i < wh; ++i) {
+        const float wq = s_mq[q0 + i] == -INFINITY ? 0.f : exp2f(s_mq[q0 + i] - Mt);   // a warp without pieces weighs nothing
+        Lt += s_lq[q0 + i] * wq;
+        O += s_acc[q0 + i][dd] * wq;
+      }
+      r = O / Lt;
+    }
+    o[bh2 * D + dd] = from_f<T>(r);
   }
 }
 
@@ -734,18 +733,26 @@ static int mma_decode_launch(const void* q, const void* kc, const void* vc, cons
                              void* o, int B, int cmax, int H, int Hk, int Smax, const KvLayout& L,
                              DecodeScratch* scratch, int* status, cudaStream_t st) {
   const int grid = num_sms();
-  if (grid * DM_WARPS > kMaxDecodeWarps) return LLAMA_ERR_UNSUPPORTED;
   auto kern = attn_decode_mma_kernel<T>;
   if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), DM_SMEM)) return rc;
   const float scale_log2 = kLog2e / sqrtf(128.f);
   const int nmax = cmax < Smax ? cmax : Smax;
+  // warps per head of the combine: enough that each loads about CB_MAX pieces
+  const long long W = (long long)grid * DM_WARPS;
+  long long pieces = W / ((long long)B * Hk) + 2;
+  const long long tiles = (nmax + DM_KEYS - 1) / DM_KEYS;
+  if (pieces > tiles) pieces = tiles;
+  int wh = 1;
+  while (wh < CW && (long long)wh * CB_MAX < pieces) wh *= 2;
+  auto combine = pieces <= 6 ? attn_decode_combine_pieces_kernel<T, 128, 6>
+                             : attn_decode_combine_pieces_kernel<T, 128, CB_MAX>;
   cudaError_t err = launch_k(kern, dim3(grid), dim3(DM_WARPS * 32), DM_SMEM, st, static_cast<const T*>(q),
                              static_cast<const T*>(kc), static_cast<const T*>(vc), nkeys, add_keys, nmax,
                              scratch->part, B, H, Hk, L, scale_log2, status);
   if (err == cudaSuccess)
-    err = launch_k(attn_decode_combine_pieces_kernel<T, 128>, dim3(H, B), dim3(128), 0, st,
-                   (const float*)scratch->part, nkeys, add_keys, nmax, static_cast<T*>(o), B, H, Hk,
-                   (long long)grid * DM_WARPS);
+    err = launch_k(combine, dim3((unsigned)((B * H + CW / wh - 1) / (CW / wh))),
+                   dim3(CW * 32), 0, st, (const float*)scratch->part, nkeys, add_keys, nmax, static_cast<T*>(o), B, H,
+                   Hk, W, wh);
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 

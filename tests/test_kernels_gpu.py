@@ -187,6 +187,8 @@ def test_attention_prefill_f32(d):
     (BF16, 128, 1, 32, 8, 131072, [131072]),                 # longest cache of the sweep
     (BF16, 128, 64, 32, 8, 1024, [1 + 16 * i for i in range(64)]),
     (F16, 128, 1, 8, 1, 65536, [65536]),                   # one kv head: every decoding warp holds a piece of it
+    (BF16, 128, 4, 32, 8, 2048, [2048, 1, 1500, 777]),       # ~20 pieces per head: two combine warps per head
+    (F16, 128, 13, 12, 6, 700, [1 + 53 * i for i in range(13)]),   # 156 heads: a partial last combine block
     (BF16, 64, 2, 8, 2, 300, [17, 300]),
     (F16, 128, 3, 32, 8, 1000, [1, 517, 1000]),
     (F16, 128, 32, 32, 8, 4224, [4097 + 4 * i for i in range(32)]),
@@ -213,6 +215,32 @@ def test_attention_decode(dtype, d, B, H, Hk, cmax, lens):
                                           np.array([n - 1]), dtype)
         assert worst <= 1.0, (b, worst)                   # every head within its rounding bound
         assert err < {BF16: 1e-2, F16: 2e-3, F32: 1e-5}[dtype]
+
+
+@pytest.mark.parametrize('B', [1, 5])
+def test_attention_decode_bad_lengths_give_nan_rows(B):
+    """A length outside [1, cmax] gives a NaN row for that sequence, latches
+    LLAMA_ERR_DEVICE_BOUNDS, and leaves the other sequences' rows correct."""
+    H, Hk, d, cmax = 32, 8, 128, 640
+    lens = [0, 300, 641, 640, 17][:B] if B > 1 else [641]
+    qv, qr = normal_values(19, 1, (B, H, d), BF16)
+    kv, kr = normal_values(19, 2, (B, Hk, cmax, d), BF16)
+    vv, vr = normal_values(19, 3, (B, Hk, cmax, d), BF16)
+    o = torch.zeros((B, H * d), dtype=torch.bfloat16, device='cuda')
+    L.llama_attention_decode(to_device(qr, BF16), to_device(kr, BF16), to_device(vr, BF16),
+                             torch.tensor(lens, dtype=torch.int32, device='cuda'), o, B, cmax, H, Hk, d, BF16)
+    assert L.llama_status(None) == L.LLAMA_ERR_DEVICE_BOUNDS
+    assert L.llama_status(None) == 0                  # cleared
+    got = o.float().cpu().numpy()
+    for b, n in enumerate(lens):
+        if not 1 <= n <= cmax:
+            assert np.isnan(got[b]).all(), b
+            continue
+        worst, err = attention_row_errors(got[b][None], qv[b][:, None, :].astype(np.float64),
+                                          kv[b][:, :n].astype(np.float64), vv[b][:, :n].astype(np.float64),
+                                          np.array([n - 1]), BF16)
+        assert worst <= 1.0, (b, worst)
+        assert err < 1e-2
 
 
 def test_attention_decode_few_tiles_after_many():
