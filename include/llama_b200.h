@@ -222,10 +222,11 @@ int llama_attention_decode(const void* q, const void* kc, const void* vc, const 
  * cudaMalloc/cudaFree inside a latency-critical loop synchronizes the whole device. This call
  * never allocates or frees device memory; everything else is the same as
  * llama_attention_decode (arguments, layouts, results, bit for bit).
- * Its split partials live in one static 4 MiB device array that every GPU which loads this
- * library keeps until the process exits. Calls needing more than 4 MiB of partials return
- * LLAMA_ERR_SHAPE: for bf16 or fp16 with d = 128 the partials take (B*Hk + 4*SMs) * (H/Hk) * (d+2) * 4
- * bytes (SMs = 148 on B200), so with H = 32, Hk = 8 every B up to 170 fits.
+ * Its split partials live in one static 8 MiB device array that every GPU which loads this
+ * library keeps until the process exits. Calls needing more than 8 MiB of partials return
+ * LLAMA_ERR_SHAPE: for bf16 or fp16 with d = 128 the partials take at most
+ * (B*Hk + 12*SMs) * (H/Hk) * (d+2) * 4 + 16 bytes (SMs = 148 on B200; (B*Hk + 4*SMs) * ... when
+ * B*Hk*ceil(cmax/32) < 512*SMs), so with H = 32, Hk = 8 every B up to 280 fits whatever cmax.
  * Device-side errors of the call (a len[b] outside [1, cmax], which also gives a NaN row; a
  * bounded wait that gave up) are latched in a static status word of its own, next to the
  * array; llama_status() returns and clears it, and allocates nothing when only this call ran.

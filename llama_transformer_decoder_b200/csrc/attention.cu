@@ -298,28 +298,92 @@ __global__ void attn_decode_combine_kernel(const float* __restrict__ part, T* __
 
 
 // ---------------------------------------- decode, 16-bit d = 128 (mma)
-// Every warp is an independent flash decoder over a contiguous range of the
-// global tile sequence: (sequence b, kv head g, 32-key tile t) in that order,
-// T tiles in all; warp w of W takes tiles [T*w/W, T*(w+1)/W), so warps differ
-// by at most one tile whatever the lengths. Cutting that sequence at warp and
-// at (b, g) boundaries gives pieces; the piece of (b, g) held by warp w is
-// stored in slot (b*Hk + g) + w, which is unique, so the partials need only
-// (B*Hk + W) slots. A warp streams its tiles through a private 3-stage ring of
-// swizzled shared memory (cp.async, zero fill past the last key) without
-// draining at piece boundaries, computes S = Q K^T and O += P V with mma.sync
-// (the G query heads of the kv head are rows 0..G-1 of a 16-row tile), and
-// writes (o, max, sum) of every piece for the combine kernel.
+// The work is the sequence of (sequence b, kv head g, 32-key tile t) triples
+// in that order, T tiles in all, split into W ranges r = [T r / W, T (r+1) / W),
+// one per decoding warp. When every warp has enough tiles, the last 25% of
+// each range is cut into two sub-chunks (15% and 10% of the range) that warps
+// claim from a counter once their own 75% is done: the first sub-chunks of all
+// ranges, then the second ones, so the last claims are the short ones. Warps on SMs that stream slower than the others (measured: the same
+// SMs every run, finishing 12-15 us after the median of a ~100 us launch)
+// thereby stream less of the tail. Each claim is issued a few tiles before the
+// warp needs it. Sub-chunk boundaries depend only on T and the chunk index,
+// never on timing. Chunk id k = r * DM_SUB + s (s = 0: the owner's part)
+// increases with tile position; cutting the chunks at (b, g) boundaries gives
+// pieces, and the piece of (b, g) in chunk k is stored in slot (b*Hk + g) + k,
+// which is unique since chunks and (b, g) ranges are both in tile order. The
+// partials need B*Hk + W * DM_SUB slots (B*Hk + W without claimed
+// sub-chunks), and the merge order is the same whichever warp ran a chunk.
+//
+// A warp streams its tiles through a private 3-stage ring of swizzled shared
+// memory (cp.async, zero fill past the last key) without draining at chunk or
+// piece boundaries, computes S = Q K^T and O += P V with mma.sync (the G query
+// heads of the kv head are rows 0..G-1 of a 16-row tile) and writes
+// (o, max, sum) of every piece for the combine kernel.
 constexpr int DM_KEYS = 32;
 constexpr int DM_STAGES = 3;
 constexpr int DM_WARPS = 4;
 constexpr int DM_TILE = DM_KEYS * 256;             // one K (or V) tile: 32 rows x 256 B
 constexpr int DM_STAGE = 2 * DM_TILE;
-constexpr int DM_SMEM = DM_WARPS * DM_STAGES * DM_STAGE;
+constexpr int DM_RING = DM_WARPS * DM_STAGES * DM_STAGE;
+// Per-sequence tile prefix and key counts in shared memory (for B up to
+// DM_SEEK_B), so that moving to a claimed chunk is a binary search, not a walk
+// over every sequence's length in global memory.
+constexpr int DM_SEEK_B = 128;
+constexpr int DM_SMEM = DM_RING + (DM_SEEK_B + 1) * 8 + DM_SEEK_B * 4;
+constexpr int DM_CLAIM_AHEAD = 3;                  // tiles before a chunk's end its successor is claimed
+static_assert(DM_STAGES == 3, "the chunk queue holds the DM_STAGES - 1 chunks the loader may run ahead, plus one");
+constexpr int DM_SUB = 3;                          // sub-chunks of a range (the owner's, then two claimed)
+// Tiles per warp for claimed sub-chunks. Below ~128 (launches under ~200 us
+// at batch 32) they measured slower inside the decode step, though faster
+// alone; above it they gain 5-7% (batch 8-32, 16k-64k keys).
+constexpr int DM_TAIL_MIN = 128;
+__host__ __device__ constexpr int dm_cut(int s) { return s == 0 ? 0 : s == 1 ? 75 : s == 2 ? 90 : 100; }
+// The last 16 bytes of the decode scratch hold the two tail counters
+// (sub-chunks claimed, warps finished; zero between launches: the last warp to
+// finish re-arms them); the partials of every decode path start at its front.
+constexpr size_t kDecodeCounterFloats = 4;
 
+// Chunk geometry of T tiles over W warps for B*Hk (sequence, kv head) pairs.
+struct DmSplit {
+  long long T, W;
+  bool tail;   // claimed sub-chunks: enough tiles per warp, and few enough ranges per (b, g) for the merge
+};
+__host__ __device__ inline DmSplit dm_split(long long T, long long W, long long BHk) {
+  return DmSplit{T, W, T >= DM_TAIL_MIN * W && BHk * 24 >= W};   // <= 24 ranges (72 pieces) per (b, g)
+}
+__host__ __device__ inline long long dm_chunks(const DmSplit& s) { return s.tail ? s.W * DM_SUB : s.W; }
+// First tile of chunk k (k = dm_chunks gives T).
+__device__ __forceinline__ long long dm_chunk_start(const DmSplit& s, long long k) {
+  if (!s.tail) return s.T * k / s.W;
+  const long long r = k / DM_SUB;
+  const int sub = (int)(k - r * DM_SUB);
+  const long long a = s.T * r / s.W;
+  if (sub == 0) return a;
+  return a + (s.T * (r + 1) / s.W - a) * dm_cut(sub) / 100;
+}
+// Chunk holding tile x < T.
+__device__ inline long long dm_chunk_of(const DmSplit& s, long long x) {
+  const long long r = ((x + 1) * s.W - 1) / s.T;
+  if (!s.tail) return r;
+  const long long a = s.T * r / s.W, len = s.T * (r + 1) / s.W - a;
+  int sub = 0;
+  while (sub < DM_SUB - 1 && a + len * dm_cut(sub + 1) / 100 <= x) ++sub;
+  return r * DM_SUB + sub;
+}
 __device__ __forceinline__ int dm_keys(const int32_t* nkeys, int b, int add, int nmax) {
   return min(nkeys[b] + add, nmax);
 }
 __device__ __forceinline__ int dm_tiles(int n) { return n > 0 ? (n + DM_KEYS - 1) / DM_KEYS : 0; }
+
+// Sequence lengths as the cursors read them: from shared memory (the CTA's
+// prefix table) when B <= DM_SEEK_B, else from global memory.
+struct DmLens {
+  const int32_t* nkeys;
+  int add, nmax, B, Hk;
+  const long long* cum;   // [B + 1] tiles before sequence b, or null
+  const int* keys;        // [B] keys of sequence b (clamped), or null
+  __device__ int n(int b) const { return keys ? keys[b] : dm_keys(nkeys, b, add, nmax); }
+};
 
 struct TileCursor {
   int b, g, t;          // sequence, kv head, tile of (b, g)
@@ -327,36 +391,46 @@ struct TileCursor {
   long long left;       // tiles left in this warp's range, counting the current one
 };
 
-__device__ void tc_seek(TileCursor& c, long long x, long long count, const int32_t* nkeys, int add, int nmax, int B,
-                        int Hk) {
+__device__ void tc_seek(TileCursor& c, long long x, long long count, const DmLens& Ls) {
   c.left = count;
+  int b = -1;
   long long acc = 0;
-  for (int b = 0; b < B; ++b) {
-    const int n = dm_keys(nkeys, b, add, nmax);
-    const int nt = dm_tiles(n);
-    const long long cnt = (long long)Hk * nt;
-    if (x < acc + cnt) {
-      const int r = (int)(x - acc);
-      c.b = b; c.n = n; c.nt = nt; c.g = r / nt; c.t = r - c.g * nt;
-      return;
+  if (Ls.cum) {   // the last sequence whose first tile is at or before x (it holds x: empty ones are skipped)
+    int lo = 0, hi = Ls.B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (Ls.cum[mid] <= x) lo = mid;
+      else hi = mid - 1;
     }
-    acc += cnt;
+    if (x < Ls.cum[lo + 1]) { b = lo; acc = Ls.cum[lo]; }
+  } else {
+    for (int bb = 0; bb < Ls.B; ++bb) {
+      const long long cnt = (long long)Ls.Hk * dm_tiles(Ls.n(bb));
+      if (x < acc + cnt) { b = bb; break; }
+      acc += cnt;
+    }
   }
-  c.left = 0;
+  if (b < 0) {
+    c.left = 0;
+    return;
+  }
+  const int n = Ls.n(b), nt = dm_tiles(n);
+  const int r = (int)(x - acc);
+  c.b = b; c.n = n; c.nt = nt; c.g = r / nt; c.t = r - c.g * nt;
 }
 
 // Advance one tile; true when the piece (this warp's part of one (b, g)) ended.
-__device__ bool tc_next(TileCursor& c, const int32_t* nkeys, int add, int nmax, int B, int Hk) {
+__device__ bool tc_next(TileCursor& c, const DmLens& Ls) {
   const bool last_in_range = --c.left <= 0;
   if (++c.t < c.nt) return last_in_range;
   c.t = 0;
-  if (++c.g == Hk) {
+  if (++c.g == Ls.Hk) {
     c.g = 0;
     do {
       ++c.b;
-      c.n = c.b < B ? dm_keys(nkeys, c.b, add, nmax) : 0;
+      c.n = c.b < Ls.B ? Ls.n(c.b) : 0;
       c.nt = dm_tiles(c.n);
-    } while (c.nt == 0 && c.b < B);
+    } while (c.nt == 0 && c.b < Ls.B);
   }
   return true;
 }
@@ -380,17 +454,23 @@ __device__ __forceinline__ void dm_load_tile(uint8_t* stage, const T* kc, const 
   }
 }
 
-template <typename T>
+// TAIL = false compiles the claims and the seek table out (the launch's size
+// bound rules claimed sub-chunks out); with TAIL = true they are used when
+// this launch's T calls for them.
+template <typename T, bool TAIL>
 __global__ void __launch_bounds__(DM_WARPS * 32, 1)
     attn_decode_mma_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
-                           const int32_t* __restrict__ nkeys, int add_keys, int nmax, float* __restrict__ part, int B,
-                           int H, int Hk, KvLayout L, float scale_log2, int* status) {
+                           const int32_t* __restrict__ nkeys, int add_keys, int nmax, float* __restrict__ part,
+                           int* __restrict__ counters, int B, int H, int Hk, KvLayout L, float scale_log2,
+                           int* status) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ __align__(128) uint8_t sm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = H / Hk;
   uint8_t* ring = sm + warp * DM_STAGES * DM_STAGE;
+  long long* s_cum = reinterpret_cast<long long*>(sm + DM_RING);
+  int* s_keys = reinterpret_cast<int*>(sm + DM_RING + (DM_SEEK_B + 1) * 8);
 
   long long total = 0;
   for (int b = 0; b < B; ++b) {
@@ -400,18 +480,80 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
   }
   const long long W = (long long)gridDim.x * DM_WARPS;
   const int w = blockIdx.x * DM_WARPS + warp;
-  const long long x0 = total * w / W, x1 = total * (w + 1) / W;
-  if (x1 <= x0) return;
+  DmSplit sp = dm_split(total, W, (long long)B * Hk);
+  if (!TAIL) sp.tail = false;   // never taken: the host's bound excludes it
+  const bool tail = sp.tail;
+  DmLens Ls{nkeys, add_keys, nmax, B, Hk, nullptr, nullptr};
+  if (tail && B <= DM_SEEK_B) {   // the prefix table: keys by thread, tile prefix by a scan in warp 0
+    for (int b = threadIdx.x; b < B; b += blockDim.x) s_keys[b] = dm_keys(nkeys, b, add_keys, nmax);
+    __syncthreads();
+    if (warp == 0) {
+      long long carry = 0;
+      for (int b0 = 0; b0 < B; b0 += 32) {
+        const int b = b0 + lane;
+        long long v = b < B ? (long long)Hk * dm_tiles(s_keys[b]) : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const long long u = __shfl_up_sync(0xffffffffu, v, off);
+          if (lane >= off) v += u;
+        }
+        if (b < B) s_cum[b + 1] = carry + v;
+        carry += __shfl_sync(0xffffffffu, v, 31);
+      }
+      if (lane == 0) s_cum[0] = 0;
+    }
+    __syncthreads();
+    Ls.cum = s_cum;
+    Ls.keys = s_keys;
+  }
+  const long long k_first = tail ? (long long)w * DM_SUB : w;   // the warp's own part of its range
+  const long long x0 = dm_chunk_start(sp, k_first), x1 = dm_chunk_start(sp, k_first + 1);
+  if (x1 <= x0) return;   // only without a tail (T < W): with one, every range holds >= DM_TAIL_MIN tiles
+  const int n_claims = tail ? (DM_SUB - 1) * (int)W : 0;
 
   TileCursor ld, cp;
-  tc_seek(ld, x0, x1 - x0, nkeys, add_keys, nmax, B, Hk);
+  tc_seek(ld, x0, x1 - x0, Ls);
   cp = ld;
+  long long k_cp = k_first;         // the consumer's chunk
+  long long k_q0 = 0, k_q1 = 0, k_q2 = 0;   // chunks the loader moved on to, not yet reached by the consumer
+  int n_q = 0;                              // (it runs at most DM_STAGES - 1 = 2 tiles ahead)
+  int pending = 0;                  // lane 0: the claim issued for the loader's next chunk
+  bool claimed = false, ld_done = false;
+  int issued = 0;
+  auto maybe_claim = [&]() {
+    if (tail && !claimed && ld.left <= DM_CLAIM_AHEAD) {
+      if (lane == 0) pending = atomicAdd(&counters[0], 1);
+      claimed = true;
+    }
+  };
+  // one tile into the ring, then step the loader (to its claimed chunk at a chunk's end)
+  auto issue = [&]() {
+    dm_load_tile(ring + (issued % DM_STAGES) * DM_STAGE, kc, vc, ld, Hk, L, lane);
+    ++issued;
+    tc_next(ld, Ls);
+    if (ld.left > 0) {
+      maybe_claim();
+      return;
+    }
+    const int c = tail ? __shfl_sync(0xffffffffu, pending, 0) : 0;
+    claimed = false;
+    if (!tail || c >= n_claims) {
+      ld_done = true;
+      return;
+    }
+    // claim c: sub-chunk 1 + c / W of range c % W
+    const long long k = (long long)(c % (int)W) * DM_SUB + 1 + c / (int)W, a = dm_chunk_start(sp, k);
+    tc_seek(ld, a, dm_chunk_start(sp, k + 1) - a, Ls);
+    if (n_q == 0) k_q0 = k;
+    else if (n_q == 1) k_q1 = k;
+    else k_q2 = k;
+    ++n_q;
+    maybe_claim();
+  };
   const int row = lane >> 2, tq = lane & 3;   // fragment row (query head within the group), column pair
   const bool real = row < G;
   uint32_t qa[8][2];
-  // the first piece's query rows before the ring fills, so that they do not
-  // queue behind every warp's first K/V tiles
-  auto load_q = [&](const TileCursor& c) {
+  auto load_q = [&](const TileCursor& c) {   // the G query rows of (b, g)
     const T* qr = q + ((size_t)c.b * H + c.g * G + (real ? row : 0)) * 128;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
@@ -419,16 +561,12 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
       qa[ks][1] = real ? *reinterpret_cast<const uint32_t*>(qr + ks * 16 + 8 + 2 * tq) : 0u;
     }
   };
-  if (cp.left > 0) load_q(cp);
-  int issued = 0;
-  bool ld_done = ld.left <= 0;
+  // the first piece's query rows before the ring fills, so that they do not
+  // queue behind every warp's first K/V tiles
+  load_q(cp);
+  maybe_claim();
   for (int i = 0; i < DM_STAGES - 1; ++i) {
-    if (!ld_done) {
-      dm_load_tile(ring + (issued % DM_STAGES) * DM_STAGE, kc, vc, ld, Hk, L, lane);
-      ++issued;
-      tc_next(ld, nkeys, add_keys, nmax, B, Hk);
-      ld_done = ld.left <= 0;
-    }
+    if (!ld_done) issue();
     cp_async_commit();
   }
 
@@ -436,7 +574,7 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
   float m_r = -INFINITY, l_r = 0.f;
   int consumed = 0;
   bool start = true, first_piece = true;
-  while (cp.left > 0) {
+  for (;;) {
     if (start) {   // new piece: reset the state and fetch the G query rows of (b, g)
       if (!first_piece) load_q(cp);
       first_piece = false;
@@ -446,12 +584,7 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
       l_r = 0.f;
       start = false;
     }
-    if (!ld_done) {   // keep DM_STAGES-1 tiles in flight
-      dm_load_tile(ring + (issued % DM_STAGES) * DM_STAGE, kc, vc, ld, Hk, L, lane);
-      ++issued;
-      tc_next(ld, nkeys, add_keys, nmax, B, Hk);
-      ld_done = ld.left <= 0;
-    }
+    if (!ld_done) issue();   // keep DM_STAGES-1 tiles in flight
     cp_async_commit();
     cp_async_wait<DM_STAGES - 1>();
     __syncwarp();
@@ -523,25 +656,41 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
     __syncwarp();   // the stage may be refilled from the next iteration on
     ++consumed;
     const int b_done = cp.b, g_done = cp.g;
-    if (tc_next(cp, nkeys, add_keys, nmax, B, Hk)) {
+    if (tc_next(cp, Ls)) {
       if (real) {
-        const size_t slot = (size_t)b_done * Hk + g_done + w;
+        const size_t slot = (size_t)b_done * Hk + g_done + k_cp;
         float* dst = part + (slot * G + row) * 130;
 #pragma unroll
         for (int n = 0; n < 16; ++n) *reinterpret_cast<float2*>(dst + n * 8 + 2 * tq) = make_float2(oacc[n][0], oacc[n][1]);
         if (tq == 0) { dst[128] = m_r; dst[129] = l_r; }
       }
       start = true;
+      if (cp.left <= 0) {   // the chunk is done: on to the next one the loader reached, if any
+        if (n_q == 0) break;
+        k_cp = k_q0;
+        k_q0 = k_q1;
+        k_q1 = k_q2;
+        --n_q;
+        const long long a = dm_chunk_start(sp, k_cp);
+        tc_seek(cp, a, dm_chunk_start(sp, k_cp + 1) - a, Ls);
+      }
     }
   }
   cp_async_wait<0>();
+  if (tail && lane == 0) {   // every warp has made its last claim: the last one out re-arms the counters
+    __threadfence();
+    if (atomicAdd(&counters[1], 1) == (int)W - 1) {
+      counters[0] = 0;
+      counters[1] = 0;
+    }
+  }
 }
 
-// Merge the pieces of every (b, h). The warps holding tiles of (b, g) are
-// owner(t0) .. owner(t0 + nt - 1), owner(x) = ((x+1)W - 1) / T: when T >= W
-// every warp's range is non-empty, so the pieces are all the warps between
-// those two; when T < W every warp holds at most one tile, so piece k is the
-// owner of tile t0 + k. A block of CW warps serves CW / wh heads (flattened
+// Merge the pieces of every (b, h). The chunks holding tiles of (b, g) are
+// chunk(t0) .. chunk(t0 + nt - 1): when every range holds tiles (T >= W;
+// claimed sub-chunks then always do) these are every chunk between the two;
+// otherwise (T < W, no claimed sub-chunks) every warp holds at most one tile,
+// so piece k is the warp of tile t0 + k. A block of CW warps serves CW / wh heads (flattened
 // b*H + h), wh warps each: warp j of a head merges its pieces
 // [cnt j / wh, cnt (j+1) / wh), loading CB pieces at a time with every load in
 // flight and keeping a running (max, sum, o) rescaled as the maximum grows;
@@ -592,9 +741,10 @@ __global__ void __launch_bounds__(CW * 32) attn_decode_combine_pieces_kernel(
     const bool bad = nt_b == 0 || total == 0 || nb < 1 || nb > nmax;
     if (j == 0 && lane == 0) s_bad[q / wh] = bad;
     if (!bad) {
-      const long long w_lo = ((t0 + 1) * W - 1) / total;
+      const DmSplit sp = dm_split(total, W, (long long)B * Hk);
+      const long long w_lo = dm_chunk_of(sp, t0);
       const bool dense = total >= W;
-      const int cnt = dense ? (int)(((t0 + nt_b) * W - 1) / total - w_lo + 1) : nt_b;
+      const int cnt = dense ? (int)(dm_chunk_of(sp, t0 + nt_b - 1) - w_lo + 1) : nt_b;
       const size_t bg = (size_t)b * Hk + g;
       const int k0 = cnt * j / wh, k1 = cnt * (j + 1) / wh;
       for (int kb = k0; kb < k1; kb += CB) {
@@ -723,9 +873,20 @@ int decode_splits(int cmax, int B, int Hk) {
 bool use_mma_decode(int d, int dtype) { return (dtype == LLAMA_BF16 || dtype == LLAMA_F16) && d == 128; }
 }  // namespace
 
+namespace {
+// Chunk geometry of a launch whose sequences hold at most cmax keys (claimed
+// sub-chunks only come in as T grows, so this bounds every launch within cmax).
+DmSplit decode_split_bound(int cmax, int B, int Hk) {
+  const long long T = (long long)B * Hk * ((cmax + DM_KEYS - 1) / DM_KEYS);
+  return dm_split(T, (long long)num_sms() * DM_WARPS, (long long)B * Hk);
+}
+}  // namespace
+
 size_t decode_scratch_floats(int cmax, int B, int H, int Hk, int d, int dtype) {
-  if (use_mma_decode(d, dtype)) return ((size_t)B * Hk + (size_t)num_sms() * DM_WARPS) * (H / Hk) * (d + 2);
-  return (size_t)B * H * decode_splits(cmax, B, Hk) * (d + 2);
+  if (use_mma_decode(d, dtype))
+    return kDecodeCounterFloats +
+           ((size_t)B * Hk + (size_t)dm_chunks(decode_split_bound(cmax, B, Hk))) * (H / Hk) * (d + 2);
+  return kDecodeCounterFloats + (size_t)B * H * decode_splits(cmax, B, Hk) * (d + 2);
 }
 
 template <typename T>
@@ -733,26 +894,29 @@ static int mma_decode_launch(const void* q, const void* kc, const void* vc, cons
                              void* o, int B, int cmax, int H, int Hk, int Smax, const KvLayout& L,
                              DecodeScratch* scratch, int* status, cudaStream_t st) {
   const int grid = num_sms();
-  auto kern = attn_decode_mma_kernel<T>;
-  if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), DM_SMEM)) return rc;
   const float scale_log2 = kLog2e / sqrtf(128.f);
   const int nmax = cmax < Smax ? cmax : Smax;
+  const DmSplit bound = decode_split_bound(nmax, B, Hk);
+  auto kern = bound.tail ? attn_decode_mma_kernel<T, true> : attn_decode_mma_kernel<T, false>;
+  if (const int rc = ensure_smem_attr(reinterpret_cast<const void*>(kern), bound.tail ? DM_SMEM : DM_RING)) return rc;
   // warps per head of the combine: enough that each loads about CB_MAX pieces
   const long long W = (long long)grid * DM_WARPS;
-  long long pieces = W / ((long long)B * Hk) + 2;
+  long long pieces = dm_chunks(bound) / ((long long)B * Hk) + (bound.tail ? DM_SUB + 1 : 2);
   const long long tiles = (nmax + DM_KEYS - 1) / DM_KEYS;
-  if (pieces > tiles) pieces = tiles;
+  if (!bound.tail && pieces > tiles) pieces = tiles;
   int wh = 1;
   while (wh < CW && (long long)wh * CB_MAX < pieces) wh *= 2;
   auto combine = pieces <= 6 ? attn_decode_combine_pieces_kernel<T, 128, 6>
                              : attn_decode_combine_pieces_kernel<T, 128, CB_MAX>;
-  cudaError_t err = launch_k(kern, dim3(grid), dim3(DM_WARPS * 32), DM_SMEM, st, static_cast<const T*>(q),
-                             static_cast<const T*>(kc), static_cast<const T*>(vc), nkeys, add_keys, nmax,
-                             scratch->part, B, H, Hk, L, scale_log2, status);
+  int* counters = reinterpret_cast<int*>(scratch->part + scratch->floats - kDecodeCounterFloats);
+  float* part = scratch->part;
+  // the seek table's shared memory only where claimed sub-chunks may be used
+  cudaError_t err = launch_k(kern, dim3(grid), dim3(DM_WARPS * 32), bound.tail ? DM_SMEM : DM_RING, st,
+                             static_cast<const T*>(q), static_cast<const T*>(kc), static_cast<const T*>(vc), nkeys,
+                             add_keys, nmax, part, counters, B, H, Hk, L, scale_log2, status);
   if (err == cudaSuccess)
-    err = launch_k(combine, dim3((unsigned)((B * H + CW / wh - 1) / (CW / wh))),
-                   dim3(CW * 32), 0, st, (const float*)scratch->part, nkeys, add_keys, nmax, static_cast<T*>(o), B, H,
-                   Hk, W, wh);
+    err = launch_k(combine, dim3((unsigned)((B * H + CW / wh - 1) / (CW / wh))), dim3(CW * 32), 0, st,
+                   (const float*)part, nkeys, add_keys, nmax, static_cast<T*>(o), B, H, Hk, W, wh);
   return err == cudaSuccess ? LLAMA_OK : LLAMA_ERR_CUDA;
 }
 
@@ -771,18 +935,19 @@ int attention_decode(const void* q, const void* kc, const void* vc, const int32_
   }
   if (kv_table) return LLAMA_ERR_UNSUPPORTED;   // paged caches: 16-bit, head_dim 128 only
   const int splits = decode_splits(cmax, B, Hk);
+  float* part = scratch->part;
   if (dtype == LLAMA_BF16) {
-    if (d == 64) return decode_launch<bf16, 64>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch->part,
+    if (d == 64) return decode_launch<bf16, 64>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, part,
                                                 splits, status, st);
   } else if (dtype == LLAMA_F16) {
-    if (d == 64) return decode_launch<f16, 64>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch->part,
+    if (d == 64) return decode_launch<f16, 64>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, part,
                                                splits, status, st);
   } else {
     if (d == 128) return decode_launch<float, 128>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax,
-                                                   scratch->part, splits, status, st);
-    if (d == 64) return decode_launch<float, 64>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch->part,
+                                                   part, splits, status, st);
+    if (d == 64) return decode_launch<float, 64>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, part,
                                                  splits, status, st);
-    if (d == 32) return decode_launch<float, 32>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, scratch->part,
+    if (d == 32) return decode_launch<float, 32>(q, kc, vc, nkeys, add_keys, o, B, cmax, H, Hk, Smax, part,
                                                  splits, status, st);
   }
   return LLAMA_ERR_UNSUPPORTED;

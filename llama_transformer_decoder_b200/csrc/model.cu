@@ -297,6 +297,13 @@ int grow_decode_scratch(DecodeScratch* ds, size_t floats) {
   ds->part = nullptr;
   ds->floats = 0;
   if (cudaMalloc(&ds->part, floats * sizeof(float)) != cudaSuccess) { cudaGetLastError(); return LLAMA_ERR_OOM; }
+  // the decode kernel's work counters in the last 16 bytes start at zero (it re-arms them itself)
+  if (cudaMemset(ds->part + floats - 4, 0, 4 * sizeof(float)) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(ds->part);
+    ds->part = nullptr;
+    return LLAMA_ERR_CUDA;
+  }
   ds->floats = floats;
   return LLAMA_OK;
 }

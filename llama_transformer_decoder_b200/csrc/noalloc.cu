@@ -2,7 +2,9 @@
 // memory. The split partials that llama_attention_decode keeps in
 // library-allocated scratch live here in one file-scope static device array
 // instead, and the call's device-side errors go to a static status word next
-// to it, so the call itself never allocates or frees device memory.
+// to it, so the call itself never allocates or frees device memory. The
+// array starts zeroed, as the decode kernel's work counters in its last 16
+// bytes must (the kernel re-arms them at the end of every launch).
 #include <map>
 #include <mutex>
 
@@ -11,7 +13,7 @@
 
 namespace {
 
-constexpr size_t kScratchBytes = 4u << 20;   // 4 MiB, held by every GPU that loads the library
+constexpr size_t kScratchBytes = 8u << 20;   // 8 MiB, held by every GPU that loads the library
 
 static __device__ __align__(256) float g_decode_scratch[kScratchBytes / sizeof(float)];
 static __device__ int g_noalloc_status;

@@ -189,6 +189,8 @@ def test_attention_prefill_f32(d):
     (F16, 128, 1, 8, 1, 65536, [65536]),                   # one kv head: every decoding warp holds a piece of it
     (BF16, 128, 4, 32, 8, 2048, [2048, 1, 1500, 777]),       # ~20 pieces per head: two combine warps per head
     (F16, 128, 13, 12, 6, 700, [1 + 53 * i for i in range(13)]),   # 156 heads: a partial last combine block
+    (F16, 128, 32, 32, 8, 16384, [16384 - 97 * i for i in range(32)]),   # claimed sub-chunks (>= 128 tiles per warp)
+    (BF16, 128, 160, 8, 2, 8192, [8192 - 7 * i for i in range(160)]),   # claimed sub-chunks, B over the seek table
     (BF16, 64, 2, 8, 2, 300, [17, 300]),
     (F16, 128, 3, 32, 8, 1000, [1, 517, 1000]),
     (F16, 128, 32, 32, 8, 4224, [4097 + 4 * i for i in range(32)]),

@@ -35,6 +35,8 @@ def _inputs(seed, B, H, Hk, d, cmax, dtype):
 
 CASES = [  # dtype, B, H, Hk, d, cmax, two sets of lengths (one per call)
     (BF16, 4, 32, 8, 128, 4096, [1, 700, 4096, 2048], [4096, 3, 1500, 999]),
+    (F16, 8, 32, 8, 128, 65536, [65536, 60000, 65000, 40000, 65536, 50000, 1, 65535],   # claimed sub-chunks,
+     [4096, 8000, 7000, 1, 8192, 8100, 7500, 6000]),                                     # then none
     (F16, 3, 8, 2, 64, 1000, [1000, 1, 517], [2, 999, 640]),
     (F32, 2, 8, 2, 32, 1000, [1000, 333], [17, 1000]),
     (F32, 2, 4, 4, 64, 900, [900, 1], [450, 899]),
@@ -82,7 +84,7 @@ def test_noalloc_decode_reports_lengths_outside_the_cache(dtype, d):
 
 
 def test_noalloc_decode_rejects_sizes_beyond_its_array():
-    B, H, Hk, d, cmax = 256, 32, 8, 128, 64        # (256*8 + 4*148)*4*(128+2)*4 B > 4 MiB of partials
+    B, H, Hk, d, cmax = 512, 32, 8, 128, 64        # (512*8 + 4*148)*4*(128+2)*4 B > 8 MiB of partials
     q = torch.zeros((B, H, d), dtype=torch.bfloat16, device='cuda')
     k = torch.zeros((B, Hk, cmax, d), dtype=torch.bfloat16, device='cuda')
     ln = torch.ones(B, dtype=torch.int32, device='cuda')
