@@ -277,11 +277,9 @@ def run_reference(args):
 
 # ---------------------------------------------------------------- our arm
 D_, F_, H_, HK_, HD_, V_ = 4096, 14336, 32, 8, 128, 128256
-# Measured DRAM bytes per launch of the chained prefill projection GEMM (one
-# layer's Wo, w1/w3, w2 and the next QKV at 2048 tokens; one ncu capture of
-# the current kernel). None until captured for the current kernel.
 # DRAM read + write bytes of one middle layer's chained launch (Wo, w1/w3,
-# w2, next QKV), from an ncu capture of a 2-layer model of the 8B shapes
+# w2, next QKV) at B=1, S=2048, from an ncu capture of a 2-layer model of the
+# 8B shapes. Other batches move other activation bytes: no figure for them.
 PAIR_GEMM_TRAFFIC = 1096.8e6 + 163.6e6
 
 
@@ -338,10 +336,12 @@ def measure_prefill(L, m, st, toks, arg, args, ws, local, NL, tf_sust, peak_src,
     roofline = {'kernel': 'gemm_chain_kernel (tcgen05 cta_group::2; per layer one launch of Wo, w1/w3, w2 and the '
                           'next layer\'s QKV, plus layer 0\'s QKV)', 'bound': 'tensor',
                 'achieved': achieved, 'peak': tf_sust, 'unit': 'TFLOP/s',
-                'frac': achieved / tf_sust if achieved else None, 'traffic': PAIR_GEMM_TRAFFIC,
-                'traffic_note': 'DRAM read+write bytes of a middle layer\'s chained launch from one ncu capture '
-                                '(1.3x its operand bytes: w1/w3 weights stream twice by design, w2\'s weight is '
-                                'partly re-read per row block)',
+                'frac': achieved / tf_sust if achieved else None,
+                'traffic': PAIR_GEMM_TRAFFIC if B == 1 else None,
+                'traffic_note': ('DRAM read+write bytes of a middle layer\'s chained launch from one ncu capture '
+                                 '(1.3x its operand bytes: w1/w3 weights stream twice by design, w2\'s weight is '
+                                 'partly re-read per row block)') if B == 1 else
+                                'not captured at this batch (the B=1 capture does not scale with the tokens)',
                 'peak_kind': f'bf16 sustained ({peak_src}); fp16 has the same nominal tensor rate',
                 'launches': gemm_launches // max(args.steps, 1),
                 'attention_tflops': attn_flops * args.steps / (attn[0] / 1e3) / 1e12 if attn[0] else None,
