@@ -690,8 +690,8 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
 // chunk(t0) .. chunk(t0 + nt - 1): when every range holds tiles (T >= W;
 // claimed sub-chunks then always do) these are every chunk between the two;
 // otherwise (T < W, no claimed sub-chunks) every warp holds at most one tile,
-// so piece k is the warp of tile t0 + k. A block of CW warps serves CW / wh heads (flattened
-// b*H + h), wh warps each: warp j of a head merges its pieces
+// so piece k is the warp of tile t0 + k. A block of CW warps serves CW / wh
+// heads (flattened b*H + h), wh warps each: warp j of a head merges its pieces
 // [cnt j / wh, cnt (j+1) / wh), loading CB pieces at a time with every load in
 // flight and keeping a running (max, sum, o) rescaled as the maximum grows;
 // the wh warps' results are then merged in warp order. The order is fixed, so
