@@ -312,6 +312,36 @@ def test_attention_decode_paged(dtype):
         assert err < (1e-2 if dtype == BF16 else 2e-3)
 
 
+def test_attention_decode_paged_claimed_sub_chunks():
+    """A paged cache long enough (>= 128 tiles of 32 keys per decoding warp)
+    for the claimed sub-chunks: claimed chunks start inside pages of other
+    sequences' ranges; sampled sequences against the oracle."""
+    dtype, B, H, Hk, d, C = F16, 24, 32, 8, 128, 14336
+    lens = [C - 97 * i for i in range(B)]
+    assert Hk * sum((n + 31) // 32 for n in lens) >= 128 * 148 * 4
+    qv, qr = normal_values(52, 1, (B, H, d), dtype)
+    kv, kr = normal_values(52, 2, (B, Hk, C, d), dtype)
+    vv, vr = normal_values(52, 3, (B, Hk, C, d), dtype)
+    n_pages = B * (C // 128) + 3
+    kp, table, max_pages = _paginate(kr, n_pages, 3)
+    vp, _, _ = _paginate(vr, n_pages, 3)
+    del kr, vr
+    o = torch.empty((B, H * d), dtype=torch.float16, device='cuda')
+    L.llama_attention_decode_paged(to_device(qr, dtype), to_device(kp, dtype), to_device(vp, dtype),
+                                   torch.from_numpy(table).cuda(), max_pages, n_pages,
+                                   torch.tensor(lens, dtype=torch.int32, device='cuda'), o, B, H, Hk, d, dtype)
+    torch.cuda.synchronize()
+    _sync_ok()
+    got = o.float().cpu().numpy()
+    for b in (0, 1, B // 2, B - 1):
+        n = lens[b]
+        worst, err = attention_row_errors(got[b][None], qv[b][:, None, :].astype(np.float64),
+                                          kv[b][:, :n].astype(np.float64), vv[b][:, :n].astype(np.float64),
+                                          np.array([n - 1]), dtype)
+        assert worst <= 1.0, (b, worst)
+        assert err < 2e-3
+
+
 def test_attention_prefill_paged_continues_a_cache():
     """Queries at positions pos0[b] .. pos0[b]+S-1 over a paged cache that
     already holds their keys (a prompt continued across page boundaries)."""
