@@ -316,8 +316,8 @@ __global__ void attn_decode_combine_kernel(const float* __restrict__ part, T* __
 //
 // A warp streams its tiles through a private 3-stage ring of swizzled shared
 // memory (cp.async, zero fill past the last key) without draining at chunk or
-// piece boundaries, computes S = Q K^T and O += P V with mma.sync (the G query
-// heads of the kv head are rows 0..G-1 of a 16-row tile) and writes
+// piece boundaries, computes S^T = K Q^T and O^T += V^T P^T with mma.sync (the
+// G query heads of the kv head are columns 0..G-1 of 8) and writes
 // (o, max, sum) of every piece for the combine kernel.
 constexpr int DM_KEYS = 32;
 constexpr int DM_STAGES = 3;
@@ -570,8 +570,12 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
     cp_async_commit();
   }
 
-  float oacc[16][2];
-  float m_r = -INFINITY, l_r = 0.f;
+  // Keys and head dims take the 16-row side of mma.m16n8k16 and the (padded)
+  // query heads its 8 columns: S^T = K Q^T, then O^T += V^T P^T, 32 products
+  // per 32-key tile where query rows padded to 16 would take 64. A thread
+  // holds the two query columns 2 tq and 2 tq + 1.
+  float oacc[8][4];          // O^T: d = 16 i + row (+8), queries 2 tq, 2 tq + 1
+  float m_r[2], l_r[2];
   int consumed = 0;
   bool start = true, first_piece = true;
   for (;;) {
@@ -579,9 +583,9 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
       if (!first_piece) load_q(cp);
       first_piece = false;
 #pragma unroll
-      for (int n = 0; n < 16; ++n) oacc[n][0] = oacc[n][1] = 0.f;
-      m_r = -INFINITY;
-      l_r = 0.f;
+      for (int i = 0; i < 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+      m_r[0] = m_r[1] = -INFINITY;
+      l_r[0] = l_r[1] = 0.f;
       start = false;
     }
     if (!ld_done) issue();   // keep DM_STAGES-1 tiles in flight
@@ -591,78 +595,97 @@ __global__ void __launch_bounds__(DM_WARPS * 32, 1)
     const uint8_t* st = ring + (consumed % DM_STAGES) * DM_STAGE;
     const uint32_t kb = smem_u32(st), vb = smem_u32(st + DM_TILE);
     const int valid = min(DM_KEYS, cp.n - cp.t * DM_KEYS);
-    // S = Q K^T for 32 keys
-    float sc[4][4];
+    // S^T = K Q^T: two 16-key row tiles; the Q fragments serve as B as they are
+    float s[2][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
+    for (int mt = 0; mt < 2; ++mt) s[mt][0] = s[mt][1] = s[mt][2] = s[mt][3] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
 #pragma unroll
-      for (int jp = 0; jp < 2; ++jp) {
-        const int r = jp * 16 + (lane & 7) + ((lane >> 4) << 3);
-        const int c = ks * 2 + ((lane >> 3) & 1);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(kb + swz(r, c), b0, b1, b2, b3);
-        mma16<T>(sc[2 * jp], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
-        mma16<T>(sc[2 * jp + 1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
+      for (int mt = 0; mt < 2; ++mt) {
+        const int r = mt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        const int c = ks * 2 + (lane >> 4);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(kb + swz(r, c), a0, a1, a2, a3);
+        mma16<T>(s[mt], a0, a1, a2, a3, qa[ks][0], qa[ks][1]);
       }
     }
-    float mx = -INFINITY;
+    // online softmax per query column over the tile's keys (rows row, row + 8
+    // of both row tiles here; the other rows sit in lanes row' = lane >> 2)
+    float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int kk = j * 8 + 2 * tq + e;
-        const float v = kk < valid ? sc[j][e] * scale_log2 : -INFINITY;
-        sc[j][e] = v;
-        mx = fmaxf(mx, v);
+      for (int i = 0; i < 4; ++i) {
+        const int kk = mt * 16 + row + ((i >> 1) << 3);
+        const float v = kk < valid ? s[mt][i] * scale_log2 : -INFINITY;
+        s[mt][i] = v;
+        mx[i & 1] = fmaxf(mx[i & 1], v);
       }
     }
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float mnew = fmaxf(m_r, mx);
-    const float corr = exp2f(m_r - mnew);
-    m_r = mnew;
-    float ls = 0.f;
-    uint32_t pa[2][2];
+    float corr[2], ls[2] = {0.f, 0.f};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float p0 = exp2f(sc[j][0] - mnew), p1 = exp2f(sc[j][1] - mnew);
-      ls += p0 + p1;
-      pa[j >> 1][j & 1] = pack2<T>(p0, p1);
+    for (int e = 0; e < 2; ++e) {
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], off));
+      const float mnew = fmaxf(m_r[e], mx[e]);
+      corr[e] = exp2f(m_r[e] - mnew);
+      m_r[e] = mnew;
     }
-    ls += __shfl_xor_sync(0xffffffffu, ls, 1);
-    ls += __shfl_xor_sync(0xffffffffu, ls, 2);
-    l_r = l_r * corr + ls;
-    // O += P V  (rows 8..15 of the tiles are zero padding)
+    // P^T as B fragments: each packed pair is a row of an 8x8 block (keys x
+    // queries) that movmatrix turns into the block's transpose
+    uint32_t pb[2][2];
 #pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
+    for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-      for (int np = 0; np < 8; ++np) {
-        const int r = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-        const int c = np * 2 + (lane >> 4);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vb + swz(r, c), b0, b1, b2, b3);
-        float t0[4] = {ks == 0 ? oacc[2 * np][0] * corr : oacc[2 * np][0],
-                       ks == 0 ? oacc[2 * np][1] * corr : oacc[2 * np][1], 0.f, 0.f};
-        float t1[4] = {ks == 0 ? oacc[2 * np + 1][0] * corr : oacc[2 * np + 1][0],
-                       ks == 0 ? oacc[2 * np + 1][1] * corr : oacc[2 * np + 1][1], 0.f, 0.f};
-        mma16<T>(t0, pa[ks][0], 0u, pa[ks][1], 0u, b0, b1);
-        mma16<T>(t1, pa[ks][0], 0u, pa[ks][1], 0u, b2, b3);
-        oacc[2 * np][0] = t0[0]; oacc[2 * np][1] = t0[1];
-        oacc[2 * np + 1][0] = t1[0]; oacc[2 * np + 1][1] = t1[1];
+      for (int h = 0; h < 2; ++h) {
+        const float p0 = exp2f(s[mt][2 * h] - m_r[0]), p1 = exp2f(s[mt][2 * h + 1] - m_r[1]);
+        ls[0] += p0;
+        ls[1] += p1;
+        const uint32_t pk = pack2<T>(p0, p1);
+        asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(pb[mt][h]) : "r"(pk));
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) ls[e] += __shfl_xor_sync(0xffffffffu, ls[e], off);
+      l_r[e] = l_r[e] * corr[e] + ls[e];
+    }
+    // O^T = O^T corr + V^T P^T: eight 16-dim row tiles, two 16-key steps
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      oacc[i][0] *= corr[0]; oacc[i][1] *= corr[1];
+      oacc[i][2] *= corr[0]; oacc[i][3] *= corr[1];
+    }
+#pragma unroll
+    for (int kt = 0; kt < 2; ++kt) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = kt * 16 + (lane & 7) + ((lane >> 4) << 3);
+        const int c = i * 2 + ((lane >> 3) & 1);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(vb + swz(r, c), a0, a1, a2, a3);
+        mma16<T>(oacc[i], a0, a1, a2, a3, pb[kt][0], pb[kt][1]);
       }
     }
     __syncwarp();   // the stage may be refilled from the next iteration on
     ++consumed;
     const int b_done = cp.b, g_done = cp.g;
     if (tc_next(cp, Ls)) {
-      if (real) {
-        const size_t slot = (size_t)b_done * Hk + g_done + k_cp;
-        float* dst = part + (slot * G + row) * 130;
+      const size_t slot = (size_t)b_done * Hk + g_done + k_cp;
 #pragma unroll
-        for (int n = 0; n < 16; ++n) *reinterpret_cast<float2*>(dst + n * 8 + 2 * tq) = make_float2(oacc[n][0], oacc[n][1]);
-        if (tq == 0) { dst[128] = m_r; dst[129] = l_r; }
+      for (int e = 0; e < 2; ++e) {
+        const int qh = 2 * tq + e;   // query head within the group
+        if (qh < G) {
+          float* dst = part + (slot * G + qh) * 130;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            dst[i * 16 + row] = oacc[i][e];
+            dst[i * 16 + row + 8] = oacc[i][2 + e];
+          }
+          if (row == 0) { dst[128] = m_r[e]; dst[129] = l_r[e]; }
+        }
       }
       start = true;
       if (cp.left <= 0) {   // the chunk is done: on to the next one the loader reached, if any
